@@ -1,0 +1,385 @@
+"""Throughput of the chunked SSD scan on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one ssd_scan_fwd over one batch of the 2.7B-shaped layer
+(B=8, L=16384, H=80, P=64, N=128, G=1, Q=256, bf16 io, fp32 state), inputs
+resident in HBM (x alone is 1.34 GB, larger than the 126 MB L2, so no flush
+is needed between steps).  With N > 1 (torchrun) every rank scans its own
+batch (independent sequences; no collective on the data path) and the time
+is the max over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the only reference there is) on
+a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SSD scan tokens/s & % of roofline (1×B200, B=8 L=16K H=80 P=64 N=128)"
+WORKLOAD = "mamba2_2p7b_layer"
+
+
+def algorithmic_bytes(wl) -> int:
+    """Bytes one scan must move at minimum: x, y, dt, B, C, A, D, init, final."""
+    Bz, L, H, P, N, G = wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.dstate, wl.ngroups
+    io = 2 if wl.io == "bf16" else 4
+    return (2 * Bz * L * H * P * io + Bz * L * H * 4 + 2 * Bz * L * G * N * io + 2 * H * 4
+            + 2 * Bz * H * N * P * 4)
+
+
+def algorithmic_flops(wl) -> float:
+    """Causal contractions per token-head: C.B^T shared by the H/G heads of a group
+    (Q*N/(2*H/G)), (S.L)X (Q*P/2), chunk state (N*P) and inter-chunk C.b (N*P); 2 flops/MAC."""
+    Bz, L, H, P, N, G, Q = wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.dstate, wl.ngroups, wl.chunk
+    mac = Q * N / (2 * H / G) + Q * P / 2 + 2 * N * P
+    return 2.0 * mac * Bz * L * H
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), float(pk.get("bf16_tflops_sustained", 0)), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "chunked_state_space_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        ent = t.get(kernel)
+        if ent and ent.get("source_hash") == kernel_source_hash():
+            return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+    return None
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML (read only) while running."""
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report nothing rather than guess
+            self.nv = None
+            self.err = str(e)
+        self.period = period_s
+
+    _NAMES = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h) if hasattr(
+                    nv, "nvmlDeviceGetCurrentClocksEventReasons") else nv.nvmlDeviceGetCurrentClocksThrottleReasons(
+                    self.h)
+                for bit, name in self._NAMES.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._thr is not None:
+            self._thr.join()
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def cpu_baseline(wl, target_s: float = 12.0):
+    """The fp64 oracle, as it stands, on a bounded sample: batch 0, all heads,
+    the first L' tokens (L' sized for about `target_s` seconds)."""
+    import oracle
+    from chunked_state_space_b200 import inputs
+    sub = inputs.custom(wl.name, batch=1, seqlen=min(wl.seqlen, 4096))
+    host = inputs.generate(sub)
+    args = [inputs.to_f64(host[k]) for k in ("x", "dt", "A", "B", "C", "D", "init")]
+    probe = 128
+    t0 = time.perf_counter()
+    oracle.scan_recurrence(args[0][:, :probe], args[1][:, :probe], args[2], args[3][:, :probe],
+                           args[4][:, :probe], args[5], args[6])
+    dt_probe = time.perf_counter() - t0
+    Lp = int(min(sub.seqlen, max(probe, probe * target_s / max(dt_probe, 1e-6))))
+    t0 = time.perf_counter()
+    oracle.scan_recurrence(args[0][:, :Lp], args[1][:, :Lp], args[2], args[3][:, :Lp], args[4][:, :Lp],
+                           args[5], args[6])
+    el = time.perf_counter() - t0
+    return {"value": Lp / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"batch 1 of {wl.batch}, first {Lp} of {wl.seqlen} tokens, all {wl.nheads} heads "
+                      f"(fp64 token recurrence, OpenMP over heads); {el:.1f} s"}
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle timed per step on a bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from chunked_state_space_b200 import inputs
+    import oracle
+    wl = inputs.WORKLOADS[WORKLOAD]
+    Lp = 256
+    sub = inputs.custom(wl.name, batch=1, seqlen=Lp)
+    host = inputs.generate(sub)
+    a = [inputs.to_f64(host[k]) for k in ("x", "dt", "A", "B", "C", "D", "init")]
+    for _ in range(args.warmup):
+        oracle.scan_recurrence(*a)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.scan_recurrence(*a)
+    el = time.perf_counter() - t0
+    val = Lp * args.steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "seqlen": wl.seqlen, "nheads": wl.nheads,
+                   "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk,
+                   "sample_per_step": f"batch 1, first {Lp} tokens, all {wl.nheads} heads"},
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"batch 1 of {wl.batch}, first {Lp} of {wl.seqlen} tokens per step"},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    from chunked_state_space_b200 import inputs, ssd
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    wl = inputs.WORKLOADS[args.workload]
+    host = inputs.generate(wl, seed=rank)          # each rank: its own independent batch
+    pinned = {}
+    for k, v in host.items():
+        t = torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16 else torch.from_numpy(v)
+        pinned[k] = t.pin_memory()
+    del host
+    d = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
+    y = torch.empty_like(d["x"])
+    fin = torch.empty((wl.batch, wl.nheads, wl.dstate, wl.headdim), dtype=torch.float32, device=dev)
+    dims = ssd.make_dims(d["x"], d["B"], wl.chunk)
+    ws = torch.empty(max(ssd.ssd_scan_workspace_size(dims), 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+
+    def step():
+        ssd.ssd_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init"], chunk=wl.chunk, y=y,
+                         final_state=fin, workspace=ws, stream=stream)
+
+    path, kernels_per_step = ssd.ssd_scan_path(dims)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    clocks = ClockSampler(local)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    per_step = [a.elapsed_time(b) for a, b in ev]
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_per_step = ms_total / args.steps
+    tokens = wl.batch * wl.seqlen * world
+    value = tokens / (ms_per_step * 1e-3)
+
+    # end to end through the public API from pinned host buffers
+    h_y = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    h_fin = torch.empty(fin.shape, dtype=fin.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = y.numel() * y.element_size() + fin.numel() * fin.element_size()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        for k, v in pinned.items():
+            d[k].copy_(v, non_blocking=True)
+        step()
+        h_y.copy_(y, non_blocking=True)
+        h_fin.copy_(fin, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = tokens / (e2e_ms * 1e-3)
+
+    hbm_peak, tc_peak, tc_sust, peak_src = load_peaks()
+    kernel_ms = statistics.mean(per_step) if path == "fused" and kernels_per_step == 1 else None
+    roofline = None
+    if kernel_ms is not None:
+        ach = algorithmic_bytes(wl) / (kernel_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
+                    "traffic": traffic_from_profile("ssd_fused"), "kernel": "ssd_fused",
+                    "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else
+                    "fallback 6650 GB/s",
+                    "tensor_tflops": algorithmic_flops(wl) / (kernel_ms * 1e-3) / 1e12,
+                    "tensor_frac_of_burst_peak": algorithmic_flops(wl) / (kernel_ms * 1e-3) / 1e12 / tc_peak}
+    else:
+        roofline = _unfused_roofline(wl, d, dims, stream, hbm_peak, peak_src)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "seqlen": wl.seqlen, "nheads": wl.nheads,
+                   "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk,
+                   "state_dtype": "f32", "path": path, "parallelism": f"dp{world} (independent batches per rank)",
+                   "l2": "inputs larger than L2 (x is 1.34 GB per rank); no flush"},
+        "clocks": clk, "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                               "d2h_bytes_per_step": d2h},
+        "gpu_launches": kernels_per_step * args.steps, "roofline": roofline,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def _unfused_roofline(wl, d, dims, stream, hbm_peak, peak_src):
+    """Time the four step kernels separately (CUDA events on the launching stream)
+    and report the dominant one against the HBM roofline."""
+    import torch
+    from chunked_state_space_b200 import ssd
+    nc = -(-wl.seqlen // wl.chunk)
+    lam = torch.empty((wl.batch, wl.nheads, nc, wl.chunk), dtype=torch.float32, device=d["x"].device)
+    st = torch.empty((wl.batch, wl.nheads, nc, wl.dstate, wl.headdim), dtype=torch.float32, device=d["x"].device)
+    y = torch.empty_like(d["x"])
+    fin = torch.empty_like(d["init"])
+    names = ["chunk_cumsum", "chunk_state", "state_passing", "chunk_scan"]
+    times = {n: [] for n in names}
+    for it in range(4):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        evs[0].record(stream)
+        ssd.ssd_chunk_cumsum(d["dt"], d["A"], dims, lam=lam, stream=stream)
+        evs[1].record(stream)
+        ssd.ssd_chunk_state(d["x"], d["B"], lam, dims, states=st, stream=stream)
+        evs[2].record(stream)
+        ssd.ssd_state_passing(st, lam, dims, init_state=d["init"], prev_states=st, final_state=fin, stream=stream)
+        evs[3].record(stream)
+        ssd.ssd_chunk_scan(d["x"], d["B"], d["C"], lam, st, dims, D=d["D"], y=y, stream=stream)
+        evs[4].record(stream)
+        torch.cuda.synchronize()
+        if it:
+            for i, n in enumerate(names):
+                times[n].append(evs[i].elapsed_time(evs[i + 1]))
+    mean = {n: statistics.mean(v) for n, v in times.items()}
+    top = max(mean, key=mean.get)
+    Bz, L, H, P, N, G = wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.dstate, wl.ngroups
+    st_bytes = Bz * H * nc * N * P * 4
+    lam_bytes = Bz * H * nc * wl.chunk * 4
+    xb = Bz * L * H * P * 2
+    bcb = Bz * L * G * N * 2
+    alg = {"chunk_cumsum": Bz * L * H * 4 + lam_bytes, "chunk_state": xb + bcb + lam_bytes + st_bytes,
+           "state_passing": 2 * st_bytes + lam_bytes // wl.chunk + 2 * Bz * H * N * P * 4,
+           "chunk_scan": 2 * xb + 2 * bcb + lam_bytes + st_bytes}
+    ach = alg[top] / (mean[top] * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
+            "traffic": traffic_from_profile(top), "kernel": top,
+            "kernel_ms": {n: round(v, 4) for n, v in mean.items()},
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else
+            "fallback 6650 GB/s"}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,213 @@
+/*
+ * ssd.h -- C ABI of the B200 chunked selective-state-space (SSD) scan library
+ *          (libssd.so, sm_100a).
+ *
+ * What it computes.  For every batch b and head h, with group g = h / (H/G):
+ *     a_t = exp(dt[b,t,h] * A[h])
+ *     h_t = a_t h_{t-1} + B[b,t,g,:] x[b,t,h,:]^T          (N x P state)
+ *     y_t = C[b,t,g,:]^T h_t + D[h] x[b,t,h,:]
+ * starting from init_state (or zero).  This is the recurrence of
+ * "分块推理：解锁循环模型并行计算，实现长序列高效处理" §2, with the per-token (selective)
+ * dt, B, C of "告别Transformer的二次方噩梦：用Mamba（S6）模型在长文本任务中实现线性时间推理"
+ * §2.1.  The library evaluates it chunk by chunk as that page's §2.1-§2.2
+ * derive: chunks of Q tokens, (1) a cumulative sum of the log-decays
+ * dt*A inside each chunk, (2) the chunk-local state b_intra(c) from a zero
+ * start, (3) the inter-chunk recursion b(c) = b_intra(c) + (prod a) b(c-1),
+ * and (4) the outputs by_intra (masked C B^T (.) L times X) plus the
+ * correction by_inter = diag(L) C(c) b(c-1).  ssd_vertical_fwd adds the
+ * page's §3.2 depth-first multi-layer schedule.
+ *
+ * Conventions shared by every entry point.
+ *  - Ownership: the caller allocates and owns every buffer.  The library
+ *    never allocates device memory and never synchronises the stream.
+ *  - Pointers: device pointers unless stated; each must be 16-byte aligned.
+ *  - Layout: contiguous row-major tensors:
+ *        x, y    [B, L, H, P]   (io dtype)      dt [B, L, H] (f32)
+ *        Bm, Cm  [B, L, G, N]   (io dtype)      A, D [H] (f32)
+ *        states  [B, H, N, P]   (f32)
+ *        lam     [B, H, nc, Q]  (f32), nc = ceil(L / Q)
+ *        chunk states / prev states [B, H, nc, N, P] (f32)
+ *  - dt must be positive and A non-positive (no softplus, bias or clamp is
+ *    applied); results for dt*A > 0 may overflow.
+ *  - L need not be a multiple of Q: the last chunk may be shorter.
+ *  - Streams: `stream` is a cudaStream_t (NULL = legacy default stream);
+ *    work is enqueued asynchronously on it.
+ *  - Errors: a status other than SSD_OK means no kernel was launched, except
+ *    SSD_ERR_CUDA (a launch failed part-way) and SSD_ERR_TIMEOUT (reported by
+ *    ssd_read_device_status after a bounded device-side wait gave up).
+ *  - Results are deterministic run to run (no atomics in reductions).
+ */
+#ifndef SSD_B200_SSD_H
+#define SSD_B200_SSD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SSD_OK = 0,
+  SSD_ERR_INVALID_ARG = 1, /* NULL where a pointer is required, bad enum, aliasing */
+  SSD_ERR_SHAPE = 2,       /* non-positive size, H % G != 0 */
+  SSD_ERR_DTYPE = 3,       /* io dtype not supported for this call */
+  SSD_ERR_ALIGN = 4,       /* pointer not 16-byte aligned */
+  SSD_ERR_UNSUPPORTED = 5, /* size outside the supported set (see ssd_dims) */
+  SSD_ERR_WORKSPACE = 6,   /* workspace NULL or smaller than the size query */
+  SSD_ERR_CUDA = 7,        /* a CUDA launch or query failed */
+  SSD_ERR_TIMEOUT = 8      /* a bounded device-side wait gave up */
+} ssd_status;
+
+typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
+
+/*
+ * Problem sizes.  Supported: batch, seqlen >= 1; 1 <= headdim (P) <= 64;
+ * 1 <= dstate (N) <= 128; 1 <= chunk (Q) <= 256; ngroups >= 1 dividing nheads.
+ * io_dtype is the dtype of x, Bm, Cm and y.  reserved must be 0.
+ */
+typedef struct ssd_dims {
+  int64_t batch;    /* B */
+  int64_t seqlen;   /* L */
+  int64_t nheads;   /* H */
+  int64_t headdim;  /* P */
+  int64_t dstate;   /* N */
+  int64_t ngroups;  /* G */
+  int64_t chunk;    /* Q */
+  int32_t io_dtype; /* ssd_dtype */
+  int32_t reserved;
+} ssd_dims;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* ssd_status_string(ssd_status s);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int ssd_version(void);
+
+/*
+ * Bytes of device workspace ssd_scan_fwd needs for `d` (written to *bytes).
+ * Errors: SSD_ERR_INVALID_ARG (NULL), SSD_ERR_SHAPE, SSD_ERR_UNSUPPORTED,
+ * SSD_ERR_DTYPE.
+ */
+ssd_status ssd_scan_workspace_size(const ssd_dims* d, size_t* bytes);
+
+/*
+ * One layer of the chunked scan, "分块推理…" §2.1-§2.2: y and the final state
+ * from x, dt, A, Bm, Cm, D and the initial state, all four steps on `stream`.
+ *   x [B,L,H,P] io, dt [B,L,H] f32, A [H] f32, Bm/Cm [B,L,G,N] io,
+ *   D [H] f32 or NULL (= 0), init_state [B,H,N,P] f32 or NULL (= 0),
+ *   y [B,L,H,P] io (written; must not overlap any input),
+ *   final_state [B,H,N,P] f32 or NULL (may alias init_state),
+ *   workspace: device scratch of at least ssd_scan_workspace_size bytes,
+ *   owned by the caller, contents need not be initialised.
+ * Picks the tensor-core path for bf16 io when the sizes allow it, else the
+ * CUDA-core path.  Errors: every status above.
+ */
+ssd_status ssd_scan_fwd(const ssd_dims* d, const void* x, const float* dt, const float* A,
+                        const void* Bm, const void* Cm, const float* D, const float* init_state,
+                        void* y, float* final_state, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/*
+ * Which implementation ssd_scan_fwd uses for `d`: *path = SSD_PATH_CUDA_CORES
+ * (four CUDA-core step kernels), SSD_PATH_TENSOR_STEPS (four step kernels,
+ * steps 2 and 4 on tcgen05 tensor cores) or SSD_PATH_FUSED (one persistent
+ * tensor-core kernel); *kernels = kernel launches per call.  Either output
+ * pointer may be NULL.  Errors: as ssd_scan_workspace_size.
+ */
+enum { SSD_PATH_CUDA_CORES = 0, SSD_PATH_TENSOR_STEPS = 1, SSD_PATH_FUSED = 2 };
+ssd_status ssd_scan_path(const ssd_dims* d, int32_t* path, int32_t* kernels);
+
+/* The same computation, forced through the four separate step kernels below
+ * (the step-testable path).  Same arguments and errors as ssd_scan_fwd. */
+ssd_status ssd_scan_fwd_unfused(const ssd_dims* d, const void* x, const float* dt, const float* A,
+                                const void* Bm, const void* Cm, const float* D,
+                                const float* init_state, void* y, float* final_state,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Step 1, the log-decay cumulative sum ("分块推理…" §2.2, the product of A_t over a
+ * chunk, taken in log space):  lam[b,h,c,i] = sum_{r=0..i} dt[b,cQ+r,h] * A[h]
+ * for i < len(c); positions past the end of a short last chunk repeat the
+ * chunk total.  Summed sequentially in fp32 so that differences
+ * lam[t] - lam[s] keep their accuracy.
+ */
+ssd_status ssd_chunk_cumsum(const ssd_dims* d, const float* dt, const float* A, float* lam,
+                            void* stream);
+
+/*
+ * Step 2, chunk-local states from a zero start ("分块推理…" §2.1, b_intra):
+ *   chunk_states[b,h,c,n,p] = sum_{s in c} exp(lam_end(c) - lam_s) Bm[b,s,g,n] x[b,s,h,p]
+ * (fp32 accumulation; tensor cores for bf16 io where supported).
+ */
+ssd_status ssd_chunk_state(const ssd_dims* d, const void* x, const void* Bm, const float* lam,
+                           float* chunk_states, void* stream);
+
+/*
+ * Step 3, the inter-chunk recursion ("分块推理…" §2.2):
+ *   b(-1) = init_state (or 0);  b(c) = chunk_states(c) + exp(lam_end(c)) b(c-1)
+ * writes prev_states(c) = b(c-1) for every chunk and final_state = b(nc-1).
+ * prev_states may alias chunk_states (updated in place); final_state may be
+ * NULL and may alias init_state.
+ */
+ssd_status ssd_state_passing(const ssd_dims* d, const float* chunk_states, const float* lam,
+                             const float* init_state, float* prev_states, float* final_state,
+                             void* stream);
+
+/*
+ * Step 4, chunk outputs ("分块推理…" §2.1-§2.2, y = by_intra + by_inter):
+ *   y_t = sum_{s<=t, s in c} (C_t . B_s) exp(lam_t - lam_s) x_s
+ *       + exp(lam_t) C_t^T prev_states(c) + D[h] x_t
+ */
+ssd_status ssd_chunk_scan(const ssd_dims* d, const void* x, const void* Bm, const void* Cm,
+                          const float* lam, const float* D, const float* prev_states, void* y,
+                          void* stream);
+
+/*
+ * Layer-to-layer normalisation of the multi-layer stack (a reading: the
+ * pages only say that layer l's output feeds layer l+1):
+ *   out[r,:] = in[r,:] / sqrt(mean_f in[r,f]^2 + eps), computed in fp32,
+ * for `rows` rows of `features` contiguous values; in/out in `io_dtype`
+ * (may alias).
+ */
+ssd_status ssd_rmsnorm(int64_t rows, int64_t features, int32_t io_dtype, const void* in, float eps,
+                       void* out, void* stream);
+
+/*
+ * Bytes of workspace ssd_vertical_fwd needs for `d`, `n_layers` and the
+ * vertical block length `vblock` (V).
+ */
+ssd_status ssd_vertical_workspace_size(const ssd_dims* d, int32_t n_layers, int64_t vblock,
+                                       size_t* bytes);
+
+/*
+ * Depth-first multi-layer schedule, "分块推理…" §3.2: the sequence is cut into
+ * V-token blocks; each block passes through layers 0..n_layers-1 before the
+ * next block starts, and every layer keeps its state b between blocks.
+ *   x0: layer-0 input [B,L,H,P] io.
+ *   dt, A, Bm, Cm, D: HOST arrays of n_layers DEVICE pointers (D[l] may be
+ *   NULL), each with the single-layer layout above.
+ *   states: HOST array of n_layers DEVICE pointers [B,H,N,P] f32: the initial
+ *   state of each layer on entry, its final state on return (in place).
+ *   y_out: the last layer's output [B,L,H,P] io.
+ * Layer l+1's input is ssd_rmsnorm(y_l) (eps = rms_eps), stored in io dtype.
+ * When V is a multiple of Q the result is bitwise equal to running the layers
+ * one after another over the whole sequence (the §3.1 horizontal schedule).
+ */
+ssd_status ssd_vertical_fwd(const ssd_dims* d, int32_t n_layers, int64_t vblock, float rms_eps,
+                            const void* x0, const float* const* dt, const float* const* A,
+                            const void* const* Bm, const void* const* Cm, const float* const* D,
+                            float* const* states, void* y_out, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
+ * Read and clear the device status word that bounded waits inside the
+ * kernels set (synchronises `stream`).  Returns SSD_OK or SSD_ERR_TIMEOUT.
+ */
+ssd_status ssd_read_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_B200_SSD_H */

@@ -1,0 +1,46 @@
+/*
+ * ssd_selftest.h -- diagnostic entry point of libssd.so (no counterpart on the
+ * pages: it checks the tensor-core building blocks the scan kernels are made
+ * of, not the scan).
+ *
+ * ssd_selftest_umma computes D[128 x N] = A[128 x K] * B[K x N] on one CTA
+ * with bf16 inputs and fp32 accumulation through tcgen05.mma, staging the
+ * operands in the layout named by `variant`:
+ *   SSD_SELFTEST_A_K_B_K            A [128][K] and B [N][K] in global, both K-major in smem
+ *   SSD_SELFTEST_A_K_B_MN           A [128][K] K-major, B [K][N] MN-major
+ *   SSD_SELFTEST_A_MN_B_MN          A [K][128] MN-major, B [K][N] MN-major
+ *   SSD_SELFTEST_A_MN_B_MN_SWAPPED  as above with the two descriptor strides exchanged
+ *                                   (expected to be wrong; documents the encoding)
+ *   SSD_SELFTEST_TS_A_TMEM_B_MN     A [128][K] placed in tensor memory, B [K][N] MN-major
+ *   SSD_SELFTEST_TMA_A_K_B_MN       as A_K_B_MN but both operands loaded by TMA
+ * A, B: device bf16, D: device fp32 [128][N]; N in {64, 128}; K in {64, 128, 256};
+ * 16-byte aligned.  Asynchronous on `stream`.  Errors: SSD_ERR_INVALID_ARG,
+ * SSD_ERR_UNSUPPORTED, SSD_ERR_ALIGN, SSD_ERR_CUDA; a bounded wait that gives
+ * up raises the status read by ssd_read_device_status.
+ */
+#ifndef SSD_B200_SSD_SELFTEST_H
+#define SSD_B200_SSD_SELFTEST_H
+
+#include "ssd.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  SSD_SELFTEST_A_K_B_K = 0,
+  SSD_SELFTEST_A_K_B_MN = 1,
+  SSD_SELFTEST_A_MN_B_MN = 2,
+  SSD_SELFTEST_A_MN_B_MN_SWAPPED = 3,
+  SSD_SELFTEST_TS_A_TMEM_B_MN = 4,
+  SSD_SELFTEST_TMA_A_K_B_MN = 5
+};
+
+ssd_status ssd_selftest_umma(int32_t variant, const void* A, const void* B, float* D, int32_t N, int32_t K,
+                             void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_B200_SSD_SELFTEST_H */

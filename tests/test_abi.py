@@ -1,0 +1,143 @@
+"""The C-ABI library (CPU only: no kernel is launched here).
+
+Checks that libssd.so loads, exports every function include/ssd.h declares,
+and that argument validation rejects bad calls with the documented status
+before anything reaches the GPU.  Pointers below are fake addresses: every
+call returns from validation before using them.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from chunked_state_space_b200 import build as ssd_build
+from chunked_state_space_b200 import ssd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for hdr in os.listdir(os.path.join(ROOT, "include")):
+        if hdr.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", hdr)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(ssd_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ssd_build.build()
+    return ssd.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "ssd_scan_fwd" in names and "ssd_vertical_fwd" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    # the binding knows the same list
+    assert set(ssd.EXPORTED) >= set(names)
+
+
+def test_status_strings_and_version(lib):
+    for code, name in enumerate(ssd.STATUS_NAMES):
+        assert ssd.status_string(code).startswith(name)
+    assert ssd.status_string(99) == "SSD_ERR_UNKNOWN"
+    assert ssd.ssd_version() == 100
+
+
+def dims(**kw):
+    d = dict(batch=2, seqlen=1000, nheads=4, headdim=64, dstate=128, ngroups=2, chunk=256, io_dtype=1,
+             reserved=0)
+    d.update(kw)
+    return ssd.Dims(**d)
+
+
+def ws_size(d):
+    n = ctypes.c_size_t(0)
+    s = ssd.lib().ssd_scan_workspace_size(ctypes.byref(d), ctypes.byref(n))
+    return s, n.value
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(batch=0), 2), (dict(seqlen=0), 2), (dict(nheads=3), 2), (dict(ngroups=0), 2),
+    (dict(headdim=65), 5), (dict(dstate=129), 5), (dict(chunk=257), 5), (dict(io_dtype=2), 3),
+    (dict(reserved=1), 1), (dict(nheads=70000, ngroups=1), 5),
+])
+def test_workspace_size_rejects(lib, kw, status):
+    s, _ = ws_size(dims(**kw))
+    assert s == status, ssd.status_string(s)
+
+
+def test_workspace_size_values(lib):
+    s, n = ws_size(dims())
+    assert s == 0
+    nc = 4
+    lam = 2 * 4 * nc * 256 * 4
+    states = 2 * 4 * nc * 128 * 64 * 4
+    assert n >= lam + states
+    assert lib.ssd_scan_workspace_size(None, ctypes.byref(ctypes.c_size_t())) == 1
+    assert lib.ssd_scan_workspace_size(ctypes.byref(dims()), None) == 1
+
+
+# fake, 256-byte aligned device addresses far apart
+BASE = 1 << 40
+GB = 1 << 30
+
+
+def call_scan(d, **over):
+    ptr = dict(x=BASE, dt=BASE + 2 * GB, A=BASE + 3 * GB, B=BASE + 4 * GB, C=BASE + 5 * GB, D=BASE + 6 * GB,
+               init=BASE + 7 * GB, y=BASE + 8 * GB, final=BASE + 9 * GB, ws=BASE + 10 * GB)
+    ptr.update(over)
+    wsb = over.get("wsbytes", 1 << 40)
+    p = lambda k: ctypes.c_void_p(ptr[k]) if ptr[k] is not None else None
+    return ssd.lib().ssd_scan_fwd(ctypes.byref(d), p("x"), p("dt"), p("A"), p("B"), p("C"), p("D"), p("init"),
+                                  p("y"), p("final"), p("ws"), wsb, None)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(x=None), 1), (dict(dt=None), 1), (dict(y=None), 1),
+    (dict(x=BASE + 8), 4), (dict(D=BASE + 6 * GB + 4), 4), (dict(final=BASE + 9 * GB + 2), 4),
+    (dict(y=BASE + 1024), 1),                     # y overlaps x
+    (dict(final=BASE + 7 * GB + 256), 1),         # final partially overlaps init
+    (dict(ws=None), 6), (dict(wsbytes=1024), 6), (dict(ws=BASE + 10 * GB + 8), 4),
+])
+def test_scan_fwd_rejects(lib, over, status):
+    s = call_scan(dims(), **over)
+    assert s == status, ssd.status_string(s)
+
+
+def test_scan_fwd_rejects_bad_dims(lib):
+    assert call_scan(dims(nheads=5)) == 2
+    assert call_scan(dims(io_dtype=7)) == 3
+    assert lib.ssd_scan_fwd(None, *([None] * 10), 0, None) == 1
+
+
+def test_step_entry_points_reject(lib):
+    d = dims()
+    p = ctypes.c_void_p(BASE)
+    assert lib.ssd_chunk_cumsum(ctypes.byref(d), None, p, p, None) == 1
+    assert lib.ssd_chunk_cumsum(ctypes.byref(d), ctypes.c_void_p(BASE + 4), p, p, None) == 4
+    assert lib.ssd_chunk_state(ctypes.byref(d), p, None, p, p, None) == 1
+    assert lib.ssd_state_passing(ctypes.byref(d), p, p, None, None, None, None) == 1
+    assert lib.ssd_chunk_scan(ctypes.byref(d), p, p, p, p, None, None, p, None) == 1
+    assert lib.ssd_rmsnorm(4, 0, 1, p, 1e-6, p, None) == 2
+    assert lib.ssd_rmsnorm(4, 16, 5, p, 1e-6, p, None) == 3
+    assert lib.ssd_rmsnorm(4, 16, 1, None, 1e-6, p, None) == 1
+    assert lib.ssd_rmsnorm(4, 16, 1, p, -1.0, p, None) == 1
+
+
+def test_vertical_rejects(lib):
+    d = dims()
+    n = ctypes.c_size_t(0)
+    assert lib.ssd_vertical_workspace_size(ctypes.byref(d), 0, 2048, ctypes.byref(n)) == 2
+    assert lib.ssd_vertical_workspace_size(ctypes.byref(d), 3, 0, ctypes.byref(n)) == 2
+    assert lib.ssd_vertical_workspace_size(ctypes.byref(d), 3, 512, ctypes.byref(n)) == 0
+    one = ctypes.c_size_t(0)
+    dv = dims(seqlen=512)
+    assert lib.ssd_scan_workspace_size(ctypes.byref(dv), ctypes.byref(one)) == 0
+    assert n.value >= one.value + 2 * 2 * 512 * 4 * 64 * 2
+    assert lib.ssd_vertical_fwd(ctypes.byref(d), 2, 512, 1e-6, None, *([None] * 6), None, None, 0, None) == 1

@@ -1,0 +1,263 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Tolerances (max|y - y_ref| / max|y_ref|, same for the final state):
+1e-5 for fp32 io, 5e-3 for bf16 io with fp32 accumulation.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from chunked_state_space_b200 import inputs
+from chunked_state_space_b200 import ssd
+from gpu_util import TOL, device_inputs, oracle_args, oracle_sampled, rel_err, to_dev, to_np64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    ssd.lib()  # fails loudly if libssd.so is missing
+    yield
+    torch.cuda.synchronize()
+
+
+def run_scan(dev, wl, unfused=False, **kw):
+    y, fin = ssd.ssd_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
+                              chunk=wl.chunk, unfused=unfused, **kw)
+    torch.cuda.synchronize()
+    return y, fin
+
+
+def check_full(wl, seed=0, paths=("default", "unfused")):
+    host = inputs.generate(wl, seed=seed)
+    dev = device_inputs(host)
+    y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host))
+    for path in paths:
+        y, fin = run_scan(dev, wl, unfused=(path == "unfused"))
+        ey, ef = rel_err(to_np64(y), y_ref), rel_err(to_np64(fin), f_ref)
+        assert ey <= TOL[wl.io], (path, ey)
+        assert ef <= TOL[wl.io], (path, ef)
+    return host, dev
+
+
+# ------------------------------------------------------------------ small workloads, whole output
+
+def test_tiny_f32_workload():
+    check_full(inputs.WORKLOADS["tiny_f32"])
+
+
+@pytest.mark.parametrize("over", [
+    dict(base="tiny_f32", batch=2, seqlen=300, nheads=4, ngroups=2, headdim=16, dstate=16, chunk=64),
+    dict(base="tiny_f32", batch=1, seqlen=1, nheads=2, chunk=64),
+    dict(base="tiny_f32", batch=1, seqlen=50, nheads=2, chunk=64),         # L < Q
+    dict(base="tiny_f32", batch=2, seqlen=33, nheads=3, ngroups=3, headdim=5, dstate=3, chunk=1),
+    dict(base="tiny_f32", batch=1, seqlen=130, nheads=2, headdim=1, dstate=1, chunk=16),
+    dict(base="tiny_f32", batch=1, seqlen=517, nheads=2, headdim=64, dstate=128, chunk=256, init_var=0.5),
+    dict(base="mamba2_130m_layer", batch=2, seqlen=700, nheads=4, ngroups=2, init_var=0.1),
+    dict(base="mamba2_130m_layer", batch=1, seqlen=1, nheads=2),
+    dict(base="mamba2_130m_layer", batch=1, seqlen=255, nheads=2, init_var=0.1),
+    dict(base="mamba2_130m_layer", batch=1, seqlen=1000, nheads=3, headdim=32, dstate=64, chunk=128),
+    dict(base="mamba2_130m_layer", batch=1, seqlen=200, nheads=2, headdim=7, dstate=9, chunk=40),
+])
+def test_shapes_and_edges(over):
+    over = dict(over)
+    base = over.pop("base")
+    check_full(inputs.custom(base, **over))
+
+
+def test_no_d_no_init_and_aliasing():
+    wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=600, nheads=2, init_var=0.1)
+    host = inputs.generate(wl)
+    dev = device_inputs(host)
+    args = oracle_args(host)
+    y_ref, f_ref = oracle.scan_recurrence(*args[:5], None, None)
+    y, fin = ssd.ssd_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], None, None, chunk=wl.chunk)
+    torch.cuda.synchronize()
+    assert rel_err(to_np64(y), y_ref) <= TOL["bf16"]
+    assert rel_err(to_np64(fin), f_ref) <= TOL["bf16"]
+    # final_state may alias init_state
+    y_ref2, f_ref2 = oracle.scan_recurrence(*args)
+    st = dev["init"].clone()
+    y2, _ = ssd.ssd_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], st, chunk=wl.chunk,
+                             final_state=st)
+    torch.cuda.synchronize()
+    assert rel_err(to_np64(y2), y_ref2) <= TOL["bf16"]
+    assert rel_err(to_np64(st), f_ref2) <= TOL["bf16"]
+
+
+def test_deterministic():
+    wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=1100, nheads=4, init_var=0.1)
+    dev = device_inputs(inputs.generate(wl))
+    y1, f1 = run_scan(dev, wl)
+    y2, f2 = run_scan(dev, wl)
+    assert torch.equal(y1, y2) and torch.equal(f1, f2)
+
+
+# ------------------------------------------------------------------ the four steps, one at a time
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_steps_match_oracle_intermediates(io):
+    if io == "f32":
+        wl = inputs.custom("tiny_f32", batch=2, seqlen=300, nheads=4, ngroups=2, init_var=0.3)
+    else:
+        wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=700, nheads=4, ngroups=2, init_var=0.1)
+    tol = TOL[io]
+    host = inputs.generate(wl)
+    dev = device_inputs(host)
+    args = oracle_args(host)
+    ref = oracle.scan_chunked(*args[:5], wl.chunk, args[5], args[6])
+    x, Bm = dev["x"], dev["B"]
+    dims = ssd.make_dims(x, Bm, wl.chunk)
+    f32 = lambda a: torch.from_numpy(a.astype(np.float32)).cuda()
+    # step 1
+    lam = ssd.ssd_chunk_cumsum(dev["dt"], dev["A"], dims)
+    torch.cuda.synchronize()
+    assert rel_err(to_np64(lam), ref["lam"]) <= 1e-6
+    # step 2 on the oracle's lam
+    cs = ssd.ssd_chunk_state(x, Bm, f32(ref["lam"]), dims)
+    torch.cuda.synchronize()
+    assert rel_err(to_np64(cs), ref["chunk_states"]) <= tol
+    # step 3 on the oracle's chunk states
+    prev, fin = ssd.ssd_state_passing(f32(ref["chunk_states"]), f32(ref["lam"]), dims, init_state=dev["init"])
+    torch.cuda.synchronize()
+    assert rel_err(to_np64(prev), ref["prev_states"]) <= 1e-5
+    assert rel_err(to_np64(fin), ref["final"]) <= 1e-5
+    # step 3 in place (prev aliases chunk states)
+    buf = f32(ref["chunk_states"])
+    ssd.ssd_state_passing(buf, f32(ref["lam"]), dims, init_state=dev["init"], prev_states=buf)
+    torch.cuda.synchronize()
+    assert rel_err(to_np64(buf), ref["prev_states"]) <= 1e-5
+    # step 4 on the oracle's prev states
+    y = ssd.ssd_chunk_scan(x, Bm, dev["C"], f32(ref["lam"]), f32(ref["prev_states"]), dims, D=dev["D"])
+    torch.cuda.synchronize()
+    assert rel_err(to_np64(y), ref["y"]) <= tol
+
+
+def test_rmsnorm_matches_oracle():
+    rng = np.random.default_rng(0)
+    a = rng.standard_normal((2, 37, 24, 64)).astype(np.float32) * 3.0
+    t = torch.from_numpy(a).cuda().to(torch.bfloat16)
+    out = ssd.ssd_rmsnorm(t, 1e-6)
+    torch.cuda.synchronize()
+    ref = oracle.rmsnorm_bf16(to_np64(t), 1e-6)
+    # both round to bf16: compare within one bf16 ulp of the normalised values
+    assert np.max(np.abs(to_np64(out) - ref)) <= 2.0 ** -7 * np.max(np.abs(ref))
+    # in place
+    t2 = t.clone()
+    ssd.ssd_rmsnorm(t2, 1e-6, out=t2)
+    torch.cuda.synchronize()
+    assert torch.equal(t2, out)
+
+
+# ------------------------------------------------------------------ the named workloads at full size
+
+def test_mamba2_130m_layer_full():
+    check_full(inputs.WORKLOADS["mamba2_130m_layer"])
+
+
+def _sample_pairs(Bz, H, n, seed):
+    rng = np.random.default_rng(seed)
+    pairs = {(0, 0), (Bz - 1, H - 1)}
+    while len(pairs) < n:
+        pairs.add((int(rng.integers(Bz)), int(rng.integers(H))))
+    return sorted(pairs)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,nsamp", [("mamba2_2p7b_layer", 12), ("long_context_layer", 6)])
+def test_full_size_sampled(name, nsamp):
+    """Full-size run in the benchmark's launch configuration; the oracle checks
+    sampled (batch, head) rows over the whole sequence and their final states."""
+    wl = inputs.WORKLOADS[name]
+    host = inputs.generate(wl)
+    dev = device_inputs(host)
+    y, fin = run_scan(dev, wl)
+    pairs = _sample_pairs(wl.batch, wl.nheads, nsamp, seed=1)
+    y_ref, f_ref = oracle_sampled(host, wl, pairs)
+    for i, (b, h) in enumerate(pairs):
+        ey = rel_err(to_np64(y[b, :, h]), y_ref[i])
+        ef = rel_err(to_np64(fin[b, h]), f_ref[i])
+        assert ey <= TOL["bf16"], (b, h, ey)
+        assert ef <= TOL["bf16"], (b, h, ef)
+    assert torch.isfinite(y.float()).all()
+    del dev, y, fin
+    torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------ multi-layer stack: vertical vs horizontal
+
+def _stack_layers(wl, n_layers):
+    layers_host = [inputs.generate(wl, layer=l, names=("dt", "A", "B", "C", "D")) for l in range(n_layers)]
+    return layers_host, [device_inputs(h) for h in layers_host]
+
+
+def _horizontal_gpu(x0, layers, states, wl, eps):
+    x = x0
+    y = None
+    for l, p in enumerate(layers):
+        y, _ = ssd.ssd_scan_fwd(x, p["dt"], p["A"], p["B"], p["C"], p["D"], states[l], chunk=wl.chunk,
+                                final_state=states[l])
+        if l + 1 < len(layers):
+            x = ssd.ssd_rmsnorm(y, eps)
+    torch.cuda.synchronize()
+    return y
+
+
+@pytest.mark.parametrize("L,V", [(1024, 256), (1000, 256), (1000, 300)])
+def test_vertical_small(L, V):
+    wl = inputs.custom("stack24_vertical", batch=2, seqlen=L, nheads=4)
+    n_layers, eps = 3, 1e-6
+    host_layers, dev_layers = _stack_layers(wl, n_layers)
+    x0h = inputs.generate(wl, names=("x",))["x"]
+    x0 = to_dev(x0h)
+    zero = lambda: [torch.zeros((wl.batch, wl.nheads, wl.dstate, wl.headdim), device="cuda")
+                    for _ in range(n_layers)]
+    st_v, st_h = zero(), zero()
+    yv = ssd.ssd_vertical_fwd(x0, dev_layers, st_v, vblock=V, chunk=wl.chunk, rms_eps=eps)
+    yh = _horizontal_gpu(x0, dev_layers, st_h, wl, eps)
+    if V % wl.chunk == 0:
+        assert torch.equal(yv, yh)
+        for a, b in zip(st_v, st_h):
+            assert torch.equal(a, b)
+    layers64 = [dict(dt=inputs.to_f64(h["dt"]), A=inputs.to_f64(h["A"]), B=inputs.to_f64(h["B"]),
+                     C=inputs.to_f64(h["C"]), D=inputs.to_f64(h["D"])) for h in host_layers]
+    y_ref, f_ref = oracle.stack_horizontal(inputs.to_f64(x0h), layers64, eps)
+    assert rel_err(to_np64(yv), y_ref) <= TOL["bf16"]
+    for a, r in zip(st_v, f_ref):
+        assert rel_err(to_np64(a), r) <= TOL["bf16"]
+
+
+@pytest.mark.slow
+def test_stack24_vertical_full():
+    """The 24-layer stack at full size: vertical == horizontal bitwise on the
+    GPU (V % Q == 0), the prefix of the full run equals a run on the prefix
+    alone (causality), and that prefix run matches the oracle for batch 0."""
+    wl = inputs.WORKLOADS["stack24_vertical"]
+    n_layers, eps, V = wl.n_layers, 1e-6, wl.vblock
+    host_layers, dev_layers = _stack_layers(wl, n_layers)
+    x0h = inputs.generate(wl, names=("x",))["x"]
+    x0 = to_dev(x0h)
+    zero = lambda Bz: [torch.zeros((Bz, wl.nheads, wl.dstate, wl.headdim), device="cuda") for _ in range(n_layers)]
+    st_v, st_h = zero(wl.batch), zero(wl.batch)
+    yv = ssd.ssd_vertical_fwd(x0, dev_layers, st_v, vblock=V, chunk=wl.chunk, rms_eps=eps)
+    torch.cuda.synchronize()
+    yh = _horizontal_gpu(x0, dev_layers, st_h, wl, eps)
+    assert torch.equal(yv, yh)
+    for a, b in zip(st_v, st_h):
+        assert torch.equal(a, b)
+    # prefix run (batch 0, 2 V-blocks)
+    Lp = 2 * V
+    pre = lambda t: t[:1, :Lp].contiguous()
+    dev_pre = [dict(dt=pre(p["dt"]), A=p["A"], B=pre(p["B"]), C=pre(p["C"]), D=p["D"]) for p in dev_layers]
+    st_p = zero(1)
+    yp = ssd.ssd_vertical_fwd(pre(x0), dev_pre, st_p, vblock=V, chunk=wl.chunk, rms_eps=eps)
+    torch.cuda.synchronize()
+    assert torch.equal(yp, yv[:1, :Lp])
+    layers64 = [dict(dt=inputs.to_f64(h["dt"][:1, :Lp]), A=inputs.to_f64(h["A"]), B=inputs.to_f64(h["B"][:1, :Lp]),
+                     C=inputs.to_f64(h["C"][:1, :Lp]), D=inputs.to_f64(h["D"])) for h in host_layers]
+    y_ref, f_ref = oracle.stack_horizontal(inputs.to_f64(x0h[:1, :Lp]), layers64, eps)
+    assert rel_err(to_np64(yp), y_ref) <= TOL["bf16"]
+    for a, r in zip(st_p, f_ref):
+        assert rel_err(to_np64(a), r) <= TOL["bf16"]

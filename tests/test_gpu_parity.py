@@ -229,35 +229,83 @@ def test_vertical_small(L, V):
         assert rel_err(to_np64(a), r) <= TOL["bf16"]
 
 
+def _stack_sensitivity(x0, layers64, eps, rel=1e-7, seed=0):
+    """How far the oracle's own last-layer output moves when every layer's output
+    is perturbed by `rel` (fp32-level) before its bf16 storage rounding."""
+    rng = np.random.default_rng(seed)
+    x = x0
+    y = None
+    for li, p in enumerate(layers64):
+        y, _ = oracle.scan_recurrence(x, p["dt"], p["A"], p["B"], p["C"], p["D"], None)
+        if li + 1 < len(layers64):
+            x = oracle.rmsnorm_bf16(oracle.round_bf16(y * (1 + rel * rng.standard_normal(y.shape))), eps)
+    return y
+
+
 @pytest.mark.slow
 def test_stack24_vertical_full():
-    """The 24-layer stack at full size: vertical == horizontal bitwise on the
-    GPU (V % Q == 0), the prefix of the full run equals a run on the prefix
-    alone (causality), and that prefix run matches the oracle for batch 0."""
+    """The 24-layer stack at full size.
+
+    1. vertical == horizontal bitwise on the GPU (V % Q == 0);
+    2. every layer, teacher-forced: the GPU's y_l and final state for a sampled
+       (batch, head) over the whole sequence match the oracle run on the GPU's
+       own bf16 input x_l (5e-3), and x_{l+1} is the RMS-normalised y_l;
+    3. end to end on a prefix against the oracle's stack, with the tolerance
+       set by the oracle's own sensitivity to fp32-level perturbations before
+       each bf16 storage rounding (the stack amplifies rounding-boundary flips).
+    """
     wl = inputs.WORKLOADS["stack24_vertical"]
     n_layers, eps, V = wl.n_layers, 1e-6, wl.vblock
     host_layers, dev_layers = _stack_layers(wl, n_layers)
     x0h = inputs.generate(wl, names=("x",))["x"]
     x0 = to_dev(x0h)
     zero = lambda Bz: [torch.zeros((Bz, wl.nheads, wl.dstate, wl.headdim), device="cuda") for _ in range(n_layers)]
-    st_v, st_h = zero(wl.batch), zero(wl.batch)
+    st_v = zero(wl.batch)
     yv = ssd.ssd_vertical_fwd(x0, dev_layers, st_v, vblock=V, chunk=wl.chunk, rms_eps=eps)
     torch.cuda.synchronize()
-    yh = _horizontal_gpu(x0, dev_layers, st_h, wl, eps)
-    assert torch.equal(yv, yh)
+    # horizontal schedule, keeping every layer's input and output
+    st_h = zero(wl.batch)
+    xs, ys = [x0], []
+    for l, p in enumerate(dev_layers):
+        y, _ = ssd.ssd_scan_fwd(xs[-1], p["dt"], p["A"], p["B"], p["C"], p["D"], st_h[l], chunk=wl.chunk,
+                                final_state=st_h[l])
+        ys.append(y)
+        if l + 1 < n_layers:
+            xs.append(ssd.ssd_rmsnorm(y, eps))
+    torch.cuda.synchronize()
+    assert torch.equal(yv, ys[-1])
     for a, b in zip(st_v, st_h):
         assert torch.equal(a, b)
-    # prefix run (batch 0, 2 V-blocks)
-    Lp = 2 * V
+    # 2. teacher-forced per layer, one sampled (batch, head) per layer, full length, one oracle call
+    rng = np.random.default_rng(2)
+    samp = [(int(rng.integers(wl.batch)), int(rng.integers(wl.nheads))) for _ in range(n_layers)]
+    f = inputs.to_f64
+    xo = np.stack([to_np64(xs[l][b, :, h]) for l, (b, h) in enumerate(samp)], axis=1)[None]
+    dto = np.stack([f(host_layers[l]["dt"][b, :, h]) for l, (b, h) in enumerate(samp)], axis=1)[None]
+    Bo = np.stack([f(host_layers[l]["B"][b, :, 0]) for l, (b, h) in enumerate(samp)], axis=1)[None]
+    Co = np.stack([f(host_layers[l]["C"][b, :, 0]) for l, (b, h) in enumerate(samp)], axis=1)[None]
+    Ao = np.array([f(host_layers[l]["A"])[h] for l, (b, h) in enumerate(samp)])
+    Do = np.array([f(host_layers[l]["D"])[h] for l, (b, h) in enumerate(samp)])
+    y_ref, f_ref = oracle.scan_recurrence(xo, dto, Ao, Bo, Co, Do, None)
+    for l, (b, h) in enumerate(samp):
+        assert rel_err(to_np64(ys[l][b, :, h]), y_ref[0, :, l]) <= TOL["bf16"], ("layer", l)
+        assert rel_err(to_np64(st_h[l][b, h]), f_ref[0, l]) <= TOL["bf16"], ("state", l)
+    for l in range(n_layers - 1):
+        tok = slice(0, 4096)
+        ref = oracle.rmsnorm_bf16(to_np64(ys[l][:1, tok]), eps)
+        got = to_np64(xs[l + 1][:1, tok])
+        assert np.max(np.abs(got - ref)) <= 2.0 ** -7 * np.max(np.abs(ref)), ("rmsnorm", l)
+    # 3. end to end on a prefix (batch 0, 1024 tokens)
+    Lp = 1024
     pre = lambda t: t[:1, :Lp].contiguous()
     dev_pre = [dict(dt=pre(p["dt"]), A=p["A"], B=pre(p["B"]), C=pre(p["C"]), D=p["D"]) for p in dev_layers]
-    st_p = zero(1)
-    yp = ssd.ssd_vertical_fwd(pre(x0), dev_pre, st_p, vblock=V, chunk=wl.chunk, rms_eps=eps)
+    yp = ssd.ssd_vertical_fwd(pre(x0), dev_pre, zero(1), vblock=V, chunk=wl.chunk, rms_eps=eps)
     torch.cuda.synchronize()
     assert torch.equal(yp, yv[:1, :Lp])
-    layers64 = [dict(dt=inputs.to_f64(h["dt"][:1, :Lp]), A=inputs.to_f64(h["A"]), B=inputs.to_f64(h["B"][:1, :Lp]),
-                     C=inputs.to_f64(h["C"][:1, :Lp]), D=inputs.to_f64(h["D"])) for h in host_layers]
-    y_ref, f_ref = oracle.stack_horizontal(inputs.to_f64(x0h[:1, :Lp]), layers64, eps)
-    assert rel_err(to_np64(yp), y_ref) <= TOL["bf16"]
-    for a, r in zip(st_p, f_ref):
-        assert rel_err(to_np64(a), r) <= TOL["bf16"]
+    layers64 = [dict(dt=f(h["dt"][:1, :Lp]), A=f(h["A"]), B=f(h["B"][:1, :Lp]), C=f(h["C"][:1, :Lp]),
+                     D=f(h["D"])) for h in host_layers]
+    x0p = f(x0h[:1, :Lp])
+    y_ref, _ = oracle.stack_horizontal(x0p, layers64, eps)
+    sens = rel_err(_stack_sensitivity(x0p, layers64, eps), y_ref)
+    err = rel_err(to_np64(yp), y_ref)
+    assert err <= max(TOL["bf16"], 3.0 * sens), (err, sens)

@@ -206,6 +206,7 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--batch", type=int, default=None, help="override the batch size (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -226,6 +227,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     wl = inputs.WORKLOADS[args.workload]
+    if args.batch:
+        wl = inputs.custom(wl.name, batch=args.batch)
     host = inputs.generate(wl, seed=rank)          # each rank: its own independent batch
     pinned = {}
     for k, v in host.items():
@@ -287,7 +290,7 @@ def main():
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.e2e_steps):
+    for _ in range(max(args.e2e_steps, 1)):
         for k, v in pinned.items():
             d[k].copy_(v, non_blocking=True)
         step()
@@ -295,7 +298,7 @@ def main():
         h_fin.copy_(fin, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    e2e_ms = e0.elapsed_time(e1) / max(args.e2e_steps, 1)
     if world > 1:
         t = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)

@@ -2,5 +2,6 @@
 // device-side globals (the status word) are visible to every kernel.
 #include "ssd_simt.cu"
 #include "ssd_tc.cu"
+#include "ssd_fused.cu"
 #include "ssd_api.cu"
 #include "ssd_selftest.cu"

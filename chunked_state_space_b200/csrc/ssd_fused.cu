@@ -1,0 +1,439 @@
+// Fused tensor-core kernel of the chunked SSD scan (sm_100a): all four steps
+// of "分块推理：解锁循环模型并行计算，实现长序列高效处理" §2.1-§2.2 in one pass, with the
+// inter-chunk state carried on chip.
+//
+// One CTA owns one (batch, head) sequence and walks it in 128-token
+// sub-chunks j (a Q = 256 chunk is two of them: the page's intra/inter split
+// applied once more inside the chunk, which is exact by its §2.3).  Per
+// sub-chunk, with lam the in-sub-chunk cumulative sum of dt*A:
+//   S       = C_j B_j^T                                   (tcgen05, 128x128x128)
+//   P       = S (.) exp(lam_t - lam_s) [s <= t]  -> bf16 in TMEM
+//   y_intra = P X_j                                       (A operand from TMEM)
+//   y_inter = C_j bf16(s_{j-1})                           (state as MN-major B)
+//   b_intra = B_j^T X'_j,  X'_j = diag(exp(lam_end - lam_s)) X_j
+//   y_t     = y_intra + exp(lam_t) y_inter + D x_t
+//   s_j     = exp(lam_end) s_{j-1} + b_intra              (fp32, registers)
+// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
+// issues MMAs, warps 2-5 (one thread per row) build lam, P and X', warps 6-9
+// (one thread per row) finish y, update the state and publish its bf16 copy.
+// TMEM holds two 256-column buffers so sub-chunk j+1's S and mask overlap
+// sub-chunk j's products and epilogue.  Every wait is bounded; a timeout
+// raises g_device_status and the roles drain without further waits.
+#include "ssd_tc.cuh"
+#include "tma.cuh"
+#include "umma.cuh"
+
+namespace ssd {
+namespace fused {
+
+using namespace umma;
+
+constexpr int T = 128;       // tokens per sub-chunk
+constexpr int P = 64;        // head dim
+constexpr int NS = 128;      // state dim
+constexpr int THREADS = 320;
+constexpr uint32_t TILE = 16384;               // [128 rows][64 bf16], 128B-swizzled
+constexpr uint32_t STAGE = 5 * TILE;           // X, B (2 blocks), C (2 blocks)
+constexpr uint32_t OFF_X = 0, OFF_B = TILE, OFF_C = 3 * TILE;
+constexpr uint32_t OFF_XP = 2 * STAGE;         // X' (single buffer)
+constexpr uint32_t OFF_PREV = OFF_XP + TILE;   // bf16 state, MN-major [n][p]
+constexpr uint32_t OFF_LAM = OFF_PREV + TILE;  // float [4][128]
+constexpr uint32_t OFF_WTOT = OFF_LAM + 4 * T * 4;
+constexpr uint32_t OFF_BAR = OFF_WTOT + 64;
+constexpr uint32_t NBAR = 14;
+constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TX_BYTES = 5 * TILE;
+
+struct Params {
+  int64_t L;
+  int H, G, nsub;
+  const float* dt;
+  int64_t sdt;
+  const float* A;
+  const float* D;
+  const float* init;
+  float* final_state;
+  __nv_bfloat16* y;
+  int64_t sy;
+};
+
+// barrier indices
+enum { FULL0 = 0, EMPTY0 = 2, SFULL0 = 4, PFULL0 = 6, CFULL0 = 8, TEMPTY0 = 10, STATEFULL = 12, DRAIN = 13 };
+
+struct Ctl {
+  uint64_t* bar;
+  volatile int* abort;
+  __device__ bool wait(int i, uint32_t parity) const {
+    if (*abort) return false;
+    uint64_t* b = bar + i;
+    if (mbar_try_wait(b, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+      if (mbar_try_wait(b, parity)) return true;
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > 1000000000ull) {
+        *abort = 1;
+        atomicExch(&g_device_status, 2);
+        return false;
+      }
+    }
+  }
+};
+
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n)); }
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    k_ssd_fused(Params p, const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
+                const __grid_constant__ CUtensorMap map_c) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(sm);
+  float* lamb = reinterpret_cast<float*>(sm + OFF_LAM);
+  float* wtot = reinterpret_cast<float*>(sm + OFF_WTOT);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
+  int* abort_flag = reinterpret_cast<int*>(sm + OFF_MISC + 4);
+  Ctl ctl{bar, abort_flag};
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;
+  const int b = bh / p.H, h = bh % p.H;
+  const int g = h / (p.H / p.G);
+  const int nsub = p.nsub;
+
+  if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[FULL0 + i], 1);
+      mbar_init(&bar[EMPTY0 + i], 1 + T);
+      mbar_init(&bar[SFULL0 + i], 1);
+      mbar_init(&bar[PFULL0 + i], T);
+      mbar_init(&bar[CFULL0 + i], 1);
+      mbar_init(&bar[TEMPTY0 + i], T);
+    }
+    mbar_init(&bar[STATEFULL], T);
+    mbar_init(&bar[DRAIN], 1);
+    fence_mbar_init();
+    prefetch_tmap(&map_x);
+    prefetch_tmap(&map_b);
+    prefetch_tmap(&map_c);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      for (int j = 0; j < nsub; ++j) {
+        const int st = j & 1;
+        if (j >= 2 && !ctl.wait(EMPTY0 + st, ((j >> 1) + 1) & 1)) break;
+        uint8_t* sx = sm + st * STAGE;
+        const int t0 = j * T;
+        mbar_arrive_expect_tx(&bar[FULL0 + st], TX_BYTES);
+        tma_load_4d(sx + OFF_X, &map_x, &bar[FULL0 + st], 0, h, t0, b);
+        tma_load_4d(sx + OFF_B, &map_b, &bar[FULL0 + st], 0, g, t0, b);
+        tma_load_4d(sx + OFF_B + TILE, &map_b, &bar[FULL0 + st], 64, g, t0, b);
+        tma_load_4d(sx + OFF_C, &map_c, &bar[FULL0 + st], 0, g, t0, b);
+        tma_load_4d(sx + OFF_C + TILE, &map_c, &bar[FULL0 + st], 64, g, t0, b);
+      }
+      // drain: the last loads of each stage must land before the CTA may exit
+      for (int j = (nsub > 2 ? nsub - 2 : 0); j < nsub; ++j) {
+        uint64_t* fb = &bar[FULL0 + (j & 1)];
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(fb, (j >> 1) & 1) && globaltimer_ns() - t0 < 1000000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idS = idesc_bf16(128, 128, false, false);
+      const uint32_t idY = idesc_bf16(128, 64, false, true);
+      const uint32_t idB = idesc_bf16(128, 64, true, true);
+      bool ok = true;
+      for (int j = 0; j <= nsub && ok; ++j) {
+        if (j < nsub) {
+          const int st = j & 1, buf = j & 1;
+          ok = ctl.wait(FULL0 + st, (j >> 1) & 1);
+          if (ok && j >= 2) ok = ctl.wait(TEMPTY0 + buf, ((j >> 1) + 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sC = sbase + st * STAGE + OFF_C, sB = sbase + st * STAGE + OFF_B;
+          const uint32_t tS = tmem + buf * 256;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t koff = (ks >> 2) * TILE + (ks & 3) * 32;
+            mma_ss(tS, smem_desc(sC + koff, 16, 1024), smem_desc(sB + koff, 16, 1024), idS, ks > 0);
+          }
+          mma_commit(&bar[SFULL0 + buf]);
+        }
+        if (j >= 1) {
+          const int jj = j - 1, st = jj & 1, buf = jj & 1;
+          ok = ctl.wait(PFULL0 + buf, (jj >> 1) & 1);
+          if (ok) ok = ctl.wait(STATEFULL, jj & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t base = tmem + buf * 256;
+          const uint32_t sX = sbase + st * STAGE + OFF_X, sC = sbase + st * STAGE + OFF_C;
+          const uint32_t sB = sbase + st * STAGE + OFF_B;
+          const uint32_t sXp = sbase + OFF_XP, sPrev = sbase + OFF_PREV;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)  // y_intra = P X
+            mma_ts(base + 128, base + ks * 8, smem_desc(sX + ks * 2048, TILE, 1024), idY, ks > 0);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {  // y_inter = C prev
+            const uint32_t koff = (ks >> 2) * TILE + (ks & 3) * 32;
+            mma_ss(base + 64, smem_desc(sC + koff, 16, 1024), smem_desc(sPrev + ks * 2048, TILE, 1024), idY,
+                   ks > 0);
+          }
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)  // b_intra = B^T X'
+            mma_ss(base + 192, smem_desc(sB + ks * 2048, TILE, 1024), smem_desc(sXp + ks * 2048, TILE, 1024), idB,
+                   ks > 0);
+          mma_commit(&bar[CFULL0 + buf]);
+          mma_commit(&bar[EMPTY0 + st]);
+        }
+      }
+      // every MMA issued must complete before TMEM is released (also on abort)
+      mma_commit(&bar[DRAIN]);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(&bar[DRAIN], 0) && globaltimer_ns() - t0 < 1000000000ull) {
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ lam, P and X'
+    const int q = warp & 3;           // TMEM lane quarter
+    const int row = q * 32 + lane;    // token row within the sub-chunk
+    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+    const float Ah = p.A[h];
+    const int row_hi = q * 32 + 31;
+    for (int j = 0; j < nsub; ++j) {
+      const int st = j & 1, buf = j & 1;
+      const int64_t tg = (int64_t)j * T + row;
+      const float dtv = tg < p.L ? p.dt[(int64_t)b * p.sdt + tg * p.H + h] : 0.f;
+      float v = dtv * Ah;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float n = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += n;
+      }
+      if (lane == 31) wtot[q] = v;
+      named_sync(1, T);
+      float pre = 0.f;
+      for (int k = 0; k < q; ++k) pre += wtot[k];
+      const float lam_t = v + pre;
+      float* lj = lamb + (j & 3) * T;
+      lj[row] = lam_t;
+      named_sync(1, T);
+      const float lam_end = lj[T - 1];
+      // X'_j = diag(exp(lam_end - lam_t)) X_j
+      bool ok = ctl.wait(FULL0 + st, (j >> 1) & 1);
+      if (ok && j >= 1) ok = ctl.wait(CFULL0 + ((j - 1) & 1), ((j - 1) >> 1) & 1);
+      if (ok) {
+        const float w = __expf(lam_end - lam_t);
+        const uint32_t sX = sbase + st * STAGE + OFF_X, sXp = sbase + OFF_XP;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t off = swz128(row, c * 8);
+          uint4 v4 = lds128(sX + off);
+          uint32_t* u = reinterpret_cast<uint32_t*>(&v4);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = bf2_to_f2(u[i]);
+            u[i] = pack_bf16(f.x * w, f.y * w);
+          }
+          sts128(sXp + off, v4);
+        }
+        fence_async_smem();
+      }
+      // P = S (.) exp(lam_t - lam_s) on s <= t, bf16, written over S
+      if (ok) ok = ctl.wait(SFULL0 + buf, (j >> 1) & 1);
+      tc_fence_after();
+      const uint32_t tS = tl + buf * 256;
+#pragma unroll 1
+      for (int k = 0; k < 8; ++k) {
+        uint32_t pk[8];
+        if (16 * k <= row_hi) {
+          uint32_t r[16];
+          tmem_ld16(tS + 16 * k, r);
+          tmem_wait_ld();
+          float f[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int s = 16 * k + i;
+            f[i] = (s <= row) ? __uint_as_float(r[i]) * __expf(lam_t - lj[s]) : 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) pk[i] = pack_bf16(f[2 * i], f[2 * i + 1]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) pk[i] = 0u;
+        }
+        tmem_st8(tS + 8 * k, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar[PFULL0 + buf]);
+    }
+  } else {
+    // ------------------------------------------------------------ y, state, final
+    const int q = warp & 3;
+    const int r = q * 32 + lane;  // state row n and output row t
+    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+    const float Dh = p.D ? p.D[h] : 0.f;
+    float s[P];
+    if (p.init) {
+      const float4* src = reinterpret_cast<const float4*>(p.init + ((int64_t)bh * NS + r) * P);
+#pragma unroll
+      for (int i = 0; i < P / 4; ++i) {
+        const float4 v = src[i];
+        s[4 * i] = v.x; s[4 * i + 1] = v.y; s[4 * i + 2] = v.z; s[4 * i + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < P; ++i) s[i] = 0.f;
+    }
+    const uint32_t sPrev = sbase + OFF_PREV;
+    auto publish_state = [&]() {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 v;
+        v.x = pack_bf16(s[8 * c + 0], s[8 * c + 1]);
+        v.y = pack_bf16(s[8 * c + 2], s[8 * c + 3]);
+        v.z = pack_bf16(s[8 * c + 4], s[8 * c + 5]);
+        v.w = pack_bf16(s[8 * c + 6], s[8 * c + 7]);
+        sts128(sPrev + swz128(r, 8 * c), v);
+      }
+      fence_async_smem();
+      mbar_arrive(&bar[STATEFULL]);
+    };
+    publish_state();
+    for (int j = 0; j < nsub; ++j) {
+      const int st = j & 1, buf = j & 1;
+      bool ok = ctl.wait(CFULL0 + buf, (j >> 1) & 1);
+      if (ok) ok = ctl.wait(FULL0 + st, (j >> 1) & 1);  // acquire the x tile for D x_t
+      tc_fence_after();
+      const float* lj = lamb + (j & 3) * T;
+      const float lam_end = lj[T - 1];
+      const float lam_t = lj[r];
+      const uint32_t base = tl + buf * 256;
+      // state: s_j = exp(lam_end) s_{j-1} + b_intra
+      const float dec = __expf(lam_end);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[16];
+        tmem_ld16(base + 192 + 16 * c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) s[16 * c + i] = fmaf(dec, s[16 * c + i], __uint_as_float(v[i]));
+      }
+      if (ok) publish_state();
+      // y_t = y_intra + exp(lam_t) y_inter + D x_t
+      const float e = __expf(lam_t);
+      const uint32_t sX = sbase + st * STAGE + OFF_X;
+      const int64_t tg = (int64_t)j * T + r;
+      uint4 outv[8];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t yi[16], ye[16];
+        tmem_ld16(base + 128 + 16 * c, yi);
+        tmem_ld16(base + 64 + 16 * c, ye);
+        tmem_wait_ld();
+#pragma unroll
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          const int cc = 2 * c + hlf;  // 8-column chunk
+          uint4 xv = lds128(sX + swz128(r, 8 * cc));
+          const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xv);
+          uint32_t* o = reinterpret_cast<uint32_t*>(&outv[cc]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 xf = bf2_to_f2(xu[i]);
+            const int k0 = hlf * 8 + 2 * i;
+            const float a0 = __uint_as_float(yi[k0]) + e * __uint_as_float(ye[k0]) + Dh * xf.x;
+            const float a1 = __uint_as_float(yi[k0 + 1]) + e * __uint_as_float(ye[k0 + 1]) + Dh * xf.y;
+            o[i] = pack_bf16(a0, a1);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar[TEMPTY0 + buf]);
+      mbar_arrive(&bar[EMPTY0 + st]);
+      if (tg < p.L) {
+        uint4* dst = reinterpret_cast<uint4*>(p.y + (int64_t)b * p.sy + (tg * p.H + h) * P);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) dst[c] = outv[c];
+      }
+    }
+    if (p.final_state) {
+      float4* dst = reinterpret_cast<float4*>(p.final_state + ((int64_t)bh * NS + r) * P);
+#pragma unroll
+      for (int i = 0; i < P / 4; ++i) dst[i] = make_float4(s[4 * i], s[4 * i + 1], s[4 * i + 2], s[4 * i + 3]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_relinquish();
+  }
+}
+
+}  // namespace fused
+
+bool fused_supported(const Problem& p) {
+  return p.io == SSD_BF16 && p.P == fused::P && p.N == fused::NS && p.Q % fused::T == 0 && p.B * p.H < (1ll << 31);
+}
+
+int fused_kernels_per_call(const Problem&) { return 1; }
+
+cudaError_t launch_fused(const Problem& p, const float* init, float* final_state, void*, cudaStream_t st) {
+  using namespace fused;
+  CUtensorMap mx, mb, mc;
+  const uint32_t box[4] = {64, 1, (uint32_t)T, 1};
+  const uint64_t dx[4] = {(uint64_t)P, (uint64_t)p.H, (uint64_t)p.L, (uint64_t)p.B};
+  const uint64_t sx[3] = {(uint64_t)P * 2, (uint64_t)p.H * P * 2, (uint64_t)p.sx * 2};
+  const uint64_t dbc[4] = {(uint64_t)NS, (uint64_t)p.G, (uint64_t)p.L, (uint64_t)p.B};
+  const uint64_t sbc[3] = {(uint64_t)NS * 2, (uint64_t)p.G * NS * 2, (uint64_t)p.sbc * 2};
+  if (!tma::encode_bf16(&mx, p.x, 4, dx, sx, box) || !tma::encode_bf16(&mb, p.Bm, 4, dbc, sbc, box) ||
+      !tma::encode_bf16(&mc, p.Cm, 4, dbc, sbc, box))
+    return cudaErrorInvalidValue;
+  Params kp;
+  kp.L = p.L;
+  kp.H = (int)p.H;
+  kp.G = (int)p.G;
+  kp.nsub = (int)ceil_div(p.L, T);
+  kp.dt = p.dt;
+  kp.sdt = p.sdt;
+  kp.A = p.A;
+  kp.D = p.D;
+  kp.init = init;
+  kp.final_state = final_state;
+  kp.y = static_cast<__nv_bfloat16*>(p.y);
+  kp.sy = p.sy;
+  cudaError_t e = cudaFuncSetAttribute(k_ssd_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  k_ssd_fused<<<(unsigned)(p.B * p.H), THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc);
+  return cudaGetLastError();
+}
+
+}  // namespace ssd

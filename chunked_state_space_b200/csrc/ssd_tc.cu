@@ -4,16 +4,12 @@
 namespace ssd {
 
 bool tc_supported(const Problem&) { return false; }
-bool fused_supported(const Problem&) { return false; }
 size_t tc_workspace_bytes(const Problem&) { return 0; }
-int fused_kernels_per_call(const Problem&) { return 1; }
+
 cudaError_t launch_chunk_state_tc(const Problem&, const float*, float*, cudaStream_t) {
   return cudaErrorNotSupported;
 }
 cudaError_t launch_chunk_scan_tc(const Problem&, const float*, const float*, cudaStream_t) {
-  return cudaErrorNotSupported;
-}
-cudaError_t launch_fused(const Problem&, const float*, float*, void*, cudaStream_t) {
   return cudaErrorNotSupported;
 }
 

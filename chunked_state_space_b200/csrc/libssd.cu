@@ -1,6 +1,7 @@
 // Single translation unit of libssd.so: the kernels share one module so that
 // device-side globals (the status word) are visible to every kernel.
 #include "ssd_simt.cu"
+#include "ssd_step.cu"
 #include "ssd_tc.cu"
 #include "ssd_fused.cu"
 #include "ssd_api.cu"

@@ -15,6 +15,7 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_to(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 size_t io_size(int io) { return io == SSD_BF16 ? 2 : 4; }
 
@@ -74,11 +75,14 @@ ssd_status cuda_status(cudaError_t e) {
 
 ssd_status validate_scan_args(const ssd_dims* d, const void* x, const float* dt, const float* A, const void* Bm,
                               const void* Cm, const float* D, const float* init, const void* y,
-                              const float* final_state) {
+                              const float* final_state, bool natural_alignment = false) {
   if (!x || !dt || !A || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;
   const void* ptrs[] = {x, dt, A, Bm, Cm, D, init, y, final_state};
-  for (const void* q : ptrs)
-    if (q && !aligned16(q)) return SSD_ERR_ALIGN;
+  const uintptr_t io_al = natural_alignment ? (d->io_dtype == SSD_BF16 ? 2 : 4) : 16;
+  const uintptr_t f_al = natural_alignment ? 4 : 16;
+  const bool is_io[] = {true, false, false, true, true, false, false, true, false};
+  for (int i = 0; i < 9; ++i)
+    if (ptrs[i] && !aligned_to(ptrs[i], is_io[i] ? io_al : f_al)) return SSD_ERR_ALIGN;
   const size_t es = io_size(d->io_dtype);
   const size_t nx = (size_t)d->batch * d->seqlen * d->nheads * d->headdim;
   const size_t nbc = (size_t)d->batch * d->seqlen * d->ngroups * d->dstate;
@@ -355,6 +359,22 @@ ssd_status ssd_vertical_fwd(const ssd_dims* d, int32_t n_layers, int64_t vblock,
     }
   }
   return SSD_OK;
+}
+
+ssd_status ssd_step(const ssd_dims* d, const void* x, const float* dt, const float* A, const void* Bm, const void* Cm,
+                    const float* D, float* state, void* y, void* stream) {
+  if (!d) return SSD_ERR_INVALID_ARG;
+  ssd_dims d1 = *d;
+  d1.seqlen = 1;
+  d1.chunk = 1;
+  ssd_status s = validate_dims(&d1);
+  if (s != SSD_OK) return s;
+  if (!state) return SSD_ERR_INVALID_ARG;
+  s = validate_scan_args(&d1, x, dt, A, Bm, Cm, D, state, y, state, /*natural_alignment=*/true);
+  if (s != SSD_OK) return s;
+  Problem p = make_problem(&d1);
+  p.x = x; p.dt = dt; p.A = A; p.Bm = Bm; p.Cm = Cm; p.D = D; p.y = y;
+  return cuda_status(launch_ssd_step(p, state, static_cast<cudaStream_t>(stream)));
 }
 
 ssd_status ssd_read_device_status(void* stream) {

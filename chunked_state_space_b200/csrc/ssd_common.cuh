@@ -56,6 +56,7 @@ cudaError_t launch_chunk_state_simt(const Problem& p, const float* lam, float* s
 cudaError_t launch_state_passing(const Problem& p, const float* states, const float* lam,
                                  const float* init, float* prev, float* final_state, cudaStream_t st);
 cudaError_t launch_chunk_scan_simt(const Problem& p, const float* lam, const float* prev, cudaStream_t st);
+cudaError_t launch_ssd_step(const Problem& p, float* state, cudaStream_t st);
 cudaError_t launch_rmsnorm(int64_t rows, int64_t features, int io, const void* in, float eps, void* out,
                            cudaStream_t st);
 

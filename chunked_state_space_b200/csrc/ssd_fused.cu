@@ -13,9 +13,13 @@
 //   b_intra = B_j^T X'_j,  X'_j = diag(exp(lam_end - lam_s)) X_j
 //   y_t     = y_intra + exp(lam_t) y_inter + D x_t
 //   s_j     = exp(lam_end) s_{j-1} + b_intra              (fp32, registers)
-// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
-// issues MMAs, warps 2-5 (one thread per row) build lam, P and X', warps 6-9
-// (one thread per row) finish y, update the state and publish its bf16 copy.
+// Warp roles (384 threads): warp 0 issues TMA loads; warp 1 owns TMEM and
+// issues MMAs; warps 2-3 load dt one sub-chunk ahead, scan lam, form the
+// per-column decay factors and X'; warps 4-7 (one thread per row) turn S
+// into P; warps 8-11 (one thread per row) finish y, update the state and
+// publish its bf16 copy.  The mask needs exp(lam_t - lam_s) only inside the
+// diagonal 32x32 blocks: below them it is exp(lam_t - lam_r) exp(lam_r - lam_s)
+// with r the last column of the block (both factors <= 1).
 // TMEM holds two 256-column buffers so sub-chunk j+1's S and mask overlap
 // sub-chunk j's products and epilogue.  Every wait is bounded; a timeout
 // raises g_device_status and the roles drain without further waits.
@@ -31,16 +35,17 @@ using namespace umma;
 constexpr int T = 128;       // tokens per sub-chunk
 constexpr int P = 64;        // head dim
 constexpr int NS = 128;      // state dim
-constexpr int THREADS = 320;
+constexpr int THREADS = 384;
 constexpr uint32_t TILE = 16384;               // [128 rows][64 bf16], 128B-swizzled
 constexpr uint32_t STAGE = 5 * TILE;           // X, B (2 blocks), C (2 blocks)
 constexpr uint32_t OFF_X = 0, OFF_B = TILE, OFF_C = 3 * TILE;
 constexpr uint32_t OFF_XP = 2 * STAGE;         // X' (single buffer)
 constexpr uint32_t OFF_PREV = OFF_XP + TILE;   // bf16 state, MN-major [n][p]
 constexpr uint32_t OFF_LAM = OFF_PREV + TILE;  // float [4][128]
-constexpr uint32_t OFF_WTOT = OFF_LAM + 4 * T * 4;
+constexpr uint32_t OFF_ECOL = OFF_LAM + 4 * T * 4;  // float [4][128]
+constexpr uint32_t OFF_WTOT = OFF_ECOL + 4 * T * 4;
 constexpr uint32_t OFF_BAR = OFF_WTOT + 64;
-constexpr uint32_t NBAR = 14;
+constexpr uint32_t NBAR = 18;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
@@ -57,10 +62,20 @@ struct Params {
   float* final_state;
   __nv_bfloat16* y;
   int64_t sy;
+  unsigned long long* trace;  // diagnostics: per-sub-chunk event clocks of CTA 0, or NULL
+};
+
+// Trace events (clock64 of CTA 0), one row of kTraceEvents per sub-chunk.
+enum {
+  EV_LOADS = 0, EV_S_ISSUED, EV_C_ISSUED, EV_MASK_START, EV_MASK_DONE, EV_LAM_READY, EV_XP_DONE, EV_C_SEEN,
+  EV_STATE_PUB, EV_EPI_DONE, kTraceEvents = 16
 };
 
 // barrier indices
-enum { FULL0 = 0, EMPTY0 = 2, SFULL0 = 4, PFULL0 = 6, CFULL0 = 8, TEMPTY0 = 10, STATEFULL = 12, DRAIN = 13 };
+enum {
+  FULL0 = 0, EMPTY0 = 2, SFULL0 = 4, PFULL0 = 6, CFULL0 = 8, TEMPTY0 = 10, STATEFULL = 12, DRAIN = 13, LAMRDY0 = 14
+};
+constexpr int AUX = 64;  // threads of warps 2-3
 
 struct Ctl {
   uint64_t* bar;
@@ -104,6 +119,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(sm);
   float* lamb = reinterpret_cast<float*>(sm + OFF_LAM);
+  float* ecolb = reinterpret_cast<float*>(sm + OFF_ECOL);
   float* wtot = reinterpret_cast<float*>(sm + OFF_WTOT);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
@@ -115,6 +131,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int b = bh / p.H, h = bh % p.H;
   const int g = h / (p.H / p.G);
   const int nsub = p.nsub;
+  unsigned long long* const trace = (p.trace && blockIdx.x == 0) ? p.trace : nullptr;
+  auto mark = [&](int j, int ev) {
+    if (trace) trace[j * kTraceEvents + ev] = clock64();
+  };
 
   if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
   if (threadIdx.x == 0) {
@@ -123,12 +143,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&bar[FULL0 + i], 1);
       mbar_init(&bar[EMPTY0 + i], 1 + T);
       mbar_init(&bar[SFULL0 + i], 1);
-      mbar_init(&bar[PFULL0 + i], T);
+      mbar_init(&bar[PFULL0 + i], T + AUX);
       mbar_init(&bar[CFULL0 + i], 1);
       mbar_init(&bar[TEMPTY0 + i], T);
     }
     mbar_init(&bar[STATEFULL], T);
     mbar_init(&bar[DRAIN], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&bar[LAMRDY0 + i], AUX);
     fence_mbar_init();
     prefetch_tmap(&map_x);
     prefetch_tmap(&map_b);
@@ -153,6 +174,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_load_4d(sx + OFF_B + TILE, &map_b, &bar[FULL0 + st], 64, g, t0, b);
         tma_load_4d(sx + OFF_C, &map_c, &bar[FULL0 + st], 0, g, t0, b);
         tma_load_4d(sx + OFF_C + TILE, &map_c, &bar[FULL0 + st], 64, g, t0, b);
+        mark(j, EV_LOADS);
       }
       // drain: the last loads of each stage must land before the CTA may exit
       for (int j = (nsub > 2 ? nsub - 2 : 0); j < nsub; ++j) {
@@ -164,40 +186,27 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Polls two queues and issues whichever is ready: the products c(jc) of
+    // sub-chunk jc (on the state's critical path, checked first) and S(js) of
+    // a later sub-chunk.  S(js) needs its stage loaded and its TMEM buffer
+    // released by the epilogue of js-2; c(jc) needs P and X' (PFULL) and the
+    // bf16 state b(jc-1) (STATEFULL).
     if (lane == 0) {
       const uint32_t idS = idesc_bf16(128, 128, false, false);
       const uint32_t idY = idesc_bf16(128, 64, false, true);
       const uint32_t idB = idesc_bf16(128, 64, true, true);
-      bool ok = true;
-      for (int j = 0; j <= nsub && ok; ++j) {
-        if (j < nsub) {
-          const int st = j & 1, buf = j & 1;
-          ok = ctl.wait(FULL0 + st, (j >> 1) & 1);
-          if (ok && j >= 2) ok = ctl.wait(TEMPTY0 + buf, ((j >> 1) + 1) & 1);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t sC = sbase + st * STAGE + OFF_C, sB = sbase + st * STAGE + OFF_B;
-          const uint32_t tS = tmem + buf * 256;
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t koff = (ks >> 2) * TILE + (ks & 3) * 32;
-            mma_ss(tS, smem_desc(sC + koff, 16, 1024), smem_desc(sB + koff, 16, 1024), idS, ks > 0);
-          }
-          mma_commit(&bar[SFULL0 + buf]);
-        }
-        if (j >= 1) {
-          const int jj = j - 1, st = jj & 1, buf = jj & 1;
-          ok = ctl.wait(PFULL0 + buf, (jj >> 1) & 1);
-          if (ok) ok = ctl.wait(STATEFULL, jj & 1);
-          if (!ok) break;
+      int js = 0, jc = 0;
+      uint64_t t_last = globaltimer_ns();
+      while (jc < nsub) {
+        bool progress = false;
+        if (jc < js && mbar_try_wait(&bar[PFULL0 + (jc & 1)], (jc >> 1) & 1) &&
+            mbar_try_wait(&bar[STATEFULL], jc & 1)) {
+          const int st = jc & 1, buf = jc & 1;
           tc_fence_after();
           const uint32_t base = tmem + buf * 256;
           const uint32_t sX = sbase + st * STAGE + OFF_X, sC = sbase + st * STAGE + OFF_C;
           const uint32_t sB = sbase + st * STAGE + OFF_B;
           const uint32_t sXp = sbase + OFF_XP, sPrev = sbase + OFF_PREV;
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)  // y_intra = P X
-            mma_ts(base + 128, base + ks * 8, smem_desc(sX + ks * 2048, TILE, 1024), idY, ks > 0);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {  // y_inter = C prev
             const uint32_t koff = (ks >> 2) * TILE + (ks & 3) * 32;
@@ -208,8 +217,40 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int ks = 0; ks < 8; ++ks)  // b_intra = B^T X'
             mma_ss(base + 192, smem_desc(sB + ks * 2048, TILE, 1024), smem_desc(sXp + ks * 2048, TILE, 1024), idB,
                    ks > 0);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)  // y_intra = P X
+            mma_ts(base + 128, base + ks * 8, smem_desc(sX + ks * 2048, TILE, 1024), idY, ks > 0);
           mma_commit(&bar[CFULL0 + buf]);
           mma_commit(&bar[EMPTY0 + st]);
+          mark(jc, EV_C_ISSUED);
+          ++jc;
+          progress = true;
+        }
+        if (js < nsub && mbar_try_wait(&bar[FULL0 + (js & 1)], (js >> 1) & 1) &&
+            (js < 2 || mbar_try_wait(&bar[TEMPTY0 + (js & 1)], ((js >> 1) + 1) & 1))) {
+          const int st = js & 1, buf = js & 1;
+          tc_fence_after();
+          const uint32_t sC = sbase + st * STAGE + OFF_C, sB = sbase + st * STAGE + OFF_B;
+          const uint32_t tS = tmem + buf * 256;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t koff = (ks >> 2) * TILE + (ks & 3) * 32;
+            mma_ss(tS, smem_desc(sC + koff, 16, 1024), smem_desc(sB + koff, 16, 1024), idS, ks > 0);
+          }
+          mma_commit(&bar[SFULL0 + buf]);
+          mark(js, EV_S_ISSUED);
+          ++js;
+          progress = true;
+        }
+        if (progress) {
+          t_last = globaltimer_ns();
+        } else {
+          if (*abort_flag) break;
+          if (globaltimer_ns() - t_last > 1000000000ull) {
+            *abort_flag = 1;
+            atomicExch(&g_device_status, 2);
+            break;
+          }
         }
       }
       // every MMA issued must complete before TMEM is released (also on abort)
@@ -218,80 +259,125 @@ __global__ void __launch_bounds__(THREADS, 1)
       while (!mbar_try_wait(&bar[DRAIN], 0) && globaltimer_ns() - t0 < 1000000000ull) {
       }
     }
-  } else if (warp < 6) {
-    // ------------------------------------------------------------ lam, P and X'
-    const int q = warp & 3;           // TMEM lane quarter
-    const int row = q * 32 + lane;    // token row within the sub-chunk
-    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ dt, lam, decay factors, X'
+    const int a = threadIdx.x - 64;  // 0..63
     const float Ah = p.A[h];
-    const int row_hi = q * 32 + 31;
+    const float* dtb = p.dt + (int64_t)b * p.sdt + h;
+    auto load_dt = [&](int j, float& d0, float& d1) {
+      const int64_t t0 = (int64_t)j * T + 2 * a;
+      d0 = (j < nsub && t0 < p.L) ? dtb[t0 * p.H] : 0.f;
+      d1 = (j < nsub && t0 + 1 < p.L) ? dtb[(t0 + 1) * p.H] : 0.f;
+    };
+    float d0, d1;
+    load_dt(0, d0, d1);
     for (int j = 0; j < nsub; ++j) {
-      const int st = j & 1, buf = j & 1;
-      const int64_t tg = (int64_t)j * T + row;
-      const float dtv = tg < p.L ? p.dt[(int64_t)b * p.sdt + tg * p.H + h] : 0.f;
-      float v = dtv * Ah;
+      const int st = j & 1, slot = j & 3;
+      float n0, n1;
+      load_dt(j + 1, n0, n1);  // one sub-chunk ahead
+      // inclusive scan of dt*A over the 128 tokens (two per thread)
+      const float l0 = d0 * Ah, l1 = d1 * Ah;
+      float v = l0 + l1;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
-        const float n = __shfl_up_sync(0xffffffffu, v, off);
-        if (lane >= off) v += n;
+        const float nb = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += nb;
       }
-      if (lane == 31) wtot[q] = v;
-      named_sync(1, T);
-      float pre = 0.f;
-      for (int k = 0; k < q; ++k) pre += wtot[k];
-      const float lam_t = v + pre;
-      float* lj = lamb + (j & 3) * T;
-      lj[row] = lam_t;
-      named_sync(1, T);
-      const float lam_end = lj[T - 1];
-      // X'_j = diag(exp(lam_end - lam_t)) X_j
+      if (lane == 31) wtot[warp - 2] = v;
+      named_sync(1, AUX);
+      const float pre = (warp == 3) ? wtot[0] : 0.f;
+      const float lam1 = v + pre;       // token 2a+1
+      const float lam0 = lam1 - l1;     // token 2a
+      float* lj = lamb + slot * T;
+      float* ec = ecolb + slot * T;
+      lj[2 * a] = lam0;
+      lj[2 * a + 1] = lam1;
+      named_sync(1, AUX);
+      // decay from each column s to the last column of its 32-block
+      const float lr = lj[(2 * a) | 31];
+      ec[2 * a] = __expf(lr - lam0);
+      ec[2 * a + 1] = __expf(lr - lam1);
+      mbar_arrive(&bar[LAMRDY0 + slot]);
+      if (a == 0) mark(j, EV_LAM_READY);
+      d0 = n0;
+      d1 = n1;
+      // X'_j = diag(exp(lam_end - lam_t)) X_j, rows a and a + 64
       bool ok = ctl.wait(FULL0 + st, (j >> 1) & 1);
       if (ok && j >= 1) ok = ctl.wait(CFULL0 + ((j - 1) & 1), ((j - 1) >> 1) & 1);
       if (ok) {
-        const float w = __expf(lam_end - lam_t);
+        const float lam_end = lj[T - 1];
         const uint32_t sX = sbase + st * STAGE + OFF_X, sXp = sbase + OFF_XP;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t off = swz128(row, c * 8);
-          uint4 v4 = lds128(sX + off);
-          uint32_t* u = reinterpret_cast<uint32_t*>(&v4);
+        for (int rr = 0; rr < 2; ++rr) {
+          const int row = a + 64 * rr;
+          const float w = __expf(lam_end - lj[row]);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 f = bf2_to_f2(u[i]);
-            u[i] = pack_bf16(f.x * w, f.y * w);
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t off = swz128(row, c * 8);
+            uint4 v4 = lds128(sX + off);
+            uint32_t* u = reinterpret_cast<uint32_t*>(&v4);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = bf2_to_f2(u[i]);
+              u[i] = pack_bf16(f.x * w, f.y * w);
+            }
+            sts128(sXp + off, v4);
           }
-          sts128(sXp + off, v4);
         }
         fence_async_smem();
       }
-      // P = S (.) exp(lam_t - lam_s) on s <= t, bf16, written over S
+      mbar_arrive(&bar[PFULL0 + st]);
+      if (a == 0) mark(j, EV_XP_DONE);
+      named_sync(1, AUX);  // wtot reuse
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ P = S (.) L
+    const int q = warp & 3;          // TMEM lane quarter = 32-row block
+    const int row = q * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+    for (int j = 0; j < nsub; ++j) {
+      const int buf = j & 1, slot = j & 3;
+      bool ok = ctl.wait(LAMRDY0 + slot, (j >> 2) & 1);
       if (ok) ok = ctl.wait(SFULL0 + buf, (j >> 1) & 1);
       tc_fence_after();
+      if (q == 3 && lane == 0) mark(j, EV_MASK_START);
+      const float* lj = lamb + slot * T;
+      const float* ec = ecolb + slot * T;
+      const float lam_t = lj[row];
       const uint32_t tS = tl + buf * 256;
 #pragma unroll 1
-      for (int k = 0; k < 8; ++k) {
-        uint32_t pk[8];
-        if (16 * k <= row_hi) {
-          uint32_t r[16];
-          tmem_ld16(tS + 16 * k, r);
+      for (int kb = 0; kb < 4; ++kb) {
+        uint32_t pk[16];
+        if (kb <= q) {
+          uint32_t r[32];
+          tmem_ld32(tS + 32 * kb, r);
           tmem_wait_ld();
-          float f[16];
+          if (kb < q) {
+            const float rowf = __expf(lam_t - lj[32 * kb + 31]);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int s = 16 * k + i;
-            f[i] = (s <= row) ? __uint_as_float(r[i]) * __expf(lam_t - lj[s]) : 0.f;
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16(__uint_as_float(r[2 * i]) * rowf * ec[32 * kb + 2 * i],
+                                __uint_as_float(r[2 * i + 1]) * rowf * ec[32 * kb + 2 * i + 1]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int s0 = 32 * kb + 2 * i;
+              const float f0 = (s0 <= row) ? __uint_as_float(r[2 * i]) * __expf(lam_t - lj[s0]) : 0.f;
+              const float f1 = (s0 + 1 <= row) ? __uint_as_float(r[2 * i + 1]) * __expf(lam_t - lj[s0 + 1]) : 0.f;
+              pk[i] = pack_bf16(f0, f1);
+            }
           }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) pk[i] = pack_bf16(f[2 * i], f[2 * i + 1]);
         } else {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) pk[i] = 0u;
+          for (int i = 0; i < 16; ++i) pk[i] = 0u;
         }
-        tmem_st8(tS + 8 * k, pk);
+        tmem_st16(tS + 16 * kb, pk);
       }
       tmem_wait_st();
       tc_fence_before();
+      (void)ok;
       mbar_arrive(&bar[PFULL0 + buf]);
+      if (q == 3 && lane == 0) mark(j, EV_MASK_DONE);
     }
   } else {
     // ------------------------------------------------------------ y, state, final
@@ -329,8 +415,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int j = 0; j < nsub; ++j) {
       const int st = j & 1, buf = j & 1;
       bool ok = ctl.wait(CFULL0 + buf, (j >> 1) & 1);
-      if (ok) ok = ctl.wait(FULL0 + st, (j >> 1) & 1);  // acquire the x tile for D x_t
+      if (ok) ok = ctl.wait(FULL0 + st, (j >> 1) & 1);            // acquire the x tile for D x_t
+      if (ok) ok = ctl.wait(LAMRDY0 + (j & 3), (j >> 2) & 1);      // and lam of this sub-chunk
       tc_fence_after();
+      if (r == 0) mark(j, EV_C_SEEN);
       const float* lj = lamb + (j & 3) * T;
       const float lam_end = lj[T - 1];
       const float lam_t = lj[r];
@@ -338,35 +426,36 @@ __global__ void __launch_bounds__(THREADS, 1)
       // state: s_j = exp(lam_end) s_{j-1} + b_intra
       const float dec = __expf(lam_end);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[16];
-        tmem_ld16(base + 192 + 16 * c, v);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        tmem_ld32(base + 192 + 32 * c, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) s[16 * c + i] = fmaf(dec, s[16 * c + i], __uint_as_float(v[i]));
+        for (int i = 0; i < 32; ++i) s[32 * c + i] = fmaf(dec, s[32 * c + i], __uint_as_float(v[i]));
       }
       if (ok) publish_state();
+      if (r == 0) mark(j, EV_STATE_PUB);
       // y_t = y_intra + exp(lam_t) y_inter + D x_t
       const float e = __expf(lam_t);
       const uint32_t sX = sbase + st * STAGE + OFF_X;
       const int64_t tg = (int64_t)j * T + r;
       uint4 outv[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t yi[16], ye[16];
-        tmem_ld16(base + 128 + 16 * c, yi);
-        tmem_ld16(base + 64 + 16 * c, ye);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t yi[32], ye[32];
+        tmem_ld32(base + 128 + 32 * c, yi);
+        tmem_ld32(base + 64 + 32 * c, ye);
         tmem_wait_ld();
 #pragma unroll
-        for (int hlf = 0; hlf < 2; ++hlf) {
-          const int cc = 2 * c + hlf;  // 8-column chunk
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int cc = 4 * c + q4;  // 8-column chunk
           uint4 xv = lds128(sX + swz128(r, 8 * cc));
           const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xv);
           uint32_t* o = reinterpret_cast<uint32_t*>(&outv[cc]);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float2 xf = bf2_to_f2(xu[i]);
-            const int k0 = hlf * 8 + 2 * i;
+            const int k0 = q4 * 8 + 2 * i;
             const float a0 = __uint_as_float(yi[k0]) + e * __uint_as_float(ye[k0]) + Dh * xf.x;
             const float a1 = __uint_as_float(yi[k0 + 1]) + e * __uint_as_float(ye[k0 + 1]) + Dh * xf.y;
             o[i] = pack_bf16(a0, a1);
@@ -376,6 +465,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       mbar_arrive(&bar[TEMPTY0 + buf]);
       mbar_arrive(&bar[EMPTY0 + st]);
+      if (r == 0) mark(j, EV_EPI_DONE);
       if (tg < p.L) {
         uint4* dst = reinterpret_cast<uint4*>(p.y + (int64_t)b * p.sy + (tg * p.H + h) * P);
 #pragma unroll
@@ -406,7 +496,15 @@ bool fused_supported(const Problem& p) {
 
 int fused_kernels_per_call(const Problem&) { return 1; }
 
+cudaError_t launch_fused_traced(const Problem& p, const float* init, float* final_state, unsigned long long* trace,
+                                cudaStream_t st);
+
 cudaError_t launch_fused(const Problem& p, const float* init, float* final_state, void*, cudaStream_t st) {
+  return launch_fused_traced(p, init, final_state, nullptr, st);
+}
+
+cudaError_t launch_fused_traced(const Problem& p, const float* init, float* final_state, unsigned long long* trace,
+                                cudaStream_t st) {
   using namespace fused;
   CUtensorMap mx, mb, mc;
   const uint32_t box[4] = {64, 1, (uint32_t)T, 1};
@@ -430,6 +528,7 @@ cudaError_t launch_fused(const Problem& p, const float* init, float* final_state
   kp.final_state = final_state;
   kp.y = static_cast<__nv_bfloat16*>(p.y);
   kp.sy = p.sy;
+  kp.trace = trace;
   cudaError_t e = cudaFuncSetAttribute(k_ssd_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
   k_ssd_fused<<<(unsigned)(p.B * p.H), THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc);

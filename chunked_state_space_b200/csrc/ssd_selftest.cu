@@ -172,3 +172,21 @@ extern "C" ssd_status ssd_selftest_umma(int32_t variant, const void* A, const vo
   }
   return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
+
+// Diagnostics for the fused kernel: the same launch as ssd_scan_fwd, with CTA
+// 0 recording the clock of every pipeline event of every sub-chunk.
+extern "C" ssd_status ssd_selftest_fused_trace(const ssd_dims* d, const void* x, const float* dt, const float* A,
+                                               const void* Bm, const void* Cm, const float* D,
+                                               const float* init_state, void* y, float* final_state,
+                                               unsigned long long* trace, int64_t trace_len, void* stream) {
+  using namespace ssd;
+  ssd_status s = validate_dims(d);
+  if (s != SSD_OK) return s;
+  s = validate_scan_args(d, x, dt, A, Bm, Cm, D, init_state, y, final_state);
+  if (s != SSD_OK) return s;
+  Problem p = make_problem(d);
+  if (!fused_supported(p)) return SSD_ERR_UNSUPPORTED;
+  if (!trace || trace_len < ceil_div(p.L, 128) * 16) return SSD_ERR_INVALID_ARG;
+  p.x = x; p.dt = dt; p.A = A; p.Bm = Bm; p.Cm = Cm; p.D = D; p.y = y;
+  return cuda_status(launch_fused_traced(p, init_state, final_state, trace, static_cast<cudaStream_t>(stream)));
+}

@@ -25,7 +25,8 @@ STATUS_NAMES = ["SSD_OK", "SSD_ERR_INVALID_ARG", "SSD_ERR_SHAPE", "SSD_ERR_DTYPE
 EXPORTED = ["ssd_status_string", "ssd_version", "ssd_scan_workspace_size", "ssd_scan_fwd",
             "ssd_scan_fwd_unfused", "ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing",
             "ssd_chunk_scan", "ssd_rmsnorm", "ssd_vertical_workspace_size", "ssd_vertical_fwd",
-            "ssd_read_device_status", "ssd_selftest_umma", "ssd_scan_path"]
+            "ssd_read_device_status", "ssd_selftest_umma", "ssd_scan_path", "ssd_step",
+            "ssd_selftest_fused_trace"]
 
 
 class SSDError(RuntimeError):
@@ -73,6 +74,8 @@ def lib() -> ctypes.CDLL:
         "ssd_read_device_status": (ctypes.c_int, [_P]),
         "ssd_selftest_umma": (ctypes.c_int, [ctypes.c_int32, _P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P]),
         "ssd_scan_path": (ctypes.c_int, [D, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]),
+        "ssd_step": (ctypes.c_int, [D] + [_P] * 9),
+        "ssd_selftest_fused_trace": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_int64, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -251,6 +254,20 @@ def ssd_vertical_fwd(x0, layers: Sequence[dict], states: Sequence[torch.Tensor],
     return y_out
 
 
+def ssd_step(x, dt, A, Bm, Cm, state, D=None, y=None, stream=None):
+    """One decode step: x [B,H,P], dt [B,H], A [H], B/C [B,G,N], state [B,H,N,P] f32
+    (updated in place).  Returns y [B,H,P]."""
+    _contig(x, dt, A, Bm, Cm, D, state, y)
+    Bz, H, P = x.shape
+    G, N = Bm.shape[1], Bm.shape[2]
+    dims = Dims(Bz, 1, H, P, N, G, 1, _io_code(x), 0)
+    if y is None:
+        y = torch.empty_like(x)
+    _check(lib().ssd_step(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D), _ptr(state),
+                          _ptr(y), _stream(stream)), "ssd_step")
+    return y
+
+
 def ssd_read_device_status(stream=None) -> int:
     return int(lib().ssd_read_device_status(_stream(stream)))
 
@@ -270,3 +287,21 @@ def ssd_selftest_umma(variant: str, A: torch.Tensor, B: torch.Tensor, N: int, K:
     _check(lib().ssd_selftest_umma(SELFTEST_VARIANTS[variant], _ptr(A), _ptr(B), _ptr(D), N, K, _stream(stream)),
            "ssd_selftest_umma")
     return D
+
+
+TRACE_EVENTS = ["loads", "S_issued", "c_issued", "mask_start", "mask_done", "lam_ready", "xp_done", "c_seen",
+                "state_pub", "epi_done"]
+
+
+def ssd_selftest_fused_trace(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, stream=None):
+    """Diagnostic: run the fused kernel with CTA 0 tracing its pipeline events.
+    Returns (y, final_state, trace [nsub, 16] int64 clocks)."""
+    dims = make_dims(x, Bm, chunk)
+    nsub = -(-dims.seqlen // 128)
+    y = torch.empty_like(x)
+    fin = torch.empty((dims.batch, dims.nheads, dims.dstate, dims.headdim), dtype=torch.float32, device=x.device)
+    trace = torch.zeros((nsub, 16), dtype=torch.int64, device=x.device)
+    _check(lib().ssd_selftest_fused_trace(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D),
+                                          _ptr(init_state), _ptr(y), _ptr(fin), _ptr(trace), trace.numel(),
+                                          _stream(stream)), "ssd_selftest_fused_trace")
+    return y, fin, trace

@@ -201,6 +201,21 @@ ssd_status ssd_vertical_fwd(const ssd_dims* d, int32_t n_layers, int64_t vblock,
                             size_t workspace_bytes, void* stream);
 
 /*
+ * Recurrent (decode) step: one token per (batch, head), the state updated in
+ * place -- the token recurrence of "分块推理…" §2 itself, the mode a model runs
+ * in when it generates with a state cache:
+ *   a = exp(dt A_h);  state = a state + B x^T;  y = C^T state + D_h x
+ *   d: sizes (seqlen and chunk are ignored), x [B,H,P] io, dt [B,H] f32,
+ *   A [H] f32, Bm/Cm [B,G,N] io, D [H] f32 or NULL, state [B,H,N,P] f32
+ *   (h_{t-1} on entry, h_t on return), y [B,H,P] io (must not overlap inputs).
+ * Pointers need only their element's natural alignment (2 or 4 bytes), so a
+ * token slice x[:, t] of a [B,L,H,P] tensor can be passed directly.
+ * Errors: as ssd_scan_fwd except SSD_ERR_WORKSPACE (no workspace).
+ */
+ssd_status ssd_step(const ssd_dims* d, const void* x, const float* dt, const float* A, const void* Bm,
+                    const void* Cm, const float* D, float* state, void* y, void* stream);
+
+/*
  * Read and clear the device status word that bounded waits inside the
  * kernels set (synchronises `stream`).  Returns SSD_OK or SSD_ERR_TIMEOUT.
  */

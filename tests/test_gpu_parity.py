@@ -207,6 +207,10 @@ def _horizontal_gpu(x0, layers, states, wl, eps):
 
 @pytest.mark.parametrize("L,V", [(1024, 256), (1000, 256), (1000, 300)])
 def test_vertical_small(L, V):
+    """3-layer stack: vertical == horizontal (bitwise when V % Q == 0), every
+    layer teacher-forced against the oracle on its own bf16 input (5e-3), and
+    the end-to-end output within the tolerance the oracle's own rounding
+    sensitivity allows."""
     wl = inputs.custom("stack24_vertical", batch=2, seqlen=L, nheads=4)
     n_layers, eps = 3, 1e-6
     host_layers, dev_layers = _stack_layers(wl, n_layers)
@@ -216,22 +220,36 @@ def test_vertical_small(L, V):
                     for _ in range(n_layers)]
     st_v, st_h = zero(), zero()
     yv = ssd.ssd_vertical_fwd(x0, dev_layers, st_v, vblock=V, chunk=wl.chunk, rms_eps=eps)
-    yh = _horizontal_gpu(x0, dev_layers, st_h, wl, eps)
+    xs, ys = [x0], []
+    for l, p in enumerate(dev_layers):
+        y, _ = ssd.ssd_scan_fwd(xs[-1], p["dt"], p["A"], p["B"], p["C"], p["D"], st_h[l], chunk=wl.chunk,
+                                final_state=st_h[l])
+        ys.append(y)
+        if l + 1 < n_layers:
+            xs.append(ssd.ssd_rmsnorm(y, eps))
+    torch.cuda.synchronize()
     if V % wl.chunk == 0:
-        assert torch.equal(yv, yh)
+        assert torch.equal(yv, ys[-1])
         for a, b in zip(st_v, st_h):
             assert torch.equal(a, b)
-    layers64 = [dict(dt=inputs.to_f64(h["dt"]), A=inputs.to_f64(h["A"]), B=inputs.to_f64(h["B"]),
-                     C=inputs.to_f64(h["C"]), D=inputs.to_f64(h["D"])) for h in host_layers]
-    y_ref, f_ref = oracle.stack_horizontal(inputs.to_f64(x0h), layers64, eps)
-    assert rel_err(to_np64(yv), y_ref) <= TOL["bf16"]
-    for a, r in zip(st_v, f_ref):
-        assert rel_err(to_np64(a), r) <= TOL["bf16"]
+    f = inputs.to_f64
+    layers64 = [dict(dt=f(h["dt"]), A=f(h["A"]), B=f(h["B"]), C=f(h["C"]), D=f(h["D"])) for h in host_layers]
+    for l, p in enumerate(layers64):
+        y_ref, f_ref = oracle.scan_recurrence(to_np64(xs[l]), p["dt"], p["A"], p["B"], p["C"], p["D"], None)
+        assert rel_err(to_np64(ys[l]), y_ref) <= TOL["bf16"], ("layer", l)
+        assert rel_err(to_np64(st_h[l]), f_ref) <= TOL["bf16"], ("state", l)
+        assert rel_err(to_np64(st_v[l]), f_ref) <= TOL["bf16"], ("vertical state", l)
+    y_ref, _ = oracle.stack_horizontal(f(x0h), layers64, eps)
+    sens = rel_err(_stack_sensitivity(f(x0h), layers64, eps), y_ref)
+    err = rel_err(to_np64(yv), y_ref)
+    assert err <= TOL["bf16"] + 2.0 * sens, (err, sens)
 
 
-def _stack_sensitivity(x0, layers64, eps, rel=1e-7, seed=0):
+def _stack_sensitivity(x0, layers64, eps, rel=2.0 ** -9, seed=0):
     """How far the oracle's own last-layer output moves when every layer's output
-    is perturbed by `rel` (fp32-level) before its bf16 storage rounding."""
+    is perturbed by relative noise of size `rel` before its bf16 storage
+    rounding.  rel = 2^-9 is the relative size of one bf16 operand rounding,
+    the error a tensor-core layer adds per element."""
     rng = np.random.default_rng(seed)
     x = x0
     y = None
@@ -251,8 +269,8 @@ def test_stack24_vertical_full():
        (batch, head) over the whole sequence match the oracle run on the GPU's
        own bf16 input x_l (5e-3), and x_{l+1} is the RMS-normalised y_l;
     3. end to end on a prefix against the oracle's stack, with the tolerance
-       set by the oracle's own sensitivity to fp32-level perturbations before
-       each bf16 storage rounding (the stack amplifies rounding-boundary flips).
+       set by the oracle's own sensitivity to bf16-operand-sized perturbations
+       before each bf16 storage rounding (the stack amplifies rounding flips).
     """
     wl = inputs.WORKLOADS["stack24_vertical"]
     n_layers, eps, V = wl.n_layers, 1e-6, wl.vblock
@@ -308,4 +326,4 @@ def test_stack24_vertical_full():
     y_ref, _ = oracle.stack_horizontal(x0p, layers64, eps)
     sens = rel_err(_stack_sensitivity(x0p, layers64, eps), y_ref)
     err = rel_err(to_np64(yp), y_ref)
-    assert err <= max(TOL["bf16"], 3.0 * sens), (err, sens)
+    assert err <= TOL["bf16"] + 2.0 * sens, (err, sens)

@@ -39,8 +39,8 @@ constexpr int THREADS = 384;
 constexpr uint32_t TILE = 16384;               // [128 rows][64 bf16], 128B-swizzled
 constexpr uint32_t STAGE = 5 * TILE;           // X, B (2 blocks), C (2 blocks)
 constexpr uint32_t OFF_X = 0, OFF_B = TILE, OFF_C = 3 * TILE;
-constexpr uint32_t OFF_XP = 2 * STAGE;         // X' (single buffer)
-constexpr uint32_t OFF_PREV = OFF_XP + TILE;   // bf16 state, MN-major [n][p]
+constexpr uint32_t OFF_XP = 2 * STAGE;         // X' (two buffers)
+constexpr uint32_t OFF_PREV = OFF_XP + 2 * TILE;  // bf16 state, MN-major [n][p]
 constexpr uint32_t OFF_LAM = OFF_PREV + TILE;  // float [4][128]
 constexpr uint32_t OFF_ECOL = OFF_LAM + 4 * T * 4;  // float [4][128]
 constexpr uint32_t OFF_WTOT = OFF_ECOL + 4 * T * 4;
@@ -199,14 +199,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint64_t t_last = globaltimer_ns();
       while (jc < nsub) {
         bool progress = false;
-        if (jc < js && mbar_try_wait(&bar[PFULL0 + (jc & 1)], (jc >> 1) & 1) &&
-            mbar_try_wait(&bar[STATEFULL], jc & 1)) {
+        if (jc < js && mbar_test_wait(&bar[PFULL0 + (jc & 1)], (jc >> 1) & 1) &&
+            mbar_test_wait(&bar[STATEFULL], jc & 1)) {
           const int st = jc & 1, buf = jc & 1;
           tc_fence_after();
           const uint32_t base = tmem + buf * 256;
           const uint32_t sX = sbase + st * STAGE + OFF_X, sC = sbase + st * STAGE + OFF_C;
           const uint32_t sB = sbase + st * STAGE + OFF_B;
-          const uint32_t sXp = sbase + OFF_XP, sPrev = sbase + OFF_PREV;
+          const uint32_t sXp = sbase + OFF_XP + (jc & 1) * TILE, sPrev = sbase + OFF_PREV;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {  // y_inter = C prev
             const uint32_t koff = (ks >> 2) * TILE + (ks & 3) * 32;
@@ -226,8 +226,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           ++jc;
           progress = true;
         }
-        if (js < nsub && mbar_try_wait(&bar[FULL0 + (js & 1)], (js >> 1) & 1) &&
-            (js < 2 || mbar_try_wait(&bar[TEMPTY0 + (js & 1)], ((js >> 1) + 1) & 1))) {
+        if (js < nsub && mbar_test_wait(&bar[FULL0 + (js & 1)], (js >> 1) & 1) &&
+            (js < 2 || mbar_test_wait(&bar[TEMPTY0 + (js & 1)], ((js >> 1) + 1) & 1))) {
           const int st = js & 1, buf = js & 1;
           tc_fence_after();
           const uint32_t sC = sbase + st * STAGE + OFF_C, sB = sbase + st * STAGE + OFF_B;
@@ -301,27 +301,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (a == 0) mark(j, EV_LAM_READY);
       d0 = n0;
       d1 = n1;
-      // X'_j = diag(exp(lam_end - lam_t)) X_j, rows a and a + 64
+      // X'_j = diag(exp(lam_end - lam_t)) X_j, rows a and a + 64, into buffer j & 1
+      // (free once the products of sub-chunk j - 2 have completed)
       bool ok = ctl.wait(FULL0 + st, (j >> 1) & 1);
-      if (ok && j >= 1) ok = ctl.wait(CFULL0 + ((j - 1) & 1), ((j - 1) >> 1) & 1);
+      if (ok && j >= 2) ok = ctl.wait(CFULL0 + st, ((j - 2) >> 1) & 1);
       if (ok) {
         const float lam_end = lj[T - 1];
-        const uint32_t sX = sbase + st * STAGE + OFF_X, sXp = sbase + OFF_XP;
+        const uint4* src = reinterpret_cast<const uint4*>(sm + st * STAGE + OFF_X);
+        uint4* dst = reinterpret_cast<uint4*>(sm + OFF_XP + st * TILE);
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
           const int row = a + 64 * rr;
           const float w = __expf(lam_end - lj[row]);
+          uint4 v4[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) v4[c] = src[swz128(row, c * 8) >> 4];
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const uint32_t off = swz128(row, c * 8);
-            uint4 v4 = lds128(sX + off);
-            uint32_t* u = reinterpret_cast<uint32_t*>(&v4);
+            uint32_t* u = reinterpret_cast<uint32_t*>(&v4[c]);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const float2 f = bf2_to_f2(u[i]);
               u[i] = pack_bf16(f.x * w, f.y * w);
             }
-            sts128(sXp + off, v4);
+            dst[swz128(row, c * 8) >> 4] = v4[c];
           }
         }
         fence_async_smem();
@@ -345,33 +348,37 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float* ec = ecolb + slot * T;
       const float lam_t = lj[row];
       const uint32_t tS = tl + buf * 256;
-#pragma unroll 1
-      for (int kb = 0; kb < 4; ++kb) {
-        uint32_t pk[16];
-        if (kb <= q) {
-          uint32_t r[32];
-          tmem_ld32(tS + 32 * kb, r);
-          tmem_wait_ld();
-          if (kb < q) {
-            const float rowf = __expf(lam_t - lj[32 * kb + 31]);
+      auto make_block = [&](int kb, const uint32_t* r, uint32_t* pk) {
+        if (kb < q) {
+          const float rowf = __expf(lam_t - lj[32 * kb + 31]);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = pack_bf16(__uint_as_float(r[2 * i]) * rowf * ec[32 * kb + 2 * i],
-                                __uint_as_float(r[2 * i + 1]) * rowf * ec[32 * kb + 2 * i + 1]);
-          } else {
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16(__uint_as_float(r[2 * i]) * rowf * ec[32 * kb + 2 * i],
+                              __uint_as_float(r[2 * i + 1]) * rowf * ec[32 * kb + 2 * i + 1]);
+        } else if (kb == q) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int s0 = 32 * kb + 2 * i;
-              const float f0 = (s0 <= row) ? __uint_as_float(r[2 * i]) * __expf(lam_t - lj[s0]) : 0.f;
-              const float f1 = (s0 + 1 <= row) ? __uint_as_float(r[2 * i + 1]) * __expf(lam_t - lj[s0 + 1]) : 0.f;
-              pk[i] = pack_bf16(f0, f1);
-            }
+          for (int i = 0; i < 16; ++i) {
+            const int s0 = 32 * kb + 2 * i;
+            const float f0 = (s0 <= row) ? __uint_as_float(r[2 * i]) * __expf(lam_t - lj[s0]) : 0.f;
+            const float f1 = (s0 + 1 <= row) ? __uint_as_float(r[2 * i + 1]) * __expf(lam_t - lj[s0 + 1]) : 0.f;
+            pk[i] = pack_bf16(f0, f1);
           }
         } else {
 #pragma unroll
           for (int i = 0; i < 16; ++i) pk[i] = 0u;
         }
+      };
+#pragma unroll 1
+      for (int kb = 0; kb < 4; kb += 2) {
+        uint32_t r0[32], r1[32], pk[16];
+        // warp-uniform: only blocks on or below the diagonal block are read
+        if (kb <= q) tmem_ld32(tS + 32 * kb, r0);
+        if (kb + 1 <= q) tmem_ld32(tS + 32 * (kb + 1), r1);
+        tmem_wait_ld();
+        make_block(kb, r0, pk);
         tmem_st16(tS + 16 * kb, pk);
+        make_block(kb + 1, r1, pk);
+        tmem_st16(tS + 16 * (kb + 1), pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -437,9 +444,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (r == 0) mark(j, EV_STATE_PUB);
       // y_t = y_intra + exp(lam_t) y_inter + D x_t
       const float e = __expf(lam_t);
-      const uint32_t sX = sbase + st * STAGE + OFF_X;
+      const uint4* xrow = reinterpret_cast<const uint4*>(sm + st * STAGE + OFF_X);
       const int64_t tg = (int64_t)j * T + r;
-      uint4 outv[8];
+      uint4* dst = reinterpret_cast<uint4*>(p.y + (int64_t)b * p.sy + (tg * p.H + h) * P);
+      const bool row_in = tg < p.L;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t yi[32], ye[32];
@@ -449,9 +457,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           const int cc = 4 * c + q4;  // 8-column chunk
-          uint4 xv = lds128(sX + swz128(r, 8 * cc));
+          const uint4 xv = xrow[swz128(r, 8 * cc) >> 4];
           const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xv);
-          uint32_t* o = reinterpret_cast<uint32_t*>(&outv[cc]);
+          uint4 ov;
+          uint32_t* o = reinterpret_cast<uint32_t*>(&ov);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float2 xf = bf2_to_f2(xu[i]);
@@ -460,17 +469,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             const float a1 = __uint_as_float(yi[k0 + 1]) + e * __uint_as_float(ye[k0 + 1]) + Dh * xf.y;
             o[i] = pack_bf16(a0, a1);
           }
+          if (row_in) dst[cc] = ov;
         }
       }
       tc_fence_before();
       mbar_arrive(&bar[TEMPTY0 + buf]);
       mbar_arrive(&bar[EMPTY0 + st]);
       if (r == 0) mark(j, EV_EPI_DONE);
-      if (tg < p.L) {
-        uint4* dst = reinterpret_cast<uint4*>(p.y + (int64_t)b * p.sy + (tg * p.H + h) * P);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) dst[c] = outv[c];
-      }
     }
     if (p.final_state) {
       float4* dst = reinterpret_cast<float4*>(p.final_state + ((int64_t)bh * NS + r) * P);

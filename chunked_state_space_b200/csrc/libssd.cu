@@ -5,4 +5,5 @@
 #include "ssd_tc.cu"
 #include "ssd_fused.cu"
 #include "ssd_api.cu"
+#include "ssd_noalloc.cu"
 #include "ssd_selftest.cu"

@@ -26,7 +26,7 @@ EXPORTED = ["ssd_status_string", "ssd_version", "ssd_scan_workspace_size", "ssd_
             "ssd_scan_fwd_unfused", "ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing",
             "ssd_chunk_scan", "ssd_rmsnorm", "ssd_vertical_workspace_size", "ssd_vertical_fwd",
             "ssd_read_device_status", "ssd_selftest_umma", "ssd_scan_path", "ssd_step",
-            "ssd_selftest_fused_trace"]
+            "ssd_selftest_fused_trace", "ssd_scan_fwd_noalloc"]
 
 
 class SSDError(RuntimeError):
@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
         "ssd_selftest_umma": (ctypes.c_int, [ctypes.c_int32, _P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P]),
         "ssd_scan_path": (ctypes.c_int, [D, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]),
         "ssd_step": (ctypes.c_int, [D] + [_P] * 9),
+        "ssd_scan_fwd_noalloc": (ctypes.c_int, [D] + [_P] * 10),
         "ssd_selftest_fused_trace": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_int64, _P]),
     }
     for name, (res, args) in sig.items():

@@ -126,6 +126,30 @@ ssd_status ssd_scan_fwd_unfused(const ssd_dims* d, const void* x, const float* d
                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The step-by-step scan (same arguments, results and errors as
+ * ssd_scan_fwd_unfused) for callers that cannot allocate device memory when
+ * they run it -- code being captured into a CUDA graph, engines or plugin
+ * hosts that plan all device memory up front, runtimes with a fixed budget.
+ * The pages have no counterpart: this is a packaging of the same kernels.
+ *   - Scratch comes from a 32 MiB buffer compiled into libssd (every GPU that
+ *     loads the library holds it until the process exits).  The call needs
+ *     4*B*H*nc*Q + 4*B*H*nc*N*P bytes (each part rounded up to 256) and returns
+ *     SSD_ERR_UNSUPPORTED, with a message on stderr, for sizes beyond that.
+ *   - The call allocates nothing (no cudaMalloc or cudaFree, no allocating
+ *     library routine).  Its first call on a device looks up the buffer's
+ *     device address with that device current; make that first call before
+ *     any stream capture.
+ *   - Every call shares the buffer and it keeps the last call's contents;
+ *     nothing in it needs to start at zero (each call writes the scratch it
+ *     reads).  Calls whose executions overlap on the GPU (other streams,
+ *     other host threads) race on it and must be serialised by the caller.
+ */
+ssd_status ssd_scan_fwd_noalloc(const ssd_dims* d, const void* x, const float* dt, const float* A,
+                                const void* Bm, const void* Cm, const float* D,
+                                const float* init_state, void* y, float* final_state,
+                                void* stream);
+
+/*
  * Step 1, the log-decay cumulative sum ("分块推理…" §2.2, the product of A_t over a
  * chunk, taken in log space):  lam[b,h,c,i] = sum_{r=0..i} dt[b,cQ+r,h] * A[h]
  * for i < len(c); positions past the end of a short last chunk repeat the

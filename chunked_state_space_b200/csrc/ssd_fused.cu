@@ -11,7 +11,7 @@
 //   y_intra = P X_j                                       (A operand from TMEM)
 //   y_inter = C_j bf16(s_{j-1})                           (state as MN-major B)
 //   b_intra = B_j^T X'_j,  X'_j = diag(exp(lam_end - lam_s)) X_j
-//   y_t     = y_intra + exp(lam_t) y_inter + D x_t
+//   y_t     = y_intra + exp(lam_t) y_inter + D x_t       (x_t re-read from L2)
 //   s_j     = exp(lam_end) s_{j-1} + b_intra              (fp32, registers)
 // Warp roles (384 threads): warp 0 issues TMA loads; warp 1 owns TMEM and
 // issues MMAs; warps 2-3 load dt one sub-chunk ahead, scan lam, form the
@@ -60,6 +60,8 @@ struct Params {
   const float* D;
   const float* init;
   float* final_state;
+  const __nv_bfloat16* x;
+  int64_t sx;
   __nv_bfloat16* y;
   int64_t sy;
   unsigned long long* trace;  // diagnostics: per-sub-chunk event clocks of CTA 0, or NULL
@@ -68,7 +70,7 @@ struct Params {
 // Trace events (clock64 of CTA 0), one row of kTraceEvents per sub-chunk.
 enum {
   EV_LOADS = 0, EV_S_ISSUED, EV_C_ISSUED, EV_MASK_START, EV_MASK_DONE, EV_LAM_READY, EV_XP_DONE, EV_C_SEEN,
-  EV_STATE_PUB, EV_EPI_DONE, kTraceEvents = 16
+  EV_STATE_PUB, EV_EPI_DONE, EV_C_READY, EV_C_MID, EV_S_READY, EV_MASK_LD, kTraceEvents = 16
 };
 
 // barrier indices
@@ -141,7 +143,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     *abort_flag = 0;
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar[FULL0 + i], 1);
-      mbar_init(&bar[EMPTY0 + i], 1 + T);
+      mbar_init(&bar[EMPTY0 + i], 1);
       mbar_init(&bar[SFULL0 + i], 1);
       mbar_init(&bar[PFULL0 + i], T + AUX);
       mbar_init(&bar[CFULL0 + i], 1);
@@ -202,6 +204,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (jc < js && mbar_test_wait(&bar[PFULL0 + (jc & 1)], (jc >> 1) & 1) &&
             mbar_test_wait(&bar[STATEFULL], jc & 1)) {
           const int st = jc & 1, buf = jc & 1;
+          mark(jc, EV_C_READY);
           tc_fence_after();
           const uint32_t base = tmem + buf * 256;
           const uint32_t sX = sbase + st * STAGE + OFF_X, sC = sbase + st * STAGE + OFF_C;
@@ -213,6 +216,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             mma_ss(base + 64, smem_desc(sC + koff, 16, 1024), smem_desc(sPrev + ks * 2048, TILE, 1024), idY,
                    ks > 0);
           }
+          mark(jc, EV_C_MID);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)  // b_intra = B^T X'
             mma_ss(base + 192, smem_desc(sB + ks * 2048, TILE, 1024), smem_desc(sXp + ks * 2048, TILE, 1024), idB,
@@ -229,6 +233,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (js < nsub && mbar_test_wait(&bar[FULL0 + (js & 1)], (js >> 1) & 1) &&
             (js < 2 || mbar_test_wait(&bar[TEMPTY0 + (js & 1)], ((js >> 1) + 1) & 1))) {
           const int st = js & 1, buf = js & 1;
+          mark(js, EV_S_READY);
           tc_fence_after();
           const uint32_t sC = sbase + st * STAGE + OFF_C, sB = sbase + st * STAGE + OFF_B;
           const uint32_t tS = tmem + buf * 256;
@@ -375,6 +380,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (kb <= q) tmem_ld32(tS + 32 * kb, r0);
         if (kb + 1 <= q) tmem_ld32(tS + 32 * (kb + 1), r1);
         tmem_wait_ld();
+        if (kb == 0 && q == 3 && lane == 0) mark(j, EV_MASK_LD);
         make_block(kb, r0, pk);
         tmem_st16(tS + 16 * kb, pk);
         make_block(kb + 1, r1, pk);
@@ -392,6 +398,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int r = q * 32 + lane;  // state row n and output row t
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
     const float Dh = p.D ? p.D[h] : 0.f;
+    // x row of the sub-chunk, loaded before waiting for its products (it is in L2
+    // from the TMA load; the wait hides the latency)
+    const __nv_bfloat16* xg = p.x + (int64_t)b * p.sx + (int64_t)h * P;
+    auto load_x = [&](int j, uint4* xv) {
+      const int64_t tg = (int64_t)j * T + r;
+      if (j < nsub && tg < p.L) {
+        const uint4* src = reinterpret_cast<const uint4*>(xg + tg * p.H * P);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) xv[c] = src[c];
+      } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) xv[c] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+    uint4 xcur[8];
     float s[P];
     if (p.init) {
       const float4* src = reinterpret_cast<const float4*>(p.init + ((int64_t)bh * NS + r) * P);
@@ -420,10 +441,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     };
     publish_state();
     for (int j = 0; j < nsub; ++j) {
-      const int st = j & 1, buf = j & 1;
+      const int buf = j & 1;
+      load_x(j, xcur);
       bool ok = ctl.wait(CFULL0 + buf, (j >> 1) & 1);
-      if (ok) ok = ctl.wait(FULL0 + st, (j >> 1) & 1);            // acquire the x tile for D x_t
-      if (ok) ok = ctl.wait(LAMRDY0 + (j & 3), (j >> 2) & 1);      // and lam of this sub-chunk
+      if (ok) ok = ctl.wait(LAMRDY0 + (j & 3), (j >> 2) & 1);      // acquire lam of this sub-chunk
       tc_fence_after();
       if (r == 0) mark(j, EV_C_SEEN);
       const float* lj = lamb + (j & 3) * T;
@@ -444,37 +465,33 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (r == 0) mark(j, EV_STATE_PUB);
       // y_t = y_intra + exp(lam_t) y_inter + D x_t
       const float e = __expf(lam_t);
-      const uint4* xrow = reinterpret_cast<const uint4*>(sm + st * STAGE + OFF_X);
       const int64_t tg = (int64_t)j * T + r;
       uint4* dst = reinterpret_cast<uint4*>(p.y + (int64_t)b * p.sy + (tg * p.H + h) * P);
       const bool row_in = tg < p.L;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t yi[32], ye[32];
-        tmem_ld32(base + 128 + 32 * c, yi);
-        tmem_ld32(base + 64 + 32 * c, ye);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t yi[16], ye[16];
+        tmem_ld16(base + 128 + 16 * c, yi);
+        tmem_ld16(base + 64 + 16 * c, ye);
         tmem_wait_ld();
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int cc = 4 * c + q4;  // 8-column chunk
-          const uint4 xv = xrow[swz128(r, 8 * cc) >> 4];
-          const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xv);
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int cc = 2 * c + h2;  // 8-column chunk
+          const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xcur[cc]);
           uint4 ov;
           uint32_t* o = reinterpret_cast<uint32_t*>(&ov);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
+            const int k0 = h2 * 8 + 2 * i;
             const float2 xf = bf2_to_f2(xu[i]);
-            const int k0 = q4 * 8 + 2 * i;
-            const float a0 = __uint_as_float(yi[k0]) + e * __uint_as_float(ye[k0]) + Dh * xf.x;
-            const float a1 = __uint_as_float(yi[k0 + 1]) + e * __uint_as_float(ye[k0 + 1]) + Dh * xf.y;
-            o[i] = pack_bf16(a0, a1);
+            o[i] = pack_bf16(fmaf(e, __uint_as_float(ye[k0]), fmaf(Dh, xf.x, __uint_as_float(yi[k0]))),
+                             fmaf(e, __uint_as_float(ye[k0 + 1]), fmaf(Dh, xf.y, __uint_as_float(yi[k0 + 1]))));
           }
           if (row_in) dst[cc] = ov;
         }
       }
       tc_fence_before();
       mbar_arrive(&bar[TEMPTY0 + buf]);
-      mbar_arrive(&bar[EMPTY0 + st]);
       if (r == 0) mark(j, EV_EPI_DONE);
     }
     if (p.final_state) {
@@ -531,6 +548,8 @@ cudaError_t launch_fused_traced(const Problem& p, const float* init, float* fina
   kp.D = p.D;
   kp.init = init;
   kp.final_state = final_state;
+  kp.x = static_cast<const __nv_bfloat16*>(p.x);
+  kp.sx = p.sx;
   kp.y = static_cast<__nv_bfloat16*>(p.y);
   kp.sy = p.sy;
   kp.trace = trace;

@@ -7,11 +7,12 @@
 // applied once more inside the chunk, which is exact by its §2.3).  Per
 // sub-chunk, with lam the in-sub-chunk cumulative sum of dt*A:
 //   S       = C_j B_j^T                                   (tcgen05, 128x128x128)
-//   P       = S (.) exp(lam_t - lam_s) [s <= t]  -> bf16 in TMEM
-//   y_intra = P X_j                                       (A operand from TMEM)
-//   y_inter = C_j bf16(s_{j-1})                           (state as MN-major B)
+//   P       = S (.) exp(lam_t - lam_s) [s <= t]  -> bf16 in TMEM, columns 0-63
+//   C'      = diag(exp(lam_t)) C_j                -> bf16 in TMEM, columns 64-127
+//   y       = P X_j + C' bf16(s_{j-1})            (both A operands from TMEM: the
+//             page's by_intra + by_inter in one accumulator)
 //   b_intra = B_j^T X'_j,  X'_j = diag(exp(lam_end - lam_s)) X_j
-//   y_t     = y_intra + exp(lam_t) y_inter + D x_t       (x_t re-read from L2)
+//   y_t     = y + D x_t                           (x_t re-read from L2, fp32)
 //   s_j     = exp(lam_end) s_{j-1} + b_intra              (fp32, registers)
 // Warp roles (384 threads): warp 0 issues TMA loads; warp 1 owns TMEM and
 // issues MMAs; warps 2-3 load dt one sub-chunk ahead, scan lam, form the
@@ -20,8 +21,8 @@
 // publish its bf16 copy.  The mask needs exp(lam_t - lam_s) only inside the
 // diagonal 32x32 blocks: below them it is exp(lam_t - lam_r) exp(lam_r - lam_s)
 // with r the last column of the block (both factors <= 1).
-// TMEM holds two 256-column buffers so sub-chunk j+1's S and mask overlap
-// sub-chunk j's products and epilogue.  Every wait is bounded; a timeout
+// TMEM holds two 256-column buffers [S -> P | C'][y][b_intra] so sub-chunk
+// j+1's S and mask overlap sub-chunk j's products and epilogue.  Every wait is bounded; a timeout
 // raises g_device_status and the roles drain without further waits.
 #include "ssd_tc.cuh"
 #include "tma.cuh"
@@ -70,7 +71,8 @@ struct Params {
 // Trace events (clock64 of CTA 0), one row of kTraceEvents per sub-chunk.
 enum {
   EV_LOADS = 0, EV_S_ISSUED, EV_C_ISSUED, EV_MASK_START, EV_MASK_DONE, EV_LAM_READY, EV_XP_DONE, EV_C_SEEN,
-  EV_STATE_PUB, EV_EPI_DONE, EV_C_READY, EV_C_MID, EV_S_READY, EV_MASK_LD, kTraceEvents = 16
+  EV_STATE_PUB, EV_EPI_DONE, EV_C_READY, EV_C_MID, EV_S_READY, EV_MASK_LD, EV_MASK_B01, EV_MASK_LD2,
+  EV_MASK_B23, EV_MASK_WST, kTraceEvents = 24
 };
 
 // barrier indices
@@ -82,18 +84,22 @@ constexpr int AUX = 64;  // threads of warps 2-3
 struct Ctl {
   uint64_t* bar;
   volatile int* abort;
+  // Sleeps in mbarrier.try_wait (hinted) and reads the timer only every 32
+  // probes, so waiting warps take almost no issue slots from working ones.
   __device__ bool wait(int i, uint32_t parity) const {
     if (*abort) return false;
     uint64_t* b = bar + i;
     if (mbar_try_wait(b, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    while (true) {
-      if (mbar_try_wait(b, parity)) return true;
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > 1000000000ull) {
-        *abort = 1;
-        atomicExch(&g_device_status, 2);
-        return false;
+    for (uint32_t spin = 1;; ++spin) {
+      if (mbar_try_wait_sleep(b, parity, 20000u)) return true;
+      if ((spin & 31) == 0) {
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > 1000000000ull) {
+          *abort = 1;
+          atomicExch(&g_device_status, 2);
+          return false;
+        }
       }
     }
   }
@@ -110,6 +116,14 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
 }
+// 2^x with the ex2.approx PTX instruction (flushes denormals; |rel err| ~ 2^-22).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+
 __device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
@@ -118,7 +132,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     k_ssd_fused(Params p, const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
                 const __grid_constant__ CUtensorMap map_c) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, derived from the __shared__ array by an offset so
+  // the compiler keeps the shared address space (LDS/STS, not generic access)
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(sm);
   float* lamb = reinterpret_cast<float*>(sm + OFF_LAM);
   float* ecolb = reinterpret_cast<float*>(sm + OFF_ECOL);
@@ -165,8 +181,22 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      // L2 prefetch runs kPrefetch sub-chunks ahead of the shared-memory loads,
+      // so a stage freed by the products of sub-chunk j-2 refills from L2
+      constexpr int kPrefetch = 3;
+      auto prefetch = [&](int jp) {
+        if (jp >= nsub) return;
+        const int tp = jp * T;
+        tma_prefetch_4d(&map_x, 0, h, tp, b);
+        tma_prefetch_4d(&map_b, 0, g, tp, b);
+        tma_prefetch_4d(&map_b, 64, g, tp, b);
+        tma_prefetch_4d(&map_c, 0, g, tp, b);
+        tma_prefetch_4d(&map_c, 64, g, tp, b);
+      };
+      for (int jp = 0; jp < kPrefetch; ++jp) prefetch(jp);
       for (int j = 0; j < nsub; ++j) {
         const int st = j & 1;
+        prefetch(j + kPrefetch);
         if (j >= 2 && !ctl.wait(EMPTY0 + st, ((j >> 1) + 1) & 1)) break;
         uint8_t* sx = sm + st * STAGE;
         const int t0 = j * T;
@@ -198,6 +228,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t idY = idesc_bf16(128, 64, false, true);
       const uint32_t idB = idesc_bf16(128, 64, true, true);
       int js = 0, jc = 0;
+      uint32_t idle = 0;
       uint64_t t_last = globaltimer_ns();
       while (jc < nsub) {
         bool progress = false;
@@ -207,23 +238,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           mark(jc, EV_C_READY);
           tc_fence_after();
           const uint32_t base = tmem + buf * 256;
-          const uint32_t sX = sbase + st * STAGE + OFF_X, sC = sbase + st * STAGE + OFF_C;
+          const uint32_t sX = sbase + st * STAGE + OFF_X;
           const uint32_t sB = sbase + st * STAGE + OFF_B;
           const uint32_t sXp = sbase + OFF_XP + (jc & 1) * TILE, sPrev = sbase + OFF_PREV;
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {  // y_inter = C prev
-            const uint32_t koff = (ks >> 2) * TILE + (ks & 3) * 32;
-            mma_ss(base + 64, smem_desc(sC + koff, 16, 1024), smem_desc(sPrev + ks * 2048, TILE, 1024), idY,
-                   ks > 0);
-          }
-          mark(jc, EV_C_MID);
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)  // b_intra = B^T X'
+          for (int ks = 0; ks < 8; ++ks)  // b_intra = B^T X'  (the state chain needs it first)
             mma_ss(base + 192, smem_desc(sB + ks * 2048, TILE, 1024), smem_desc(sXp + ks * 2048, TILE, 1024), idB,
                    ks > 0);
+          mark(jc, EV_C_MID);
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks)  // y_intra = P X
+          for (int ks = 0; ks < 8; ++ks)  // y = P X
             mma_ts(base + 128, base + ks * 8, smem_desc(sX + ks * 2048, TILE, 1024), idY, ks > 0);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)  // y += C' prev
+            mma_ts(base + 128, base + 64 + ks * 8, smem_desc(sPrev + ks * 2048, TILE, 1024), idY, 1u);
           mma_commit(&bar[CFULL0 + buf]);
           mma_commit(&bar[EMPTY0 + st]);
           mark(jc, EV_C_ISSUED);
@@ -248,14 +276,18 @@ __global__ void __launch_bounds__(THREADS, 1)
           progress = true;
         }
         if (progress) {
-          t_last = globaltimer_ns();
-        } else {
+          idle = 0;
+        } else if ((++idle & 63) == 0) {
+          const uint64_t now = globaltimer_ns();
+          if (idle == 64) t_last = now;
           if (*abort_flag) break;
-          if (globaltimer_ns() - t_last > 1000000000ull) {
+          if (now - t_last > 1000000000ull) {
             *abort_flag = 1;
             atomicExch(&g_device_status, 2);
             break;
           }
+        } else {
+          __nanosleep(20);
         }
       }
       // every MMA issued must complete before TMEM is released (also on abort)
@@ -293,15 +325,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float pre = (warp == 3) ? wtot[0] : 0.f;
       const float lam1 = v + pre;       // token 2a+1
       const float lam0 = lam1 - l1;     // token 2a
+      // lam is kept in log2 units (lam * log2 e) so every decay is one ex2
       float* lj = lamb + slot * T;
       float* ec = ecolb + slot * T;
-      lj[2 * a] = lam0;
-      lj[2 * a + 1] = lam1;
+      lj[2 * a] = lam0 * kLog2e;
+      lj[2 * a + 1] = lam1 * kLog2e;
       named_sync(1, AUX);
       // decay from each column s to the last column of its 32-block
       const float lr = lj[(2 * a) | 31];
-      ec[2 * a] = __expf(lr - lam0);
-      ec[2 * a + 1] = __expf(lr - lam1);
+      ec[2 * a] = ex2(lr - lj[2 * a]);
+      ec[2 * a + 1] = ex2(lr - lj[2 * a + 1]);
       mbar_arrive(&bar[LAMRDY0 + slot]);
       if (a == 0) mark(j, EV_LAM_READY);
       d0 = n0;
@@ -311,13 +344,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = ctl.wait(FULL0 + st, (j >> 1) & 1);
       if (ok && j >= 2) ok = ctl.wait(CFULL0 + st, ((j - 2) >> 1) & 1);
       if (ok) {
-        const float lam_end = lj[T - 1];
+        const float lam_end = lj[T - 1];  // log2 units
         const uint4* src = reinterpret_cast<const uint4*>(sm + st * STAGE + OFF_X);
         uint4* dst = reinterpret_cast<uint4*>(sm + OFF_XP + st * TILE);
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
           const int row = a + 64 * rr;
-          const float w = __expf(lam_end - lj[row]);
+          const float w = ex2(lam_end - lj[row]);
           uint4 v4[8];
 #pragma unroll
           for (int c = 0; c < 8; ++c) v4[c] = src[swz128(row, c * 8) >> 4];
@@ -325,7 +358,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int c = 0; c < 8; ++c) {
             uint32_t* u = reinterpret_cast<uint32_t*>(&v4[c]);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < 4; ++i) {  // fp32 product, one rounding (the state accumulates it)
               const float2 f = bf2_to_f2(u[i]);
               u[i] = pack_bf16(f.x * w, f.y * w);
             }
@@ -349,24 +382,63 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (ok) ok = ctl.wait(SFULL0 + buf, (j >> 1) & 1);
       tc_fence_after();
       if (q == 3 && lane == 0) mark(j, EV_MASK_START);
-      const float* lj = lamb + slot * T;
+      if (ok) ok = ctl.wait(FULL0 + (j & 1), (j >> 1) & 1);  // the C tile, for C'
+      const float* lj = lamb + slot * T;   // log2 units
       const float* ec = ecolb + slot * T;
       const float lam_t = lj[row];
       const uint32_t tS = tl + buf * 256;
+      // C' row = exp(lam_t) C[row, :] into columns 64-127 (packed bf16 pairs, the A
+      // operand layout); those S columns are dead for this lane quarter once its
+      // mask has read them (quarters 0-1 never need them)
+      auto write_cprime = [&]() {
+        const __nv_bfloat162 e2 = __float2bfloat162_rn(ex2(lam_t));
+        const uint4* crow = reinterpret_cast<const uint4*>(sm + (j & 1) * STAGE + OFF_C);
+#pragma unroll
+        for (int kb2 = 0; kb2 < 2; ++kb2) {
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t w[16];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint4 v = crow[(kb2 * TILE + swz128(row, 8 * (4 * h2 + c))) >> 4];
+              __nv_bfloat162* u = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) u[i] = __hmul2(u[i], e2);
+              w[4 * c + 0] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
+            }
+            tmem_st16(tS + 64 + 32 * kb2 + 16 * h2, w);
+          }
+        }
+      };
+      if (q < 2) write_cprime();
+      const float4* ec4 = reinterpret_cast<const float4*>(ec);
+      const float4* lj4 = reinterpret_cast<const float4*>(lj);
+      // P block kb (32 columns) of this row from the S values r[0..31]
       auto make_block = [&](int kb, const uint32_t* r, uint32_t* pk) {
         if (kb < q) {
-          const float rowf = __expf(lam_t - lj[32 * kb + 31]);
+          // below the diagonal block: exp(lam_t - lam_s) = 2^(lt - l_end(kb)) * ec[s]
+          const float rowf = ex2(lam_t - lj[32 * kb + 31]);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16(__uint_as_float(r[2 * i]) * rowf * ec[32 * kb + 2 * i],
-                              __uint_as_float(r[2 * i + 1]) * rowf * ec[32 * kb + 2 * i + 1]);
+          for (int v = 0; v < 8; ++v) {
+            const float4 c = ec4[8 * kb + v];
+            pk[2 * v] = pack_bf16(__uint_as_float(r[4 * v]) * (rowf * c.x), __uint_as_float(r[4 * v + 1]) * (rowf * c.y));
+            pk[2 * v + 1] =
+                pack_bf16(__uint_as_float(r[4 * v + 2]) * (rowf * c.z), __uint_as_float(r[4 * v + 3]) * (rowf * c.w));
+          }
         } else if (kb == q) {
+          // diagonal block: direct decays, clamped at 0 above the diagonal and then zeroed
+          const int rl = row - 32 * kb;  // column index of the diagonal within the block
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int s0 = 32 * kb + 2 * i;
-            const float f0 = (s0 <= row) ? __uint_as_float(r[2 * i]) * __expf(lam_t - lj[s0]) : 0.f;
-            const float f1 = (s0 + 1 <= row) ? __uint_as_float(r[2 * i + 1]) * __expf(lam_t - lj[s0 + 1]) : 0.f;
-            pk[i] = pack_bf16(f0, f1);
+          for (int v = 0; v < 8; ++v) {
+            const float4 l = lj4[8 * kb + v];
+            const float e0 = ex2(fminf(lam_t - l.x, 0.f)), e1 = ex2(fminf(lam_t - l.y, 0.f));
+            const float e2 = ex2(fminf(lam_t - l.z, 0.f)), e3 = ex2(fminf(lam_t - l.w, 0.f));
+            const float f0 = (4 * v + 0 <= rl) ? __uint_as_float(r[4 * v + 0]) * e0 : 0.f;
+            const float f1 = (4 * v + 1 <= rl) ? __uint_as_float(r[4 * v + 1]) * e1 : 0.f;
+            const float f2 = (4 * v + 2 <= rl) ? __uint_as_float(r[4 * v + 2]) * e2 : 0.f;
+            const float f3 = (4 * v + 3 <= rl) ? __uint_as_float(r[4 * v + 3]) * e3 : 0.f;
+            pk[2 * v] = pack_bf16(f0, f1);
+            pk[2 * v + 1] = pack_bf16(f2, f3);
           }
         } else {
 #pragma unroll
@@ -380,13 +452,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (kb <= q) tmem_ld32(tS + 32 * kb, r0);
         if (kb + 1 <= q) tmem_ld32(tS + 32 * (kb + 1), r1);
         tmem_wait_ld();
-        if (kb == 0 && q == 3 && lane == 0) mark(j, EV_MASK_LD);
+        if (q == 3 && lane == 0) mark(j, kb == 0 ? EV_MASK_LD : EV_MASK_LD2);
         make_block(kb, r0, pk);
         tmem_st16(tS + 16 * kb, pk);
         make_block(kb + 1, r1, pk);
         tmem_st16(tS + 16 * (kb + 1), pk);
+        if (q == 3 && lane == 0) mark(j, kb == 0 ? EV_MASK_B01 : EV_MASK_B23);
       }
+      if (q >= 2) write_cprime();
       tmem_wait_st();
+      if (q == 3 && lane == 0) mark(j, EV_MASK_WST);
       tc_fence_before();
       (void)ok;
       mbar_arrive(&bar[PFULL0 + buf]);
@@ -449,10 +524,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (r == 0) mark(j, EV_C_SEEN);
       const float* lj = lamb + (j & 3) * T;
       const float lam_end = lj[T - 1];
-      const float lam_t = lj[r];
       const uint32_t base = tl + buf * 256;
       // state: s_j = exp(lam_end) s_{j-1} + b_intra
-      const float dec = __expf(lam_end);
+      const float dec = ex2(lam_end);  // lam in log2 units
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t v[32];
@@ -463,16 +537,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (ok) publish_state();
       if (r == 0) mark(j, EV_STATE_PUB);
-      // y_t = y_intra + exp(lam_t) y_inter + D x_t
-      const float e = __expf(lam_t);
+      // y_t = y + D x_t
       const int64_t tg = (int64_t)j * T + r;
       uint4* dst = reinterpret_cast<uint4*>(p.y + (int64_t)b * p.sy + (tg * p.H + h) * P);
       const bool row_in = tg < p.L;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t yi[16], ye[16];
+        uint32_t yi[16];
         tmem_ld16(base + 128 + 16 * c, yi);
-        tmem_ld16(base + 64 + 16 * c, ye);
         tmem_wait_ld();
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -484,8 +556,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int i = 0; i < 4; ++i) {
             const int k0 = h2 * 8 + 2 * i;
             const float2 xf = bf2_to_f2(xu[i]);
-            o[i] = pack_bf16(fmaf(e, __uint_as_float(ye[k0]), fmaf(Dh, xf.x, __uint_as_float(yi[k0]))),
-                             fmaf(e, __uint_as_float(ye[k0 + 1]), fmaf(Dh, xf.y, __uint_as_float(yi[k0 + 1]))));
+            o[i] = pack_bf16(fmaf(Dh, xf.x, __uint_as_float(yi[k0])), fmaf(Dh, xf.y, __uint_as_float(yi[k0 + 1])));
           }
           if (row_in) dst[cc] = ov;
         }

@@ -291,17 +291,18 @@ def ssd_selftest_umma(variant: str, A: torch.Tensor, B: torch.Tensor, N: int, K:
 
 
 TRACE_EVENTS = ["loads", "S_issued", "c_issued", "mask_start", "mask_done", "lam_ready", "xp_done", "c_seen",
-                "state_pub", "epi_done"]
+                "state_pub", "epi_done", "c_ready", "c_mid", "S_ready", "mask_ld", "mask_b01", "mask_ld2", "mask_b23",
+                "mask_wait_st"]
 
 
 def ssd_selftest_fused_trace(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, stream=None):
     """Diagnostic: run the fused kernel with CTA 0 tracing its pipeline events.
-    Returns (y, final_state, trace [nsub, 16] int64 clocks)."""
+    Returns (y, final_state, trace [nsub, 24] int64 clocks)."""
     dims = make_dims(x, Bm, chunk)
     nsub = -(-dims.seqlen // 128)
     y = torch.empty_like(x)
     fin = torch.empty((dims.batch, dims.nheads, dims.dstate, dims.headdim), dtype=torch.float32, device=x.device)
-    trace = torch.zeros((nsub, 16), dtype=torch.int64, device=x.device)
+    trace = torch.zeros((nsub, 24), dtype=torch.int64, device=x.device)
     _check(lib().ssd_selftest_fused_trace(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D),
                                           _ptr(init_state), _ptr(y), _ptr(fin), _ptr(trace), trace.numel(),
                                           _stream(stream)), "ssd_selftest_fused_trace")

@@ -44,10 +44,13 @@ ssd_status ssd_selftest_umma(int32_t variant, const void* A, const void* B, floa
  * arguments; the problem must be one the fused kernel takes, else
  * SSD_ERR_UNSUPPORTED) and has the CTA of batch 0, head 0 write the SM clock
  * (clock64) of each pipeline event of each 128-token sub-chunk j to
- * trace[16*j + e] (device buffer of trace_len >= 16*ceil(L/128) uint64):
+ * trace[24*j + e] (device buffer of trace_len >= 24*ceil(L/128) uint64):
  * e = 0 loads issued, 1 S issued, 2 products issued, 3 mask started, 4 mask
  * done, 5 lam ready, 6 X' done, 7 products seen by the epilogue, 8 state
- * published, 9 epilogue done.  Used to find the critical path.
+ * published, 9 epilogue done, 10 products ready to issue, 11 first third of
+ * the products issued, 12 S ready to issue, 13-17 points inside the mask
+ * (first TMEM read, blocks 0-1 written, second read, blocks 2-3 written,
+ * stores complete).  Used to find the critical path.
  */
 ssd_status ssd_selftest_fused_trace(const ssd_dims* d, const void* x, const float* dt, const float* A,
                                     const void* Bm, const void* Cm, const float* D, const float* init_state,

@@ -32,6 +32,22 @@ METRIC = "SSD scan tokens/s & % of roofline (1×B200, B=8 L=16K H=80 P=64 N=128)
 WORKLOAD = "mamba2_2p7b_layer"
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The largest `value` over all ranks (plain value on a single process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's batch: every rank scans its own independent sequences."""
+    return int(rank)
+
+
 def algorithmic_bytes(wl) -> int:
     """Bytes one scan must move at minimum: x, y, dt, B, C, A, D, init, final."""
     Bz, L, H, P, N, G = wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.dstate, wl.ngroups
@@ -229,7 +245,7 @@ def main():
     wl = inputs.WORKLOADS[args.workload]
     if args.batch:
         wl = inputs.custom(wl.name, batch=args.batch)
-    host = inputs.generate(wl, seed=rank)          # each rank: its own independent batch
+    host = inputs.generate(wl, seed=rank_seed(rank))  # each rank: its own independent batch
     pinned = {}
     for k, v in host.items():
         t = torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16 else torch.from_numpy(v)
@@ -272,10 +288,7 @@ def main():
         dist.barrier()
     ms_total = t_start.elapsed_time(t_end)
     per_step = [a.elapsed_time(b) for a, b in ev]
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dev)
     ms_per_step = ms_total / args.steps
     tokens = wl.batch * wl.seqlen * world
     value = tokens / (ms_per_step * 1e-3)
@@ -299,10 +312,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / max(args.e2e_steps, 1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev)
     e2e_value = tokens / (e2e_ms * 1e-3)
 
     hbm_peak, tc_peak, tc_sust, peak_src = load_peaks()

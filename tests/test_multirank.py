@@ -1,0 +1,93 @@
+"""The multi-rank host logic of bench.py, on CPU with gloo (world size 2).
+
+On the GPU machine bench.py runs one process per GPU under torchrun; every rank
+scans its own batch (no collective on the data path) and only the timing is
+reduced (max over ranks).  These tests run that reduction and the rank
+conventions with the gloo backend on 127.0.0.1.
+"""
+import datetime
+import os
+import socket
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        got = bench.max_over_ranks(10.0 + 5.0 * rank, torch.device("cpu"))
+        q.put((rank, got, bench.rank_seed(rank)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    res.sort()
+    assert [r[1] for r in res] == [15.0, 15.0]        # every rank sees the max
+    assert res[0][2] != res[1][2]                      # distinct batches
+
+
+def test_single_process_max_is_identity():
+    import torch
+    import bench
+    assert bench.max_over_ranks(3.5, torch.device("cpu")) == 3.5
+
+
+def test_rank_batches_are_independent():
+    from chunked_state_space_b200 import inputs
+    import bench
+    wl = inputs.custom("mamba2_2p7b_layer", batch=1, seqlen=256)
+    a = inputs.generate(wl, seed=bench.rank_seed(0), names=("x",))["x"]
+    b = inputs.generate(wl, seed=bench.rank_seed(1), names=("x",))["x"]
+    assert not np.array_equal(a, b)
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
+
+
+def test_reference_arm_rank0_prints_one_line():
+    import json
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3"], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"

@@ -52,9 +52,18 @@ constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TX_BYTES = 5 * TILE;
 
+// Modes: the whole scan (one CTA per (batch, head) sequence), or one CTA per
+// (batch, head, chunk) for the step kernels -- chunk states from a zero start
+// (step 2) or chunk outputs from given previous states (step 4) -- with the
+// log-decay sums read from step 1's output instead of scanned from dt.
+enum { MODE_SCAN = 0, MODE_CHUNK_STATE = 1, MODE_CHUNK_SCAN = 2 };
+
 struct Params {
+  int mode;
   int64_t L;
   int H, G, nsub;
+  int64_t nc, Q;         // chunking of the step kernels
+  const float* lam_in;   // step-1 log-decay sums [B,H,nc,Q] (step modes)
   const float* dt;
   int64_t sdt;
   const float* A;
@@ -145,10 +154,18 @@ __global__ void __launch_bounds__(THREADS, 1)
   Ctl ctl{bar, abort_flag};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
-  const int b = bh / p.H, h = bh % p.H;
+  const bool chunked = p.mode != MODE_SCAN;
+  const int64_t bh = chunked ? (int64_t)blockIdx.x / p.nc : (int64_t)blockIdx.x;
+  const int64_t cidx = chunked ? (int64_t)blockIdx.x % p.nc : 0;   // chunk of this CTA (step modes)
+  const int b = (int)(bh / p.H), h = (int)(bh % p.H);
   const int g = h / (p.H / p.G);
-  const int nsub = p.nsub;
+  const int t_base = (int)(cidx * p.Q);                          // first token of this CTA
+  const int nsub = chunked ? (int)ceil_div(min((int64_t)p.Q, p.L - t_base), (int64_t)T) : p.nsub;
+  const int64_t cslot = bh * p.nc + cidx;                       // [B,H,nc] index (step modes)
+  const float* init_ptr = chunked ? (p.mode == MODE_CHUNK_SCAN ? p.init + cslot * NS * P : nullptr)
+                                  : (p.init ? p.init + bh * NS * P : nullptr);
+  float* final_ptr = chunked ? (p.mode == MODE_CHUNK_STATE ? p.final_state + cslot * NS * P : nullptr)
+                             : (p.final_state ? p.final_state + bh * NS * P : nullptr);
   unsigned long long* const trace = (p.trace && blockIdx.x == 0) ? p.trace : nullptr;
   auto mark = [&](int j, int ev) {
     if (trace) trace[j * kTraceEvents + ev] = clock64();
@@ -186,7 +203,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       constexpr int kPrefetch = 3;
       auto prefetch = [&](int jp) {
         if (jp >= nsub) return;
-        const int tp = jp * T;
+        const int tp = t_base + jp * T;
         tma_prefetch_4d(&map_x, 0, h, tp, b);
         tma_prefetch_4d(&map_b, 0, g, tp, b);
         tma_prefetch_4d(&map_b, 64, g, tp, b);
@@ -199,7 +216,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         prefetch(j + kPrefetch);
         if (j >= 2 && !ctl.wait(EMPTY0 + st, ((j >> 1) + 1) & 1)) break;
         uint8_t* sx = sm + st * STAGE;
-        const int t0 = j * T;
+        const int t0 = t_base + j * T;
         mbar_arrive_expect_tx(&bar[FULL0 + st], TX_BYTES);
         tma_load_4d(sx + OFF_X, &map_x, &bar[FULL0 + st], 0, h, t0, b);
         tma_load_4d(sx + OFF_B, &map_b, &bar[FULL0 + st], 0, g, t0, b);
@@ -299,13 +316,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp < 4) {
     // ------------------------------------------------------------ dt, lam, decay factors, X'
     const int a = threadIdx.x - 64;  // 0..63
-    const float Ah = p.A[h];
+    const float Ah = chunked ? 0.f : p.A[h];  // A (and dt) are read only by the whole scan
     const float* dtb = p.dt + (int64_t)b * p.sdt + h;
     auto load_dt = [&](int j, float& d0, float& d1) {
       const int64_t t0 = (int64_t)j * T + 2 * a;
-      d0 = (j < nsub && t0 < p.L) ? dtb[t0 * p.H] : 0.f;
-      d1 = (j < nsub && t0 + 1 < p.L) ? dtb[(t0 + 1) * p.H] : 0.f;
+      d0 = (!chunked && j < nsub && t0 < p.L) ? dtb[t0 * p.H] : 0.f;
+      d1 = (!chunked && j < nsub && t0 + 1 < p.L) ? dtb[(t0 + 1) * p.H] : 0.f;
     };
+    const float* lamc = chunked ? p.lam_in + cslot * p.Q : nullptr;
     float d0, d1;
     load_dt(0, d0, d1);
     for (int j = 0; j < nsub; ++j) {
@@ -323,8 +341,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 31) wtot[warp - 2] = v;
       named_sync(1, AUX);
       const float pre = (warp == 3) ? wtot[0] : 0.f;
-      const float lam1 = v + pre;       // token 2a+1
-      const float lam0 = lam1 - l1;     // token 2a
+      float lam1 = v + pre;       // token 2a+1
+      float lam0 = lam1 - l1;     // token 2a
+      if (chunked) {              // step modes: sub-chunk-local sums from step 1's output
+        const float* ls = lamc + j * T;
+        const float base0 = (j == 0) ? 0.f : ls[-1];
+        lam0 = ls[2 * a] - base0;
+        lam1 = ls[2 * a + 1] - base0;
+      }
       // lam is kept in log2 units (lam * log2 e) so every decay is one ex2
       float* lj = lamb + slot * T;
       float* ec = ecolb + slot * T;
@@ -477,7 +501,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // from the TMA load; the wait hides the latency)
     const __nv_bfloat16* xg = p.x + (int64_t)b * p.sx + (int64_t)h * P;
     auto load_x = [&](int j, uint4* xv) {
-      const int64_t tg = (int64_t)j * T + r;
+      const int64_t tg = (int64_t)t_base + (int64_t)j * T + r;
       if (j < nsub && tg < p.L) {
         const uint4* src = reinterpret_cast<const uint4*>(xg + tg * p.H * P);
 #pragma unroll
@@ -489,8 +513,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     };
     uint4 xcur[8];
     float s[P];
-    if (p.init) {
-      const float4* src = reinterpret_cast<const float4*>(p.init + ((int64_t)bh * NS + r) * P);
+    if (init_ptr) {
+      const float4* src = reinterpret_cast<const float4*>(init_ptr + (int64_t)r * P);
 #pragma unroll
       for (int i = 0; i < P / 4; ++i) {
         const float4 v = src[i];
@@ -538,9 +562,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (ok) publish_state();
       if (r == 0) mark(j, EV_STATE_PUB);
       // y_t = y + D x_t
-      const int64_t tg = (int64_t)j * T + r;
+      const int64_t tg = (int64_t)t_base + (int64_t)j * T + r;
       uint4* dst = reinterpret_cast<uint4*>(p.y + (int64_t)b * p.sy + (tg * p.H + h) * P);
-      const bool row_in = tg < p.L;
+      const bool row_in = p.y != nullptr && tg < p.L;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t yi[16];
@@ -565,8 +589,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive(&bar[TEMPTY0 + buf]);
       if (r == 0) mark(j, EV_EPI_DONE);
     }
-    if (p.final_state) {
-      float4* dst = reinterpret_cast<float4*>(p.final_state + ((int64_t)bh * NS + r) * P);
+    if (final_ptr) {
+      float4* dst = reinterpret_cast<float4*>(final_ptr + (int64_t)r * P);
 #pragma unroll
       for (int i = 0; i < P / 4; ++i) dst[i] = make_float4(s[4 * i], s[4 * i + 1], s[4 * i + 2], s[4 * i + 3]);
     }
@@ -587,18 +611,45 @@ bool fused_supported(const Problem& p) {
   return p.io == SSD_BF16 && p.P == fused::P && p.N == fused::NS && p.Q % fused::T == 0 && p.B * p.H < (1ll << 31);
 }
 
+bool tc_supported(const Problem& p) { return fused_supported(p) && p.B * p.H * p.nc < (1ll << 31); }
+
 int fused_kernels_per_call(const Problem&) { return 1; }
 
-cudaError_t launch_fused_traced(const Problem& p, const float* init, float* final_state, unsigned long long* trace,
-                                cudaStream_t st);
-
-cudaError_t launch_fused(const Problem& p, const float* init, float* final_state, void*, cudaStream_t st) {
-  return launch_fused_traced(p, init, final_state, nullptr, st);
-}
+static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
+                               void* y, unsigned long long* trace, cudaStream_t st);
 
 cudaError_t launch_fused_traced(const Problem& p, const float* init, float* final_state, unsigned long long* trace,
                                 cudaStream_t st) {
+  return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, trace, st);
+}
+
+cudaError_t launch_fused(const Problem& p, const float* init, float* final_state, void*, cudaStream_t st) {
+  return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, nullptr, st);
+}
+
+// Step 2 on tensor cores: one CTA per (batch, head, chunk), zero start, the
+// chunk's end state written to states[b,h,c].
+cudaError_t launch_chunk_state_tc(const Problem& p, const float* lam, float* states, cudaStream_t st) {
+  return launch_mode(p, fused::MODE_CHUNK_STATE, lam, nullptr, states, nullptr, nullptr, st);
+}
+
+// Step 4 on tensor cores: one CTA per (batch, head, chunk), starting from
+// prev[b,h,c], writing the chunk's outputs.
+cudaError_t launch_chunk_scan_tc(const Problem& p, const float* lam, const float* prev, cudaStream_t st) {
+  return launch_mode(p, fused::MODE_CHUNK_SCAN, lam, prev, nullptr, p.y, nullptr, st);
+}
+
+static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
+                               void* y, unsigned long long* trace, cudaStream_t st) {
   using namespace fused;
+  // every pointer the mode reads must be present (the step entry points pass
+  // only the tensors of their step)
+  if (!p.x || !p.Bm) return cudaErrorInvalidValue;
+  if (mode == MODE_SCAN && (!p.dt || !p.A || !p.Cm || !y)) return cudaErrorInvalidValue;
+  if (mode == MODE_CHUNK_STATE && (!lam || !final_state)) return cudaErrorInvalidValue;
+  if (mode == MODE_CHUNK_SCAN && (!lam || !init || !p.Cm || !y)) return cudaErrorInvalidValue;
+  // the chunk-state mode never uses C: its C tiles are read from B (valid memory)
+  const void* cptr = (mode == MODE_CHUNK_STATE) ? p.Bm : p.Cm;
   CUtensorMap mx, mb, mc;
   const uint32_t box[4] = {64, 1, (uint32_t)T, 1};
   const uint64_t dx[4] = {(uint64_t)P, (uint64_t)p.H, (uint64_t)p.L, (uint64_t)p.B};
@@ -606,9 +657,13 @@ cudaError_t launch_fused_traced(const Problem& p, const float* init, float* fina
   const uint64_t dbc[4] = {(uint64_t)NS, (uint64_t)p.G, (uint64_t)p.L, (uint64_t)p.B};
   const uint64_t sbc[3] = {(uint64_t)NS * 2, (uint64_t)p.G * NS * 2, (uint64_t)p.sbc * 2};
   if (!tma::encode_bf16(&mx, p.x, 4, dx, sx, box) || !tma::encode_bf16(&mb, p.Bm, 4, dbc, sbc, box) ||
-      !tma::encode_bf16(&mc, p.Cm, 4, dbc, sbc, box))
+      !tma::encode_bf16(&mc, cptr, 4, dbc, sbc, box))
     return cudaErrorInvalidValue;
   Params kp;
+  kp.mode = mode;
+  kp.nc = p.nc;
+  kp.Q = p.Q;
+  kp.lam_in = lam;
   kp.L = p.L;
   kp.H = (int)p.H;
   kp.G = (int)p.G;
@@ -621,12 +676,13 @@ cudaError_t launch_fused_traced(const Problem& p, const float* init, float* fina
   kp.final_state = final_state;
   kp.x = static_cast<const __nv_bfloat16*>(p.x);
   kp.sx = p.sx;
-  kp.y = static_cast<__nv_bfloat16*>(p.y);
+  kp.y = static_cast<__nv_bfloat16*>(y);
   kp.sy = p.sy;
   kp.trace = trace;
   cudaError_t e = cudaFuncSetAttribute(k_ssd_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  k_ssd_fused<<<(unsigned)(p.B * p.H), THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc);
+  const int64_t ctas = mode == fused::MODE_SCAN ? p.B * p.H : p.B * p.H * p.nc;
+  k_ssd_fused<<<(unsigned)ctas, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc);
   return cudaGetLastError();
 }
 

@@ -97,12 +97,19 @@ def test_deterministic():
 
 # ------------------------------------------------------------------ the four steps, one at a time
 
-@pytest.mark.parametrize("io", ["f32", "bf16"])
-def test_steps_match_oracle_intermediates(io):
-    if io == "f32":
+@pytest.mark.parametrize("case", ["f32", "bf16_tensor_cores", "bf16_cuda_cores"])
+def test_steps_match_oracle_intermediates(case):
+    """Each step kernel on the oracle's inputs to that step.  bf16 with P = 64,
+    N = 128, Q % 128 = 0 runs steps 2 and 4 on tcgen05; other bf16 shapes on
+    CUDA cores."""
+    if case == "f32":
         wl = inputs.custom("tiny_f32", batch=2, seqlen=300, nheads=4, ngroups=2, init_var=0.3)
-    else:
+    elif case == "bf16_tensor_cores":
         wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=700, nheads=4, ngroups=2, init_var=0.1)
+    else:
+        wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=700, nheads=4, ngroups=2, headdim=32, dstate=64,
+                           chunk=128, init_var=0.1)
+    io = wl.io
     tol = TOL[io]
     host = inputs.generate(wl)
     dev = device_inputs(host)

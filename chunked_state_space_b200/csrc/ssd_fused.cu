@@ -133,6 +133,33 @@ __device__ __forceinline__ float ex2(float x) {
 }
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Packed fp32x2 arithmetic (sm_100): two lanes of fp32 per instruction, each
+// lane rounded like the scalar operation.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 c;
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rc, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rc;\n\t}"
+      : "=f"(c.x), "=f"(c.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return c;
+}
+
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
 __device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
@@ -383,8 +410,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint32_t* u = reinterpret_cast<uint32_t*>(&v4[c]);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {  // fp32 product, one rounding (the state accumulates it)
-              const float2 f = bf2_to_f2(u[i]);
-              u[i] = pack_bf16(f.x * w, f.y * w);
+              const float2 f = mul2(bf2_to_f2(u[i]), make_float2(w, w));
+              u[i] = pack_bf16(f.x, f.y);
             }
             dst[swz128(row, c * 8) >> 4] = v4[c];
           }
@@ -442,12 +469,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (kb < q) {
           // below the diagonal block: exp(lam_t - lam_s) = 2^(lt - l_end(kb)) * ec[s]
           const float rowf = ex2(lam_t - lj[32 * kb + 31]);
+          const float2 rf2 = make_float2(rowf, rowf);
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
             const float4 c = ec4[8 * kb + v];
-            pk[2 * v] = pack_bf16(__uint_as_float(r[4 * v]) * (rowf * c.x), __uint_as_float(r[4 * v + 1]) * (rowf * c.y));
-            pk[2 * v + 1] =
-                pack_bf16(__uint_as_float(r[4 * v + 2]) * (rowf * c.z), __uint_as_float(r[4 * v + 3]) * (rowf * c.w));
+            const float2 a = mul2(mul2(make_float2(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1])),
+                                       make_float2(c.x, c.y)), rf2);
+            const float2 bb = mul2(mul2(make_float2(__uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])),
+                                        make_float2(c.z, c.w)), rf2);
+            pk[2 * v] = pack_bf16(a.x, a.y);
+            pk[2 * v + 1] = pack_bf16(bb.x, bb.y);
           }
         } else if (kb == q) {
           // diagonal block: direct decays, clamped at 0 above the diagonal and then zeroed
@@ -557,7 +588,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_ld32(base + 192 + 32 * c, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[32 * c + i] = fmaf(dec, s[32 * c + i], __uint_as_float(v[i]));
+        for (int i = 0; i < 32; i += 2) {
+          const float2 o = fma2(make_float2(dec, dec), make_float2(s[32 * c + i], s[32 * c + i + 1]),
+                                make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])));
+          s[32 * c + i] = o.x;
+          s[32 * c + i + 1] = o.y;
+        }
       }
       if (ok) publish_state();
       if (r == 0) mark(j, EV_STATE_PUB);
@@ -580,7 +616,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int i = 0; i < 4; ++i) {
             const int k0 = h2 * 8 + 2 * i;
             const float2 xf = bf2_to_f2(xu[i]);
-            o[i] = pack_bf16(fmaf(Dh, xf.x, __uint_as_float(yi[k0])), fmaf(Dh, xf.y, __uint_as_float(yi[k0 + 1])));
+            const float2 yo = fma2(make_float2(Dh, Dh), xf,
+                                   make_float2(__uint_as_float(yi[k0]), __uint_as_float(yi[k0 + 1])));
+            o[i] = pack_bf16(yo.x, yo.y);
           }
           if (row_in) dst[cc] = ov;
         }

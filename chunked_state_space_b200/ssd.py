@@ -26,7 +26,7 @@ EXPORTED = ["ssd_status_string", "ssd_version", "ssd_scan_workspace_size", "ssd_
             "ssd_scan_fwd_unfused", "ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing",
             "ssd_chunk_scan", "ssd_rmsnorm", "ssd_vertical_workspace_size", "ssd_vertical_fwd",
             "ssd_read_device_status", "ssd_selftest_umma", "ssd_scan_path", "ssd_step",
-            "ssd_selftest_fused_trace", "ssd_scan_fwd_noalloc"]
+            "ssd_selftest_fused_trace", "ssd_scan_fwd_noalloc", "ssd_selftest_mask_timing"]
 
 
 class SSDError(RuntimeError):
@@ -76,6 +76,7 @@ def lib() -> ctypes.CDLL:
         "ssd_scan_path": (ctypes.c_int, [D, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]),
         "ssd_step": (ctypes.c_int, [D] + [_P] * 9),
         "ssd_scan_fwd_noalloc": (ctypes.c_int, [D] + [_P] * 10),
+        "ssd_selftest_mask_timing": (ctypes.c_int, [ctypes.c_int32, _P, _P, _P]),
         "ssd_selftest_fused_trace": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_int64, _P]),
     }
     for name, (res, args) in sig.items():
@@ -307,3 +308,12 @@ def ssd_selftest_fused_trace(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: i
                                           _ptr(init_state), _ptr(y), _ptr(fin), _ptr(trace), trace.numel(),
                                           _stream(stream)), "ssd_selftest_fused_trace")
     return y, fin, trace
+
+
+def ssd_selftest_mask_timing(variant: int, stream=None):
+    """Diagnostic: SM clocks per repetition of one mask building block (see
+    include/ssd_selftest.h), one value per thread of the 4-warp CTA."""
+    cyc = torch.zeros(128, dtype=torch.int64, device="cuda")
+    sink = torch.zeros(128, dtype=torch.float32, device="cuda")
+    _check(lib().ssd_selftest_mask_timing(variant, _ptr(cyc), _ptr(sink), _stream(stream)), "ssd_selftest_mask_timing")
+    return cyc

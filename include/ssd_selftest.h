@@ -57,6 +57,17 @@ ssd_status ssd_selftest_fused_trace(const ssd_dims* d, const void* x, const floa
                                     void* y, float* final_state, unsigned long long* trace, int64_t trace_len,
                                     void* stream);
 
+/*
+ * ssd_selftest_mask_timing times, on one CTA of 4 warps, 64 repetitions of one
+ * building block of the fused kernel's mask (variant 0: two 32-column TMEM
+ * loads; 1: plus the off-diagonal block arithmetic; 2: plus two 16-column
+ * TMEM stores; 3: off-diagonal arithmetic alone; 4: diagonal-block arithmetic
+ * alone; 5: sixteen 16-byte shared-memory row loads) and writes the SM clocks
+ * per repetition of each thread to cycles[128] (device int64); sink[128]
+ * (device f32) receives a checksum that keeps the work alive.
+ */
+ssd_status ssd_selftest_mask_timing(int32_t variant, long long* cycles, float* sink, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -8,11 +8,10 @@
 // sub-chunk, with lam the in-sub-chunk cumulative sum of dt*A:
 //   S       = C_j B_j^T                                   (tcgen05, 128x128x128)
 //   P       = S (.) exp(lam_t - lam_s) [s <= t]  -> bf16 in TMEM, columns 0-63
-//   C'      = diag(exp(lam_t)) C_j                -> bf16 in TMEM, columns 64-127
-//   y       = P X_j + C' bf16(s_{j-1})            (both A operands from TMEM: the
-//             page's by_intra + by_inter in one accumulator)
+//   y_intra = P X_j                               (A operand from TMEM)
+//   y_inter = C_j bf16(s_{j-1})                   (into S columns 64-127, dead by then)
 //   b_intra = B_j^T X'_j,  X'_j = diag(exp(lam_end - lam_s)) X_j
-//   y_t     = y + D x_t                           (x_t re-read from L2, fp32)
+//   y_t     = y_intra + exp(lam_t) y_inter + D x_t    (fp32; x_t re-read from L2)
 //   s_j     = exp(lam_end) s_{j-1} + b_intra              (fp32, registers)
 // Warp roles (384 threads): warp 0 issues TMA loads; warp 1 owns TMEM and
 // issues MMAs; warps 2-3 load dt one sub-chunk ahead, scan lam, form the
@@ -21,7 +20,7 @@
 // publish its bf16 copy.  The mask needs exp(lam_t - lam_s) only inside the
 // diagonal 32x32 blocks: below them it is exp(lam_t - lam_r) exp(lam_r - lam_s)
 // with r the last column of the block (both factors <= 1).
-// TMEM holds two 256-column buffers [S -> P | C'][y][b_intra] so sub-chunk
+// TMEM holds two 256-column buffers [S -> P | y_inter][y_intra][b_intra] so sub-chunk
 // j+1's S and mask overlap sub-chunk j's products and epilogue.  Every wait is bounded; a timeout
 // raises g_device_status and the roles drain without further waits.
 #include "ssd_tc.cuh"
@@ -291,11 +290,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                    ks > 0);
           mark(jc, EV_C_MID);
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks)  // y = P X
+          for (int ks = 0; ks < 8; ++ks)  // y_intra = P X
             mma_ts(base + 128, base + ks * 8, smem_desc(sX + ks * 2048, TILE, 1024), idY, ks > 0);
+          const uint32_t sC = sbase + st * STAGE + OFF_C;
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks)  // y += C' prev
-            mma_ts(base + 128, base + 64 + ks * 8, smem_desc(sPrev + ks * 2048, TILE, 1024), idY, 1u);
+          for (int ks = 0; ks < 8; ++ks) {  // y_inter = C prev  (K = dstate)
+            const uint32_t koff = (ks >> 2) * TILE + (ks & 3) * 32;
+            mma_ss(base + 64, smem_desc(sC + koff, 16, 1024), smem_desc(sPrev + ks * 2048, TILE, 1024), idY, ks > 0);
+          }
           mma_commit(&bar[CFULL0 + buf]);
           mma_commit(&bar[EMPTY0 + st]);
           mark(jc, EV_C_ISSUED);
@@ -433,35 +435,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (ok) ok = ctl.wait(SFULL0 + buf, (j >> 1) & 1);
       tc_fence_after();
       if (q == 3 && lane == 0) mark(j, EV_MASK_START);
-      if (ok) ok = ctl.wait(FULL0 + (j & 1), (j >> 1) & 1);  // the C tile, for C'
       const float* lj = lamb + slot * T;   // log2 units
       const float* ec = ecolb + slot * T;
       const float lam_t = lj[row];
       const uint32_t tS = tl + buf * 256;
-      // C' row = exp(lam_t) C[row, :] into columns 64-127 (packed bf16 pairs, the A
-      // operand layout); those S columns are dead for this lane quarter once its
-      // mask has read them (quarters 0-1 never need them)
-      auto write_cprime = [&]() {
-        const __nv_bfloat162 e2 = __float2bfloat162_rn(ex2(lam_t));
-        const uint4* crow = reinterpret_cast<const uint4*>(sm + (j & 1) * STAGE + OFF_C);
-#pragma unroll
-        for (int kb2 = 0; kb2 < 2; ++kb2) {
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            uint32_t w[16];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint4 v = crow[(kb2 * TILE + swz128(row, 8 * (4 * h2 + c))) >> 4];
-              __nv_bfloat162* u = reinterpret_cast<__nv_bfloat162*>(&v);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) u[i] = __hmul2(u[i], e2);
-              w[4 * c + 0] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
-            }
-            tmem_st16(tS + 64 + 32 * kb2 + 16 * h2, w);
-          }
-        }
-      };
-      if (q < 2) write_cprime();
       const float4* ec4 = reinterpret_cast<const float4*>(ec);
       const float4* lj4 = reinterpret_cast<const float4*>(lj);
       // P block kb (32 columns) of this row from the S values r[0..31]
@@ -514,7 +491,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_st16(tS + 16 * (kb + 1), pk);
         if (q == 3 && lane == 0) mark(j, kb == 0 ? EV_MASK_B01 : EV_MASK_B23);
       }
-      if (q >= 2) write_cprime();
       tmem_wait_st();
       if (q == 3 && lane == 0) mark(j, EV_MASK_WST);
       tc_fence_before();
@@ -597,14 +573,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (ok) publish_state();
       if (r == 0) mark(j, EV_STATE_PUB);
-      // y_t = y + D x_t
+      // y_t = y_intra + exp(lam_t) y_inter + D x_t
+      const float et = ex2(lj[r]);
       const int64_t tg = (int64_t)t_base + (int64_t)j * T + r;
       uint4* dst = reinterpret_cast<uint4*>(p.y + (int64_t)b * p.sy + (tg * p.H + h) * P);
       const bool row_in = p.y != nullptr && tg < p.L;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t yi[16];
+        uint32_t yi[16], ye[16];
         tmem_ld16(base + 128 + 16 * c, yi);
+        tmem_ld16(base + 64 + 16 * c, ye);
         tmem_wait_ld();
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -616,8 +594,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int i = 0; i < 4; ++i) {
             const int k0 = h2 * 8 + 2 * i;
             const float2 xf = bf2_to_f2(xu[i]);
-            const float2 yo = fma2(make_float2(Dh, Dh), xf,
-                                   make_float2(__uint_as_float(yi[k0]), __uint_as_float(yi[k0 + 1])));
+            float2 yo = fma2(make_float2(Dh, Dh), xf, make_float2(__uint_as_float(yi[k0]), __uint_as_float(yi[k0 + 1])));
+            yo = fma2(make_float2(et, et), make_float2(__uint_as_float(ye[k0]), __uint_as_float(ye[k0 + 1])), yo);
             o[i] = pack_bf16(yo.x, yo.y);
           }
           if (row_in) dst[cc] = ov;

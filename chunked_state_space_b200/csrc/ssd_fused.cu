@@ -13,8 +13,8 @@
 //   b_intra = B_j^T X'_j,  X'_j = diag(exp(lam_end - lam_s)) X_j
 //   y_t     = y_intra + exp(lam_t) y_inter + D x_t    (fp32; x_t re-read from L2)
 //   s_j     = exp(lam_end) s_{j-1} + b_intra              (fp32, registers)
-// Warp roles (384 threads): warp 0 issues TMA loads; warp 1 owns TMEM and
-// issues MMAs; warps 2-3 load dt one sub-chunk ahead, scan lam, form the
+// Warp roles (384 threads): warp 2 issues TMA loads; warp 3 owns TMEM and
+// issues MMAs; warps 0-1 load dt one sub-chunk ahead, scan lam, form the
 // per-column decay factors and X'; warps 4-7 (one thread per row) turn S
 // into P; warps 8-11 (one thread per row) finish y, update the state and
 // publish its bf16 copy.  The mask needs exp(lam_t - lam_s) only inside the
@@ -73,7 +73,8 @@ struct Params {
   int64_t sx;
   __nv_bfloat16* y;
   int64_t sy;
-  unsigned long long* trace;  // diagnostics: per-sub-chunk event clocks of CTA 0, or NULL
+  unsigned long long* trace;  // diagnostics: per-sub-chunk event clocks of CTA 0, then
+                              // [start ns, end ns, SM] of every CTA; or NULL
 };
 
 // Trace events (clock64 of CTA 0), one row of kTraceEvents per sub-chunk.
@@ -87,7 +88,11 @@ enum {
 enum {
   FULL0 = 0, EMPTY0 = 2, SFULL0 = 4, PFULL0 = 6, CFULL0 = 8, TEMPTY0 = 10, STATEFULL = 12, DRAIN = 13, LAMRDY0 = 14
 };
-constexpr int AUX = 64;  // threads of warps 2-3
+constexpr int AUX = 64;  // threads of warps 0-1
+// Warp w runs on SM sub-partition w % 4 and may only touch TMEM lane quarter
+// w % 4, so the rows with the most mask work (quarter 3) share a sub-partition
+// with the lightest single-thread role.
+constexpr int W_TMA = 2, W_MMA = 3;
 
 struct Ctl {
   uint64_t* bar;
@@ -196,8 +201,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   auto mark = [&](int j, int ev) {
     if (trace) trace[j * kTraceEvents + ev] = clock64();
   };
+  unsigned long long* const cta_rec =
+      p.trace ? p.trace + (int64_t)p.nsub * kTraceEvents + 3 * (int64_t)blockIdx.x : nullptr;
+  if (cta_rec && threadIdx.x == 0) {
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    cta_rec[0] = globaltimer_ns();
+    cta_rec[2] = smid;
+  }
 
-  if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
+  if (warp == W_MMA) tmem_alloc(tmem_slot, TMEM_COLS);
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int i = 0; i < 2; ++i) {
@@ -221,7 +234,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == W_TMA) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       // L2 prefetch runs kPrefetch sub-chunks ahead of the shared-memory loads,
@@ -259,7 +272,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == W_MMA) {
     // ------------------------------------------------------------ MMA issuer
     // Polls two queues and issues whichever is ready: the products c(jc) of
     // sub-chunk jc (on the state's critical path, checked first) and S(js) of
@@ -344,7 +357,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ dt, lam, decay factors, X'
-    const int a = threadIdx.x - 64;  // 0..63
+    const int a = threadIdx.x;  // 0..63 (warps 0-1)
     const float Ah = chunked ? 0.f : p.A[h];  // A (and dt) are read only by the whole scan
     const float* dtb = p.dt + (int64_t)b * p.sdt + h;
     auto load_dt = [&](int j, float& d0, float& d1) {
@@ -367,9 +380,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         const float nb = __shfl_up_sync(0xffffffffu, v, off);
         if (lane >= off) v += nb;
       }
-      if (lane == 31) wtot[warp - 2] = v;
+      if (lane == 31) wtot[warp] = v;
       named_sync(1, AUX);
-      const float pre = (warp == 3) ? wtot[0] : 0.f;
+      const float pre = (warp == 1) ? wtot[0] : 0.f;
       float lam1 = v + pre;       // token 2a+1
       float lam0 = lam1 - l1;     // token 2a
       if (chunked) {              // step modes: sub-chunk-local sums from step 1's output
@@ -614,11 +627,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == W_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
     tmem_relinquish();
   }
+  if (cta_rec && threadIdx.x == 0) cta_rec[1] = globaltimer_ns();
 }
 
 }  // namespace fused

@@ -186,7 +186,8 @@ extern "C" ssd_status ssd_selftest_fused_trace(const ssd_dims* d, const void* x,
   if (s != SSD_OK) return s;
   Problem p = make_problem(d);
   if (!fused_supported(p)) return SSD_ERR_UNSUPPORTED;
-  if (!trace || trace_len < ceil_div(p.L, 128) * fused::kTraceEvents) return SSD_ERR_INVALID_ARG;
+  const int64_t ctas = p.B * p.H;
+  if (!trace || trace_len < ceil_div(p.L, 128) * fused::kTraceEvents + 3 * ctas) return SSD_ERR_INVALID_ARG;
   p.x = x; p.dt = dt; p.A = A; p.Bm = Bm; p.Cm = Cm; p.D = D; p.y = y;
   return cuda_status(launch_fused_traced(p, init_state, final_state, trace, static_cast<cudaStream_t>(stream)));
 }

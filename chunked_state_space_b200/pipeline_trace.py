@@ -29,12 +29,25 @@ def run(workload: str = "mamba2_2p7b_layer", batch: int | None = None, repeats: 
         return torch.from_numpy(a).cuda()
 
     d = {k: dev(v) for k, v in host.items()}
-    tr = None
+    tr = ctas = None
     for _ in range(repeats):
-        _, _, tr = ssd.ssd_selftest_fused_trace(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init"],
-                                                chunk=wl.chunk)
+        _, _, tr, ctas = ssd.ssd_selftest_fused_trace(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init"],
+                                                      chunk=wl.chunk)
     torch.cuda.synchronize()
-    return tr.cpu().numpy().astype(np.int64)
+    return tr.cpu().numpy().astype(np.int64), ctas.cpu().numpy().astype(np.int64)
+
+
+def cta_summary(ctas: np.ndarray) -> dict:
+    """Spread of CTA durations and how the launch filled the SMs."""
+    t0 = ctas[:, 0].min()
+    dur = (ctas[:, 1] - ctas[:, 0]) / 1e3
+    return {
+        "kernel span us": (ctas[:, 1].max() - t0) / 1e3,
+        "CTA duration us (min/median/max)": (dur.min(), float(np.median(dur)), dur.max()),
+        "CTAs per SM (max)": int(np.bincount(ctas[:, 2]).max()),
+        "SMs used": int(len(np.unique(ctas[:, 2]))),
+        "sum of CTA time / (SMs x span)": float(dur.sum() / (len(np.unique(ctas[:, 2])) * (ctas[:, 1].max() - t0) / 1e3)),
+    }
 
 
 def summarize(t: np.ndarray) -> dict:
@@ -61,9 +74,11 @@ def main():
     ap.add_argument("--workload", default="mamba2_2p7b_layer")
     ap.add_argument("--batch", type=int, default=None)
     args = ap.parse_args()
-    t = run(args.workload, args.batch)
+    t, ctas = run(args.workload, args.batch)
     for k, v in summarize(t).items():
         print(f"{k:40s} {v:8d} clk")
+    for k, v in cta_summary(ctas).items():
+        print(f"{k:40s} {v}")
 
 
 if __name__ == "__main__":

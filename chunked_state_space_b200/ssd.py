@@ -298,16 +298,18 @@ TRACE_EVENTS = ["loads", "S_issued", "c_issued", "mask_start", "mask_done", "lam
 
 def ssd_selftest_fused_trace(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, stream=None):
     """Diagnostic: run the fused kernel with CTA 0 tracing its pipeline events.
-    Returns (y, final_state, trace [nsub, 24] int64 clocks)."""
+    Returns (y, final_state, trace [nsub, 24] int64 clocks, ctas [B*H, 3] int64
+    (start ns, end ns, SM) of every CTA)."""
     dims = make_dims(x, Bm, chunk)
     nsub = -(-dims.seqlen // 128)
     y = torch.empty_like(x)
     fin = torch.empty((dims.batch, dims.nheads, dims.dstate, dims.headdim), dtype=torch.float32, device=x.device)
-    trace = torch.zeros((nsub, 24), dtype=torch.int64, device=x.device)
+    ntr = nsub * 24
+    trace = torch.zeros(ntr + 3 * dims.batch * dims.nheads, dtype=torch.int64, device=x.device)
     _check(lib().ssd_selftest_fused_trace(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D),
                                           _ptr(init_state), _ptr(y), _ptr(fin), _ptr(trace), trace.numel(),
                                           _stream(stream)), "ssd_selftest_fused_trace")
-    return y, fin, trace
+    return y, fin, trace[:ntr].view(nsub, 24), trace[ntr:].view(-1, 3)
 
 
 def ssd_selftest_mask_timing(variant: int, stream=None):

@@ -50,7 +50,10 @@ ssd_status ssd_selftest_umma(int32_t variant, const void* A, const void* B, floa
  * published, 9 epilogue done, 10 products ready to issue, 11 first third of
  * the products issued, 12 S ready to issue, 13-17 points inside the mask
  * (first TMEM read, blocks 0-1 written, second read, blocks 2-3 written,
- * stores complete).  Used to find the critical path.
+ * stores complete).  After those 24*ceil(L/128) values, every CTA c (batch
+ * b, head h: c = b*H + h) writes trace[24*ceil(L/128) + 3c + {0, 1, 2}] =
+ * its start and end (globaltimer, ns) and its SM index; trace_len must cover
+ * them.  Used to find the critical path and the spread of CTA durations.
  */
 ssd_status ssd_selftest_fused_trace(const ssd_dims* d, const void* x, const float* dt, const float* A,
                                     const void* Bm, const void* Cm, const float* D, const float* init_state,

@@ -283,6 +283,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t idS = idesc_bf16(128, 128, false, false);
       const uint32_t idY = idesc_bf16(128, 64, false, true);
       const uint32_t idB = idesc_bf16(128, 64, true, true);
+      // Descriptors of stage 0, computed once: each MMA only advances the start
+      // address (one 64-bit add on the issuing thread's critical path).
+      const uint64_t dC = smem_desc(sbase + OFF_C, 16, 1024);      // K-major (A of S and y_inter)
+      const uint64_t dBk = smem_desc(sbase + OFF_B, 16, 1024);     // K-major (B of S)
+      const uint64_t dBmn = smem_desc(sbase + OFF_B, TILE, 1024);  // MN-major (A of b_intra)
+      const uint64_t dX = smem_desc(sbase + OFF_X, TILE, 1024);    // MN-major (B of y_intra)
+      const uint64_t dXp = smem_desc(sbase + OFF_XP, TILE, 1024);  // MN-major (B of b_intra)
+      const uint64_t dPrev = smem_desc(sbase + OFF_PREV, TILE, 1024);
       int js = 0, jc = 0;
       uint32_t idle = 0;
       uint64_t t_last = globaltimer_ns();
@@ -294,23 +302,19 @@ __global__ void __launch_bounds__(THREADS, 1)
           mark(jc, EV_C_READY);
           tc_fence_after();
           const uint32_t base = tmem + buf * 256;
-          const uint32_t sX = sbase + st * STAGE + OFF_X;
-          const uint32_t sB = sbase + st * STAGE + OFF_B;
-          const uint32_t sXp = sbase + OFF_XP + (jc & 1) * TILE, sPrev = sbase + OFF_PREV;
+          const uint64_t cB = desc_advance(dBmn, st * STAGE), cXp = desc_advance(dXp, (jc & 1) * TILE);
+          const uint64_t cX = desc_advance(dX, st * STAGE), cC = desc_advance(dC, st * STAGE);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)  // b_intra = B^T X'  (the state chain needs it first)
-            mma_ss(base + 192, smem_desc(sB + ks * 2048, TILE, 1024), smem_desc(sXp + ks * 2048, TILE, 1024), idB,
-                   ks > 0);
+            mma_ss(base + 192, desc_advance(cB, ks * 2048), desc_advance(cXp, ks * 2048), idB, ks > 0);
           mark(jc, EV_C_MID);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)  // y_intra = P X
-            mma_ts(base + 128, base + ks * 8, smem_desc(sX + ks * 2048, TILE, 1024), idY, ks > 0);
-          const uint32_t sC = sbase + st * STAGE + OFF_C;
+            mma_ts(base + 128, base + ks * 8, desc_advance(cX, ks * 2048), idY, ks > 0);
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {  // y_inter = C prev  (K = dstate)
-            const uint32_t koff = (ks >> 2) * TILE + (ks & 3) * 32;
-            mma_ss(base + 64, smem_desc(sC + koff, 16, 1024), smem_desc(sPrev + ks * 2048, TILE, 1024), idY, ks > 0);
-          }
+          for (int ks = 0; ks < 8; ++ks)  // y_inter = C prev  (K = dstate)
+            mma_ss(base + 64, desc_advance(cC, (ks >> 2) * TILE + (ks & 3) * 32), desc_advance(dPrev, ks * 2048), idY,
+                   ks > 0);
           mma_commit(&bar[CFULL0 + buf]);
           mma_commit(&bar[EMPTY0 + st]);
           mark(jc, EV_C_ISSUED);
@@ -322,12 +326,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int st = js & 1, buf = js & 1;
           mark(js, EV_S_READY);
           tc_fence_after();
-          const uint32_t sC = sbase + st * STAGE + OFF_C, sB = sbase + st * STAGE + OFF_B;
           const uint32_t tS = tmem + buf * 256;
+          const uint64_t sCd = desc_advance(dC, st * STAGE), sBd = desc_advance(dBk, st * STAGE);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
             const uint32_t koff = (ks >> 2) * TILE + (ks & 3) * 32;
-            mma_ss(tS, smem_desc(sC + koff, 16, 1024), smem_desc(sB + koff, 16, 1024), idS, ks > 0);
+            mma_ss(tS, desc_advance(sCd, koff), desc_advance(sBd, koff), idS, ks > 0);
           }
           mma_commit(&bar[SFULL0 + buf]);
           mark(js, EV_S_ISSUED);

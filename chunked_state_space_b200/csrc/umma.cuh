@@ -14,6 +14,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 namespace ssd {
@@ -205,6 +206,11 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   d |= (uint64_t)(swizzle & 7) << 61;
   return d;
 }
+
+// The descriptor of the same operand `bytes` further on: the start-address
+// field is the low 14 bits of address >> 4, and shared-memory addresses stay
+// below 256 KB, so the add never carries into the LBO field.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D: D format [4,6)=1,
 // A format [7,10)=1, B format [10,13)=1, A major bit 15, B major bit 16

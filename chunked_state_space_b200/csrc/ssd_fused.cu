@@ -75,6 +75,8 @@ struct Params {
   int64_t sy;
   unsigned long long* trace;  // diagnostics: per-sub-chunk event clocks of CTA 0, then
                               // [start ns, end ns, SM] of every CTA; or NULL
+  int withhold_loads;         // self-test of the timeout path: issue no TMA loads, so
+                              // every wait on them runs out (0 in every other launch)
 };
 
 // Trace events (clock64 of CTA 0), one row of kTraceEvents per sub-chunk.
@@ -250,7 +252,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_prefetch_4d(&map_c, 64, g, tp, b);
       };
       for (int jp = 0; jp < kPrefetch; ++jp) prefetch(jp);
-      for (int j = 0; j < nsub; ++j) {
+      const int nload = p.withhold_loads ? 0 : nsub;
+      for (int j = 0; j < nload; ++j) {
         const int st = j & 1;
         prefetch(j + kPrefetch);
         if (j >= 2 && !ctl.wait(EMPTY0 + st, ((j >> 1) + 1) & 1)) break;
@@ -265,7 +268,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         mark(j, EV_LOADS);
       }
       // drain: the last loads of each stage must land before the CTA may exit
-      for (int j = (nsub > 2 ? nsub - 2 : 0); j < nsub; ++j) {
+      for (int j = (nload > 2 ? nload - 2 : 0); j < nload; ++j) {
         uint64_t* fb = &bar[FULL0 + (j & 1)];
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(fb, (j >> 1) & 1) && globaltimer_ns() - t0 < 1000000000ull) {
@@ -650,11 +653,15 @@ bool tc_supported(const Problem& p) { return fused_supported(p) && p.B * p.H * p
 int fused_kernels_per_call(const Problem&) { return 1; }
 
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
-                               void* y, unsigned long long* trace, cudaStream_t st);
+                               void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads = 0);
 
 cudaError_t launch_fused_traced(const Problem& p, const float* init, float* final_state, unsigned long long* trace,
                                 cudaStream_t st) {
   return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, trace, st);
+}
+
+cudaError_t launch_fused_withheld(const Problem& p, const float* init, float* final_state, cudaStream_t st) {
+  return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, nullptr, st, 1);
 }
 
 cudaError_t launch_fused(const Problem& p, const float* init, float* final_state, void*, cudaStream_t st) {
@@ -674,7 +681,7 @@ cudaError_t launch_chunk_scan_tc(const Problem& p, const float* lam, const float
 }
 
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
-                               void* y, unsigned long long* trace, cudaStream_t st) {
+                               void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads) {
   using namespace fused;
   // every pointer the mode reads must be present (the step entry points pass
   // only the tensors of their step)
@@ -713,6 +720,7 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   kp.y = static_cast<__nv_bfloat16*>(y);
   kp.sy = p.sy;
   kp.trace = trace;
+  kp.withhold_loads = withhold_loads;
   cudaError_t e = cudaFuncSetAttribute(k_ssd_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int64_t ctas = mode == fused::MODE_SCAN ? p.B * p.H : p.B * p.H * p.nc;

@@ -192,6 +192,24 @@ extern "C" ssd_status ssd_selftest_fused_trace(const ssd_dims* d, const void* x,
   return cuda_status(launch_fused_traced(p, init_state, final_state, trace, static_cast<cudaStream_t>(stream)));
 }
 
+// Timeout path of the fused kernel: the same launch as ssd_scan_fwd with its
+// TMA loads withheld, so every wait on them runs out (after about a second)
+// and the kernel records SSD_ERR_TIMEOUT in the device status word and
+// returns; nothing faults and the context stays usable.
+extern "C" ssd_status ssd_selftest_timeout(const ssd_dims* d, const void* x, const float* dt, const float* A,
+                                           const void* Bm, const void* Cm, const float* D, const float* init_state,
+                                           void* y, float* final_state, void* stream) {
+  using namespace ssd;
+  ssd_status s = validate_dims(d);
+  if (s != SSD_OK) return s;
+  s = validate_scan_args(d, x, dt, A, Bm, Cm, D, init_state, y, final_state);
+  if (s != SSD_OK) return s;
+  Problem p = make_problem(d);
+  if (!fused_supported(p)) return SSD_ERR_UNSUPPORTED;
+  p.x = x; p.dt = dt; p.A = A; p.Bm = Bm; p.Cm = Cm; p.D = D; p.y = y;
+  return cuda_status(launch_fused_withheld(p, init_state, final_state, static_cast<cudaStream_t>(stream)));
+}
+
 // ---------------------------------------------------------------------------
 // Micro-timing of the mask's building blocks on one CTA (4 warps, one TMEM
 // lane quarter each), away from the rest of the fused kernel: 64 repetitions

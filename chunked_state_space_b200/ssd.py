@@ -26,7 +26,8 @@ EXPORTED = ["ssd_status_string", "ssd_version", "ssd_scan_workspace_size", "ssd_
             "ssd_scan_fwd_unfused", "ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing",
             "ssd_chunk_scan", "ssd_rmsnorm", "ssd_vertical_workspace_size", "ssd_vertical_fwd",
             "ssd_read_device_status", "ssd_selftest_umma", "ssd_scan_path", "ssd_step",
-            "ssd_selftest_fused_trace", "ssd_scan_fwd_noalloc", "ssd_selftest_mask_timing"]
+            "ssd_selftest_fused_trace", "ssd_scan_fwd_noalloc", "ssd_selftest_mask_timing",
+            "ssd_selftest_timeout"]
 
 
 class SSDError(RuntimeError):
@@ -78,6 +79,7 @@ def lib() -> ctypes.CDLL:
         "ssd_scan_fwd_noalloc": (ctypes.c_int, [D] + [_P] * 10),
         "ssd_selftest_mask_timing": (ctypes.c_int, [ctypes.c_int32, _P, _P, _P]),
         "ssd_selftest_fused_trace": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_int64, _P]),
+        "ssd_selftest_timeout": (ctypes.c_int, [D] + [_P] * 10),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -310,6 +312,16 @@ def ssd_selftest_fused_trace(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: i
                                           _ptr(init_state), _ptr(y), _ptr(fin), _ptr(trace), trace.numel(),
                                           _stream(stream)), "ssd_selftest_fused_trace")
     return y, fin, trace[:ntr].view(nsub, 24), trace[ntr:].view(-1, 3)
+
+
+def ssd_selftest_timeout(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, stream=None) -> None:
+    """Diagnostic: launch the fused kernel with its TMA loads withheld, so its
+    bounded waits run out; read the outcome with ssd_read_device_status."""
+    dims = make_dims(x, Bm, chunk)
+    y = torch.empty_like(x)
+    fin = torch.empty((dims.batch, dims.nheads, dims.dstate, dims.headdim), dtype=torch.float32, device=x.device)
+    _check(lib().ssd_selftest_timeout(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D),
+                                      _ptr(init_state), _ptr(y), _ptr(fin), _stream(stream)), "ssd_selftest_timeout")
 
 
 def ssd_selftest_mask_timing(variant: int, stream=None):

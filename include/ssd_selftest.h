@@ -71,6 +71,21 @@ ssd_status ssd_selftest_fused_trace(const ssd_dims* d, const void* x, const floa
  */
 ssd_status ssd_selftest_mask_timing(int32_t variant, long long* cycles, float* sink, void* stream);
 
+/*
+ * ssd_selftest_timeout exercises the bounded waits of ssd_scan_fwd's fused
+ * tensor-core kernel: same arguments and validation as ssd_scan_fwd (the
+ * problem must be one the fused kernel takes, else SSD_ERR_UNSUPPORTED), but
+ * the kernel issues none of its TMA loads, so every wait on them gives up
+ * after about one second.  The launch itself returns SSD_OK; the following
+ * ssd_read_device_status(stream) must return SSD_ERR_TIMEOUT (and clears the
+ * word).  y and final_state are left undefined.  No fault, trap or unbounded
+ * wait is involved: the kernel drains and exits, and later launches in the
+ * same context run normally.
+ */
+ssd_status ssd_selftest_timeout(const ssd_dims* d, const void* x, const float* dt, const float* A, const void* Bm,
+                                const void* Cm, const float* D, const float* init_state, void* y, float* final_state,
+                                void* stream);
+
 #ifdef __cplusplus
 }
 #endif

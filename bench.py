@@ -9,6 +9,12 @@ is needed between steps).  With N > 1 (torchrun) every rank scans its own
 batch (independent sequences; no collective on the data path) and the time
 is the max over ranks.  Rank 0 prints one JSON line.
 
+--workload picks another seeded workload: a layer whose inputs fit in L2 is
+timed with a 512 MB L2 flush between steps (per-step CUDA events exclude the
+flush); the 24-layer stack is timed as one ssd_vertical_fwd over all layers
+(depth-first schedule), with the horizontal schedule and a CUDA-graph replay
+of the vertical one reported beside it.
+
 --impl reference times the fp64 CPU oracle (the only reference there is) on
 a bounded sample of the same workload on the host cores.
 """
@@ -54,6 +60,11 @@ def algorithmic_bytes(wl) -> int:
     io = 2 if wl.io == "bf16" else 4
     return (2 * Bz * L * H * P * io + Bz * L * H * 4 + 2 * Bz * L * G * N * io + 2 * H * 4
             + 2 * Bz * H * N * P * 4)
+
+
+def l2_resident(wl) -> bool:
+    """Inputs and outputs of one scan fit in the 126 MB L2 (flush between steps)."""
+    return algorithmic_bytes(wl) < 256 * 2 ** 20
 
 
 def algorithmic_flops(wl) -> float:
@@ -158,9 +169,23 @@ class ClockSampler:
 def cpu_baseline(wl, target_s: float = 12.0):
     """The fp64 oracle, as it stands, on a bounded sample of the workload: whole
     batches (all heads, full length) one after another until about `target_s`
-    seconds of CPU work, or the whole batch."""
+    seconds of CPU work, or the whole batch.  For a multi-layer stack: one
+    sequence of layer 0 over its full length, tokens/s divided by the layer
+    count (every layer costs the same)."""
     import oracle
     from chunked_state_space_b200 import inputs
+    if wl.n_layers > 1:
+        one = inputs.custom(wl.name, batch=1)
+        host = inputs.generate(one, seed=1000)
+        args = [inputs.to_f64(host[k]) for k in ("x", "dt", "A", "B", "C", "D", "init")]
+        del host
+        t0 = time.perf_counter()
+        oracle.scan_recurrence(*args)
+        el = time.perf_counter() - t0
+        return {"value": wl.seqlen / el / wl.n_layers, "unit": "tokens/s", "cores": oracle.num_threads(),
+                "kind": "oracle",
+                "sample": f"1 of {wl.batch} sequences of layer 0, full length {wl.seqlen}, all {wl.nheads} heads, "
+                          f"scaled by 1/{wl.n_layers} layers (fp64 token recurrence); {el:.1f} s"}
     tokens, el, nb = 0, 0.0, 0
     for b in range(wl.batch):
         one = inputs.custom(wl.name, batch=1)
@@ -245,6 +270,8 @@ def main():
     wl = inputs.WORKLOADS[args.workload]
     if args.batch:
         wl = inputs.custom(wl.name, batch=args.batch)
+    if wl.n_layers > 1:
+        return run_stack(args, wl, dev, rank, world)
     host = inputs.generate(wl, seed=rank_seed(rank))  # each rank: its own independent batch
     pinned = {}
     for k, v in host.items():
@@ -264,31 +291,8 @@ def main():
                          final_state=fin, workspace=ws, stream=stream)
 
     path, kernels_per_step = ssd.ssd_scan_path(dims)
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-
-    clocks = ClockSampler(local)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    clocks.start()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    clk = clocks.stop()
-    if world > 1:
-        dist.barrier()
-    ms_total = t_start.elapsed_time(t_end)
-    per_step = [a.elapsed_time(b) for a, b in ev]
-    ms_total = max_over_ranks(ms_total, dev)
+    flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev) if l2_resident(wl) else None
+    per_step, ms_total, clk = timed_steps(step, args, stream, dev, local, world, flush)
     ms_per_step = ms_total / args.steps
     tokens = wl.batch * wl.seqlen * world
     value = tokens / (ms_per_step * 1e-3)
@@ -336,10 +340,189 @@ def main():
         "config": {"workload": wl.name, "batch": wl.batch, "seqlen": wl.seqlen, "nheads": wl.nheads,
                    "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk,
                    "state_dtype": "f32", "path": path, "parallelism": f"dp{world} (independent batches per rank)",
-                   "l2": "inputs larger than L2 (x is 1.34 GB per rank); no flush"},
+                   "l2": ("512 MB L2 flush between steps (inputs fit in L2); per-step events exclude it"
+                          if flush is not None else
+                          f"inputs larger than L2 ({algorithmic_bytes(wl) / 1e9:.2f} GB per rank); no flush")},
         "clocks": clk, "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                                "d2h_bytes_per_step": d2h},
         "gpu_launches": kernels_per_step * args.steps, "roofline": roofline,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def timed_steps(step, args, stream, dev, local, world, flush=None):
+    """Warm-up, then exactly args.steps steps bracketed by barrier + synchronize,
+    CUDA events on the launching stream around every step; NVML clocks sampled
+    meanwhile.  With `flush` (a buffer larger than L2) it is rewritten before
+    every step and the time is the sum of the per-step events (flush excluded);
+    else the time between the first and last event.  Max over ranks."""
+    import torch
+    import torch.distributed as dist
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    per_step = [a.elapsed_time(b) for a, b in ev]
+    ms_total = sum(per_step) if flush is not None else t_start.elapsed_time(t_end)
+    return per_step, max_over_ranks(ms_total, dev), clk
+
+
+def run_stack(args, wl, dev, rank, world):
+    """The 24-layer stack: one step = ssd_vertical_fwd over all layers and the
+    whole sequence (V-token blocks, per-layer carried states, RMS norm between
+    layers).  Reported beside it: the horizontal schedule (layer by layer) and
+    a CUDA-graph replay of the vertical schedule."""
+    import torch
+    import torch.distributed as dist
+    from chunked_state_space_b200 import inputs, ssd
+    local = dev.index
+    stream = torch.cuda.current_stream(dev)
+    seed = rank_seed(rank)
+    eps = 1e-6
+    names = ("dt", "A", "B", "C", "D")
+    host_layers = [inputs.generate(wl, seed=seed, layer=l, names=names) for l in range(wl.n_layers)]
+    x0h = inputs.generate(wl, seed=seed, names=("x",))["x"]
+
+    def pin(v):
+        t = torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16 else torch.from_numpy(v)
+        return t.pin_memory()
+
+    p_layers = [{k: pin(v) for k, v in h.items()} for h in host_layers]
+    p_x0 = pin(x0h)
+    del host_layers, x0h
+    layers = [{k: v.to(dev, non_blocking=True) for k, v in p.items()} for p in p_layers]
+    x0 = p_x0.to(dev, non_blocking=True)
+    states = [torch.zeros((wl.batch, wl.nheads, wl.dstate, wl.headdim), dtype=torch.float32, device=dev)
+              for _ in range(wl.n_layers)]
+    y = torch.empty_like(x0)
+    dims = ssd.make_dims(x0, layers[0]["B"], wl.chunk)
+    ws = torch.empty(ssd.ssd_vertical_workspace_size(dims, wl.n_layers, wl.vblock), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize(dev)
+
+    def vertical():
+        ssd.ssd_vertical_fwd(x0, layers, states, vblock=wl.vblock, chunk=wl.chunk, rms_eps=eps, y_out=y,
+                             workspace=ws, stream=stream)
+
+    per_step, ms_total, clk = timed_steps(vertical, args, stream, dev, local, world)
+    ms_per_step = ms_total / args.steps
+    tokens = wl.batch * wl.seqlen * world
+    value = tokens / (ms_per_step * 1e-3)
+    nblk = -(-wl.seqlen // wl.vblock)
+    launches = nblk * (2 * wl.n_layers - 1)
+
+    # horizontal schedule: layer by layer over the whole sequence
+    xh = torch.empty_like(x0)
+
+    def horizontal():
+        x = x0
+        for l, p in enumerate(layers):
+            ssd.ssd_scan_fwd(x, p["dt"], p["A"], p["B"], p["C"], p["D"], states[l], chunk=wl.chunk, y=y,
+                             final_state=states[l], stream=stream)
+            if l + 1 < wl.n_layers:
+                ssd.ssd_rmsnorm(y, eps, out=xh, stream=stream)
+                x = xh
+
+    hs = argparse.Namespace(steps=max(2, args.steps // 2), warmup=args.warmup)
+    _, h_total, _ = timed_steps(horizontal, hs, stream, dev, local, world)
+    h_ms = h_total / hs.steps
+
+    # the vertical schedule captured once in a CUDA graph and replayed
+    graph_ms = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            ssd.ssd_vertical_fwd(x0, layers, states, vblock=wl.vblock, chunk=wl.chunk, rms_eps=eps, y_out=y,
+                                 workspace=ws, stream=side)
+        stream.wait_stream(side)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.graph(g, stream=side):
+            ssd.ssd_vertical_fwd(x0, layers, states, vblock=wl.vblock, chunk=wl.chunk, rms_eps=eps, y_out=y,
+                                 workspace=ws, stream=side)
+        torch.cuda.synchronize(dev)
+        _, g_total, _ = timed_steps(g.replay, hs, stream, dev, local, world)
+        graph_ms = g_total / hs.steps
+        del g
+    except Exception as e:  # reported, not hidden: the eager figure stands
+        graph_ms = f"capture failed: {type(e).__name__}: {e}"[:200]
+
+    # end to end through the public API from pinned host buffers
+    h_y = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    h_states = [torch.empty(s.shape, dtype=s.dtype, pin_memory=True) for s in states]
+    h2d = p_x0.numel() * p_x0.element_size() + sum(v.numel() * v.element_size() for p in p_layers
+                                                    for v in p.values())
+    d2h = y.numel() * y.element_size() + sum(s.numel() * s.element_size() for s in states)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(max(args.e2e_steps, 1)):
+        x0.copy_(p_x0, non_blocking=True)
+        for p, dl in zip(p_layers, layers):
+            for k, v in p.items():
+                dl[k].copy_(v, non_blocking=True)
+        for s in states:
+            s.zero_()
+        vertical()
+        h_y.copy_(y, non_blocking=True)
+        for hs_, s in zip(h_states, states):
+            hs_.copy_(s, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / max(args.e2e_steps, 1), dev)
+
+    hbm_peak, tc_peak, tc_sust, peak_src = load_peaks()
+    layer_wl = inputs.custom(wl.name, n_layers=1)
+    alg = algorithmic_bytes(layer_wl) * wl.n_layers
+    ach = alg / (ms_per_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "seqlen": wl.seqlen, "nheads": wl.nheads,
+                   "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk,
+                   "n_layers": wl.n_layers, "vblock": wl.vblock, "schedule": "vertical (ssd_vertical_fwd)",
+                   "horizontal_ms_per_step": h_ms, "vertical_graph_ms_per_step": graph_ms,
+                   "parallelism": f"dp{world} (independent batches per rank)",
+                   "l2": f"inputs larger than L2 ({alg / 1e9:.2f} GB per step); no flush"},
+        "clocks": clk, "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                               "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches * args.steps,
+        "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
+                     "traffic": None, "kernel": "whole step (k_ssd_fused per block and layer, k_rmsnorm between)",
+                     "algorithmic_bytes": f"{wl.n_layers} x one layer's scan bytes; the RMS norm traffic between "
+                                          "layers is not counted",
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else
+                     "fallback 6650 GB/s"},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
@@ -382,8 +565,9 @@ def _unfused_roofline(wl, d, dims, stream, hbm_peak, peak_src):
     Bz, L, H, P, N, G = wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.dstate, wl.ngroups
     st_bytes = Bz * H * nc * N * P * 4
     lam_bytes = Bz * H * nc * wl.chunk * 4
-    xb = Bz * L * H * P * 2
-    bcb = Bz * L * G * N * 2
+    io = 2 if wl.io == "bf16" else 4
+    xb = Bz * L * H * P * io
+    bcb = Bz * L * G * N * io
     alg = {"chunk_cumsum": Bz * L * H * 4 + lam_bytes, "chunk_state": xb + bcb + lam_bytes + st_bytes,
            "state_passing": 2 * st_bytes + lam_bytes // wl.chunk + 2 * Bz * H * N * P * 4,
            "chunk_scan": 2 * xb + 2 * bcb + lam_bytes + st_bytes}

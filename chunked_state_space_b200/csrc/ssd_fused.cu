@@ -23,6 +23,8 @@
 // TMEM holds two 256-column buffers [S -> P | y_inter][y_intra][b_intra] so sub-chunk
 // j+1's S and mask overlap sub-chunk j's products and epilogue.  Every wait is bounded; a timeout
 // raises g_device_status and the roles drain without further waits.
+#include <atomic>
+
 #include "ssd_tc.cuh"
 #include "tma.cuh"
 #include "umma.cuh"
@@ -721,8 +723,18 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   kp.sy = p.sy;
   kp.trace = trace;
   kp.withhold_loads = withhold_loads;
-  cudaError_t e = cudaFuncSetAttribute(k_ssd_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  // the shared-memory opt-in once per device (not stream work; keeps launches
+  // free of other API calls, e.g. inside a CUDA graph capture)
+  static std::atomic<unsigned long long> attr_set{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_set.load() & bit)) {
+    e = cudaFuncSetAttribute(k_ssd_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set.fetch_or(bit);
+  }
   const int64_t ctas = mode == fused::MODE_SCAN ? p.B * p.H : p.B * p.H * p.nc;
   k_ssd_fused<<<(unsigned)ctas, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc);
   return cudaGetLastError();

@@ -3,6 +3,9 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
+#include <vector>
+
 #include "ssd_common.cuh"
 #include "ssd_tc.cuh"
 
@@ -281,8 +284,150 @@ ssd_status ssd_vertical_workspace_size(const ssd_dims* d, int32_t n_layers, int6
   s = ssd_scan_workspace_size(&dv, &one);
   if (s != SSD_OK) return s;
   const size_t act = align_up(io_size(d->io_dtype) * (size_t)d->batch * dv.seqlen * d->nheads * d->headdim);
-  *bytes = align_up(one) + 2 * act;
+  // the wavefront schedule keeps two activation blocks per layer boundary
+  const size_t nact = n_layers > 2 ? 2 * (size_t)(n_layers - 1) : 2;
+  *bytes = align_up(one) + nact * act;
   return SSD_OK;
+}
+
+namespace {
+
+// Streams and events of the wavefront schedule, one set per device, created on
+// first use and kept for the life of the process.  `mu` is held while a call
+// enqueues its work, so calls from several host threads never interleave
+// their event records.
+struct WavefrontPool {
+  std::mutex mu;
+  std::vector<cudaStream_t> streams;  // one per layer
+  std::vector<cudaEvent_t> out;       // [layer]: block's output of that layer is normalised and ready
+  std::vector<cudaEvent_t> freed;     // [layer][2]: the layer finished reading its input buffer of that parity
+  cudaEvent_t fork = nullptr;
+
+  cudaError_t grow(int n) {
+    if (!fork) {
+      cudaError_t e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming);
+      if (e != cudaSuccess) return e;
+    }
+    while ((int)streams.size() < n) {
+      cudaStream_t s;
+      cudaEvent_t a, b, c;
+      cudaError_t e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&a, cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&b, cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c, cudaEventDisableTiming);
+      if (e != cudaSuccess) return e;
+      streams.push_back(s);
+      out.push_back(a);
+      freed.push_back(b);
+      freed.push_back(c);
+    }
+    return cudaSuccess;
+  }
+};
+
+WavefrontPool* wavefront_pool(int device) {
+  static std::mutex mu;
+  static std::vector<WavefrontPool*> pools;
+  std::lock_guard<std::mutex> lock(mu);
+  if (device < 0) return nullptr;
+  if ((int)pools.size() <= device) pools.resize(device + 1, nullptr);
+  if (!pools[device]) pools[device] = new WavefrontPool();
+  return pools[device];
+}
+
+}  // namespace
+
+// Wavefront form of the depth-first schedule (fused kernel only: it needs no
+// scratch, so launches of different layers may run at the same time).  Layer
+// l runs on its own stream, blocks in order, so its state passes from block k
+// to block k+1 by stream order.  Block k of layer l waits for block k of layer
+// l-1 (its input, normalised) and, before it overwrites the input buffer of
+// layer l+1 of parity k % 2, for layer l+1 to have finished block k-2 (the
+// last reader of that buffer).  Every (block, layer) runs the same kernel on
+// the same data as the one-block-at-a-time order, so results are identical.
+static ssd_status vertical_wavefront(const ssd_dims* d, int32_t n_layers, int64_t V, float rms_eps, const void* x0,
+                                     const float* const* dt, const float* const* A, const void* const* Bm,
+                                     const void* const* Cm, const float* const* D, float* const* states, void* y_out,
+                                     void* workspace, cudaStream_t st) {
+  int device = 0;
+  cudaError_t e = cudaGetDevice(&device);
+  if (e != cudaSuccess) return cuda_status(e);
+  WavefrontPool* pool = wavefront_pool(device);
+  std::lock_guard<std::mutex> lock(pool->mu);
+  e = pool->grow(n_layers);
+  if (e != cudaSuccess) return cuda_status(e);
+
+  const Problem full = make_problem(d);
+  ssd_dims dv = *d;
+  dv.seqlen = V;
+  size_t one = 0;
+  ssd_scan_workspace_size(&dv, &one);
+  const size_t es = io_size(d->io_dtype);
+  const size_t act = align_up(es * (size_t)d->batch * V * d->nheads * d->headdim);
+  char* ring = static_cast<char*>(workspace) + align_up(one);
+  // input buffer of layer l (1 <= l < n_layers) for blocks of parity q
+  auto in_buf = [&](int l, int64_t q) { return ring + ((size_t)(l - 1) * 2 + (size_t)q) * act; };
+  const int64_t HP = full.H * full.P;
+
+  // fork: every layer stream starts after the work already on `st`
+  e = cudaEventRecord(pool->fork, st);
+  for (int l = 0; l < n_layers && e == cudaSuccess; ++l) e = cudaStreamWaitEvent(pool->streams[l], pool->fork, 0);
+  if (e != cudaSuccess) return cuda_status(e);
+
+  ssd_status s = SSD_OK;
+  int64_t k = 0;
+  for (int64_t k0 = 0; k0 < full.L && s == SSD_OK; k0 += V, ++k) {
+    const int64_t Vk = (full.L - k0) < V ? (full.L - k0) : V;
+    ssd_dims dk = *d;
+    dk.seqlen = Vk;
+    for (int l = 0; l < n_layers; ++l) {
+      cudaStream_t sl = pool->streams[l];
+      const bool last = (l == n_layers - 1);
+      Problem p = make_problem(&dk);
+      if (l == 0) {
+        p.x = static_cast<const char*>(x0) + es * k0 * HP;
+        p.sx = full.L * HP;
+      } else {
+        p.x = in_buf(l, k & 1);
+        p.sx = Vk * HP;
+        e = cudaStreamWaitEvent(sl, pool->out[l - 1], 0);  // input of this block is ready
+      }
+      if (e == cudaSuccess && !last && k >= 2)  // layer l+1 is done with block k-2's buffer
+        e = cudaStreamWaitEvent(sl, pool->freed[2 * (l + 1) + (k & 1)], 0);
+      if (e != cudaSuccess) return cuda_status(e);
+      p.dt = dt[l] + k0 * full.H;
+      p.sdt = full.L * full.H;
+      p.A = A[l];
+      p.Bm = static_cast<const char*>(Bm[l]) + es * k0 * full.G * full.N;
+      p.Cm = static_cast<const char*>(Cm[l]) + es * k0 * full.G * full.N;
+      p.sbc = full.L * full.G * full.N;
+      p.D = D ? D[l] : nullptr;
+      if (last) {
+        p.y = static_cast<char*>(y_out) + es * k0 * HP;
+        p.sy = full.L * HP;
+      } else {
+        p.y = in_buf(l + 1, k & 1);
+        p.sy = Vk * HP;
+      }
+      s = cuda_status(launch_fused(p, states[l], states[l], nullptr, sl));
+      if (s == SSD_OK && !last) s = cuda_status(launch_rmsnorm(d->batch * Vk, HP, d->io_dtype, p.y, rms_eps, p.y, sl));
+      if (s != SSD_OK) break;
+      e = cudaEventRecord(pool->out[l], sl);
+      if (e == cudaSuccess && l > 0) e = cudaEventRecord(pool->freed[2 * l + (k & 1)], sl);
+      if (e != cudaSuccess) {
+        s = cuda_status(e);
+        break;
+      }
+    }
+  }
+  // join: `st` continues after every layer stream (also after a failed launch,
+  // so that no stream is left forked from a capture)
+  for (int l = 0; l < n_layers; ++l) {
+    cudaError_t ej = cudaEventRecord(pool->out[l], pool->streams[l]);
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(st, pool->out[l], 0);
+    if (ej != cudaSuccess && s == SSD_OK) s = cuda_status(ej);
+  }
+  return s;
 }
 
 ssd_status ssd_vertical_fwd(const ssd_dims* d, int32_t n_layers, int64_t vblock, float rms_eps, const void* x0,
@@ -308,6 +453,8 @@ ssd_status ssd_vertical_fwd(const ssd_dims* d, int32_t n_layers, int64_t vblock,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Problem full = make_problem(d);
   const int64_t V = vblock < d->seqlen ? vblock : d->seqlen;
+  if (n_layers > 1 && fused_supported(full))
+    return vertical_wavefront(d, n_layers, V, rms_eps, x0, dt, A, Bm, Cm, D, states, y_out, workspace, st);
   ssd_dims dv = *d;
   dv.seqlen = V;
   size_t one = 0;

@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_prefetch_4d(&map_c, 64, g, tp, b);
       };
       for (int jp = 0; jp < kPrefetch; ++jp) prefetch(jp);
-      const int nload = p.withhold_loads ? 0 : nsub;
+      const int nload = nsub & (p.withhold_loads - 1);  // 0 or nsub (withhold_loads is 0 or 1)
       for (int j = 0; j < nload; ++j) {
         const int st = j & 1;
         prefetch(j + kPrefetch);

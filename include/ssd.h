@@ -199,7 +199,9 @@ ssd_status ssd_rmsnorm(int64_t rows, int64_t features, int32_t io_dtype, const v
 
 /*
  * Bytes of workspace ssd_vertical_fwd needs for `d`, `n_layers` and the
- * vertical block length `vblock` (V).
+ * vertical block length `vblock` (V): the single-block scan scratch plus two
+ * V-token activation blocks per layer boundary ([B,V,H,P] io each; at least
+ * two).
  */
 ssd_status ssd_vertical_workspace_size(const ssd_dims* d, int32_t n_layers, int64_t vblock,
                                        size_t* bytes);
@@ -217,6 +219,16 @@ ssd_status ssd_vertical_workspace_size(const ssd_dims* d, int32_t n_layers, int6
  * Layer l+1's input is ssd_rmsnorm(y_l) (eps = rms_eps), stored in io dtype.
  * When V is a multiple of Q the result is bitwise equal to running the layers
  * one after another over the whole sequence (the §3.1 horizontal schedule).
+ * Execution: with more than one layer and a problem the fused tensor-core
+ * kernel takes, the (block, layer) launches run as a wavefront: layer l on a
+ * stream of its own, block k of layer l after block k of layer l-1, so
+ * different layers' blocks overlap on the GPU.  Those streams and their
+ * events belong to the library (one set per device, created on first use,
+ * kept until the process exits); every call forks them from `stream` and
+ * joins them back into it, so the call stays asynchronous, orders like a
+ * single-stream call, and can be captured into a CUDA graph.  Calls from
+ * several host threads on one device are serialised while they enqueue.
+ * Otherwise the blocks and layers run one after another on `stream`.
  */
 ssd_status ssd_vertical_fwd(const ssd_dims* d, int32_t n_layers, int64_t vblock, float rms_eps,
                             const void* x0, const float* const* dt, const float* const* A,

@@ -432,6 +432,12 @@ def run_stack(args, wl, dev, rank, world):
 
     per_step, ms_total, clk = timed_steps(vertical, args, stream, dev, local, world)
     ms_per_step = ms_total / args.steps
+    # host time to enqueue one vertical step (the launches and event operations)
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    vertical()
+    host_ms = (time.perf_counter() - t0) * 1e3
+    torch.cuda.synchronize(dev)
     tokens = wl.batch * wl.seqlen * world
     value = tokens / (ms_per_step * 1e-3)
     nblk = -(-wl.seqlen // wl.vblock)
@@ -512,6 +518,7 @@ def run_stack(args, wl, dev, rank, world):
                    "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk,
                    "n_layers": wl.n_layers, "vblock": wl.vblock, "schedule": "vertical (ssd_vertical_fwd)",
                    "horizontal_ms_per_step": h_ms, "vertical_graph_ms_per_step": graph_ms,
+                   "vertical_host_enqueue_ms": host_ms,
                    "parallelism": f"dp{world} (independent batches per rank)",
                    "l2": f"inputs larger than L2 ({alg / 1e9:.2f} GB per step); no flush"},
         "clocks": clk, "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,

@@ -345,7 +345,7 @@ WavefrontPool* wavefront_pool(int device) {
 // layer l+1 of parity k % 2, for layer l+1 to have finished block k-2 (the
 // last reader of that buffer).  Every (block, layer) runs the same kernel on
 // the same data as the one-block-at-a-time order, so results are identical.
-static ssd_status vertical_wavefront(const ssd_dims* d, int32_t n_layers, int64_t V, float rms_eps, const void* x0,
+static ssd_status vertical_wavefront(const ssd_dims* d_, int32_t n_layers, int64_t V, float rms_eps, const void* x0,
                                      const float* const* dt, const float* const* A, const void* const* Bm,
                                      const void* const* Cm, const float* const* D, float* const* states, void* y_out,
                                      void* workspace, cudaStream_t st) {
@@ -357,13 +357,13 @@ static ssd_status vertical_wavefront(const ssd_dims* d, int32_t n_layers, int64_
   e = pool->grow(n_layers);
   if (e != cudaSuccess) return cuda_status(e);
 
-  const Problem full = make_problem(d);
-  ssd_dims dv = *d;
+  const Problem full = make_problem(d_);
+  ssd_dims dv = *d_;
   dv.seqlen = V;
   size_t one = 0;
   ssd_scan_workspace_size(&dv, &one);
-  const size_t es = io_size(d->io_dtype);
-  const size_t act = align_up(es * (size_t)d->batch * V * d->nheads * d->headdim);
+  const size_t es = io_size(d_->io_dtype);
+  const size_t act = align_up(es * (size_t)d_->batch * V * d_->nheads * d_->headdim);
   char* ring = static_cast<char*>(workspace) + align_up(one);
   // input buffer of layer l (1 <= l < n_layers) for blocks of parity q
   auto in_buf = [&](int l, int64_t q) { return ring + ((size_t)(l - 1) * 2 + (size_t)q) * act; };
@@ -374,13 +374,23 @@ static ssd_status vertical_wavefront(const ssd_dims* d, int32_t n_layers, int64_
   for (int l = 0; l < n_layers && e == cudaSuccess; ++l) e = cudaStreamWaitEvent(pool->streams[l], pool->fork, 0);
   if (e != cudaSuccess) return cuda_status(e);
 
+  // Enqueued by anti-diagonals d = k + l (the order the wavefront runs in), so
+  // that the hardware queues the layer streams share never hold a wait in
+  // front of work that is already runnable; inside a diagonal the layers go
+  // downwards, so each wait binds to the record it means: block k of layer l
+  // waits for block k of layer l-1, which block k+1 of layer l-1 (same
+  // diagonal) re-records only afterwards.
   ssd_status s = SSD_OK;
-  int64_t k = 0;
-  for (int64_t k0 = 0; k0 < full.L && s == SSD_OK; k0 += V, ++k) {
-    const int64_t Vk = (full.L - k0) < V ? (full.L - k0) : V;
-    ssd_dims dk = *d;
-    dk.seqlen = Vk;
-    for (int l = 0; l < n_layers; ++l) {
+  const int64_t nblk = (full.L + V - 1) / V;
+  for (int64_t d = 0; d < nblk + n_layers - 1 && s == SSD_OK; ++d) {
+    const int l_hi = (int)(d < n_layers - 1 ? d : n_layers - 1);
+    const int l_lo = (int)(d - (nblk - 1) > 0 ? d - (nblk - 1) : 0);
+    for (int l = l_hi; l >= l_lo; --l) {
+      const int64_t k = d - l;
+      const int64_t k0 = k * V;
+      const int64_t Vk = (full.L - k0) < V ? (full.L - k0) : V;
+      ssd_dims dk = *d_;
+      dk.seqlen = Vk;
       cudaStream_t sl = pool->streams[l];
       const bool last = (l == n_layers - 1);
       Problem p = make_problem(&dk);
@@ -394,7 +404,10 @@ static ssd_status vertical_wavefront(const ssd_dims* d, int32_t n_layers, int64_
       }
       if (e == cudaSuccess && !last && k >= 2)  // layer l+1 is done with block k-2's buffer
         e = cudaStreamWaitEvent(sl, pool->freed[2 * (l + 1) + (k & 1)], 0);
-      if (e != cudaSuccess) return cuda_status(e);
+      if (e != cudaSuccess) {
+        s = cuda_status(e);
+        break;
+      }
       p.dt = dt[l] + k0 * full.H;
       p.sdt = full.L * full.H;
       p.A = A[l];
@@ -410,7 +423,8 @@ static ssd_status vertical_wavefront(const ssd_dims* d, int32_t n_layers, int64_
         p.sy = Vk * HP;
       }
       s = cuda_status(launch_fused(p, states[l], states[l], nullptr, sl));
-      if (s == SSD_OK && !last) s = cuda_status(launch_rmsnorm(d->batch * Vk, HP, d->io_dtype, p.y, rms_eps, p.y, sl));
+      if (s == SSD_OK && !last)
+        s = cuda_status(launch_rmsnorm(d_->batch * Vk, HP, d_->io_dtype, p.y, rms_eps, p.y, sl));
       if (s != SSD_OK) break;
       e = cudaEventRecord(pool->out[l], sl);
       if (e == cudaSuccess && l > 0) e = cudaEventRecord(pool->freed[2 * l + (k & 1)], sl);

@@ -699,8 +699,8 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   const uint64_t sx[3] = {(uint64_t)P * 2, (uint64_t)p.H * P * 2, (uint64_t)p.sx * 2};
   const uint64_t dbc[4] = {(uint64_t)NS, (uint64_t)p.G, (uint64_t)p.L, (uint64_t)p.B};
   const uint64_t sbc[3] = {(uint64_t)NS * 2, (uint64_t)p.G * NS * 2, (uint64_t)p.sbc * 2};
-  if (!tma::encode_bf16(&mx, p.x, 4, dx, sx, box) || !tma::encode_bf16(&mb, p.Bm, 4, dbc, sbc, box) ||
-      !tma::encode_bf16(&mc, cptr, 4, dbc, sbc, box))
+  if (!tma::encode_bf16_4d_cached(&mx, p.x, dx, sx, box) || !tma::encode_bf16_4d_cached(&mb, p.Bm, dbc, sbc, box) ||
+      !tma::encode_bf16_4d_cached(&mc, cptr, dbc, sbc, box))
     return cudaErrorInvalidValue;
   Params kp;
   kp.mode = mode;

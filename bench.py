@@ -248,6 +248,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--batch", type=int, default=None, help="override the batch size (profiling runs)")
+    ap.add_argument("--vblock", type=int, default=None, help="override the vertical block V (layer stacks)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="layer stacks: skip the horizontal and graph-replay figures (sweeps)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -270,6 +273,8 @@ def main():
     wl = inputs.WORKLOADS[args.workload]
     if args.batch:
         wl = inputs.custom(wl.name, batch=args.batch)
+    if args.vblock:
+        wl = inputs.custom(wl.name, batch=wl.batch, vblock=args.vblock)
     if wl.n_layers > 1:
         return run_stack(args, wl, dev, rank, world)
     host = inputs.generate(wl, seed=rank_seed(rank))  # each rank: its own independent batch
@@ -456,12 +461,15 @@ def run_stack(args, wl, dev, rank, world):
                 x = xh
 
     hs = argparse.Namespace(steps=max(2, args.steps // 2), warmup=args.warmup)
-    _, h_total, _ = timed_steps(horizontal, hs, stream, dev, local, world)
-    h_ms = h_total / hs.steps
+    h_ms = graph_ms = None
+    if not args.no_extras:
+        _, h_total, _ = timed_steps(horizontal, hs, stream, dev, local, world)
+        h_ms = h_total / hs.steps
 
     # the vertical schedule captured once in a CUDA graph and replayed
-    graph_ms = None
     try:
+        if args.no_extras:
+            raise StopIteration
         g = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream(dev)
         side.wait_stream(stream)
@@ -477,6 +485,8 @@ def run_stack(args, wl, dev, rank, world):
         _, g_total, _ = timed_steps(g.replay, hs, stream, dev, local, world)
         graph_ms = g_total / hs.steps
         del g
+    except StopIteration:
+        pass
     except Exception as e:  # reported, not hidden: the eager figure stands
         graph_ms = f"capture failed: {type(e).__name__}: {e}"[:200]
 

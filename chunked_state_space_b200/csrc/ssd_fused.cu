@@ -47,7 +47,7 @@ constexpr uint32_t OFF_LAM = OFF_PREV + TILE;  // float [4][128]
 constexpr uint32_t OFF_ECOL = OFF_LAM + 4 * T * 4;  // float [4][128]
 constexpr uint32_t OFF_WTOT = OFF_ECOL + 4 * T * 4;
 constexpr uint32_t OFF_BAR = OFF_WTOT + 64;
-constexpr uint32_t NBAR = 18;
+constexpr uint32_t NBAR = 20;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
@@ -90,7 +90,8 @@ enum {
 
 // barrier indices
 enum {
-  FULL0 = 0, EMPTY0 = 2, SFULL0 = 4, PFULL0 = 6, CFULL0 = 8, TEMPTY0 = 10, STATEFULL = 12, DRAIN = 13, LAMRDY0 = 14
+  FULL0 = 0, EMPTY0 = 2, SFULL0 = 4, PFULL0 = 6, CFULL0 = 8, TEMPTY0 = 10, STATEFULL = 12, DRAIN = 13, LAMRDY0 = 14,
+  YFREE0 = 18  // [X' buffer]: the y tile staged there has been read by its TMA store
 };
 constexpr int AUX = 64;  // threads of warps 0-1
 // Warp w runs on SM sub-partition w % 4 and may only touch TMEM lane quarter
@@ -174,7 +175,7 @@ __device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
 
 __global__ void __launch_bounds__(THREADS, 1)
     k_ssd_fused(Params p, const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
-                const __grid_constant__ CUtensorMap map_c) {
+                const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_y) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the __shared__ array by an offset so
   // the compiler keeps the shared address space (LDS/STS, not generic access)
@@ -224,6 +225,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&bar[PFULL0 + i], T + AUX);
       mbar_init(&bar[CFULL0 + i], 1);
       mbar_init(&bar[TEMPTY0 + i], T);
+      mbar_init(&bar[YFREE0 + i], 1);
     }
     mbar_init(&bar[STATEFULL], T);
     mbar_init(&bar[DRAIN], 1);
@@ -415,9 +417,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       d0 = n0;
       d1 = n1;
       // X'_j = diag(exp(lam_end - lam_t)) X_j, rows a and a + 64, into buffer j & 1
-      // (free once the products of sub-chunk j - 2 have completed)
+      // (free once the products of sub-chunk j - 2 have completed and its y tile,
+      // staged in the same buffer, has been read by the TMA store)
       bool ok = ctl.wait(FULL0 + st, (j >> 1) & 1);
       if (ok && j >= 2) ok = ctl.wait(CFULL0 + st, ((j - 2) >> 1) & 1);
+      if (ok && j >= 2) ok = ctl.wait(YFREE0 + st, ((j - 2) >> 1) & 1);  // y(j-2) staged here is stored
       if (ok) {
         const float lam_end = lj[T - 1];  // log2 units
         const uint4* src = reinterpret_cast<const uint4*>(sm + st * STAGE + OFF_X);
@@ -595,11 +599,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (ok) publish_state();
       if (r == 0) mark(j, EV_STATE_PUB);
-      // y_t = y_intra + exp(lam_t) y_inter + D x_t
+      // y_t = y_intra + exp(lam_t) y_inter + D x_t, staged as a 128-B-swizzled tile
+      // in the X' buffer of this sub-chunk (free: its products have completed) and
+      // written by one TMA store, coalesced, rows past L clipped by the copy.  Per-
+      // row global stores (32 rows 10 KB apart per warp instruction) held up the
+      // masking warps' shared-memory loads in the same memory pipe.
       const float et = ex2(lj[r]);
-      const int64_t tg = (int64_t)t_base + (int64_t)j * T + r;
-      uint4* dst = reinterpret_cast<uint4*>(p.y + (int64_t)b * p.sy + (tg * p.H + h) * P);
-      const bool row_in = p.y != nullptr && tg < p.L;
+      const uint32_t ystage = sbase + OFF_XP + buf * TILE;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t yi[16], ye[16];
@@ -620,13 +626,24 @@ __global__ void __launch_bounds__(THREADS, 1)
             yo = fma2(make_float2(et, et), make_float2(__uint_as_float(ye[k0]), __uint_as_float(ye[k0 + 1])), yo);
             o[i] = pack_bf16(yo.x, yo.y);
           }
-          if (row_in) dst[cc] = ov;
+          sts128(ystage + swz128(r, 8 * cc), ov);
         }
       }
       tc_fence_before();
       mbar_arrive(&bar[TEMPTY0 + buf]);
+      fence_async_smem();
+      named_sync(2, T);  // the 128 rows are staged
+      if (r == 0) {
+        if (p.y) {
+          tma_store_4d(&map_y, sm + OFF_XP + buf * TILE, 0, h, t_base + j * T, b);
+          tma_store_commit();
+          tma_store_wait_read0();
+        }
+        mbar_arrive(&bar[YFREE0 + buf]);
+      }
       if (r == 0) mark(j, EV_EPI_DONE);
     }
+    if (r == 0) tma_store_wait0();  // the y tiles are in global memory before the CTA exits
     if (final_ptr) {
       float4* dst = reinterpret_cast<float4*>(final_ptr + (int64_t)r * P);
 #pragma unroll
@@ -693,7 +710,7 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   if (mode == MODE_CHUNK_SCAN && (!lam || !init || !p.Cm || !y)) return cudaErrorInvalidValue;
   // the chunk-state mode never uses C: its C tiles are read from B (valid memory)
   const void* cptr = (mode == MODE_CHUNK_STATE) ? p.Bm : p.Cm;
-  CUtensorMap mx, mb, mc;
+  CUtensorMap mx, mb, mc, my;
   const uint32_t box[4] = {64, 1, (uint32_t)T, 1};
   const uint64_t dx[4] = {(uint64_t)P, (uint64_t)p.H, (uint64_t)p.L, (uint64_t)p.B};
   const uint64_t sx[3] = {(uint64_t)P * 2, (uint64_t)p.H * P * 2, (uint64_t)p.sx * 2};
@@ -702,6 +719,12 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   if (!tma::encode_bf16_4d_cached(&mx, p.x, dx, sx, box) || !tma::encode_bf16_4d_cached(&mb, p.Bm, dbc, sbc, box) ||
       !tma::encode_bf16_4d_cached(&mc, cptr, dbc, sbc, box))
     return cudaErrorInvalidValue;
+  if (y) {  // y has x's shape and layout, with its own batch stride
+    const uint64_t sy[3] = {(uint64_t)P * 2, (uint64_t)p.H * P * 2, (uint64_t)p.sy * 2};
+    if (!tma::encode_bf16_4d_cached(&my, y, dx, sy, box)) return cudaErrorInvalidValue;
+  } else {
+    my = mx;  // never used: no y is stored
+  }
   Params kp;
   kp.mode = mode;
   kp.nc = p.nc;
@@ -736,7 +759,7 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
     attr_set.fetch_or(bit);
   }
   const int64_t ctas = mode == fused::MODE_SCAN ? p.B * p.H : p.B * p.H * p.nc;
-  k_ssd_fused<<<(unsigned)ctas, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc);
+  k_ssd_fused<<<(unsigned)ctas, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
   return cudaGetLastError();
 }
 

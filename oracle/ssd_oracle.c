@@ -17,7 +17,7 @@
  *  [P3] "告别Transformer的二次方噩梦：用Mamba（S6）模型在长文本任务中实现线性时间推理"
  *       §2.1 (dt, B, C depend on the input, i.e. vary per token).
  *
- * Readings where the pages are silent (each listed in the design doc):
+ * Readings where the pages are silent:
  *  - decay is a per-head scalar a_t = exp(dt_t * A_h) (dt per token and head);
  *  - the input enters as the outer product B_t x_t^T with no dt factor;
  *  - state per (batch, head) is an N x P matrix; y_t = C_t^T h_t + D_h x_t;

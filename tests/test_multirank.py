@@ -1,6 +1,6 @@
 """The multi-rank host logic of bench.py, on CPU with gloo (world size 2).
 
-On the GPU machine bench.py runs one process per GPU under torchrun; every rank
+On a multi-GPU node bench.py runs one process per GPU under torchrun; every rank
 scans its own batch (no collective on the data path) and only the timing is
 reduced (max over ranks).  These tests run that reduction and the rank
 conventions with the gloo backend on 127.0.0.1.

@@ -140,4 +140,13 @@ def test_vertical_rejects(lib):
     dv = dims(seqlen=512)
     assert lib.ssd_scan_workspace_size(ctypes.byref(dv), ctypes.byref(one)) == 0
     assert n.value >= one.value + 2 * 2 * 512 * 4 * 64 * 2
+    # the wavefront keeps two V-token activation blocks per layer boundary
+    act = 2 * 512 * 4 * 64 * 2  # B * V * H * P * bf16 for dims() (batch 2, 4 heads, P 64)
+    sizes = {}
+    for layers in (1, 2, 3, 24):
+        m = ctypes.c_size_t(0)
+        assert lib.ssd_vertical_workspace_size(ctypes.byref(d), layers, 512, ctypes.byref(m)) == 0
+        sizes[layers] = m.value
+    assert sizes[1] == sizes[2] and sizes[2] >= one.value + 2 * act
+    assert sizes[24] - sizes[3] == 2 * (24 - 3) * act
     assert lib.ssd_vertical_fwd(ctypes.byref(d), 2, 512, 1e-6, None, *([None] * 6), None, None, 0, None) == 1

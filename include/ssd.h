@@ -226,8 +226,10 @@ ssd_status ssd_vertical_workspace_size(const ssd_dims* d, int32_t n_layers, int6
  * events belong to the library (one set per device, created on first use,
  * kept until the process exits); every call forks them from `stream` and
  * joins them back into it, so the call stays asynchronous, orders like a
- * single-stream call, and can be captured into a CUDA graph.  Calls from
- * several host threads on one device are serialised while they enqueue.
+ * single-stream call, and can be captured into a CUDA graph (make the first
+ * call on a device outside a capture: it creates the streams and events).
+ * Calls from several host threads on one device are serialised while they
+ * enqueue.
  * Otherwise the blocks and layers run one after another on `stream`.
  */
 ssd_status ssd_vertical_fwd(const ssd_dims* d, int32_t n_layers, int64_t vblock, float rms_eps,

@@ -84,13 +84,17 @@ def load_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+FUSED_KERNEL_SOURCES = ("ssd_fused.cu", "ssd_common.cuh", "ssd_tc.cuh", "tma.cuh", "umma.cuh")
+
+
 def kernel_source_hash() -> str:
+    """Hash of the sources the fused kernel is compiled from (its file and the
+    headers it includes): a recorded ncu traffic figure applies while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "chunked_state_space_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in FUSED_KERNEL_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -310,14 +314,21 @@ def main():
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
+    # ssd_scan_fwd_host: the batch streams through the device one sequence at a
+    # time, copies in and out overlapped with the scan
+    host_ws = torch.empty(ssd.ssd_scan_fwd_host_workspace_size(dims), dtype=torch.uint8, device=dev)
+
+    def e2e_step():
+        ssd.ssd_scan_fwd_host(pinned["x"], pinned["dt"], pinned["A"], pinned["B"], pinned["C"], pinned["D"],
+                              pinned["init"], chunk=wl.chunk, y=h_y, final_state=h_fin, workspace=host_ws,
+                              stream=stream)
+
+    e2e_step()  # creates the copy streams outside the timed region
+    torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(max(args.e2e_steps, 1)):
-        for k, v in pinned.items():
-            d[k].copy_(v, non_blocking=True)
-        step()
-        h_y.copy_(y, non_blocking=True)
-        h_fin.copy_(fin, non_blocking=True)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / max(args.e2e_steps, 1)

@@ -6,4 +6,5 @@
 #include "ssd_fused.cu"
 #include "ssd_api.cu"
 #include "ssd_noalloc.cu"
+#include "ssd_hostio.cu"
 #include "ssd_selftest.cu"

@@ -27,7 +27,7 @@ EXPORTED = ["ssd_status_string", "ssd_version", "ssd_scan_workspace_size", "ssd_
             "ssd_chunk_scan", "ssd_rmsnorm", "ssd_vertical_workspace_size", "ssd_vertical_fwd",
             "ssd_read_device_status", "ssd_selftest_umma", "ssd_scan_path", "ssd_step",
             "ssd_selftest_fused_trace", "ssd_scan_fwd_noalloc", "ssd_selftest_mask_timing",
-            "ssd_selftest_timeout"]
+            "ssd_selftest_timeout", "ssd_scan_fwd_host", "ssd_scan_fwd_host_workspace_size"]
 
 
 class SSDError(RuntimeError):
@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
         "ssd_scan_workspace_size": (ctypes.c_int, [D, ctypes.POINTER(ctypes.c_size_t)]),
         "ssd_scan_fwd": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_size_t, _P]),
         "ssd_scan_fwd_unfused": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_size_t, _P]),
+        "ssd_scan_fwd_host": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_size_t, _P]),
+        "ssd_scan_fwd_host_workspace_size": (ctypes.c_int, [D, _P]),
         "ssd_chunk_cumsum": (ctypes.c_int, [D, _P, _P, _P, _P]),
         "ssd_chunk_state": (ctypes.c_int, [D, _P, _P, _P, _P, _P]),
         "ssd_state_passing": (ctypes.c_int, [D, _P, _P, _P, _P, _P, _P]),
@@ -170,6 +172,37 @@ def ssd_scan_fwd(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, y=
     s = fn(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D), _ptr(init_state), _ptr(y),
            _ptr(final_state), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check(s, "ssd_scan_fwd_unfused" if unfused else "ssd_scan_fwd")
+    return y, final_state
+
+
+def ssd_scan_fwd_host_workspace_size(dims: Dims) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().ssd_scan_fwd_host_workspace_size(ctypes.byref(dims), ctypes.byref(n)),
+           "ssd_scan_fwd_host_workspace_size")
+    return int(n.value)
+
+
+def ssd_scan_fwd_host(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, y=None, final_state=None,
+                      workspace=None, stream=None, want_final: bool = True, device=None):
+    """ssd_scan_fwd on HOST tensors (pinned for overlapped copies): the batch streams
+    through a device workspace one sequence at a time.  Returns host (y, final_state);
+    they are complete once `stream` (default: the current stream) has finished."""
+    for t in (x, dt, A, Bm, Cm, D, init_state, y, final_state):
+        if t is not None and t.is_cuda:
+            raise SSDError(1, "ssd_scan_fwd_host takes host tensors")
+    _contig(x, dt, A, Bm, Cm, D, init_state, y, final_state)
+    dims = make_dims(x, Bm, chunk)
+    pin = x.is_pinned()
+    if y is None:
+        y = torch.empty(x.shape, dtype=x.dtype, pin_memory=pin)
+    if final_state is None and want_final:
+        final_state = torch.empty((dims.batch, dims.nheads, dims.dstate, dims.headdim), dtype=torch.float32,
+                                  pin_memory=pin)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    ws = _workspace(ssd_scan_fwd_host_workspace_size(dims), dev, workspace)
+    _check(lib().ssd_scan_fwd_host(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D),
+                                   _ptr(init_state), _ptr(y), _ptr(final_state), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream)), "ssd_scan_fwd_host")
     return y, final_state
 
 

@@ -109,6 +109,32 @@ ssd_status ssd_scan_fwd(const ssd_dims* d, const void* x, const float* dt, const
                         void* stream);
 
 /*
+ * Bytes of DEVICE workspace ssd_scan_fwd_host needs for `d`: A and D, and two
+ * one-sequence slice buffers (inputs, outputs and the scan's scratch).
+ */
+ssd_status ssd_scan_fwd_host_workspace_size(const ssd_dims* d, size_t* bytes);
+
+/*
+ * ssd_scan_fwd with every tensor in HOST memory (same shapes, layouts and
+ * meaning; init_state, final_state and D may be NULL as there), the copies
+ * overlapped with the scan: the batch flows through the device workspace one
+ * sequence at a time, slice b+1 copied in and slice b-1 copied out while slice
+ * b is scanned on `stream`.  Host buffers should be page-locked
+ * (cudaHostAlloc / cudaHostRegister): pageable memory works but its copies do
+ * not overlap.  The host buffers must stay valid and unchanged until the work
+ * on `stream` completes; y and final_state are written by then.  Results equal
+ * ssd_scan_fwd's bitwise.  The two copy streams and their events belong to the
+ * library (one set per device, created on first use, kept until the process
+ * exits); each call forks them from `stream` and joins them back.  Calls from
+ * several host threads on one device are serialised while they enqueue.
+ * Errors: as ssd_scan_fwd; SSD_ERR_WORKSPACE if the device workspace is NULL
+ * or smaller than ssd_scan_fwd_host_workspace_size.
+ */
+ssd_status ssd_scan_fwd_host(const ssd_dims* d, const void* x, const float* dt, const float* A, const void* Bm,
+                             const void* Cm, const float* D, const float* init_state, void* y, float* final_state,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Which implementation ssd_scan_fwd uses for `d`: *path = SSD_PATH_CUDA_CORES
  * (four CUDA-core step kernels), SSD_PATH_TENSOR_STEPS (four step kernels,
  * steps 2 and 4 on tcgen05 tensor cores) or SSD_PATH_FUSED (one persistent

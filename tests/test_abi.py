@@ -150,3 +150,24 @@ def test_vertical_rejects(lib):
     assert sizes[1] == sizes[2] and sizes[2] >= one.value + 2 * act
     assert sizes[24] - sizes[3] == 2 * (24 - 3) * act
     assert lib.ssd_vertical_fwd(ctypes.byref(d), 2, 512, 1e-6, None, *([None] * 6), None, None, 0, None) == 1
+
+
+def test_host_io_entry_rejects(lib):
+    d = dims()
+    n = ctypes.c_size_t(0)
+    assert lib.ssd_scan_fwd_host_workspace_size(ctypes.byref(d), ctypes.byref(n)) == 0
+    one = ctypes.c_size_t(0)
+    d1 = dims(batch=1)
+    assert lib.ssd_scan_workspace_size(ctypes.byref(d1), ctypes.byref(one)) == 0
+    # A, D and two one-sequence buffers (x, y, dt, B, C, init, final) plus scratch
+    L, H, P, N, G = 1000, 4, 64, 128, 2
+    per_slice = 2 * L * H * P * 2 + L * H * 4 + 2 * L * G * N * 2 + 2 * H * N * P * 4 + one.value
+    assert n.value >= 2 * per_slice
+    assert lib.ssd_scan_fwd_host_workspace_size(ctypes.byref(d), None) == 1
+    assert lib.ssd_scan_fwd_host_workspace_size(ctypes.byref(dims(nheads=5)), ctypes.byref(n)) == 2
+    host = ctypes.c_void_p(0x10000)  # never dereferenced: validation returns first
+    args = [host] * 5 + [None, None, host, None]
+    assert lib.ssd_scan_fwd_host(ctypes.byref(d), None, *args[1:], None, 0, None) == 1       # x NULL
+    assert lib.ssd_scan_fwd_host(ctypes.byref(d), *args, None, 0, None) == 6                 # no workspace
+    assert lib.ssd_scan_fwd_host(ctypes.byref(d), *args, ctypes.c_void_p(BASE), 1024, None) == 6
+    assert lib.ssd_scan_fwd_host(ctypes.byref(d), *args, ctypes.c_void_p(BASE + 8), n.value, None) == 4

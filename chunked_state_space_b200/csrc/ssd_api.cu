@@ -53,6 +53,9 @@ Problem make_problem(const ssd_dims* d) {
   p.sdt = p.L * p.H;
   p.sbc = p.L * p.G * p.N;
   p.sy = p.L * p.H * p.P;
+  p.ldx = p.ldy = p.H * p.P;
+  p.lddt = p.H;
+  p.ldbc = p.G * p.N;
   return p;
 }
 
@@ -207,6 +210,45 @@ ssd_status ssd_scan_fwd(const ssd_dims* d, const void* x, const float* dt, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (fused_supported(p)) return cuda_status(launch_fused(p, init_state, final_state, workspace, st));
   return run_unfused(p, init_state, final_state, static_cast<char*>(workspace), st);
+}
+
+ssd_status ssd_scan_fwd_strided(const ssd_dims* d, const void* x, int64_t x_bstride, int64_t x_tstride,
+                                const float* dt, int64_t dt_bstride, int64_t dt_tstride, const float* A, const void* Bm,
+                                const void* Cm, int64_t bc_bstride, int64_t bc_tstride, const float* D,
+                                const float* init_state, void* y, int64_t y_bstride, int64_t y_tstride,
+                                float* final_state, void* stream) {
+  ssd_status s = validate_dims(d);
+  if (s != SSD_OK) return s;
+  Problem p = make_problem(d);
+  if (!fused_supported(p)) return SSD_ERR_UNSUPPORTED;  // the tensor-core path only
+  if (!x || !dt || !A || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;
+  const int64_t HP = p.H * p.P, GN = p.G * p.N;
+  // a token's heads (groups) stay dense; tokens may be further apart, batches too
+  if (x_tstride < HP || y_tstride < HP || dt_tstride < p.H || bc_tstride < GN) return SSD_ERR_SHAPE;
+  if (x_bstride < (p.L - 1) * x_tstride + HP || y_bstride < (p.L - 1) * y_tstride + HP ||
+      dt_bstride < (p.L - 1) * dt_tstride + p.H || bc_bstride < (p.L - 1) * bc_tstride + GN)
+    return SSD_ERR_SHAPE;
+  // TMA strides are multiples of 16 bytes: 8 bf16 elements
+  if ((x_tstride | x_bstride | y_tstride | y_bstride | bc_tstride | bc_bstride) & 7) return SSD_ERR_ALIGN;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(Bm) || !aligned16(Cm) || !aligned16(A) ||
+      (D && !aligned16(D)) || !aligned_to(dt, 4) || (init_state && !aligned16(init_state)) ||
+      (final_state && !aligned16(final_state)))
+    return SSD_ERR_ALIGN;
+  // y must not overlap an input (extents from first to last element touched)
+  const size_t es = io_size(d->io_dtype);
+  const Range ry = range_of(y, es * (size_t)((p.B - 1) * y_bstride + (p.L - 1) * y_tstride + HP));
+  const Range rin[] = {range_of(x, es * (size_t)((p.B - 1) * x_bstride + (p.L - 1) * x_tstride + HP)),
+                       range_of(Bm, es * (size_t)((p.B - 1) * bc_bstride + (p.L - 1) * bc_tstride + GN)),
+                       range_of(Cm, es * (size_t)((p.B - 1) * bc_bstride + (p.L - 1) * bc_tstride + GN)),
+                       range_of(dt, 4 * (size_t)((p.B - 1) * dt_bstride + (p.L - 1) * dt_tstride + p.H))};
+  for (const Range& r : rin)
+    if (overlaps(ry, r)) return SSD_ERR_INVALID_ARG;
+  p.x = x; p.dt = dt; p.A = A; p.Bm = Bm; p.Cm = Cm; p.D = D; p.y = y;
+  p.sx = x_bstride; p.ldx = x_tstride;
+  p.sdt = dt_bstride; p.lddt = dt_tstride;
+  p.sbc = bc_bstride; p.ldbc = bc_tstride;
+  p.sy = y_bstride; p.ldy = y_tstride;
+  return cuda_status(launch_fused(p, init_state, final_state, nullptr, static_cast<cudaStream_t>(stream)));
 }
 
 ssd_status ssd_chunk_cumsum(const ssd_dims* d, const float* dt, const float* A, float* lam, void* stream) {

@@ -26,6 +26,9 @@ struct Problem {
   const float* D;
   void* y;
   int64_t sy;  // batch stride of y (default L*H*P)
+  // token strides (elements); the contiguous layout has ldx = ldy = H*P,
+  // lddt = H, ldbc = G*N.  Only the fused tensor-core kernel reads them.
+  int64_t ldx, lddt, ldbc, ldy;
 };
 
 template <typename T>

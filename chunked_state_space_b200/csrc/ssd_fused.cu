@@ -66,13 +66,13 @@ struct Params {
   int64_t nc, Q;         // chunking of the step kernels
   const float* lam_in;   // step-1 log-decay sums [B,H,nc,Q] (step modes)
   const float* dt;
-  int64_t sdt;
+  int64_t sdt, lddt;  // batch and token strides of dt
   const float* A;
   const float* D;
   const float* init;
   float* final_state;
   const __nv_bfloat16* x;
-  int64_t sx;
+  int64_t sx, ldx;    // batch and token strides of x
   __nv_bfloat16* y;
   int64_t sy;
   unsigned long long* trace;  // diagnostics: per-sub-chunk event clocks of CTA 0, then
@@ -373,8 +373,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const float* dtb = p.dt + (int64_t)b * p.sdt + h;
     auto load_dt = [&](int j, float& d0, float& d1) {
       const int64_t t0 = (int64_t)j * T + 2 * a;
-      d0 = (!chunked && j < nsub && t0 < p.L) ? dtb[t0 * p.H] : 0.f;
-      d1 = (!chunked && j < nsub && t0 + 1 < p.L) ? dtb[(t0 + 1) * p.H] : 0.f;
+      d0 = (!chunked && j < nsub && t0 < p.L) ? dtb[t0 * p.lddt] : 0.f;
+      d1 = (!chunked && j < nsub && t0 + 1 < p.L) ? dtb[(t0 + 1) * p.lddt] : 0.f;
     };
     const float* lamc = chunked ? p.lam_in + cslot * p.Q : nullptr;
     float d0, d1;
@@ -536,7 +536,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto load_x = [&](int j, uint4* xv) {
       const int64_t tg = (int64_t)t_base + (int64_t)j * T + r;
       if (j < nsub && tg < p.L) {
-        const uint4* src = reinterpret_cast<const uint4*>(xg + tg * p.H * P);
+        const uint4* src = reinterpret_cast<const uint4*>(xg + tg * p.ldx);
 #pragma unroll
         for (int c = 0; c < 8; ++c) xv[c] = src[c];
       } else {
@@ -713,14 +713,14 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   CUtensorMap mx, mb, mc, my;
   const uint32_t box[4] = {64, 1, (uint32_t)T, 1};
   const uint64_t dx[4] = {(uint64_t)P, (uint64_t)p.H, (uint64_t)p.L, (uint64_t)p.B};
-  const uint64_t sx[3] = {(uint64_t)P * 2, (uint64_t)p.H * P * 2, (uint64_t)p.sx * 2};
+  const uint64_t sx[3] = {(uint64_t)P * 2, (uint64_t)p.ldx * 2, (uint64_t)p.sx * 2};
   const uint64_t dbc[4] = {(uint64_t)NS, (uint64_t)p.G, (uint64_t)p.L, (uint64_t)p.B};
-  const uint64_t sbc[3] = {(uint64_t)NS * 2, (uint64_t)p.G * NS * 2, (uint64_t)p.sbc * 2};
+  const uint64_t sbc[3] = {(uint64_t)NS * 2, (uint64_t)p.ldbc * 2, (uint64_t)p.sbc * 2};
   if (!tma::encode_bf16_4d_cached(&mx, p.x, dx, sx, box) || !tma::encode_bf16_4d_cached(&mb, p.Bm, dbc, sbc, box) ||
       !tma::encode_bf16_4d_cached(&mc, cptr, dbc, sbc, box))
     return cudaErrorInvalidValue;
   if (y) {  // y has x's shape and layout, with its own batch stride
-    const uint64_t sy[3] = {(uint64_t)P * 2, (uint64_t)p.H * P * 2, (uint64_t)p.sy * 2};
+    const uint64_t sy[3] = {(uint64_t)P * 2, (uint64_t)p.ldy * 2, (uint64_t)p.sy * 2};
     if (!tma::encode_bf16_4d_cached(&my, y, dx, sy, box)) return cudaErrorInvalidValue;
   } else {
     my = mx;  // never used: no y is stored
@@ -736,12 +736,14 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   kp.nsub = (int)ceil_div(p.L, T);
   kp.dt = p.dt;
   kp.sdt = p.sdt;
+  kp.lddt = p.lddt;
   kp.A = p.A;
   kp.D = p.D;
   kp.init = init;
   kp.final_state = final_state;
   kp.x = static_cast<const __nv_bfloat16*>(p.x);
   kp.sx = p.sx;
+  kp.ldx = p.ldx;
   kp.y = static_cast<__nv_bfloat16*>(y);
   kp.sy = p.sy;
   kp.trace = trace;

@@ -27,7 +27,8 @@ EXPORTED = ["ssd_status_string", "ssd_version", "ssd_scan_workspace_size", "ssd_
             "ssd_chunk_scan", "ssd_rmsnorm", "ssd_vertical_workspace_size", "ssd_vertical_fwd",
             "ssd_read_device_status", "ssd_selftest_umma", "ssd_scan_path", "ssd_step",
             "ssd_selftest_fused_trace", "ssd_scan_fwd_noalloc", "ssd_selftest_mask_timing",
-            "ssd_selftest_timeout", "ssd_scan_fwd_host", "ssd_scan_fwd_host_workspace_size"]
+            "ssd_selftest_timeout", "ssd_scan_fwd_host", "ssd_scan_fwd_host_workspace_size",
+            "ssd_scan_fwd_strided"]
 
 
 class SSDError(RuntimeError):
@@ -43,6 +44,7 @@ class Dims(ctypes.Structure):
 
 
 _P = ctypes.c_void_p
+_I64 = ctypes.c_int64
 _lib = None
 
 
@@ -64,6 +66,8 @@ def lib() -> ctypes.CDLL:
         "ssd_scan_fwd_unfused": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_size_t, _P]),
         "ssd_scan_fwd_host": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_size_t, _P]),
         "ssd_scan_fwd_host_workspace_size": (ctypes.c_int, [D, _P]),
+        "ssd_scan_fwd_strided": (ctypes.c_int, [D, _P, _I64, _I64, _P, _I64, _I64, _P, _P, _P, _I64, _I64, _P, _P,
+                                                _P, _I64, _I64, _P, _P]),
         "ssd_chunk_cumsum": (ctypes.c_int, [D, _P, _P, _P, _P]),
         "ssd_chunk_state": (ctypes.c_int, [D, _P, _P, _P, _P, _P]),
         "ssd_state_passing": (ctypes.c_int, [D, _P, _P, _P, _P, _P, _P]),
@@ -203,6 +207,31 @@ def ssd_scan_fwd_host(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 25
     _check(lib().ssd_scan_fwd_host(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D),
                                    _ptr(init_state), _ptr(y), _ptr(final_state), _ptr(ws),
                                    ws.numel() * ws.element_size(), _stream(stream)), "ssd_scan_fwd_host")
+    return y, final_state
+
+
+def ssd_scan_fwd_strided(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, y=None, final_state=None,
+                         stream=None, want_final: bool = True):
+    """ssd_scan_fwd on strided views (tensor-core path): x [B,L,H,P], dt [B,L,H],
+    B/C [B,L,G,N] and y may have any batch and token strides as long as each
+    token's heads (groups) are dense, e.g. slices of one fused projection output.
+    Bm and Cm must share their strides."""
+    if Bm.stride() != Cm.stride():
+        raise SSDError(2, "B and C must have the same strides")
+    for t, inner in ((x, (x.shape[3], 1)), (Bm, (Bm.shape[3], 1)), (dt, (1,))):
+        if tuple(t.stride()[2:]) != inner:
+            raise SSDError(2, "each token's heads/groups must be dense")
+    _contig(A, D, init_state, final_state)
+    dims = make_dims(x, Bm, chunk)
+    if y is None:
+        y = torch.empty(x.shape, dtype=x.dtype, device=x.device)
+    if final_state is None and want_final:
+        final_state = torch.empty((dims.batch, dims.nheads, dims.dstate, dims.headdim), dtype=torch.float32,
+                                  device=x.device)
+    _check(lib().ssd_scan_fwd_strided(ctypes.byref(dims), _ptr(x), x.stride(0), x.stride(1), _ptr(dt), dt.stride(0),
+                                      dt.stride(1), _ptr(A), _ptr(Bm), _ptr(Cm), Bm.stride(0), Bm.stride(1), _ptr(D),
+                                      _ptr(init_state), _ptr(y), y.stride(0), y.stride(1), _ptr(final_state),
+                                      _stream(stream)), "ssd_scan_fwd_strided")
     return y, final_state
 
 

@@ -109,6 +109,29 @@ ssd_status ssd_scan_fwd(const ssd_dims* d, const void* x, const float* dt, const
                         void* stream);
 
 /*
+ * ssd_scan_fwd on strided tensors (tensor-core path only: bf16 io, P = 64,
+ * N = 128, Q a multiple of 128; else SSD_ERR_UNSUPPORTED), e.g. x, B and C as
+ * column slices of one fused projection output [B, L, H*P + 2*G*N].  Each of
+ * x, dt, Bm/Cm (one stride pair for both) and y takes a batch stride and a
+ * token stride in ELEMENTS; inside a token the heads (groups) stay dense:
+ *   x[b, t, h, p]  at x  + b*x_bstride  + t*x_tstride  + h*P + p
+ *   dt[b, t, h]    at dt + b*dt_bstride + t*dt_tstride + h
+ *   Bm[b, t, g, n] at Bm + b*bc_bstride + t*bc_tstride + g*N + n (Cm alike)
+ *   y like x with y_bstride, y_tstride.
+ * A, D, init_state, final_state are contiguous as in ssd_scan_fwd.  Token
+ * strides must be at least the dense row (H*P, H, G*N), batch strides at
+ * least a whole sequence (else SSD_ERR_SHAPE); the bf16 strides must be
+ * multiples of 8 elements (TMA: 16 bytes) and the pointers 16-byte aligned
+ * (dt: 4 bytes) (else SSD_ERR_ALIGN); y must not overlap x, dt, Bm or Cm
+ * (SSD_ERR_INVALID_ARG).  No workspace is needed.
+ */
+ssd_status ssd_scan_fwd_strided(const ssd_dims* d, const void* x, int64_t x_bstride, int64_t x_tstride,
+                                const float* dt, int64_t dt_bstride, int64_t dt_tstride, const float* A,
+                                const void* Bm, const void* Cm, int64_t bc_bstride, int64_t bc_tstride,
+                                const float* D, const float* init_state, void* y, int64_t y_bstride,
+                                int64_t y_tstride, float* final_state, void* stream);
+
+/*
  * Bytes of DEVICE workspace ssd_scan_fwd_host needs for `d`: A and D, and two
  * one-sequence slice buffers (inputs, outputs and the scan's scratch).
  */

@@ -171,3 +171,22 @@ def test_host_io_entry_rejects(lib):
     assert lib.ssd_scan_fwd_host(ctypes.byref(d), *args, None, 0, None) == 6                 # no workspace
     assert lib.ssd_scan_fwd_host(ctypes.byref(d), *args, ctypes.c_void_p(BASE), 1024, None) == 6
     assert lib.ssd_scan_fwd_host(ctypes.byref(d), *args, ctypes.c_void_p(BASE + 8), n.value, None) == 4
+
+
+def test_strided_entry_rejects(lib):
+    d = dims(seqlen=1024, ngroups=1)
+    L, H, P, N, G = 1024, 4, 64, 128, 1
+    W = H * P + 2 * G * N                      # a fused [x | B | C] row
+    f = lambda **kw: lib.ssd_scan_fwd_strided(
+        ctypes.byref(kw.get("d", d)), ctypes.c_void_p(kw.get("x", BASE)), kw.get("xb", L * W), kw.get("xt", W),
+        ctypes.c_void_p(BASE + 2 * GB), kw.get("dtb", L * H), kw.get("dtt", H), ctypes.c_void_p(BASE + 3 * GB),
+        ctypes.c_void_p(BASE + 2 * H * P), ctypes.c_void_p(BASE + 2 * (H * P + G * N)), L * W, W,
+        None, None, ctypes.c_void_p(kw.get("y", BASE + 4 * GB)), kw.get("yb", L * H * P), kw.get("yt", H * P),
+        None, None)
+    assert f(d=dims(headdim=32, seqlen=1024, ngroups=1)) == 5   # tensor-core shapes only
+    assert f(xt=H * P - 8) == 2                                  # token stride below a dense row
+    assert f(xb=L * W - W) == 2                                  # batch stride below a sequence
+    assert f(xt=W + 4, xb=L * (W + 4)) == 4                      # not a multiple of 8 elements
+    assert f(x=BASE + 8) == 4                                    # misaligned pointer
+    assert f(y=BASE + 2 * H * P) == 1                            # y overlaps the inputs
+    assert f(x=0) == 1                                           # NULL x

@@ -55,9 +55,9 @@ class _Oracle:
     def __init__(self, path: str):
         lib = ctypes.CDLL(path)
         lib.oracle_scan_recurrence.restype = None
-        lib.oracle_scan_recurrence.argtypes = [_I] * 6 + [_P] * 9
+        lib.oracle_scan_recurrence.argtypes = [_I] * 6 + [_P] * 9 + [ctypes.c_int]
         lib.oracle_scan_chunked.restype = None
-        lib.oracle_scan_chunked.argtypes = [_I] * 7 + [_P] * 14
+        lib.oracle_scan_chunked.argtypes = [_I] * 7 + [_P] * 14 + [ctypes.c_int]
         lib.oracle_round_bf16.restype = None
         lib.oracle_round_bf16.argtypes = [_I, _P, _P]
         lib.oracle_rmsnorm_bf16.restype = None
@@ -101,19 +101,22 @@ def num_threads(o: Optional[_Oracle] = None) -> int:
     return int((o or load()).lib.oracle_num_threads())
 
 
-def scan_recurrence(x, dt, A, Bm, Cm, D=None, init=None, want_final=True, o: Optional[_Oracle] = None):
-    """Token-by-token fp64 recurrence.  Returns (y [B,L,H,P], final [B,H,N,P] or None)."""
+def scan_recurrence(x, dt, A, Bm, Cm, D=None, init=None, want_final=True, o: Optional[_Oracle] = None,
+                    input_dt: bool = False):
+    """Token-by-token fp64 recurrence.  Returns (y [B,L,H,P], final [B,H,N,P] or None).
+    input_dt: the input term is dt_t B_t x_t^T (the skip keeps D x_t)."""
     o = o or load()
     x, dt, A, Bm, Cm, D, init = map(_f64, (x, dt, A, Bm, Cm, D, init))
     Bz, L, H, P, N, G = _dims(x, Bm)
     y = np.empty((Bz, L, H, P))
     fin = np.empty((Bz, H, N, P)) if want_final else None
     o.lib.oracle_scan_recurrence(Bz, L, H, P, N, G, _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm),
-                                 _ptr(D), _ptr(init), _ptr(y), _ptr(fin))
+                                 _ptr(D), _ptr(init), _ptr(y), _ptr(fin), int(bool(input_dt)))
     return y, fin
 
 
-def scan_chunked(x, dt, A, Bm, Cm, Q, D=None, init=None, o: Optional[_Oracle] = None) -> dict:
+def scan_chunked(x, dt, A, Bm, Cm, Q, D=None, init=None, o: Optional[_Oracle] = None,
+                 input_dt: bool = False) -> dict:
     """Chunked fp64 evaluation with every intermediate of the decomposition."""
     o = o or load()
     x, dt, A, Bm, Cm, D, init = map(_f64, (x, dt, A, Bm, Cm, D, init))
@@ -131,7 +134,7 @@ def scan_chunked(x, dt, A, Bm, Cm, Q, D=None, init=None, o: Optional[_Oracle] = 
     o.lib.oracle_scan_chunked(Bz, L, H, P, N, G, Q, _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm),
                               _ptr(D), _ptr(init), _ptr(out["lam"]), _ptr(out["chunk_states"]),
                               _ptr(out["prev_states"]), _ptr(out["y_intra"]), _ptr(out["y_inter"]),
-                              _ptr(out["y"]), _ptr(out["final"]))
+                              _ptr(out["y"]), _ptr(out["final"]), int(bool(input_dt)))
     return out
 
 

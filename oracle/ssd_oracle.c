@@ -19,7 +19,10 @@
  *
  * Readings where the pages are silent:
  *  - decay is a per-head scalar a_t = exp(dt_t * A_h) (dt per token and head);
- *  - the input enters as the outer product B_t x_t^T with no dt factor;
+ *  - the input enters as the outer product B_t x_t^T with no dt factor; the
+ *    optional variant (input_dt = 1) scales it by dt_t, B_t (dt_t x_t)^T, the
+ *    input-dependent step of [P3] §2.1 scaling the input as well as the decay,
+ *    while the skip keeps D_h x_t;
  *  - state per (batch, head) is an N x P matrix; y_t = C_t^T h_t + D_h x_t;
  *  - head h reads B/C group g = h / (H / G);
  *  - the last chunk may be shorter than Q (ragged L);
@@ -54,7 +57,7 @@
 void oracle_scan_recurrence(int64_t Bz, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G,
                             const double* x, const double* dt, const double* A,
                             const double* Bm, const double* Cm, const double* D,
-                            const double* init, double* y, double* final_state) {
+                            const double* init, double* y, double* final_state, int input_dt) {
   const int64_t hpg = H / G;
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t bh = 0; bh < Bz * H; ++bh) {
@@ -67,6 +70,7 @@ void oracle_scan_recurrence(int64_t Bz, int64_t L, int64_t H, int64_t P, int64_t
     const double d = D ? D[h] : 0.0;
     for (int64_t t = 0; t < L; ++t) {
       const double a = exp(dt[(b * L + t) * H + h] * A[h]);
+      const double u = input_dt ? dt[(b * L + t) * H + h] : 1.0;  /* the input term's factor */
       const double* xt = x + IX4(b, t, h, 0, L, H, P);
       const double* bt = Bm + IX4(b, t, g, 0, L, G, N);
       const double* ct = Cm + IX4(b, t, g, 0, L, G, N);
@@ -74,7 +78,7 @@ void oracle_scan_recurrence(int64_t Bz, int64_t L, int64_t H, int64_t P, int64_t
       for (int64_t n = 0; n < N; ++n) {
         double* row = st + n * P;
         const double bn = bt[n];
-        for (int64_t p = 0; p < P; ++p) row[p] = a * row[p] + bn * xt[p];
+        for (int64_t p = 0; p < P; ++p) row[p] = a * row[p] + u * bn * xt[p];
       }
       for (int64_t p = 0; p < P; ++p) yt[p] = d * xt[p];
       for (int64_t n = 0; n < N; ++n) {
@@ -106,7 +110,8 @@ void oracle_scan_chunked(int64_t Bz, int64_t L, int64_t H, int64_t P, int64_t N,
                          int64_t Q, const double* x, const double* dt, const double* A,
                          const double* Bm, const double* Cm, const double* D, const double* init,
                          double* lam, double* chunk_states, double* prev_states,
-                         double* y_intra, double* y_inter, double* y, double* final_state) {
+                         double* y_intra, double* y_inter, double* y, double* final_state,
+                         int input_dt) {
   const int64_t hpg = H / G;
   const int64_t nc = (L + Q - 1) / Q;
 #pragma omp parallel for schedule(dynamic, 1)
@@ -147,7 +152,7 @@ void oracle_scan_chunked(int64_t Bz, int64_t L, int64_t H, int64_t P, int64_t N,
           double cb = 0.0;
           for (int64_t n = 0; n < N; ++n) cb += ct[n] * bs[n];
           const double* xs = x + IX4(b, s, h, 0, L, H, P);
-          const double w = cb * Lts;
+          const double w = cb * Lts * (input_dt ? dt[(b * L + s) * H + h] : 1.0);
           for (int64_t p = 0; p < P; ++p) yi[p] += w * xs[p];
         }
         /* by_inter: diag(L) inclusive decay times C_t^T prev */
@@ -173,6 +178,7 @@ void oracle_scan_chunked(int64_t Bz, int64_t L, int64_t H, int64_t P, int64_t N,
         const int64_t s = c0 + j;
         const double* bs = Bm + IX4(b, s, g, 0, L, G, N);
         const double* xs = x + IX4(b, s, h, 0, L, H, P);
+        if (input_dt) w *= dt[(b * L + s) * H + h];
         for (int64_t n = 0; n < N; ++n)
           for (int64_t p = 0; p < P; ++p) bin[n * P + p] += w * bs[n] * xs[p];
       }

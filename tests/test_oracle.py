@@ -48,9 +48,10 @@ def run_rec(p, o=None):
     return oracle.scan_recurrence(p["x"], p["dt"], p["A"], p["Bm"], p["Cm"], p["D"], p["init"], o=o)
 
 
-def brute_force(p):
-    """y_t = C_t^T[(prod_{r<=t} a_r) h0 + sum_{s<=t}(prod_{r=s+1..t} a_r) B_s x_s^T] + D x_t,
-    evaluated as an explicit double sum over (t, s); final state = bracket at t = L-1."""
+def brute_force(p, input_dt=False):
+    """y_t = C_t^T[(prod_{r<=t} a_r) h0 + sum_{s<=t}(prod_{r=s+1..t} a_r) u_s B_s x_s^T] + D x_t,
+    evaluated as an explicit double sum over (t, s); final state = bracket at t = L-1.
+    u_s = dt_s for the dt-scaled input variant, else 1."""
     x, dt, A, Bm, Cm, D, h0 = (p[k] for k in ("x", "dt", "A", "Bm", "Cm", "D", "init"))
     Bz, L, H, P = x.shape
     G, N = Bm.shape[2:]
@@ -65,7 +66,8 @@ def brute_force(p):
                 if h0 is not None:
                     st += np.prod(a[: t + 1]) * h0[b, h]
                 for s in range(t + 1):
-                    st += np.prod(a[s + 1: t + 1]) * np.outer(Bm[b, s, g], x[b, s, h])
+                    u = dt[b, s, h] if input_dt else 1.0
+                    st += np.prod(a[s + 1: t + 1]) * u * np.outer(Bm[b, s, g], x[b, s, h])
                 y[b, t, h] = Cm[b, t, g] @ st + (D[h] if D is not None else 0.0) * x[b, t, h]
                 if t == L - 1:
                     fin[b, h] = st
@@ -378,3 +380,38 @@ def test_tiny_workload_chunked_equals_recurrence():
     assert rel(out["y"], y) < 1e-12
     assert rel(out["final"], fin) < 1e-12
     assert np.all(np.isfinite(y)) and np.max(np.abs(y)) > 0.1
+
+
+# ---------------------------------------------------------------- the dt-scaled input variant
+
+def test_input_dt_brute_force():
+    """h_t = a_t h_{t-1} + dt_t B_t x_t^T, y_t = C_t^T h_t + D x_t against the explicit double sum."""
+    p = rand_problem(seed=11, Bz=2, L=19, H=4, P=3, N=2, G=2)
+    y, f = oracle.scan_recurrence(p["x"], p["dt"], p["A"], p["Bm"], p["Cm"], p["D"], p["init"], input_dt=True)
+    yb, fb = brute_force(p, input_dt=True)
+    assert rel(y, yb) < 1e-12 and rel(f, fb) < 1e-12
+    # the variant differs from the plain scan (the pin would not see a dropped factor otherwise)
+    y0, _ = oracle.scan_recurrence(p["x"], p["dt"], p["A"], p["Bm"], p["Cm"], p["D"], p["init"])
+    assert rel(y, y0) > 1e-3
+
+
+def test_input_dt_prefix_sum():
+    """A = 0 (a = 1): h_t = h0 + sum_{s<=t} dt_s B_s x_s^T, a dt-weighted prefix sum."""
+    p = rand_problem(seed=12, Bz=1, L=23, H=2, P=2, N=3, G=1)
+    A = np.zeros_like(p["A"])
+    y, f = oracle.scan_recurrence(p["x"], p["dt"], A, p["Bm"], p["Cm"], p["D"], p["init"], input_dt=True)
+    x, dt, Bm, Cm, D, h0 = p["x"], p["dt"], p["Bm"], p["Cm"], p["D"], p["init"]
+    for h in range(2):
+        terms = dt[0, :, h, None, None] * Bm[0, :, 0, :, None] * x[0, :, h, None, :]   # [L, N, P]
+        st = h0[0, h][None] + np.cumsum(terms, axis=0)
+        yy = np.einsum("tn,tnp->tp", Cm[0, :, 0], st) + D[h] * x[0, :, h]
+        assert rel(y[0, :, h], yy) < 1e-12
+        assert rel(f[0, h], st[-1]) < 1e-12
+
+
+@pytest.mark.parametrize("Q", [1, 4, 16, 19])
+def test_input_dt_chunked_equals_recurrence(Q):
+    p = rand_problem(seed=13, Bz=2, L=37, H=4, P=2, N=3, G=2)
+    y, f = oracle.scan_recurrence(p["x"], p["dt"], p["A"], p["Bm"], p["Cm"], p["D"], p["init"], input_dt=True)
+    out = oracle.scan_chunked(p["x"], p["dt"], p["A"], p["Bm"], p["Cm"], Q, p["D"], p["init"], input_dt=True)
+    assert rel(out["y"], y) < 1e-12 and rel(out["final"], f) < 1e-12

@@ -18,7 +18,11 @@ from test_oracle import _read_golden, brute_force, rand_problem, rel
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "ssd_oracle.c")
 
 MUTANTS = {
-    "decay_dropped": ("row[p] = a * row[p] + bn * xt[p];", "row[p] = row[p] + bn * xt[p];"),
+    "decay_dropped": ("row[p] = a * row[p] + u * bn * xt[p];", "row[p] = row[p] + u * bn * xt[p];"),
+    "input_dt_factor_dropped": ("const double u = input_dt ? dt[(b * L + t) * H + h] : 1.0;", "const double u = 1.0;"),
+    "input_dt_chunked_intra_dropped": ("const double w = cb * Lts * (input_dt ? dt[(b * L + s) * H + h] : 1.0);",
+                                       "const double w = cb * Lts;"),
+    "input_dt_chunked_state_dropped": ("if (input_dt) w *= dt[(b * L + s) * H + h];", ""),
     "group_index": ("const int64_t b = bh / H, h = bh % H, g = h / hpg;",
                     "const int64_t b = bh / H, h = bh % H, g = h % G;"),
     "b_c_swapped": ("const double bn = bt[n];", "const double bn = ct[n];"),
@@ -79,6 +83,23 @@ def _pins(o):
                 return False
         return True
     check("chunked_vs_recurrence", chunked)
+
+    def input_dt_brute():
+        y, f = oracle.scan_recurrence(p["x"], p["dt"], p["A"], p["Bm"], p["Cm"], p["D"], p["init"], o=o,
+                                      input_dt=True)
+        yb, fb = brute_force(p, input_dt=True)
+        return rel(y, yb) < 1e-12 and rel(f, fb) < 1e-12
+    check("input_dt_brute_force", input_dt_brute)
+
+    def input_dt_chunked():
+        yb, fb = brute_force(p, input_dt=True)
+        for Q in (4, 16):
+            out = oracle.scan_chunked(p["x"], p["dt"], p["A"], p["Bm"], p["Cm"], Q, p["D"], p["init"], o=o,
+                                      input_dt=True)
+            if not (rel(out["y"], yb) < 1e-12 and rel(out["final"], fb) < 1e-12):
+                return False
+        return True
+    check("input_dt_chunked", input_dt_chunked)
 
     def lam():
         out = oracle.scan_chunked(p["x"], p["dt"], p["A"], p["Bm"], p["Cm"], 5, p["D"], p["init"], o=o)

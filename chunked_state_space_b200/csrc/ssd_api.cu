@@ -24,7 +24,7 @@ size_t io_size(int io) { return io == SSD_BF16 ? 2 : 4; }
 
 ssd_status validate_dims(const ssd_dims* d) {
   if (!d) return SSD_ERR_INVALID_ARG;
-  if (d->reserved != 0) return SSD_ERR_INVALID_ARG;
+  if ((d->flags & ~SSD_FLAG_INPUT_DT) != 0) return SSD_ERR_INVALID_ARG;
   if (d->io_dtype != SSD_F32 && d->io_dtype != SSD_BF16) return SSD_ERR_DTYPE;
   if (d->batch < 1 || d->seqlen < 1 || d->nheads < 1 || d->headdim < 1 || d->dstate < 1 || d->ngroups < 1 ||
       d->chunk < 1)
@@ -56,6 +56,7 @@ Problem make_problem(const ssd_dims* d) {
   p.ldx = p.ldy = p.H * p.P;
   p.lddt = p.H;
   p.ldbc = p.G * p.N;
+  p.input_dt = (d->flags & SSD_FLAG_INPUT_DT) ? 1 : 0;
   return p;
 }
 
@@ -187,6 +188,7 @@ ssd_status ssd_scan_fwd_unfused(const ssd_dims* d, const void* x, const float* d
   if (s != SSD_OK) return s;
   s = validate_scan_args(d, x, dt, A, Bm, Cm, D, init_state, y, final_state);
   if (s != SSD_OK) return s;
+  if (d->flags & SSD_FLAG_INPUT_DT) return SSD_ERR_UNSUPPORTED;  // the tensor-core path only
   Problem p = make_problem(d);
   if (!workspace || workspace_bytes < unfused_ws_bytes(p)) return SSD_ERR_WORKSPACE;
   if (!aligned16(workspace)) return SSD_ERR_ALIGN;
@@ -209,6 +211,7 @@ ssd_status ssd_scan_fwd(const ssd_dims* d, const void* x, const float* dt, const
   p.x = x; p.dt = dt; p.A = A; p.Bm = Bm; p.Cm = Cm; p.D = D; p.y = y;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (fused_supported(p)) return cuda_status(launch_fused(p, init_state, final_state, workspace, st));
+  if (p.input_dt) return SSD_ERR_UNSUPPORTED;  // the dt-scaled input: tensor-core path only
   return run_unfused(p, init_state, final_state, static_cast<char*>(workspace), st);
 }
 
@@ -254,6 +257,7 @@ ssd_status ssd_scan_fwd_strided(const ssd_dims* d, const void* x, int64_t x_bstr
 ssd_status ssd_chunk_cumsum(const ssd_dims* d, const float* dt, const float* A, float* lam, void* stream) {
   ssd_status s = validate_dims(d);
   if (s != SSD_OK) return s;
+  if (d->flags & SSD_FLAG_INPUT_DT) return SSD_ERR_UNSUPPORTED;
   if (!dt || !A || !lam) return SSD_ERR_INVALID_ARG;
   if (!aligned16(dt) || !aligned16(A) || !aligned16(lam)) return SSD_ERR_ALIGN;
   Problem p = make_problem(d);
@@ -265,6 +269,7 @@ ssd_status ssd_chunk_state(const ssd_dims* d, const void* x, const void* Bm, con
                            void* stream) {
   ssd_status s = validate_dims(d);
   if (s != SSD_OK) return s;
+  if (d->flags & SSD_FLAG_INPUT_DT) return SSD_ERR_UNSUPPORTED;
   if (!x || !Bm || !lam || !chunk_states) return SSD_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(Bm) || !aligned16(lam) || !aligned16(chunk_states)) return SSD_ERR_ALIGN;
   Problem p = make_problem(d);
@@ -278,6 +283,7 @@ ssd_status ssd_state_passing(const ssd_dims* d, const float* chunk_states, const
                              float* prev_states, float* final_state, void* stream) {
   ssd_status s = validate_dims(d);
   if (s != SSD_OK) return s;
+  if (d->flags & SSD_FLAG_INPUT_DT) return SSD_ERR_UNSUPPORTED;
   if (!chunk_states || !lam || !prev_states) return SSD_ERR_INVALID_ARG;
   const void* ptrs[] = {chunk_states, lam, init_state, prev_states, final_state};
   for (const void* q : ptrs)
@@ -291,6 +297,7 @@ ssd_status ssd_chunk_scan(const ssd_dims* d, const void* x, const void* Bm, cons
                           const float* D, const float* prev_states, void* y, void* stream) {
   ssd_status s = validate_dims(d);
   if (s != SSD_OK) return s;
+  if (d->flags & SSD_FLAG_INPUT_DT) return SSD_ERR_UNSUPPORTED;
   if (!x || !Bm || !Cm || !lam || !prev_states || !y) return SSD_ERR_INVALID_ARG;
   const void* ptrs[] = {x, Bm, Cm, lam, D, prev_states, y};
   for (const void* q : ptrs)
@@ -508,6 +515,7 @@ ssd_status ssd_vertical_fwd(const ssd_dims* d, int32_t n_layers, int64_t vblock,
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Problem full = make_problem(d);
+  if (full.input_dt && !fused_supported(full)) return SSD_ERR_UNSUPPORTED;
   const int64_t V = vblock < d->seqlen ? vblock : d->seqlen;
   if (n_layers > 1 && fused_supported(full))
     return vertical_wavefront(d, n_layers, V, rms_eps, x0, dt, A, Bm, Cm, D, states, y_out, workspace, st);

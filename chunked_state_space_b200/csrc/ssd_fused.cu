@@ -11,6 +11,8 @@
 //   y_intra = P X_j                               (A operand from TMEM)
 //   y_inter = C_j bf16(s_{j-1})                   (into S columns 64-127, dead by then)
 //   b_intra = B_j^T X'_j,  X'_j = diag(exp(lam_end - lam_s)) X_j
+//   (with the dt-scaled input every column s of P and row s of X' also
+//   carries dt_s)
 //   y_t     = y_intra + exp(lam_t) y_inter + D x_t    (fp32; x_t re-read from L2)
 //   s_j     = exp(lam_end) s_{j-1} + b_intra              (fp32, registers)
 // Warp roles (384 threads): warp 2 issues TMA loads; warp 3 owns TMEM and
@@ -45,7 +47,8 @@ constexpr uint32_t OFF_XP = 2 * STAGE;         // X' (two buffers)
 constexpr uint32_t OFF_PREV = OFF_XP + 2 * TILE;  // bf16 state, MN-major [n][p]
 constexpr uint32_t OFF_LAM = OFF_PREV + TILE;  // float [4][128]
 constexpr uint32_t OFF_ECOL = OFF_LAM + 4 * T * 4;  // float [4][128]
-constexpr uint32_t OFF_WTOT = OFF_ECOL + 4 * T * 4;
+constexpr uint32_t OFF_DTS = OFF_ECOL + 4 * T * 4;   // float [4][128]: the input term's dt (1 without the flag)
+constexpr uint32_t OFF_WTOT = OFF_DTS + 4 * T * 4;
 constexpr uint32_t OFF_BAR = OFF_WTOT + 64;
 constexpr uint32_t NBAR = 20;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
@@ -67,6 +70,7 @@ struct Params {
   const float* lam_in;   // step-1 log-decay sums [B,H,nc,Q] (step modes)
   const float* dt;
   int64_t sdt, lddt;  // batch and token strides of dt
+  int input_dt;       // the input term is dt_t B_t x_t^T
   const float* A;
   const float* D;
   const float* init;
@@ -183,6 +187,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t sbase = smem_u32(sm);
   float* lamb = reinterpret_cast<float*>(sm + OFF_LAM);
   float* ecolb = reinterpret_cast<float*>(sm + OFF_ECOL);
+  float* dtsb = reinterpret_cast<float*>(sm + OFF_DTS);
   float* wtot = reinterpret_cast<float*>(sm + OFF_WTOT);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
@@ -405,13 +410,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       // lam is kept in log2 units (lam * log2 e) so every decay is one ex2
       float* lj = lamb + slot * T;
       float* ec = ecolb + slot * T;
+      float* dts = dtsb + slot * T;
       lj[2 * a] = lam0 * kLog2e;
       lj[2 * a + 1] = lam1 * kLog2e;
+      // the input term's factor per column: dt_s with the flag, else 1 (exact)
+      const bool xdt = p.input_dt && !chunked;
+      const float f0 = xdt ? d0 : 1.f, f1 = xdt ? d1 : 1.f;
+      dts[2 * a] = f0;
+      dts[2 * a + 1] = f1;
       named_sync(1, AUX);
-      // decay from each column s to the last column of its 32-block
+      // decay from each column s to the last column of its 32-block (times the
+      // column's input factor, which every product with column s carries)
       const float lr = lj[(2 * a) | 31];
-      ec[2 * a] = ex2(lr - lj[2 * a]);
-      ec[2 * a + 1] = ex2(lr - lj[2 * a + 1]);
+      ec[2 * a] = ex2(lr - lj[2 * a]) * f0;
+      ec[2 * a + 1] = ex2(lr - lj[2 * a + 1]) * f1;
       mbar_arrive(&bar[LAMRDY0 + slot]);
       if (a == 0) mark(j, EV_LAM_READY);
       d0 = n0;
@@ -429,7 +441,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
           const int row = a + 64 * rr;
-          const float w = ex2(lam_end - lj[row]);
+          const float w = ex2(lam_end - lj[row]) * dts[row];
           uint4 v4[8];
 #pragma unroll
           for (int c = 0; c < 8; ++c) v4[c] = src[swz128(row, c * 8) >> 4];
@@ -467,6 +479,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t tS = tl + buf * 256;
       const float4* ec4 = reinterpret_cast<const float4*>(ec);
       const float4* lj4 = reinterpret_cast<const float4*>(lj);
+      const float4* dt4 = reinterpret_cast<const float4*>(dtsb + slot * T);
       // P block kb (32 columns) of this row from the S values r[0..31]
       auto make_block = [&](int kb, const uint32_t* r, uint32_t* pk) {
         if (kb < q) {
@@ -489,8 +502,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
             const float4 l = lj4[8 * kb + v];
-            const float e0 = ex2(fminf(lam_t - l.x, 0.f)), e1 = ex2(fminf(lam_t - l.y, 0.f));
-            const float e2 = ex2(fminf(lam_t - l.z, 0.f)), e3 = ex2(fminf(lam_t - l.w, 0.f));
+            const float4 fx = dt4[8 * kb + v];  // the columns' input factors (1 without the flag)
+            const float e0 = ex2(fminf(lam_t - l.x, 0.f)) * fx.x, e1 = ex2(fminf(lam_t - l.y, 0.f)) * fx.y;
+            const float e2 = ex2(fminf(lam_t - l.z, 0.f)) * fx.z, e3 = ex2(fminf(lam_t - l.w, 0.f)) * fx.w;
             const float f0 = (4 * v + 0 <= rl) ? __uint_as_float(r[4 * v + 0]) * e0 : 0.f;
             const float f1 = (4 * v + 1 <= rl) ? __uint_as_float(r[4 * v + 1]) * e1 : 0.f;
             const float f2 = (4 * v + 2 <= rl) ? __uint_as_float(r[4 * v + 2]) * e2 : 0.f;
@@ -737,6 +751,7 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   kp.dt = p.dt;
   kp.sdt = p.sdt;
   kp.lddt = p.lddt;
+  kp.input_dt = p.input_dt;
   kp.A = p.A;
   kp.D = p.D;
   kp.init = init;

@@ -56,6 +56,7 @@ extern "C" ssd_status ssd_scan_fwd_noalloc(const ssd_dims* d, const void* x, con
   using namespace ssd;
   ssd_status s = validate_dims(d);
   if (s != SSD_OK) return s;
+  if (d->flags & SSD_FLAG_INPUT_DT) return SSD_ERR_UNSUPPORTED;  // the step-by-step path
   s = validate_scan_args(d, x, dt, A, Bm, Cm, D, init_state, y, final_state);
   if (s != SSD_OK) return s;
   Problem p = make_problem(d);

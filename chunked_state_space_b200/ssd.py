@@ -40,7 +40,7 @@ class SSDError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int64),
                 ("headdim", ctypes.c_int64), ("dstate", ctypes.c_int64), ("ngroups", ctypes.c_int64),
-                ("chunk", ctypes.c_int64), ("io_dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("chunk", ctypes.c_int64), ("io_dtype", ctypes.c_int32), ("flags", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p
@@ -124,12 +124,15 @@ def _io_code(t: torch.Tensor) -> int:
     raise SSDError(3, f"unsupported io dtype {t.dtype}")
 
 
-def make_dims(x: torch.Tensor, Bm: torch.Tensor, chunk: int) -> Dims:
+FLAG_INPUT_DT = 1  # SSD_FLAG_INPUT_DT: the input term is dt_t B_t x_t^T
+
+
+def make_dims(x: torch.Tensor, Bm: torch.Tensor, chunk: int, input_dt: bool = False) -> Dims:
     if x.dim() != 4 or Bm.dim() != 4:
         raise SSDError(2, "x must be [B,L,H,P] and B/C [B,L,G,N]")
     Bz, L, H, P = x.shape
     G, N = Bm.shape[2], Bm.shape[3]
-    return Dims(Bz, L, H, P, N, G, int(chunk), _io_code(x), 0)
+    return Dims(Bz, L, H, P, N, G, int(chunk), _io_code(x), FLAG_INPUT_DT if input_dt else 0)
 
 
 def _contig(*ts):
@@ -161,10 +164,11 @@ def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]):
 
 
 def ssd_scan_fwd(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, y=None, final_state=None,
-                 workspace=None, stream=None, want_final: bool = True, unfused: bool = False):
-    """y, final_state = scan(x, dt, A, B, C, D, init_state) with chunk size `chunk`."""
+                 workspace=None, stream=None, want_final: bool = True, unfused: bool = False, input_dt: bool = False):
+    """y, final_state = scan(x, dt, A, B, C, D, init_state) with chunk size `chunk`.
+    input_dt: the input term is dt_t B_t x_t^T (tensor-core path)."""
     _contig(x, dt, A, Bm, Cm, D, init_state, y, final_state)
-    dims = make_dims(x, Bm, chunk)
+    dims = make_dims(x, Bm, chunk, input_dt)
     if y is None:
         y = torch.empty_like(x)
     if final_state is None and want_final:
@@ -187,7 +191,7 @@ def ssd_scan_fwd_host_workspace_size(dims: Dims) -> int:
 
 
 def ssd_scan_fwd_host(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, y=None, final_state=None,
-                      workspace=None, stream=None, want_final: bool = True, device=None):
+                      workspace=None, stream=None, want_final: bool = True, device=None, input_dt: bool = False):
     """ssd_scan_fwd on HOST tensors (pinned for overlapped copies): the batch streams
     through a device workspace one sequence at a time.  Returns host (y, final_state);
     they are complete once `stream` (default: the current stream) has finished."""
@@ -195,7 +199,7 @@ def ssd_scan_fwd_host(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 25
         if t is not None and t.is_cuda:
             raise SSDError(1, "ssd_scan_fwd_host takes host tensors")
     _contig(x, dt, A, Bm, Cm, D, init_state, y, final_state)
-    dims = make_dims(x, Bm, chunk)
+    dims = make_dims(x, Bm, chunk, input_dt)
     pin = x.is_pinned()
     if y is None:
         y = torch.empty(x.shape, dtype=x.dtype, pin_memory=pin)
@@ -211,7 +215,7 @@ def ssd_scan_fwd_host(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 25
 
 
 def ssd_scan_fwd_strided(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, y=None, final_state=None,
-                         stream=None, want_final: bool = True):
+                         stream=None, want_final: bool = True, input_dt: bool = False):
     """ssd_scan_fwd on strided views (tensor-core path): x [B,L,H,P], dt [B,L,H],
     B/C [B,L,G,N] and y may have any batch and token strides as long as each
     token's heads (groups) are dense, e.g. slices of one fused projection output.
@@ -222,7 +226,7 @@ def ssd_scan_fwd_strided(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int =
         if tuple(t.stride()[2:]) != inner:
             raise SSDError(2, "each token's heads/groups must be dense")
     _contig(A, D, init_state, final_state)
-    dims = make_dims(x, Bm, chunk)
+    dims = make_dims(x, Bm, chunk, input_dt)
     if y is None:
         y = torch.empty(x.shape, dtype=x.dtype, device=x.device)
     if final_state is None and want_final:
@@ -299,11 +303,11 @@ def ssd_vertical_workspace_size(dims: Dims, n_layers: int, vblock: int) -> int:
 
 
 def ssd_vertical_fwd(x0, layers: Sequence[dict], states: Sequence[torch.Tensor], vblock: int, chunk: int = 256,
-                     rms_eps: float = 1e-6, y_out=None, workspace=None, stream=None):
+                     rms_eps: float = 1e-6, y_out=None, workspace=None, stream=None, input_dt: bool = False):
     """Depth-first multi-layer schedule.  layers[l] has dt, A, B, C and optionally D;
     states[l] ([B,H,N,P] f32) holds layer l's initial state and receives its final state."""
     n = len(layers)
-    dims = make_dims(x0, layers[0]["B"], chunk)
+    dims = make_dims(x0, layers[0]["B"], chunk, input_dt)
     _contig(x0, *[t for p in layers for t in (p["dt"], p["A"], p["B"], p["C"], p.get("D"))], *states)
     if y_out is None:
         y_out = torch.empty_like(x0)
@@ -320,13 +324,13 @@ def ssd_vertical_fwd(x0, layers: Sequence[dict], states: Sequence[torch.Tensor],
     return y_out
 
 
-def ssd_step(x, dt, A, Bm, Cm, state, D=None, y=None, stream=None):
+def ssd_step(x, dt, A, Bm, Cm, state, D=None, y=None, stream=None, input_dt: bool = False):
     """One decode step: x [B,H,P], dt [B,H], A [H], B/C [B,G,N], state [B,H,N,P] f32
     (updated in place).  Returns y [B,H,P]."""
     _contig(x, dt, A, Bm, Cm, D, state, y)
     Bz, H, P = x.shape
     G, N = Bm.shape[1], Bm.shape[2]
-    dims = Dims(Bz, 1, H, P, N, G, 1, _io_code(x), 0)
+    dims = Dims(Bz, 1, H, P, N, G, 1, _io_code(x), FLAG_INPUT_DT if input_dt else 0)
     if y is None:
         y = torch.empty_like(x)
     _check(lib().ssd_step(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D), _ptr(state),

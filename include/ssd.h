@@ -64,7 +64,8 @@ typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
 /*
  * Problem sizes.  Supported: batch, seqlen >= 1; 1 <= headdim (P) <= 64;
  * 1 <= dstate (N) <= 128; 1 <= chunk (Q) <= 256; ngroups >= 1 dividing nheads.
- * io_dtype is the dtype of x, Bm, Cm and y.  reserved must be 0.
+ * io_dtype is the dtype of x, Bm, Cm and y.  flags: 0 or SSD_FLAG_INPUT_DT
+ * (any other bit is SSD_ERR_INVALID_ARG).
  */
 typedef struct ssd_dims {
   int64_t batch;    /* B */
@@ -75,8 +76,19 @@ typedef struct ssd_dims {
   int64_t ngroups;  /* G */
   int64_t chunk;    /* Q */
   int32_t io_dtype; /* ssd_dtype */
-  int32_t reserved;
+  int32_t flags;    /* ssd_flags */
 } ssd_dims;
+
+/*
+ * SSD_FLAG_INPUT_DT: the input enters scaled by dt, h_t = a_t h_{t-1} +
+ * dt_t B_t x_t^T (the discretisation of the selective-scan page: the
+ * input-dependent step Delta scales the input term as well as the decay);
+ * the skip stays D_h x_t with the unscaled x.  Taken by ssd_scan_fwd,
+ * ssd_scan_fwd_strided, ssd_scan_fwd_host and ssd_vertical_fwd when the
+ * tensor-core path takes the shape, and by ssd_step; every other entry point
+ * (and ssd_scan_fwd on the CUDA-core path) returns SSD_ERR_UNSUPPORTED.
+ */
+typedef enum { SSD_FLAG_INPUT_DT = 1 } ssd_flags;
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* ssd_status_string(ssd_status s);

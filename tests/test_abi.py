@@ -51,7 +51,7 @@ def test_status_strings_and_version(lib):
 
 def dims(**kw):
     d = dict(batch=2, seqlen=1000, nheads=4, headdim=64, dstate=128, ngroups=2, chunk=256, io_dtype=1,
-             reserved=0)
+             flags=0)
     d.update(kw)
     return ssd.Dims(**d)
 
@@ -65,7 +65,7 @@ def ws_size(d):
 @pytest.mark.parametrize("kw,status", [
     (dict(batch=0), 2), (dict(seqlen=0), 2), (dict(nheads=3), 2), (dict(ngroups=0), 2),
     (dict(headdim=65), 5), (dict(dstate=129), 5), (dict(chunk=257), 5), (dict(io_dtype=2), 3),
-    (dict(reserved=1), 1), (dict(nheads=70000, ngroups=1), 5),
+    (dict(flags=2), 1), (dict(nheads=70000, ngroups=1), 5),
 ])
 def test_workspace_size_rejects(lib, kw, status):
     s, _ = ws_size(dims(**kw))
@@ -190,3 +190,17 @@ def test_strided_entry_rejects(lib):
     assert f(x=BASE + 8) == 4                                    # misaligned pointer
     assert f(y=BASE + 2 * H * P) == 1                            # y overlaps the inputs
     assert f(x=0) == 1                                           # NULL x
+
+
+def test_input_dt_flag_only_on_the_tensor_core_path(lib):
+    fl = dict(flags=1)
+    # bf16, P 64, N 128, Q 256: the tensor-core path takes it (validation passes; no launch here)
+    assert call_scan(dims(**fl), x=None) == 1
+    # the CUDA-core path does not take the flag
+    assert call_scan(dims(headdim=32, **fl)) == 5
+    assert call_scan(dims(io_dtype=0, **fl)) == 5
+    d = dims(**fl)
+    p = ctypes.c_void_p(BASE)
+    assert lib.ssd_chunk_cumsum(ctypes.byref(d), p, p, p, None) == 5
+    ptrs = [ctypes.c_void_p(BASE + k * GB) for k in (0, 2, 3, 4, 5, 6, 7, 8, 9, 10)]  # as in call_scan
+    assert lib.ssd_scan_fwd_unfused(ctypes.byref(d), *ptrs, 1 << 40, None) == 5

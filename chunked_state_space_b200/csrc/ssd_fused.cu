@@ -177,6 +177,9 @@ __device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
 
+// XDT: the dt-scaled input variant, a separate instantiation so that the plain
+// scan carries none of its per-column factors.
+template <bool XDT>
 __global__ void __launch_bounds__(THREADS, 1)
     k_ssd_fused(Params p, const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
                 const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_y) {
@@ -413,17 +416,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       float* dts = dtsb + slot * T;
       lj[2 * a] = lam0 * kLog2e;
       lj[2 * a + 1] = lam1 * kLog2e;
-      // the input term's factor per column: dt_s with the flag, else 1 (exact)
-      const bool xdt = p.input_dt && !chunked;
-      const float f0 = xdt ? d0 : 1.f, f1 = xdt ? d1 : 1.f;
-      dts[2 * a] = f0;
-      dts[2 * a + 1] = f1;
+      if constexpr (XDT) {  // the input term's factor per column: dt_s
+        dts[2 * a] = d0;
+        dts[2 * a + 1] = d1;
+      }
       named_sync(1, AUX);
       // decay from each column s to the last column of its 32-block (times the
       // column's input factor, which every product with column s carries)
       const float lr = lj[(2 * a) | 31];
-      ec[2 * a] = ex2(lr - lj[2 * a]) * f0;
-      ec[2 * a + 1] = ex2(lr - lj[2 * a + 1]) * f1;
+      ec[2 * a] = ex2(lr - lj[2 * a]);
+      ec[2 * a + 1] = ex2(lr - lj[2 * a + 1]);
+      if constexpr (XDT) {
+        ec[2 * a] *= d0;
+        ec[2 * a + 1] *= d1;
+      }
       mbar_arrive(&bar[LAMRDY0 + slot]);
       if (a == 0) mark(j, EV_LAM_READY);
       d0 = n0;
@@ -441,7 +447,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
           const int row = a + 64 * rr;
-          const float w = ex2(lam_end - lj[row]) * dts[row];
+          float w = ex2(lam_end - lj[row]);
+          if constexpr (XDT) w *= dts[row];
           uint4 v4[8];
 #pragma unroll
           for (int c = 0; c < 8; ++c) v4[c] = src[swz128(row, c * 8) >> 4];
@@ -502,9 +509,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
             const float4 l = lj4[8 * kb + v];
-            const float4 fx = dt4[8 * kb + v];  // the columns' input factors (1 without the flag)
-            const float e0 = ex2(fminf(lam_t - l.x, 0.f)) * fx.x, e1 = ex2(fminf(lam_t - l.y, 0.f)) * fx.y;
-            const float e2 = ex2(fminf(lam_t - l.z, 0.f)) * fx.z, e3 = ex2(fminf(lam_t - l.w, 0.f)) * fx.w;
+            float e0 = ex2(fminf(lam_t - l.x, 0.f)), e1 = ex2(fminf(lam_t - l.y, 0.f));
+            float e2 = ex2(fminf(lam_t - l.z, 0.f)), e3 = ex2(fminf(lam_t - l.w, 0.f));
+            if constexpr (XDT) {  // the columns' input factors
+              const float4 fx = dt4[8 * kb + v];
+              e0 *= fx.x; e1 *= fx.y; e2 *= fx.z; e3 *= fx.w;
+            }
             const float f0 = (4 * v + 0 <= rl) ? __uint_as_float(r[4 * v + 0]) * e0 : 0.f;
             const float f1 = (4 * v + 1 <= rl) ? __uint_as_float(r[4 * v + 1]) * e1 : 0.f;
             const float f2 = (4 * v + 2 <= rl) ? __uint_as_float(r[4 * v + 2]) * e2 : 0.f;
@@ -771,12 +781,17 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   if (e != cudaSuccess) return e;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set.load() & bit)) {
-    e = cudaFuncSetAttribute(k_ssd_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    e = cudaFuncSetAttribute(k_ssd_fused<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_ssd_fused<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set.fetch_or(bit);
   }
   const int64_t ctas = mode == fused::MODE_SCAN ? p.B * p.H : p.B * p.H * p.nc;
-  k_ssd_fused<<<(unsigned)ctas, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+  if (p.input_dt && mode == fused::MODE_SCAN)
+    k_ssd_fused<true><<<(unsigned)ctas, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+  else
+    k_ssd_fused<false><<<(unsigned)ctas, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
   return cudaGetLastError();
 }
 

@@ -96,6 +96,23 @@ def test_golden_scalar_recurrence():
         np.testing.assert_allclose(out["final"].ravel(), g["final"], rtol=0, atol=1e-14)
 
 
+def test_golden_scalar_recurrence_input_dt():
+    g = _read_golden("scalar_recurrence_input_dt.txt")
+    L = len(g["dt"])
+    x = g["x"].reshape(1, L, 1, 1)
+    dt = g["dt"].reshape(1, L, 1)
+    Bm = g["B"].reshape(1, L, 1, 1)
+    Cm = g["C"].reshape(1, L, 1, 1)
+    h0 = g["h0"].reshape(1, 1, 1, 1)
+    y, fin = oracle.scan_recurrence(x, dt, g["A"], Bm, Cm, g["D"], h0, input_dt=True)
+    np.testing.assert_allclose(y.ravel(), g["y"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(fin.ravel(), g["final"], rtol=0, atol=1e-14)
+    for Q in (1, 2, 3, 4):
+        out = oracle.scan_chunked(x, dt, g["A"], Bm, Cm, Q, g["D"], h0, input_dt=True)
+        np.testing.assert_allclose(out["y"].ravel(), g["y"], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(out["final"].ravel(), g["final"], rtol=0, atol=1e-14)
+
+
 def test_golden_outer_product_orientation():
     g = _read_golden("outer_product_orientation.txt")
     N, P = int(g["N"][0]), int(g["P"][0])

@@ -101,6 +101,16 @@ def _pins(o):
         return True
     check("input_dt_chunked", input_dt_chunked)
 
+    gd = _read_golden("scalar_recurrence_input_dt.txt")
+
+    def golden_input_dt():
+        Ld = len(gd["dt"])
+        y, f = oracle.scan_recurrence(gd["x"].reshape(1, Ld, 1, 1), gd["dt"].reshape(1, Ld, 1), gd["A"],
+                                      gd["B"].reshape(1, Ld, 1, 1), gd["C"].reshape(1, Ld, 1, 1), gd["D"],
+                                      gd["h0"].reshape(1, 1, 1, 1), o=o, input_dt=True)
+        return np.allclose(y.ravel(), gd["y"], atol=1e-12) and np.allclose(f.ravel(), gd["final"], atol=1e-12)
+    check("golden_input_dt", golden_input_dt)
+
     def lam():
         out = oracle.scan_chunked(p["x"], p["dt"], p["A"], p["Bm"], p["Cm"], 5, p["D"], p["init"], o=o)
         a = np.exp(p["dt"][0, :5, 0] * p["A"][0])

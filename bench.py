@@ -253,6 +253,10 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--batch", type=int, default=None, help="override the batch size (profiling runs)")
     ap.add_argument("--vblock", type=int, default=None, help="override the vertical block V (layer stacks)")
+    ap.add_argument("--input-dt", action="store_true",
+                    help="the dt-scaled input variant (SSD_FLAG_INPUT_DT)")
+    ap.add_argument("--strided", action="store_true",
+                    help="x, B, C as column slices of one fused [B, L, H*P + 2*G*N] tensor (ssd_scan_fwd_strided)")
     ap.add_argument("--no-extras", action="store_true",
                     help="layer stacks: skip the horizontal and graph-replay figures (sweeps)")
     args = ap.parse_args()
@@ -297,7 +301,21 @@ def main():
 
     def step():
         ssd.ssd_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init"], chunk=wl.chunk, y=y,
-                         final_state=fin, workspace=ws, stream=stream)
+                         final_state=fin, workspace=ws, stream=stream, input_dt=args.input_dt)
+
+    if args.strided:  # x, B, C as views of one fused projection output
+        HP, GN = wl.nheads * wl.headdim, wl.ngroups * wl.dstate
+        xbc = torch.empty((wl.batch, wl.seqlen, HP + 2 * GN), dtype=d["x"].dtype, device=dev)
+        xbc[:, :, :HP] = d["x"].reshape(wl.batch, wl.seqlen, HP)
+        xbc[:, :, HP:HP + GN] = d["B"].reshape(wl.batch, wl.seqlen, GN)
+        xbc[:, :, HP + GN:] = d["C"].reshape(wl.batch, wl.seqlen, GN)
+        xv = xbc[:, :, :HP].unflatten(2, (wl.nheads, wl.headdim))
+        bv = xbc[:, :, HP:HP + GN].unflatten(2, (wl.ngroups, wl.dstate))
+        cv = xbc[:, :, HP + GN:].unflatten(2, (wl.ngroups, wl.dstate))
+
+        def step():  # noqa: F811
+            ssd.ssd_scan_fwd_strided(xv, d["dt"], d["A"], bv, cv, d["D"], d["init"], chunk=wl.chunk, y=y,
+                                     final_state=fin, stream=stream, input_dt=args.input_dt)
 
     path, kernels_per_step = ssd.ssd_scan_path(dims)
     flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev) if l2_resident(wl) else None
@@ -321,7 +339,7 @@ def main():
     def e2e_step():
         ssd.ssd_scan_fwd_host(pinned["x"], pinned["dt"], pinned["A"], pinned["B"], pinned["C"], pinned["D"],
                               pinned["init"], chunk=wl.chunk, y=h_y, final_state=h_fin, workspace=host_ws,
-                              stream=stream)
+                              stream=stream, input_dt=args.input_dt)
 
     e2e_step()  # creates the copy streams outside the timed region
     torch.cuda.synchronize(dev)
@@ -356,6 +374,7 @@ def main():
         "config": {"workload": wl.name, "batch": wl.batch, "seqlen": wl.seqlen, "nheads": wl.nheads,
                    "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk,
                    "state_dtype": "f32", "path": path, "parallelism": f"dp{world} (independent batches per rank)",
+                   "variant": ("input_dt " if args.input_dt else "") + ("strided" if args.strided else "") or "plain",
                    "l2": ("512 MB L2 flush between steps (inputs fit in L2); per-step events exclude it"
                           if flush is not None else
                           f"inputs larger than L2 ({algorithmic_bytes(wl) / 1e9:.2f} GB per rank); no flush")},

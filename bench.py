@@ -84,15 +84,19 @@ def load_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-FUSED_KERNEL_SOURCES = ("ssd_fused.cu", "ssd_common.cuh", "ssd_tc.cuh", "tma.cuh", "umma.cuh")
+KERNEL_SOURCES = {
+    "ssd_fused": ("ssd_fused.cu", "ssd_common.cuh", "ssd_tc.cuh", "tma.cuh", "umma.cuh"),
+    "ssd_pair": ("ssd_pair.cu", "ssd_common.cuh", "ssd_tc.cuh", "tma.cuh", "umma.cuh"),
+}
+PATH_KERNEL = {"fused": "ssd_fused", "fused_pair": "ssd_pair"}
 
 
-def kernel_source_hash() -> str:
-    """Hash of the sources the fused kernel is compiled from (its file and the
+def kernel_source_hash(kernel: str = "ssd_fused") -> str:
+    """Hash of the sources a fused kernel is compiled from (its file and the
     headers it includes): a recorded ncu traffic figure applies while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "chunked_state_space_b200", "csrc")
-    for name in FUSED_KERNEL_SOURCES:
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -108,7 +112,7 @@ def traffic_from_profile(kernel: str):
         with open(path) as f:
             t = json.load(f)
         ent = t.get(kernel)
-        if ent and ent.get("source_hash") == kernel_source_hash():
+        if ent and ent.get("source_hash") == kernel_source_hash(kernel):
             return float(ent["dram_bytes_per_launch"])
     except Exception:
         return None
@@ -257,6 +261,8 @@ def main():
                     help="the dt-scaled input variant (SSD_FLAG_INPUT_DT)")
     ap.add_argument("--strided", action="store_true",
                     help="x, B, C as column slices of one fused [B, L, H*P + 2*G*N] tensor (ssd_scan_fwd_strided)")
+    ap.add_argument("--one-head", action="store_true",
+                    help="the one-head-per-CTA fused kernel even where the two-head kernel applies (comparison)")
     ap.add_argument("--no-extras", action="store_true",
                     help="layer stacks: skip the horizontal and graph-replay figures (sweeps)")
     args = ap.parse_args()
@@ -294,14 +300,15 @@ def main():
     d = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
     y = torch.empty_like(d["x"])
     fin = torch.empty((wl.batch, wl.nheads, wl.dstate, wl.headdim), dtype=torch.float32, device=dev)
-    dims = ssd.make_dims(d["x"], d["B"], wl.chunk)
+    dims = ssd.make_dims(d["x"], d["B"], wl.chunk, args.input_dt, args.one_head)
     ws = torch.empty(max(ssd.ssd_scan_workspace_size(dims), 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     torch.cuda.synchronize(dev)
 
     def step():
         ssd.ssd_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init"], chunk=wl.chunk, y=y,
-                         final_state=fin, workspace=ws, stream=stream, input_dt=args.input_dt)
+                         final_state=fin, workspace=ws, stream=stream, input_dt=args.input_dt,
+                         one_head=args.one_head)
 
     if args.strided:  # x, B, C as views of one fused projection output
         HP, GN = wl.nheads * wl.headdim, wl.ngroups * wl.dstate
@@ -315,7 +322,8 @@ def main():
 
         def step():  # noqa: F811
             ssd.ssd_scan_fwd_strided(xv, d["dt"], d["A"], bv, cv, d["D"], d["init"], chunk=wl.chunk, y=y,
-                                     final_state=fin, stream=stream, input_dt=args.input_dt)
+                                     final_state=fin, stream=stream, input_dt=args.input_dt,
+                                     one_head=args.one_head)
 
     path, kernels_per_step = ssd.ssd_scan_path(dims)
     flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev) if l2_resident(wl) else None
@@ -354,12 +362,13 @@ def main():
     e2e_value = tokens / (e2e_ms * 1e-3)
 
     hbm_peak, tc_peak, tc_sust, peak_src = load_peaks()
-    kernel_ms = statistics.mean(per_step) if path == "fused" and kernels_per_step == 1 else None
+    kernel_ms = statistics.mean(per_step) if path in ssd.FUSED_PATHS and kernels_per_step == 1 else None
     roofline = None
     if kernel_ms is not None:
+        kname = PATH_KERNEL[path]
         ach = algorithmic_bytes(wl) / (kernel_ms * 1e-3) / 1e9
         roofline = {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
-                    "traffic": traffic_from_profile("ssd_fused"), "kernel": "ssd_fused",
+                    "traffic": traffic_from_profile(kname), "kernel": "k_" + kname,
                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else
                     "fallback 6650 GB/s",
                     "tensor_tflops": algorithmic_flops(wl) / (kernel_ms * 1e-3) / 1e12,
@@ -374,7 +383,8 @@ def main():
         "config": {"workload": wl.name, "batch": wl.batch, "seqlen": wl.seqlen, "nheads": wl.nheads,
                    "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk,
                    "state_dtype": "f32", "path": path, "parallelism": f"dp{world} (independent batches per rank)",
-                   "variant": ("input_dt " if args.input_dt else "") + ("strided" if args.strided else "") or "plain",
+                   "variant": (("input_dt " if args.input_dt else "") + ("strided " if args.strided else "") +
+                               ("one_head" if args.one_head else "")).strip() or "plain",
                    "l2": ("512 MB L2 flush between steps (inputs fit in L2); per-step events exclude it"
                           if flush is not None else
                           f"inputs larger than L2 ({algorithmic_bytes(wl) / 1e9:.2f} GB per rank); no flush")},

@@ -24,7 +24,7 @@ size_t io_size(int io) { return io == SSD_BF16 ? 2 : 4; }
 
 ssd_status validate_dims(const ssd_dims* d) {
   if (!d) return SSD_ERR_INVALID_ARG;
-  if ((d->flags & ~SSD_FLAG_INPUT_DT) != 0) return SSD_ERR_INVALID_ARG;
+  if ((d->flags & ~(SSD_FLAG_INPUT_DT | SSD_FLAG_ONE_HEAD_PER_CTA)) != 0) return SSD_ERR_INVALID_ARG;
   if (d->io_dtype != SSD_F32 && d->io_dtype != SSD_BF16) return SSD_ERR_DTYPE;
   if (d->batch < 1 || d->seqlen < 1 || d->nheads < 1 || d->headdim < 1 || d->dstate < 1 || d->ngroups < 1 ||
       d->chunk < 1)
@@ -57,6 +57,7 @@ Problem make_problem(const ssd_dims* d) {
   p.lddt = p.H;
   p.ldbc = p.G * p.N;
   p.input_dt = (d->flags & SSD_FLAG_INPUT_DT) ? 1 : 0;
+  p.single_head = (d->flags & SSD_FLAG_ONE_HEAD_PER_CTA) ? 1 : 0;
   return p;
 }
 
@@ -171,7 +172,7 @@ ssd_status ssd_scan_path(const ssd_dims* d, int32_t* path, int32_t* kernels) {
   const Problem p = make_problem(d);
   int32_t pa = SSD_PATH_CUDA_CORES, k = 4;
   if (fused_supported(p)) {
-    pa = SSD_PATH_FUSED;
+    pa = uses_pair_kernel(p) ? SSD_PATH_FUSED_PAIR : SSD_PATH_FUSED;
     k = fused_kernels_per_call(p);
   } else if (tc_supported(p)) {
     pa = SSD_PATH_TENSOR_STEPS;
@@ -210,7 +211,8 @@ ssd_status ssd_scan_fwd(const ssd_dims* d, const void* x, const float* dt, const
   if (!aligned16(workspace)) return SSD_ERR_ALIGN;
   p.x = x; p.dt = dt; p.A = A; p.Bm = Bm; p.Cm = Cm; p.D = D; p.y = y;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (fused_supported(p)) return cuda_status(launch_fused(p, init_state, final_state, workspace, st));
+  if (fused_supported(p))
+    return cuda_status(launch_fused(p, init_state, final_state, workspace, workspace_bytes, st));
   if (p.input_dt) return SSD_ERR_UNSUPPORTED;  // the dt-scaled input: tensor-core path only
   return run_unfused(p, init_state, final_state, static_cast<char*>(workspace), st);
 }
@@ -251,7 +253,7 @@ ssd_status ssd_scan_fwd_strided(const ssd_dims* d, const void* x, int64_t x_bstr
   p.sdt = dt_bstride; p.lddt = dt_tstride;
   p.sbc = bc_bstride; p.ldbc = bc_tstride;
   p.sy = y_bstride; p.ldy = y_tstride;
-  return cuda_status(launch_fused(p, init_state, final_state, nullptr, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_fused(p, init_state, final_state, nullptr, 0, static_cast<cudaStream_t>(stream)));
 }
 
 ssd_status ssd_chunk_cumsum(const ssd_dims* d, const float* dt, const float* A, float* lam, void* stream) {
@@ -471,7 +473,7 @@ static ssd_status vertical_wavefront(const ssd_dims* d_, int32_t n_layers, int64
         p.y = in_buf(l + 1, k & 1);
         p.sy = Vk * HP;
       }
-      s = cuda_status(launch_fused(p, states[l], states[l], nullptr, sl));
+      s = cuda_status(launch_fused(p, states[l], states[l], nullptr, 0, sl));
       if (s == SSD_OK && !last)
         s = cuda_status(launch_rmsnorm(d_->batch * Vk, HP, d_->io_dtype, p.y, rms_eps, p.y, sl));
       if (s != SSD_OK) break;
@@ -559,7 +561,7 @@ ssd_status ssd_vertical_fwd(const ssd_dims* d, int32_t n_layers, int64_t vblock,
         p.sy = Vk * HP;
       }
       if (fused_supported(p))
-        s = cuda_status(launch_fused(p, states[l], states[l], ws, st));
+        s = cuda_status(launch_fused(p, states[l], states[l], nullptr, 0, st));
       else
         s = run_unfused(p, states[l], states[l], ws, st);
       if (s != SSD_OK) return s;

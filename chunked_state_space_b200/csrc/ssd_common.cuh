@@ -29,7 +29,8 @@ struct Problem {
   // token strides (elements); the contiguous layout has ldx = ldy = H*P,
   // lddt = H, ldbc = G*N.  Only the fused tensor-core kernel reads them.
   int64_t ldx, lddt, ldbc, ldy;
-  int input_dt;  // SSD_FLAG_INPUT_DT: the input term is dt_t B_t x_t^T
+  int input_dt;     // SSD_FLAG_INPUT_DT: the input term is dt_t B_t x_t^T
+  int single_head;  // SSD_FLAG_ONE_HEAD_PER_CTA: never the two-head kernel
 };
 
 template <typename T>

@@ -695,6 +695,13 @@ bool tc_supported(const Problem& p) { return fused_supported(p) && p.B * p.H * p
 
 int fused_kernels_per_call(const Problem&) { return 1; }
 
+bool uses_pair_kernel(const Problem& p) { return !p.single_head && pair_supported(p); }
+
+// The one-head kernel keeps the running state on chip (whole scan) or reads and
+// writes only the caller's step tensors (step modes): no workspace.  The
+// two-head kernel needs one for its carries when it splits sequences.
+size_t tc_workspace_bytes(const Problem& p) { return uses_pair_kernel(p) ? pair_workspace_bytes(p) : 0; }
+
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
                                void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads = 0);
 
@@ -704,10 +711,13 @@ cudaError_t launch_fused_traced(const Problem& p, const float* init, float* fina
 }
 
 cudaError_t launch_fused_withheld(const Problem& p, const float* init, float* final_state, cudaStream_t st) {
+  if (uses_pair_kernel(p)) return launch_pair(p, init, final_state, nullptr, 0, st, 1);
   return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, nullptr, st, 1);
 }
 
-cudaError_t launch_fused(const Problem& p, const float* init, float* final_state, void*, cudaStream_t st) {
+cudaError_t launch_fused(const Problem& p, const float* init, float* final_state, void* workspace,
+                         size_t workspace_bytes, cudaStream_t st) {
+  if (uses_pair_kernel(p)) return launch_pair(p, init, final_state, workspace, workspace_bytes, st, 0);
   return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, nullptr, st);
 }
 

@@ -210,108 +210,24 @@ extern "C" ssd_status ssd_selftest_timeout(const ssd_dims* d, const void* x, con
   return cuda_status(launch_fused_withheld(p, init_state, final_state, static_cast<cudaStream_t>(stream)));
 }
 
-// ---------------------------------------------------------------------------
-// Micro-timing of the mask's building blocks on one CTA (4 warps, one TMEM
-// lane quarter each), away from the rest of the fused kernel: 64 repetitions
-// of one variant, SM clocks per repetition written to cycles[thread].
-//   0: two 32-column TMEM loads + wait
-//   1: variant 0 + off-diagonal block math on both blocks
-//   2: variant 1 + two 16-column TMEM stores of the packed result
-//   3: off-diagonal block math only (registers, no TMEM)
-//   4: diagonal block math only (registers, no TMEM)
-//   5: 16 shared-memory 16-byte loads of one row (the C' read)
-namespace ssd {
-__global__ void __launch_bounds__(128) k_selftest_mask_timing(int variant, long long* cycles, float* sink) {
-  using namespace umma;
-  __shared__ uint32_t tmem_slot;
-  __shared__ __align__(16) float colv[2 * 128];
-  __shared__ __align__(16) uint8_t rowbuf[32768];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < 256; i += 128) colv[i] = 0.5f + 0.001f * i;
-  for (int i = threadIdx.x; i < 32768 / 4; i += 128) reinterpret_cast<uint32_t*>(rowbuf)[i] = 0x3f803f80u + i;
-  if (warp == 0) tmem_alloc(&tmem_slot, 256);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tl = tmem_slot + ((uint32_t)(warp * 32) << 16);
-  const float* ec = colv;
-  const float* lj = colv + 128;
-  const float lam_t = 0.25f * lane;
-  const int row = warp * 32 + lane;
-  float acc = 0.f;
-  uint32_t r0[32], r1[32], pk[16];
-  for (int i = 0; i < 32; ++i) { r0[i] = __float_as_uint(1.0f + i); r1[i] = __float_as_uint(2.0f + i); }
-  auto offdiag = [&](const uint32_t* r, int kb) {
-    const float rowf = fused::ex2(lam_t - lj[32 * kb + 31]);
-    const float4* ec4 = reinterpret_cast<const float4*>(ec);
-#pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      const float4 c = ec4[8 * kb + v];
-      pk[2 * v] = pack_bf16(__uint_as_float(r[4 * v]) * (rowf * c.x), __uint_as_float(r[4 * v + 1]) * (rowf * c.y));
-      pk[2 * v + 1] = pack_bf16(__uint_as_float(r[4 * v + 2]) * (rowf * c.z), __uint_as_float(r[4 * v + 3]) * (rowf * c.w));
-    }
-  };
-  auto diag = [&](const uint32_t* r, int kb) {
-    const float4* lj4 = reinterpret_cast<const float4*>(lj);
-    const int rl = row - 32 * kb;
-#pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      const float4 l = lj4[8 * kb + v];
-      const float e0 = fused::ex2(fminf(lam_t - l.x, 0.f)), e1 = fused::ex2(fminf(lam_t - l.y, 0.f));
-      const float e2 = fused::ex2(fminf(lam_t - l.z, 0.f)), e3 = fused::ex2(fminf(lam_t - l.w, 0.f));
-      const float f0 = (4 * v + 0 <= rl) ? __uint_as_float(r[4 * v + 0]) * e0 : 0.f;
-      const float f1 = (4 * v + 1 <= rl) ? __uint_as_float(r[4 * v + 1]) * e1 : 0.f;
-      const float f2 = (4 * v + 2 <= rl) ? __uint_as_float(r[4 * v + 2]) * e2 : 0.f;
-      const float f3 = (4 * v + 3 <= rl) ? __uint_as_float(r[4 * v + 3]) * e3 : 0.f;
-      pk[2 * v] = pack_bf16(f0, f1);
-      pk[2 * v + 1] = pack_bf16(f2, f3);
-    }
-  };
-  __syncthreads();
-  const long long t0 = clock64();
-  for (int it = 0; it < 64; ++it) {
-    if (variant <= 2) {
-      tmem_ld32(tl + 0, r0);
-      tmem_ld32(tl + 32, r1);
-      tmem_wait_ld();
-    }
-    if (variant == 1 || variant == 2 || variant == 3) {
-      offdiag(r0, it & 1);
-      if (variant == 2) tmem_st16(tl + 128, pk);
-      for (int i = 0; i < 16; ++i) acc += __uint_as_float(pk[i] & 0xFFFF0000u);
-      offdiag(r1, (it + 1) & 1);
-      if (variant == 2) tmem_st16(tl + 144, pk);
-      for (int i = 0; i < 16; ++i) acc += __uint_as_float(pk[i] & 0xFFFF0000u);
-    } else if (variant == 4) {
-      diag(r0, it & 3);
-      for (int i = 0; i < 16; ++i) acc += __uint_as_float(pk[i] & 0xFFFF0000u);
-    } else if (variant == 5) {
-      const uint4* src = reinterpret_cast<const uint4*>(rowbuf);
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const uint4 v = src[((c >> 3) * 16384 + swz128(row, 8 * (c & 7))) >> 4];  // < 32768 bytes
-        acc += __uint_as_float(v.x) + __uint_as_float(v.w);
-      }
-    } else if (variant == 0) {
-      for (int i = 0; i < 32; ++i) acc += __uint_as_float(r0[i]) + __uint_as_float(r1[i]);
-    }
-  }
-  if (variant == 2) tmem_wait_st();
-  const long long t1 = clock64();
-  cycles[threadIdx.x] = (t1 - t0) / 64;
-  sink[threadIdx.x] = acc;
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem_slot, 256);
-    tmem_relinquish();
-  }
-}
-}  // namespace ssd
-
-extern "C" ssd_status ssd_selftest_mask_timing(int32_t variant, long long* cycles, float* sink, void* stream) {
-  if (!cycles || !sink || variant < 0 || variant > 5) return SSD_ERR_INVALID_ARG;
-  ssd::k_selftest_mask_timing<<<1, 128, 0, static_cast<cudaStream_t>(stream)>>>(variant, cycles, sink);
-  return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+// Carry path of the two-head kernel: the split schedule of ssd_scan_fwd with no
+// carry ever published, so every CTA that starts inside a sequence waits for
+// its predecessor's state until its bounded wait runs out (about two seconds),
+// records SSD_ERR_TIMEOUT and drains; nothing faults.
+extern "C" ssd_status ssd_selftest_carry_timeout(const ssd_dims* d, const void* x, const float* dt, const float* A,
+                                                 const void* Bm, const void* Cm, const float* D,
+                                                 const float* init_state, void* y, float* final_state,
+                                                 void* workspace, size_t workspace_bytes, void* stream) {
+  using namespace ssd;
+  ssd_status s = validate_dims(d);
+  if (s != SSD_OK) return s;
+  s = validate_scan_args(d, x, dt, A, Bm, Cm, D, init_state, y, final_state);
+  if (s != SSD_OK) return s;
+  Problem p = make_problem(d);
+  if (!uses_pair_kernel(p) || pair_workspace_bytes(p) == 0) return SSD_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < pair_workspace_bytes(p)) return SSD_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0) return SSD_ERR_ALIGN;
+  p.x = x; p.dt = dt; p.A = A; p.Bm = Bm; p.Cm = Cm; p.D = D; p.y = y;
+  return cuda_status(
+      launch_pair(p, init_state, final_state, workspace, workspace_bytes, static_cast<cudaStream_t>(stream), 2));
 }

@@ -8,16 +8,29 @@ namespace ssd {
 // True when the tcgen05 step kernels cover this problem (bf16 io and the
 // tile sizes they are written for).
 bool tc_supported(const Problem& p);
-// True when the fused single-pass kernel covers this problem.
+// True when a fused single-pass kernel covers this problem (the one-head
+// kernel always does; the two-head kernel when pair_supported also holds).
 bool fused_supported(const Problem& p);
+// True when the two-heads-per-CTA kernel covers it (even heads per group).
+bool pair_supported(const Problem& p);
+// True when launch_fused runs the two-head kernel for this problem.
+bool uses_pair_kernel(const Problem& p);
 // Kernel launches of one fused call.
 int fused_kernels_per_call(const Problem& p);
-// Workspace bytes the tensor-core paths need (0 if unsupported).
+// Workspace bytes the tensor-core paths need (0 if unsupported): the two-head
+// kernel's carries between CTAs when it splits sequences across them.
 size_t tc_workspace_bytes(const Problem& p);
+size_t pair_workspace_bytes(const Problem& p);
 
 cudaError_t launch_chunk_state_tc(const Problem& p, const float* lam, float* states, cudaStream_t st);
 cudaError_t launch_chunk_scan_tc(const Problem& p, const float* lam, const float* prev, cudaStream_t st);
+// The whole scan in one launch.  With a workspace of pair_workspace_bytes
+// the two-head kernel splits sequences evenly across the SMs; without one
+// (NULL / too small) every CTA runs whole sequences.
 cudaError_t launch_fused(const Problem& p, const float* init, float* final_state, void* workspace,
-                         cudaStream_t st);
+                         size_t workspace_bytes, cudaStream_t st);
+// withhold: 0 normal; 1 no TMA loads; 2 no carries published (self-tests of the bounded waits)
+cudaError_t launch_pair(const Problem& p, const float* init, float* final_state, void* workspace,
+                        size_t workspace_bytes, cudaStream_t st, int withhold);
 
 }  // namespace ssd

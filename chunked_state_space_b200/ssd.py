@@ -26,9 +26,9 @@ EXPORTED = ["ssd_status_string", "ssd_version", "ssd_scan_workspace_size", "ssd_
             "ssd_scan_fwd_unfused", "ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing",
             "ssd_chunk_scan", "ssd_rmsnorm", "ssd_vertical_workspace_size", "ssd_vertical_fwd",
             "ssd_read_device_status", "ssd_selftest_umma", "ssd_scan_path", "ssd_step",
-            "ssd_selftest_fused_trace", "ssd_scan_fwd_noalloc", "ssd_selftest_mask_timing",
+            "ssd_selftest_fused_trace", "ssd_scan_fwd_noalloc",
             "ssd_selftest_timeout", "ssd_scan_fwd_host", "ssd_scan_fwd_host_workspace_size",
-            "ssd_scan_fwd_strided"]
+            "ssd_scan_fwd_strided", "ssd_selftest_carry_timeout"]
 
 
 class SSDError(RuntimeError):
@@ -83,9 +83,9 @@ def lib() -> ctypes.CDLL:
         "ssd_scan_path": (ctypes.c_int, [D, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]),
         "ssd_step": (ctypes.c_int, [D] + [_P] * 9),
         "ssd_scan_fwd_noalloc": (ctypes.c_int, [D] + [_P] * 10),
-        "ssd_selftest_mask_timing": (ctypes.c_int, [ctypes.c_int32, _P, _P, _P]),
         "ssd_selftest_fused_trace": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_int64, _P]),
         "ssd_selftest_timeout": (ctypes.c_int, [D] + [_P] * 10),
+        "ssd_selftest_carry_timeout": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_size_t, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -124,15 +124,18 @@ def _io_code(t: torch.Tensor) -> int:
     raise SSDError(3, f"unsupported io dtype {t.dtype}")
 
 
-FLAG_INPUT_DT = 1  # SSD_FLAG_INPUT_DT: the input term is dt_t B_t x_t^T
+FLAG_INPUT_DT = 1        # SSD_FLAG_INPUT_DT: the input term is dt_t B_t x_t^T
+FLAG_ONE_HEAD_PER_CTA = 2  # SSD_FLAG_ONE_HEAD_PER_CTA: never the two-head kernel
 
 
-def make_dims(x: torch.Tensor, Bm: torch.Tensor, chunk: int, input_dt: bool = False) -> Dims:
+def make_dims(x: torch.Tensor, Bm: torch.Tensor, chunk: int, input_dt: bool = False,
+              one_head: bool = False) -> Dims:
     if x.dim() != 4 or Bm.dim() != 4:
         raise SSDError(2, "x must be [B,L,H,P] and B/C [B,L,G,N]")
     Bz, L, H, P = x.shape
     G, N = Bm.shape[2], Bm.shape[3]
-    return Dims(Bz, L, H, P, N, G, int(chunk), _io_code(x), FLAG_INPUT_DT if input_dt else 0)
+    flags = (FLAG_INPUT_DT if input_dt else 0) | (FLAG_ONE_HEAD_PER_CTA if one_head else 0)
+    return Dims(Bz, L, H, P, N, G, int(chunk), _io_code(x), flags)
 
 
 def _contig(*ts):
@@ -141,7 +144,8 @@ def _contig(*ts):
             raise SSDError(1, "tensors must be contiguous")
 
 
-PATH_NAMES = {0: "cuda_cores", 1: "tensor_steps", 2: "fused"}
+PATH_NAMES = {0: "cuda_cores", 1: "tensor_steps", 2: "fused", 3: "fused_pair"}
+FUSED_PATHS = ("fused", "fused_pair")
 
 
 def ssd_scan_path(dims: Dims):
@@ -164,11 +168,13 @@ def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]):
 
 
 def ssd_scan_fwd(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, y=None, final_state=None,
-                 workspace=None, stream=None, want_final: bool = True, unfused: bool = False, input_dt: bool = False):
+                 workspace=None, stream=None, want_final: bool = True, unfused: bool = False, input_dt: bool = False,
+                 one_head: bool = False):
     """y, final_state = scan(x, dt, A, B, C, D, init_state) with chunk size `chunk`.
-    input_dt: the input term is dt_t B_t x_t^T (tensor-core path)."""
+    input_dt: the input term is dt_t B_t x_t^T (tensor-core path).
+    one_head: the one-head-per-CTA fused kernel even where the two-head one applies."""
     _contig(x, dt, A, Bm, Cm, D, init_state, y, final_state)
-    dims = make_dims(x, Bm, chunk, input_dt)
+    dims = make_dims(x, Bm, chunk, input_dt, one_head)
     if y is None:
         y = torch.empty_like(x)
     if final_state is None and want_final:
@@ -215,7 +221,7 @@ def ssd_scan_fwd_host(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 25
 
 
 def ssd_scan_fwd_strided(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, y=None, final_state=None,
-                         stream=None, want_final: bool = True, input_dt: bool = False):
+                         stream=None, want_final: bool = True, input_dt: bool = False, one_head: bool = False):
     """ssd_scan_fwd on strided views (tensor-core path): x [B,L,H,P], dt [B,L,H],
     B/C [B,L,G,N] and y may have any batch and token strides as long as each
     token's heads (groups) are dense, e.g. slices of one fused projection output.
@@ -226,7 +232,7 @@ def ssd_scan_fwd_strided(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int =
         if tuple(t.stride()[2:]) != inner:
             raise SSDError(2, "each token's heads/groups must be dense")
     _contig(A, D, init_state, final_state)
-    dims = make_dims(x, Bm, chunk, input_dt)
+    dims = make_dims(x, Bm, chunk, input_dt, one_head)
     if y is None:
         y = torch.empty(x.shape, dtype=x.dtype, device=x.device)
     if final_state is None and want_final:
@@ -380,20 +386,27 @@ def ssd_selftest_fused_trace(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: i
     return y, fin, trace[:ntr].view(nsub, 24), trace[ntr:].view(-1, 3)
 
 
-def ssd_selftest_timeout(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, stream=None) -> None:
-    """Diagnostic: launch the fused kernel with its TMA loads withheld, so its
-    bounded waits run out; read the outcome with ssd_read_device_status."""
-    dims = make_dims(x, Bm, chunk)
+def ssd_selftest_timeout(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, stream=None,
+                         one_head: bool = False) -> None:
+    """Diagnostic: launch the fused kernel (the two-head one where it applies,
+    unless one_head) with its TMA loads withheld, so its bounded waits run out;
+    read the outcome with ssd_read_device_status."""
+    dims = make_dims(x, Bm, chunk, one_head=one_head)
     y = torch.empty_like(x)
     fin = torch.empty((dims.batch, dims.nheads, dims.dstate, dims.headdim), dtype=torch.float32, device=x.device)
     _check(lib().ssd_selftest_timeout(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D),
                                       _ptr(init_state), _ptr(y), _ptr(fin), _stream(stream)), "ssd_selftest_timeout")
 
 
-def ssd_selftest_mask_timing(variant: int, stream=None):
-    """Diagnostic: SM clocks per repetition of one mask building block (see
-    include/ssd_selftest.h), one value per thread of the 4-warp CTA."""
-    cyc = torch.zeros(128, dtype=torch.int64, device="cuda")
-    sink = torch.zeros(128, dtype=torch.float32, device="cuda")
-    _check(lib().ssd_selftest_mask_timing(variant, _ptr(cyc), _ptr(sink), _stream(stream)), "ssd_selftest_mask_timing")
-    return cyc
+def ssd_selftest_carry_timeout(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, stream=None) -> None:
+    """Diagnostic: launch the two-head kernel with its split schedule but with no
+    carry ever published, so every wait for one runs out; read the outcome with
+    ssd_read_device_status."""
+    dims = make_dims(x, Bm, chunk)
+    y = torch.empty_like(x)
+    fin = torch.empty((dims.batch, dims.nheads, dims.dstate, dims.headdim), dtype=torch.float32, device=x.device)
+    ws = _workspace(ssd_scan_workspace_size(dims), x.device, None)
+    _check(lib().ssd_selftest_carry_timeout(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm),
+                                            _ptr(D), _ptr(init_state), _ptr(y), _ptr(fin), _ptr(ws),
+                                            ws.numel() * ws.element_size(), _stream(stream)),
+           "ssd_selftest_carry_timeout")

@@ -36,6 +36,12 @@
  *    SSD_ERR_CUDA (a launch failed part-way) and SSD_ERR_TIMEOUT (reported by
  *    ssd_read_device_status after a bounded device-side wait gave up).
  *  - Results are deterministic run to run (no atomics in reductions).
+ *  - Per-device set-up: on its first call on a device the library records a
+ *    few things it keeps for the life of the process (the kernels' shared-
+ *    memory opt-in, the built-in scratch buffer's device address, the streams
+ *    and events of the wavefront and host-copy schedules).  Resetting the
+ *    device (cudaDeviceReset) after that first call is not supported: the
+ *    recorded state would belong to the destroyed context.
  */
 #ifndef SSD_B200_SSD_H
 #define SSD_B200_SSD_H
@@ -64,8 +70,8 @@ typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
 /*
  * Problem sizes.  Supported: batch, seqlen >= 1; 1 <= headdim (P) <= 64;
  * 1 <= dstate (N) <= 128; 1 <= chunk (Q) <= 256; ngroups >= 1 dividing nheads.
- * io_dtype is the dtype of x, Bm, Cm and y.  flags: 0 or SSD_FLAG_INPUT_DT
- * (any other bit is SSD_ERR_INVALID_ARG).
+ * io_dtype is the dtype of x, Bm, Cm and y.  flags: a combination of
+ * ssd_flags (any other bit is SSD_ERR_INVALID_ARG).
  */
 typedef struct ssd_dims {
   int64_t batch;    /* B */
@@ -87,8 +93,12 @@ typedef struct ssd_dims {
  * ssd_scan_fwd_strided, ssd_scan_fwd_host and ssd_vertical_fwd when the
  * tensor-core path takes the shape, and by ssd_step; every other entry point
  * (and ssd_scan_fwd on the CUDA-core path) returns SSD_ERR_UNSUPPORTED.
+ *
+ * SSD_FLAG_ONE_HEAD_PER_CTA: run the one-head-per-CTA fused kernel even where
+ * the two-head kernel takes the shape (same results within rounding; for
+ * comparing the two kernels).  Changes nothing on other paths.
  */
-typedef enum { SSD_FLAG_INPUT_DT = 1 } ssd_flags;
+typedef enum { SSD_FLAG_INPUT_DT = 1, SSD_FLAG_ONE_HEAD_PER_CTA = 2 } ssd_flags;
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* ssd_status_string(ssd_status s);
@@ -172,11 +182,16 @@ ssd_status ssd_scan_fwd_host(const ssd_dims* d, const void* x, const float* dt, 
 /*
  * Which implementation ssd_scan_fwd uses for `d`: *path = SSD_PATH_CUDA_CORES
  * (four CUDA-core step kernels), SSD_PATH_TENSOR_STEPS (four step kernels,
- * steps 2 and 4 on tcgen05 tensor cores) or SSD_PATH_FUSED (one persistent
- * tensor-core kernel); *kernels = kernel launches per call.  Either output
- * pointer may be NULL.  Errors: as ssd_scan_workspace_size.
+ * steps 2 and 4 on tcgen05 tensor cores), SSD_PATH_FUSED (one tensor-core
+ * kernel, one (batch, head) sequence per CTA) or SSD_PATH_FUSED_PAIR (one
+ * tensor-core kernel, two heads of a group per CTA sharing their B and C
+ * tiles; with the workspace of ssd_scan_workspace_size it cuts the
+ * concatenated sequences into equal ranges, one persistent CTA per SM, and
+ * hands the state across range boundaries through the workspace);
+ * *kernels = kernel launches per call.  Either output pointer may be NULL.
+ * Errors: as ssd_scan_workspace_size.
  */
-enum { SSD_PATH_CUDA_CORES = 0, SSD_PATH_TENSOR_STEPS = 1, SSD_PATH_FUSED = 2 };
+enum { SSD_PATH_CUDA_CORES = 0, SSD_PATH_TENSOR_STEPS = 1, SSD_PATH_FUSED = 2, SSD_PATH_FUSED_PAIR = 3 };
 ssd_status ssd_scan_path(const ssd_dims* d, int32_t* path, int32_t* kernels);
 
 /* The same computation, forced through the four separate step kernels below
@@ -199,7 +214,8 @@ ssd_status ssd_scan_fwd_unfused(const ssd_dims* d, const void* x, const float* d
  *   - The call allocates nothing (no cudaMalloc or cudaFree, no allocating
  *     library routine).  Its first call on a device looks up the buffer's
  *     device address with that device current; make that first call before
- *     any stream capture.
+ *     any stream capture, and do not reset the device afterwards (the address
+ *     is kept per device for the life of the process).
  *   - Every call shares the buffer and it keeps the last call's contents;
  *     nothing in it needs to start at zero (each call writes the scratch it
  *     reads).  Calls whose executions overlap on the GPU (other streams,

@@ -61,20 +61,11 @@ ssd_status ssd_selftest_fused_trace(const ssd_dims* d, const void* x, const floa
                                     void* stream);
 
 /*
- * ssd_selftest_mask_timing times, on one CTA of 4 warps, 64 repetitions of one
- * building block of the fused kernel's mask (variant 0: two 32-column TMEM
- * loads; 1: plus the off-diagonal block arithmetic; 2: plus two 16-column
- * TMEM stores; 3: off-diagonal arithmetic alone; 4: diagonal-block arithmetic
- * alone; 5: sixteen 16-byte shared-memory row loads) and writes the SM clocks
- * per repetition of each thread to cycles[128] (device int64); sink[128]
- * (device f32) receives a checksum that keeps the work alive.
- */
-ssd_status ssd_selftest_mask_timing(int32_t variant, long long* cycles, float* sink, void* stream);
-
-/*
  * ssd_selftest_timeout exercises the bounded waits of ssd_scan_fwd's fused
- * tensor-core kernel: same arguments and validation as ssd_scan_fwd (the
- * problem must be one the fused kernel takes, else SSD_ERR_UNSUPPORTED), but
+ * tensor-core kernel (the two-head kernel where it takes the shape, unless
+ * d->flags has SSD_FLAG_ONE_HEAD_PER_CTA; else the one-head kernel): same
+ * arguments and validation as ssd_scan_fwd (the problem must be one a fused
+ * kernel takes, else SSD_ERR_UNSUPPORTED), but
  * the kernel issues none of its TMA loads, so every wait on them gives up
  * after about one second.  The launch itself returns SSD_OK; the following
  * ssd_read_device_status(stream) must return SSD_ERR_TIMEOUT (and clears the
@@ -85,6 +76,24 @@ ssd_status ssd_selftest_mask_timing(int32_t variant, long long* cycles, float* s
 ssd_status ssd_selftest_timeout(const ssd_dims* d, const void* x, const float* dt, const float* A, const void* Bm,
                                 const void* Cm, const float* D, const float* init_state, void* y, float* final_state,
                                 void* stream);
+
+/*
+ * ssd_selftest_carry_timeout exercises the one wait of the two-head fused
+ * kernel that is not on a barrier of its own CTA: in its split schedule a CTA
+ * whose range starts inside a sequence waits for the previous CTA to publish
+ * that sequence's state (the page's inter-chunk recursion, "分块推理…" §2.2,
+ * handed across CTAs).  Same arguments and validation as ssd_scan_fwd plus
+ * the workspace; the problem must be one the two-head kernel splits (even
+ * heads per group, more head pairs than SMs; else SSD_ERR_UNSUPPORTED).  No
+ * carry is ever published, so those waits give up after about two seconds;
+ * the launch returns SSD_OK and the following ssd_read_device_status(stream)
+ * returns SSD_ERR_TIMEOUT.  y and final_state are left undefined; nothing
+ * faults and the context stays usable.
+ */
+ssd_status ssd_selftest_carry_timeout(const ssd_dims* d, const void* x, const float* dt, const float* A,
+                                      const void* Bm, const void* Cm, const float* D, const float* init_state,
+                                      void* y, float* final_state, void* workspace, size_t workspace_bytes,
+                                      void* stream);
 
 #ifdef __cplusplus
 }

@@ -65,7 +65,7 @@ def ws_size(d):
 @pytest.mark.parametrize("kw,status", [
     (dict(batch=0), 2), (dict(seqlen=0), 2), (dict(nheads=3), 2), (dict(ngroups=0), 2),
     (dict(headdim=65), 5), (dict(dstate=129), 5), (dict(chunk=257), 5), (dict(io_dtype=2), 3),
-    (dict(flags=2), 1), (dict(nheads=70000, ngroups=1), 5),
+    (dict(flags=4), 1), (dict(nheads=70000, ngroups=1), 5),
 ])
 def test_workspace_size_rejects(lib, kw, status):
     s, _ = ws_size(dims(**kw))
@@ -204,3 +204,14 @@ def test_input_dt_flag_only_on_the_tensor_core_path(lib):
     assert lib.ssd_chunk_cumsum(ctypes.byref(d), p, p, p, None) == 5
     ptrs = [ctypes.c_void_p(BASE + k * GB) for k in (0, 2, 3, 4, 5, 6, 7, 8, 9, 10)]  # as in call_scan
     assert lib.ssd_scan_fwd_unfused(ctypes.byref(d), *ptrs, 1 << 40, None) == 5
+
+
+def test_noalloc_rejects_sizes_beyond_its_buffer(lib):
+    # The 2.7B-shaped layer needs about 1.4 GB of step-by-step scratch, far beyond
+    # the built-in buffer: refused by the size check, before the buffer's device
+    # address is looked up and before anything is launched (so no GPU is needed).
+    d = dims(batch=8, seqlen=16384, nheads=80, ngroups=1)
+    ptrs = [ctypes.c_void_p(BASE + k * (1 << 34)) for k in range(9)]
+    assert lib.ssd_scan_fwd_noalloc(ctypes.byref(d), *ptrs, None) == 5
+    # a size that fits passes validation; a NULL x is still refused first
+    assert lib.ssd_scan_fwd_noalloc(ctypes.byref(dims()), None, *ptrs[1:], None) == 1

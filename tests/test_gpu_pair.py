@@ -1,0 +1,94 @@
+"""The two-heads-per-CTA fused kernel (SSD_PATH_FUSED_PAIR) against the fp64
+oracle.
+
+Two heads of one group share a CTA, their B/C tiles and S = C B^T.  With the
+caller's workspace and more head pairs than SMs the kernel cuts the
+concatenated sequences into equal ranges, one persistent CTA per SM, and a
+CTA that starts inside a sequence takes its initial state from the CTA before
+it (the inter-chunk recursion of "分块推理…" §2.2 handed across CTAs).  These
+cases cover one pair, ragged and one-token sequences, several pairs per
+group, the dt-scaled input, and the split schedule with many range
+boundaries; each is compared with the oracle at the bf16 tolerance, and the
+split schedule bitwise with the whole-sequence schedule (same arithmetic,
+the carry passes through memory in fp32)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from chunked_state_space_b200 import inputs, ssd
+from gpu_util import TOL, device_inputs, oracle_args, rel_err, to_np64
+
+pytestmark = pytest.mark.gpu
+
+
+def _scan(dev, wl, **kw):
+    y, fin = ssd.ssd_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
+                              chunk=wl.chunk, **kw)
+    torch.cuda.synchronize()
+    return y, fin
+
+
+@pytest.mark.parametrize("over", [
+    dict(batch=1, seqlen=700, nheads=2, ngroups=1, init_var=0.1),     # one pair, ragged tail
+    dict(batch=2, seqlen=1, nheads=4, ngroups=2),                      # one token
+    dict(batch=2, seqlen=129, nheads=8, ngroups=2, init_var=0.1),      # 4 heads per group, 2 sub-chunks
+    dict(batch=1, seqlen=2048, nheads=6, ngroups=3),                   # exact sub-chunks
+    dict(batch=1, seqlen=1000, nheads=4, ngroups=1, chunk=128),        # Q = 128
+])
+@pytest.mark.parametrize("input_dt", [False, True])
+def test_pair_kernel_matches_oracle(over, input_dt):
+    wl = inputs.custom("mamba2_130m_layer", **over)
+    host = inputs.generate(wl)
+    dev = device_inputs(host)
+    assert ssd.ssd_scan_path(ssd.make_dims(dev["x"], dev["B"], wl.chunk, input_dt))[0] == "fused_pair"
+    y, fin = _scan(dev, wl, input_dt=input_dt)
+    y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host), input_dt=input_dt)
+    assert rel_err(to_np64(y), y_ref) <= TOL["bf16"]
+    assert rel_err(to_np64(fin), f_ref) <= TOL["bf16"]
+    # the one-head kernel on the same inputs (both are checked against the oracle)
+    assert ssd.ssd_scan_path(ssd.make_dims(dev["x"], dev["B"], wl.chunk, input_dt, True))[0] == "fused"
+    y1, f1 = _scan(dev, wl, input_dt=input_dt, one_head=True)
+    assert rel_err(to_np64(y1), y_ref) <= TOL["bf16"]
+    assert rel_err(to_np64(f1), f_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("over", [
+    dict(batch=2, seqlen=300, nheads=160, ngroups=1, init_var=0.1),   # 160 pairs of 3 sub-chunks: ~1 per CTA
+    dict(batch=1, seqlen=1000, nheads=300, ngroups=2),                # 150 pairs of 8 sub-chunks
+    dict(batch=3, seqlen=640, nheads=100, ngroups=5, init_var=0.1),   # 150 pairs, 20 heads per group
+])
+def test_split_schedule_matches_oracle_and_whole_sequences(over):
+    wl = inputs.custom("mamba2_130m_layer", **over)
+    host = inputs.generate(wl)
+    dev = device_inputs(host)
+    dims = ssd.make_dims(dev["x"], dev["B"], wl.chunk)
+    assert ssd.ssd_scan_path(dims)[0] == "fused_pair"
+    y, fin = _scan(dev, wl)
+    y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host))
+    ey, ef = rel_err(to_np64(y), y_ref), rel_err(to_np64(fin), f_ref)
+    # per sequence too: a wrong carry spoils a few sequences, not the global max
+    got, ref = to_np64(y), y_ref
+    per = np.max(np.abs(got - ref), axis=(1, 3)) / np.maximum(np.max(np.abs(ref), axis=(1, 3)), 1e-30)
+    assert ey <= TOL["bf16"], ey
+    assert ef <= TOL["bf16"], ef
+    assert per.max() <= TOL["bf16"], (np.unravel_index(per.argmax(), per.shape), per.max())
+    # the strided entry point has no workspace: every CTA runs whole sequences
+    ys, fs = ssd.ssd_scan_fwd_strided(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
+                                      chunk=wl.chunk)
+    torch.cuda.synchronize()
+    assert torch.equal(ys, y)
+    assert torch.equal(fs, fin)
+
+
+def test_split_schedule_repeatable_and_workspace_reused():
+    """Back-to-back calls on one workspace (the carry flags are reset by each
+    call) give identical results."""
+    wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=300, nheads=160, ngroups=1, init_var=0.1)
+    dev = device_inputs(inputs.generate(wl))
+    dims = ssd.make_dims(dev["x"], dev["B"], wl.chunk)
+    ws = torch.empty(ssd.ssd_scan_workspace_size(dims), dtype=torch.uint8, device="cuda")
+    ws.fill_(0xFF)  # contents need not be initialised
+    outs = [_scan(dev, wl, workspace=ws) for _ in range(3)]
+    for y, f in outs[1:]:
+        assert torch.equal(y, outs[0][0]) and torch.equal(f, outs[0][1])

@@ -22,7 +22,10 @@ SSD_OK = 0
 SSD_ERR_TIMEOUT = 8
 
 
-def test_withheld_loads_time_out_and_context_survives():
+@pytest.mark.parametrize("one_head", [False, True])
+def test_withheld_loads_time_out_and_context_survives(one_head):
+    """Both fused kernels: the two-head one (default for this shape) and the
+    one-head one."""
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     wl = inputs.custom("mamba2_130m_layer", batch=1, seqlen=512, nheads=2)
     host = inputs.generate(wl)
@@ -31,7 +34,7 @@ def test_withheld_loads_time_out_and_context_survives():
 
     t0 = time.monotonic()
     ssd.ssd_selftest_timeout(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
-                             chunk=wl.chunk)
+                             chunk=wl.chunk, one_head=one_head)
     status = ssd.ssd_read_device_status()  # synchronises the stream
     elapsed = time.monotonic() - t0
     assert status == SSD_ERR_TIMEOUT
@@ -39,6 +42,32 @@ def test_withheld_loads_time_out_and_context_survives():
     assert ssd.ssd_read_device_status() == SSD_OK  # reading cleared the word
 
     # the context is intact: a normal scan right after matches the oracle
+    y, fin = ssd.ssd_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
+                              chunk=wl.chunk)
+    torch.cuda.synchronize()
+    assert ssd.ssd_read_device_status() == SSD_OK
+    y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host))
+    assert rel_err(to_np64(y), y_ref) <= TOL["bf16"]
+    assert rel_err(to_np64(fin), f_ref) <= TOL["bf16"]
+
+
+def test_carry_wait_times_out_and_context_survives():
+    """The two-head kernel's split schedule with no carry ever published: every
+    CTA that starts inside a sequence gives up waiting for its predecessor's
+    state after about two seconds; the host reads SSD_ERR_TIMEOUT, and a normal
+    scan (with its carries) then matches the oracle in the same context."""
+    wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=300, nheads=160, ngroups=1, init_var=0.1)
+    host = inputs.generate(wl)
+    dev = device_inputs(host)
+    assert ssd.ssd_read_device_status() == SSD_OK
+    t0 = time.monotonic()
+    ssd.ssd_selftest_carry_timeout(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
+                                   chunk=wl.chunk)
+    status = ssd.ssd_read_device_status()
+    elapsed = time.monotonic() - t0
+    assert status == SSD_ERR_TIMEOUT
+    assert elapsed < 30.0, elapsed
+    assert ssd.ssd_read_device_status() == SSD_OK
     y, fin = ssd.ssd_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
                               chunk=wl.chunk)
     torch.cuda.synchronize()

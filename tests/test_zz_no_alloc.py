@@ -5,16 +5,19 @@ libssd.so instead of a caller workspace.
 
 The test calls it through the C ABI twice in a row, on different inputs, and
 compares each result with ssd_scan_fwd_unfused (same kernels, caller
-workspace) within the parity tolerances.  The file is named so that pytest
-collects it last; it also passes alone in a fresh process.
+workspace) and with the fp64 oracle, within the parity tolerances.  The file
+is named so that pytest collects it last; it also passes alone in a fresh
+process.  The refusal of sizes beyond the built-in buffer needs no GPU and is
+checked in the CPU tier (tests/test_abi.py).
 """
 import ctypes
 
 import pytest
 import torch
 
+import oracle
 from chunked_state_space_b200 import inputs, ssd
-from gpu_util import TOL, device_inputs, rel_err, to_np64
+from gpu_util import TOL, device_inputs, oracle_args, rel_err, to_np64
 
 pytestmark = pytest.mark.gpu
 
@@ -39,7 +42,8 @@ def test_noalloc_matches_unfused_twice(name, over):
     assert torch.cuda.is_available()
     wl = inputs.custom(name, **over)
     for seed in (0, 1):  # two calls in a row; the second must not see the first's scratch
-        dev = device_inputs(inputs.generate(wl, seed=seed))
+        host = inputs.generate(wl, seed=seed)
+        dev = device_inputs(host)
         s, y, fin = _noalloc(dev, wl)
         assert s == 0, ssd.status_string(s)
         y_ref, f_ref = ssd.ssd_scan_fwd_unfused(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"],
@@ -47,14 +51,7 @@ def test_noalloc_matches_unfused_twice(name, over):
         torch.cuda.synchronize()
         assert rel_err(to_np64(y), to_np64(y_ref)) <= TOL[wl.io]
         assert rel_err(to_np64(fin), to_np64(f_ref)) <= TOL[wl.io]
+        y64, f64 = oracle.scan_recurrence(*oracle_args(host))
+        assert rel_err(to_np64(y), y64) <= TOL[wl.io]
+        assert rel_err(to_np64(fin), f64) <= TOL[wl.io]
 
-
-def test_noalloc_rejects_sizes_beyond_its_buffer():
-    # the 2.7B-shaped layer needs about 1.4 GB of scratch: refused before any launch
-    wl = inputs.custom("mamba2_2p7b_layer", seqlen=256)
-    dims = ssd.Dims(wl.batch, 16384, wl.nheads, wl.headdim, wl.dstate, wl.ngroups, wl.chunk, ssd.SSD_BF16, 0)
-    big = 1 << 40
-    p = lambda k: ctypes.c_void_p(big + k * (1 << 34))
-    s = ssd.lib().ssd_scan_fwd_noalloc(ctypes.byref(dims), p(0), p(1), p(2), p(3), p(4), p(5), p(6), p(7), p(8),
-                                       None)
-    assert s == 5, ssd.status_string(s)

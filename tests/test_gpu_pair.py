@@ -11,7 +11,6 @@ group, the dt-scaled input, and the split schedule with many range
 boundaries; each is compared with the oracle at the bf16 tolerance, and the
 split schedule bitwise with the whole-sequence schedule (same arithmetic,
 the carry passes through memory in fp32)."""
-import numpy as np
 import pytest
 import torch
 
@@ -67,13 +66,11 @@ def test_split_schedule_matches_oracle_and_whole_sequences(over):
     y, fin = _scan(dev, wl)
     y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host))
     ey, ef = rel_err(to_np64(y), y_ref), rel_err(to_np64(fin), f_ref)
-    # per sequence too: a wrong carry spoils a few sequences, not the global max
-    got, ref = to_np64(y), y_ref
-    per = np.max(np.abs(got - ref), axis=(1, 3)) / np.maximum(np.max(np.abs(ref), axis=(1, 3)), 1e-30)
     assert ey <= TOL["bf16"], ey
     assert ef <= TOL["bf16"], ef
-    assert per.max() <= TOL["bf16"], (np.unravel_index(per.argmax(), per.shape), per.max())
-    # the strided entry point has no workspace: every CTA runs whole sequences
+    # The carries themselves: the strided entry point has no workspace, so
+    # there every CTA runs whole sequences.  The split must give the same
+    # bits (a wrong or late carry changes whole sequences by O(1)).
     ys, fs = ssd.ssd_scan_fwd_strided(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
                                       chunk=wl.chunk)
     torch.cuda.synchronize()

@@ -273,8 +273,7 @@ def _horizontal_gpu(x0, layers, states, wl, eps):
 def test_vertical_small(L, V):
     """3-layer stack: vertical == horizontal (bitwise when V % Q == 0), every
     layer teacher-forced against the oracle on its own bf16 input (5e-3), and
-    the end-to-end output within the tolerance the oracle's own rounding
-    sensitivity allows."""
+    the end-to-end output within the bound of _check_end_to_end."""
     wl = inputs.custom("stack24_vertical", batch=2, seqlen=L, nheads=4)
     n_layers, eps = 3, 1e-6
     host_layers, dev_layers = _stack_layers(wl, n_layers)
@@ -303,19 +302,40 @@ def test_vertical_small(L, V):
         assert rel_err(to_np64(ys[l]), y_ref) <= TOL["bf16"], ("layer", l)
         assert rel_err(to_np64(st_h[l]), f_ref) <= TOL["bf16"], ("state", l)
         assert rel_err(to_np64(st_v[l]), f_ref) <= TOL["bf16"], ("vertical state", l)
-    y_ref, _ = oracle.stack_horizontal(f(x0h), layers64, eps)
-    sens = rel_err(_stack_sensitivity(f(x0h), layers64, eps), y_ref)
-    err = rel_err(to_np64(yv), y_ref)
-    assert err <= TOL["bf16"] + 2.0 * sens, f"end-to-end err {err:.3e}, one-flip sensitivity {sens:.3e}"
+    _check_end_to_end(f(x0h), layers64, eps, to_np64(yv), tag=f"3-layer stack L={L} V={V}")
 
 
-def _stack_sensitivity(x0, layers64, eps, rel=1e-7, seed=0):
-    """How far the oracle's own last-layer output moves when every layer's output
-    is perturbed by relative noise of size `rel` before its bf16 storage
-    rounding.  rel = 1e-7 is about one fp32 rounding: it changes nothing but
-    which way the values that sit next to a bf16 rounding boundary round, so
-    the result is the spread between two exact-up-to-fp32 evaluations of the
-    same stack (the one-flip sensitivity of the bf16 storage between layers)."""
+def _check_end_to_end(x0, layers64, eps, y_end, tag="stack"):
+    """End-to-end comparison of a GPU layer stack with the oracle's stack.
+
+    Every GPU layer is checked on its own (teacher-forced, 5e-3) elsewhere; the
+    whole stack also carries each layer's error into the layers after it.  The
+    bound models a correct bf16 implementation: each layer's output deviates
+    from the exact map by about one bf16 rounding per element (the kernel
+    multiplies bf16 operands P, X' and a bf16 copy of the state; the RMS
+    relative error of one bf16 rounding is about 2^-9), and the oracle measures
+    how far such independent per-layer noise moves its own last output (sens).
+    Asserted: err <= 5e-3 + 2 * sens(2^-9).  The spread from rounding-boundary
+    flips alone, sens(1e-7), is printed beside it: it leaves out the layers'
+    compute errors, which every layer is allowed and which later layers
+    amplify."""
+    y_ref, _ = oracle.stack_horizontal(x0, layers64, eps)
+    sens = rel_err(_stack_sensitivity(x0, layers64, eps, rel=2.0 ** -9), y_ref)
+    flip = rel_err(_stack_sensitivity(x0, layers64, eps, rel=1e-7), y_ref)
+    err = rel_err(y_end, y_ref)
+    bound = TOL["bf16"] + 2.0 * sens
+    print(f"{tag}: end-to-end err {err:.3e}, bound {bound:.3e} (sens(2^-9) {sens:.3e}; flips alone "
+          f"sens(1e-7) {flip:.3e})")
+    assert err <= bound, f"end-to-end err {err:.3e} > {bound:.3e} (sens {sens:.3e}, flips {flip:.3e})"
+
+
+def _stack_sensitivity(x0, layers64, eps, rel, seed=0):
+    """The oracle's own last-layer output when every layer's output is
+    perturbed by independent relative noise of size `rel` (seeded Gaussian)
+    before its bf16 storage rounding.  rel = 2^-9: about one bf16 rounding per
+    element, the error a correct bf16 layer adds; rel = 1e-7: about one fp32
+    rounding, which only changes which way values next to a bf16 rounding
+    boundary round."""
     rng = np.random.default_rng(seed)
     x = x0
     y = None
@@ -334,10 +354,8 @@ def test_stack24_vertical_full():
     2. every layer, teacher-forced: the GPU's y_l and final state for a sampled
        (batch, head) over the whole sequence match the oracle run on the GPU's
        own bf16 input x_l (5e-3), and x_{l+1} is the RMS-normalised y_l;
-    3. end to end on a prefix against the oracle's stack, within 5e-3 plus twice
-       the oracle's own one-flip sensitivity: how far its output moves when each
-       layer's output is perturbed by 1e-7 (relative) before its bf16 storage
-       rounding, which only changes the direction of boundary roundings.
+    3. end to end on a prefix against the oracle's stack, within the bound of
+       _check_end_to_end.
     """
     wl = inputs.WORKLOADS["stack24_vertical"]
     n_layers, eps, V = wl.n_layers, 1e-6, wl.vblock
@@ -380,7 +398,8 @@ def test_stack24_vertical_full():
         ref = oracle.rmsnorm_bf16(to_np64(ys[l][:1, tok]), eps)
         got = to_np64(xs[l + 1][:1, tok])
         assert np.max(np.abs(got - ref)) <= 2.0 ** -7 * np.max(np.abs(ref)), ("rmsnorm", l)
-    # 3. end to end on a prefix (batch 0, 1024 tokens)
+    # 3. end to end on a prefix (batch 0, 1024 tokens); the prefix is causal, so
+    # it equals the first 1024 tokens of the full run
     Lp = 1024
     pre = lambda t: t[:1, :Lp].contiguous()
     dev_pre = [dict(dt=pre(p["dt"]), A=p["A"], B=pre(p["B"]), C=pre(p["C"]), D=p["D"]) for p in dev_layers]
@@ -389,10 +408,4 @@ def test_stack24_vertical_full():
     assert torch.equal(yp, yv[:1, :Lp])
     layers64 = [dict(dt=f(h["dt"][:1, :Lp]), A=f(h["A"]), B=f(h["B"][:1, :Lp]), C=f(h["C"][:1, :Lp]),
                      D=f(h["D"])) for h in host_layers]
-    x0p = f(x0h[:1, :Lp])
-    y_ref, _ = oracle.stack_horizontal(x0p, layers64, eps)
-    sens = rel_err(_stack_sensitivity(x0p, layers64, eps), y_ref)
-    err = rel_err(to_np64(yp), y_ref)
-    print(f"stack24 end to end (batch 0, {Lp} tokens): err {err:.3e}, one-flip sensitivity {sens:.3e}, "
-          f"bound {TOL['bf16'] + 2.0 * sens:.3e}")
-    assert err <= TOL["bf16"] + 2.0 * sens, f"end-to-end err {err:.3e}, one-flip sensitivity {sens:.3e}"
+    _check_end_to_end(f(x0h[:1, :Lp]), layers64, eps, to_np64(yp), tag=f"stack24 (batch 0, {Lp} tokens)")

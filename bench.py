@@ -261,6 +261,11 @@ def main():
                     help="the dt-scaled input variant (SSD_FLAG_INPUT_DT)")
     ap.add_argument("--strided", action="store_true",
                     help="x, B, C as column slices of one fused [B, L, H*P + 2*G*N] tensor (ssd_scan_fwd_strided)")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the decode step ssd_step (one token per call, state in place) at the workload's "
+                         "batch, heads and sizes instead of the scan")
+    ap.add_argument("--unfused", action="store_true",
+                    help="time the four step kernels (ssd_scan_fwd_unfused) instead of the fused kernel")
     ap.add_argument("--one-head", action="store_true",
                     help="the one-head-per-CTA fused kernel even where the two-head kernel applies (comparison)")
     ap.add_argument("--no-extras", action="store_true",
@@ -291,6 +296,8 @@ def main():
         wl = inputs.custom(wl.name, batch=wl.batch, vblock=args.vblock)
     if wl.n_layers > 1:
         return run_stack(args, wl, dev, rank, world)
+    if args.decode:
+        return run_decode(args, wl, dev, rank, world)
     host = inputs.generate(wl, seed=rank_seed(rank))  # each rank: its own independent batch
     pinned = {}
     for k, v in host.items():
@@ -308,7 +315,7 @@ def main():
     def step():
         ssd.ssd_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init"], chunk=wl.chunk, y=y,
                          final_state=fin, workspace=ws, stream=stream, input_dt=args.input_dt,
-                         one_head=args.one_head)
+                         one_head=args.one_head, unfused=args.unfused)
 
     if args.strided:  # x, B, C as views of one fused projection output
         HP, GN = wl.nheads * wl.headdim, wl.ngroups * wl.dstate
@@ -326,6 +333,8 @@ def main():
                                      one_head=args.one_head)
 
     path, kernels_per_step = ssd.ssd_scan_path(dims)
+    if args.unfused:
+        path, kernels_per_step = "tensor_steps" if path in ssd.FUSED_PATHS else path, 4
     flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev) if l2_resident(wl) else None
     per_step, ms_total, clk = timed_steps(step, args, stream, dev, local, world, flush)
     ms_per_step = ms_total / args.steps
@@ -398,6 +407,53 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+    return 0
+
+
+def run_decode(args, wl, dev, rank, world):
+    """The decode step: one ssd_step per (batch, head) and token, the fp32 state
+    updated in place.  HBM-bound on the state (read and written once per call):
+    2*B*H*N*P*4 bytes plus the token's x, y, dt, B, C.  The state of one layer
+    fits in L2, so a 512 MB flush runs between steps (a model with many layers
+    streams each layer's state from HBM)."""
+    import torch
+    from chunked_state_space_b200 import inputs, ssd
+    Bz, H, P, N, G = wl.batch, wl.nheads, wl.headdim, wl.dstate, wl.ngroups
+    one = inputs.custom(wl.name, seqlen=1)
+    host = inputs.generate(one, seed=rank_seed(rank))
+    d = {k: (torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16 else
+             torch.from_numpy(v)).to(dev) for k, v in host.items()}
+    x, dt, Bm, Cm = d["x"][:, 0].contiguous(), d["dt"][:, 0].contiguous(), d["B"][:, 0].contiguous(), \
+        d["C"][:, 0].contiguous()
+    state = d["init"].clone()
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        ssd.ssd_step(x, dt, d["A"], Bm, Cm, state, D=d["D"], y=y, stream=stream, input_dt=args.input_dt)
+
+    per_step, ms_total, clk = timed_steps(step, args, stream, dev, dev.index, world, flush)
+    ms = ms_total / args.steps
+    io = 2 if wl.io == "bf16" else 4
+    nbytes = 2 * Bz * H * N * P * 4 + 2 * Bz * H * P * io + Bz * H * 4 + 2 * Bz * G * N * io + 8 * H
+    hbm_peak, _, _, peak_src = load_peaks()
+    ach = nbytes / (statistics.mean(per_step) * 1e-3) / 1e9
+    line = {
+        "metric": "SSD decode step tokens/s (ssd_step, one token per sequence per call)",
+        "value": Bz * world / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.io == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": wl.name + " decode", "batch": Bz, "nheads": H, "headdim": P, "dstate": N,
+                   "ngroups": G, "state_dtype": "f32",
+                   "l2": "512 MB L2 flush between steps (the state fits in L2); per-step events exclude it"},
+        "clocks": clk, "gpu_launches": args.steps,
+        "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
+                     "traffic": None, "kernel": "k_ssd_step_v4", "bytes_per_launch": nbytes,
+                     "peak_source": peak_src},
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
     return 0
 
 

@@ -16,6 +16,9 @@ pytestmark = pytest.mark.gpu
     ("tiny_f32", dict(batch=1, seqlen=20, nheads=3, ngroups=1, headdim=5, dstate=7, init_var=0.3)),
     ("mamba2_130m_layer", dict(batch=2, seqlen=24, nheads=4, ngroups=2, init_var=0.1)),
     ("mamba2_2p7b_layer", dict(seqlen=6)),
+    # 128-bit kernel with 3 column groups (256 threads do not split evenly) and with 1
+    ("tiny_f32", dict(batch=2, seqlen=12, nheads=2, ngroups=1, headdim=12, dstate=100, init_var=0.3)),
+    ("mamba2_130m_layer", dict(batch=1, seqlen=10, nheads=2, ngroups=1, headdim=4, dstate=128, init_var=0.1)),
 ])
 def test_decode_steps_match_oracle(name, over):
     wl = inputs.custom(name, **over)
@@ -52,3 +55,26 @@ def test_decode_continues_a_prefill():
     y = torch.cat(ys, dim=1)
     assert rel_err(to_np64(y), y_ref) <= TOL["bf16"]
     assert rel_err(to_np64(st), f_ref) <= TOL["bf16"]
+
+
+def test_decode_state_view_not_16_byte_aligned():
+    """A state that is only 4-byte aligned (a view one float into a buffer) takes
+    the scalar kernel and gives the same results as the 128-bit kernel."""
+    wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=8, nheads=4, ngroups=2, init_var=0.1)
+    host = inputs.generate(wl)
+    dev = device_inputs(host)
+    n = dev["init"].numel()
+    buf = torch.empty(n + 1, dtype=torch.float32, device="cuda")
+    st_u = buf[1:].view(dev["init"].shape)
+    st_u.copy_(dev["init"])
+    st_a = dev["init"].clone()
+    for t in range(wl.seqlen):
+        args = (dev["x"][:, t].contiguous(), dev["dt"][:, t].contiguous(), dev["A"], dev["B"][:, t].contiguous(),
+                dev["C"][:, t].contiguous())
+        ya = ssd.ssd_step(*args, st_a, D=dev["D"])
+        yu = ssd.ssd_step(*args, st_u, D=dev["D"])
+        torch.cuda.synchronize()
+        assert rel_err(to_np64(yu), to_np64(ya)) <= 1e-6
+    assert rel_err(to_np64(st_u), to_np64(st_a)) <= 1e-6
+    y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host))
+    assert rel_err(to_np64(st_u), f_ref) <= TOL["bf16"]

@@ -14,21 +14,29 @@
 //   b_intra    = B_k^T [X'_a | X'_b],  X'_h = diag(exp(lam_end - lam_s)) X_h   (N = 128)
 //   y_intra_h  = P_h X_h                                  (A operand from TMEM)
 //   y_t        = y_intra + exp(lam_t) y_inter + D x_t      (fp32)
-//   s_h(k)     = exp(lam_end) s_h(k-1) + b_intra_h         (fp32, registers)
+//   s_h(k)     = exp(lam_end) s_h(k-1) + b_intra_h         (fp32, in TMEM: the b_intra
+//                                                           MMA accumulates onto the scaled state)
 // (with the dt-scaled input every column s of P and row s of X' also carries dt_s).
 //
-// Warp roles (512 threads): warp 0 issues TMA loads (x of both heads in two
-// stages, B/C in one) and L2 prefetches; warp 1 owns TMEM and issues the MMAs
-// in the order S, y_inter, b_intra, y_intra; warps 2-3 load dt, scan lam and
-// write X'; warps 4-7 turn S into P_a and P_b (one thread per row); warps
-// 8-11 / 12-15 finish y and the state of head a / b (one thread per row).
-// The x tile of a head is also where its y tile is staged for the TMA store:
-// each epilogue thread reads its own x row and overwrites it with its y row.
+// Warp roles (384 threads): warp 0 runs every TMA transfer -- loads of x (two
+// stages, both heads), B and C (one buffer), L2 prefetches, and the stores of
+// finished y tiles; warp 1 owns TMEM and issues the MMAs in the order S,
+// y_inter, b_intra, y_intra; warps 2-3 load dt, scan lam and write X'; warps
+// 4-7 / 8-11 are the warps of head a / b (warp w owns TMEM lane quarter w % 4,
+// one thread per row): they turn S into that head's P, then update its state
+// and finish its y.  The two heads' masks thus run side by side, two warps
+// per SM sub-partition.  The x tile of a head is also where its y tile is
+// staged for the TMA store: each thread reads its own x row and overwrites it
+// with its y row; the producer stores the tile once all 128 rows are staged,
+// so no head warp waits for a store.
 //
 // TMEM (512 columns): two 128-column regions SP[0], SP[1] take turns -- S(k)
 // goes to SP[k&1], P(k) to SP[1-(k&1)], y_intra(k) back to SP[k&1] -- so S of
 // the next sub-chunk starts while this one's outputs are being read; y_inter
-// and b_intra have 128 columns each.
+// has 128 columns, and the running fp32 state of both heads lives in the last
+// 128 (after b_intra(k) it holds s(k); the head warps read it, publish its
+// bf16 copy for y_inter(k+1), and write exp(lam_end(k+1)) s(k) back for the
+// b_intra(k+1) MMA to accumulate onto).
 //
 // Work split: the (batch, head pair) sequences are concatenated into one list
 // of sub-chunks and cut into equal ranges, one per CTA (persistent launch of
@@ -56,7 +64,7 @@ using namespace umma;
 constexpr int T = 128;   // tokens per sub-chunk
 constexpr int P = 64;    // head dim
 constexpr int NS = 128;  // state dim
-constexpr int THREADS = 512;
+constexpr int THREADS = 384;
 constexpr uint32_t TILE = 16384;  // [128 rows][64 bf16], 128B-swizzled
 
 constexpr uint32_t OFF_B = 0;                    // B tile: n-blocks 0-63, 64-127
@@ -75,21 +83,21 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_SP = 0, TM_YI = 256, TM_BI = 384;  // SP[i] at 128*i
 
 enum {
-  BCFULL = 0,   // B/C tiles landed (tx)
-  SFULL = 1,    // S complete
-  BIFULL = 2,   // y_inter and b_intra complete (B/C and X' free, b_intra readable)
-  YFULL = 3,    // y_intra complete
-  PFULL = 4,    // P of both heads written (128 mask threads)
-  XPFULL = 5,   // X' written (64 aux threads)
-  BIEMPTY = 6,  // b_intra read (256 epilogue threads)
+  BCFULL = 0,     // B/C tiles landed (tx)
+  SFULL = 1,      // S complete
+  BIFULL = 2,     // y_inter and b_intra complete (B/C, X' and the bf16 state free; s(k) readable)
+  YFULL = 3,      // y_intra of both heads complete
+  PFULL = 4,      // P of both heads written (256 head threads)
+  XPFULL = 5,     // X' written (64 aux threads)
+  BIREADY = 6,    // the state region holds exp(lam_end(k)) s(k-1) for b_intra(k) (256)
   STATEFULL = 7,  // bf16 state published (256)
-  YEMPTY = 8,   // y_intra, y_inter read (256)
-  XFULL0 = 9,   // [stage] x tiles landed (tx)
-  XEMPTY0 = 11,  // [stage] y tiles of both heads stored from the x buffer (2)
-  LAMRDY0 = 13,  // [slot 4] tables written (64 aux threads)
+  YEMPTY = 8,     // y_inter read (256)
+  XFULL0 = 9,     // [stage] x tiles landed (tx)
+  YSTAGED0 = 11,  // [head] 128 y rows of the head staged in its x tile (128)
+  LAMRDY0 = 13,   // [slot 4] tables written (64 aux threads)
   DRAIN = 17
 };
-constexpr int AUX = 64, MASKT = 128, EPIT = 256;
+constexpr int AUX = 64, HEADT = 128, EPIT = 256;
 constexpr int W_TMA = 0, W_MMA = 1;
 
 struct Params {
@@ -248,6 +256,18 @@ __device__ __forceinline__ void st_release(int* p, int v) {
   asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+
+// Wait until at most `n` bulk store groups of this thread are still reading
+// shared memory (n = 0, 1 or 2).
+__device__ __forceinline__ void store_wait_read(int n) {
+  if (n <= 0)
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+  else if (n == 1)
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+  else
+    asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory");
+}
+
 template <bool XDT>
 __global__ void __launch_bounds__(THREADS, 1)
     k_ssd_pair(Params p, const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
@@ -278,14 +298,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&bar[SFULL], 1);
     mbar_init(&bar[BIFULL], 1);
     mbar_init(&bar[YFULL], 1);
-    mbar_init(&bar[PFULL], MASKT);
+    mbar_init(&bar[PFULL], EPIT);
     mbar_init(&bar[XPFULL], AUX);
-    mbar_init(&bar[BIEMPTY], EPIT);
+    mbar_init(&bar[BIREADY], EPIT);
     mbar_init(&bar[STATEFULL], EPIT);
     mbar_init(&bar[YEMPTY], EPIT);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar[XFULL0 + i], 1);
-      mbar_init(&bar[XEMPTY0 + i], 2);
+      mbar_init(&bar[YSTAGED0 + i], HEADT);
     }
     for (int i = 0; i < 4; ++i) mbar_init(&bar[LAMRDY0 + i], AUX);
     mbar_init(&bar[DRAIN], 1);
@@ -300,23 +320,25 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  auto coords = [&](int64_t k, int& b, int& h0, int& g, int& t0) {
+    int64_t u;
+    int j;
+    bool f, l, ci, co;
+    rg.at(k, u, j, f, l, ci, co);
+    b = (int)(u / hpp);
+    h0 = (int)(u % hpp) * 2;
+    g = h0 / (p.H / p.G);
+    t0 = j * T;
+  };
+
   if (warp == W_TMA) {
     // ------------------------------------------------------------ TMA producer
-    // Two queues polled in turn: B/C of sub-chunk kb (one buffer, free once
-    // y_inter and b_intra of kb-1 completed) and x of sub-chunk kx (two stages,
-    // free once both heads' y tiles of kx-2 were stored from them).
+    // Three queues polled in turn: y stores (head a then b of sub-chunk ky, once
+    // its 128 rows are staged), B/C of sub-chunk kb (one buffer, free once
+    // y_inter and b_intra of kb-1 completed), x of sub-chunk kx (two stages, free
+    // once both heads' y tiles of kx-2 have been read by their stores).
     if (lane == 0) {
       constexpr int kPrefetch = 3;
-      auto coords = [&](int64_t k, int& b, int& h0, int& g, int& t0) {
-        int64_t u;
-        int j;
-        bool f, l, ci, co;
-        rg.at(k, u, j, f, l, ci, co);
-        b = (int)(u / hpp);
-        h0 = (int)(u % hpp) * 2;
-        g = h0 / (p.H / p.G);
-        t0 = j * T;
-      };
       auto prefetch = [&](int64_t k) {
         if (k >= K) return;
         int b, h0, g, t0;
@@ -330,12 +352,29 @@ __global__ void __launch_bounds__(THREADS, 1)
       };
       for (int64_t k = 0; k < kPrefetch; ++k) prefetch(k);
       const bool loads = p.withhold != 1;
-      int64_t kb = 0, kx = 0, pf = kPrefetch;
+      int64_t kb = 0, kx = 0, ky = 0, pf = kPrefetch;
+      int hy = 0;          // next head to store of sub-chunk ky
+      int64_t groups = 0;  // store groups committed (one per head tile)
       uint32_t idle = 0;
       uint64_t t_last = globaltimer_ns();
-      while ((kb < K || kx < K) && !*abort_flag) {
+      while ((kb < K || kx < K || ky < K) && !*abort_flag) {
         bool progress = false;
-        if (kx < K && kx <= kb + 1 && (kx < 2 || mbar_test_wait(&bar[XEMPTY0 + (kx & 1)], ((kx - 2) >> 1) & 1))) {
+        if (ky < K && mbar_test_wait(&bar[YSTAGED0 + hy], (uint32_t)(ky & 1))) {
+          int b, h0, g, t0;
+          coords(ky, b, h0, g, t0);
+          tma_store_4d(&map_y, sm + OFF_X + (ky & 1) * 2 * TILE + hy * TILE, 0, h0 + hy, t0, b);
+          tma_store_commit();
+          ++groups;
+          if (++hy == 2) {
+            hy = 0;
+            ++ky;
+          }
+          progress = true;
+        }
+        // x(kx) reuses the stage of x(kx-2): both y tiles of kx-2 must have been
+        // stored (issued) and read; groups issued after them may stay in flight
+        if (kx < K && kx <= kb + 1 && (kx < 2 || ky > kx - 2)) {
+          if (kx >= 2) store_wait_read((int)(groups - 2 * (kx - 1)));
           int b, h0, g, t0;
           coords(kx, b, h0, g, t0);
           const int st = (int)(kx & 1);
@@ -375,8 +414,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           __nanosleep(32);
         }
       }
-      // every load issued must land before the CTA may exit (bounded: the
-      // tiles are valid memory, so they land unless the device is wedged)
+      // every load issued must land and every store complete before the CTA
+      // may exit (bounded: valid tiles land unless the device is wedged)
+      tma_store_wait0();
       if (loads) {
         const uint64_t t0 = globaltimer_ns();
         if (kb > 0)
@@ -426,17 +466,18 @@ __global__ void __launch_bounds__(THREADS, 1)
             mma_ss(tmem + TM_YI, desc_advance(dC, (ks >> 2) * TILE + (ks & 3) * 32), desc_advance(dSt, ks * 2048),
                    idYI, ks > 0);
         }
-        // b_intra(k) = B^T [X'_a | X'_b]: needs X'(k) and b_intra(k-1) read
+        // state(k) = exp(lam_end) state(k-1) + B^T [X'_a | X'_b]: needs X'(k) and the
+        // scaled state written back by the head warps
         if (ok) ok = ctl.wait(XPFULL, ph);
-        if (ok && k > 0) ok = ctl.wait(BIEMPTY, php);
+        if (ok) ok = ctl.wait(BIREADY, ph);
         if (ok) {
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            mma_ss(tmem + TM_BI, desc_advance(dBmn, ks * 2048), desc_advance(dXp, ks * 2048), idBI, ks > 0);
+            mma_ss(tmem + TM_BI, desc_advance(dBmn, ks * 2048), desc_advance(dXp, ks * 2048), idBI, 1);
           mma_commit(&bar[BIFULL]);  // also: B/C, X' and the bf16 state are free again
         }
-        // y_intra(k) of both heads into SP[pi] (S there was read by the mask)
+        // y_intra(k) of both heads into SP[pi] (both masks have read S there)
         if (ok) ok = ctl.wait(PFULL, ph);
         if (ok) {
           tc_fence_after();
@@ -550,16 +591,18 @@ __global__ void __launch_bounds__(THREADS, 1)
             float w = ex2(lam_end - lj[row]);
             if constexpr (XDT) w *= tab(slot, h, 2)[row];
             const float2 w2 = make_float2(w, w);
+            uint4 v4[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) v4[c] = lds128(src + swz128(row, c * 8));
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-              uint4 v4 = lds128(src + swz128(row, c * 8));
-              uint32_t* u = reinterpret_cast<uint32_t*>(&v4);
+              uint32_t* u = reinterpret_cast<uint32_t*>(&v4[c]);
 #pragma unroll
               for (int i = 0; i < 4; ++i) {  // fp32 product, one rounding
                 const float2 f = mul2(bf2_to_f2(u[i]), w2);
                 u[i] = pack_bf16(f.x, f.y);
               }
-              sts128(dst + swz128(row, c * 8), v4);
+              sts128(dst + swz128(row, c * 8), v4[c]);
             }
           }
         }
@@ -568,106 +611,37 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive(&bar[XPFULL]);
       named_sync(1, AUX);  // wtot reuse
     }
-  } else if (warp < 8) {
-    // ------------------------------------------------------------ P_a, P_b = S (.) L_a, L_b
-    const int q = warp & 3;  // TMEM lane quarter = 32-row block
-    const int row = q * 32 + lane;
-    const uint32_t lq = (uint32_t)(q * 32) << 16;
-    for (int64_t k = 0; k < K; ++k) {
-      const int slot = (int)(k & 3), pi = (int)(k & 1);
-      bool ok = ctl.wait(LAMRDY0 + slot, (uint32_t)((k >> 2) & 1));
-      if (ok) ok = ctl.wait(SFULL, (uint32_t)(k & 1));
-      if (ok && k > 0) ok = ctl.wait(YEMPTY, (uint32_t)((k - 1) & 1));  // y_intra(k-1) in SP[1-pi] read
-      tc_fence_after();
-      const uint32_t tS = tmem + lq + TM_SP + 128 * pi, tP = tmem + lq + TM_SP + 128 * (1 - pi);
-      float lam_t[2];
-      lam_t[0] = tab(slot, 0, 0)[row];
-      lam_t[1] = tab(slot, 1, 0)[row];
-#pragma unroll 1
-      for (int kb = 0; kb < 4; ++kb) {
-        uint32_t pk[2][16];
-        if (kb <= q) {  // warp-uniform
-          uint32_t r[32];
-          tmem_ld32(tS + 32 * kb, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const float4* lj4 = reinterpret_cast<const float4*>(tab(slot, h, 0));
-            if (kb < q) {
-              // below the diagonal block: exp(lam_t - lam_s) = 2^(lt - l_end(kb)) * ec[s]
-              const float4* ec4 = reinterpret_cast<const float4*>(tab(slot, h, 1));
-              const float rowf = ex2(lam_t[h] - tab(slot, h, 0)[32 * kb + 31]);
-              const float2 rf2 = make_float2(rowf, rowf);
-#pragma unroll
-              for (int v = 0; v < 8; ++v) {
-                const float4 c = ec4[8 * kb + v];
-                const float2 a0 = mul2(mul2(make_float2(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1])),
-                                            make_float2(c.x, c.y)),
-                                       rf2);
-                const float2 a1 = mul2(
-                    mul2(make_float2(__uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])),
-                         make_float2(c.z, c.w)),
-                    rf2);
-                pk[h][2 * v] = pack_bf16(a0.x, a0.y);
-                pk[h][2 * v + 1] = pack_bf16(a1.x, a1.y);
-              }
-            } else {
-              // diagonal block: direct decays, clamped at 0 above the diagonal and then zeroed
-              const int rl = row - 32 * kb;
-#pragma unroll
-              for (int v = 0; v < 8; ++v) {
-                const float4 l = lj4[8 * kb + v];
-                float e0 = ex2(fminf(lam_t[h] - l.x, 0.f)), e1 = ex2(fminf(lam_t[h] - l.y, 0.f));
-                float e2 = ex2(fminf(lam_t[h] - l.z, 0.f)), e3 = ex2(fminf(lam_t[h] - l.w, 0.f));
-                if constexpr (XDT) {
-                  const float4 fx = reinterpret_cast<const float4*>(tab(slot, h, 2))[8 * kb + v];
-                  e0 *= fx.x;
-                  e1 *= fx.y;
-                  e2 *= fx.z;
-                  e3 *= fx.w;
-                }
-                const float f0 = (4 * v + 0 <= rl) ? __uint_as_float(r[4 * v + 0]) * e0 : 0.f;
-                const float f1 = (4 * v + 1 <= rl) ? __uint_as_float(r[4 * v + 1]) * e1 : 0.f;
-                const float f2 = (4 * v + 2 <= rl) ? __uint_as_float(r[4 * v + 2]) * e2 : 0.f;
-                const float f3 = (4 * v + 3 <= rl) ? __uint_as_float(r[4 * v + 3]) * e3 : 0.f;
-                pk[h][2 * v] = pack_bf16(f0, f1);
-                pk[h][2 * v + 1] = pack_bf16(f2, f3);
-              }
-            }
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) pk[0][i] = pk[1][i] = 0u;
-        }
-        tmem_st16(tP + 16 * kb, pk[0]);
-        tmem_st16(tP + 64 + 16 * kb, pk[1]);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      (void)ok;
-      mbar_arrive(&bar[PFULL]);
-    }
   } else {
-    // ------------------------------------------------------------ y, state, final (head hl)
-    const int hl = (warp - 8) >> 2;  // 0: warps 8-11, 1: warps 12-15
-    const int q = warp & 3;
-    const int r = q * 32 + lane;     // state row n and output row t
-    const int et = threadIdx.x - 256;  // 0..255 over both heads
+    // ------------------------------------------------------------ the warps of head hl
+    const int hl = (warp - 4) >> 2;  // 0: warps 4-7, 1: warps 8-11
+    const int q = warp & 3;          // TMEM lane quarter
+    const int r = q * 32 + lane;     // S / P / y row t and state row n
+    const int et = threadIdx.x - 128;  // 0..255 over both heads
     const uint32_t lq = (uint32_t)(q * 32) << 16;
     const uint32_t sSt = sbase + OFF_ST + hl * TILE;
-    float s[P];
-    auto publish_state = [&]() {
+    const uint32_t tSt = tmem + lq + TM_BI + 64 * hl;  // this head's fp32 state, row r
+    // Columns 32c..32c+31 of the state row: the bf16 copy into the MN-major
+    // operand tile of y_inter, and dec times the values back into TMEM.
+    auto publish_half = [&](int c, const uint32_t* v) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 v;
-        v.x = pack_bf16(s[8 * c + 0], s[8 * c + 1]);
-        v.y = pack_bf16(s[8 * c + 2], s[8 * c + 3]);
-        v.z = pack_bf16(s[8 * c + 4], s[8 * c + 5]);
-        v.w = pack_bf16(s[8 * c + 6], s[8 * c + 7]);
-        sts128(sSt + swz128(r, 8 * c), v);
+      for (int c8 = 0; c8 < 4; ++c8) {
+        uint4 w;
+        w.x = pack_bf16(__uint_as_float(v[8 * c8 + 0]), __uint_as_float(v[8 * c8 + 1]));
+        w.y = pack_bf16(__uint_as_float(v[8 * c8 + 2]), __uint_as_float(v[8 * c8 + 3]));
+        w.z = pack_bf16(__uint_as_float(v[8 * c8 + 4]), __uint_as_float(v[8 * c8 + 5]));
+        w.w = pack_bf16(__uint_as_float(v[8 * c8 + 6]), __uint_as_float(v[8 * c8 + 7]));
+        sts128(sSt + swz128(r, 32 * c + 8 * c8), w);
       }
-      fence_async_smem();
-      mbar_arrive(&bar[STATEFULL]);
+    };
+    auto scale_back = [&](int c, uint32_t* v, float dec) {
+      const float2 dec2 = make_float2(dec, dec);
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        const float2 o = mul2(dec2, make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])));
+        v[i] = __float_as_uint(o.x);
+        v[i + 1] = __float_as_uint(o.y);
+      }
+      tmem_st32(tSt + 32 * c, v);
     };
     float Dh = 0.f;
     int64_t u = -1;
@@ -677,6 +651,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool first, last, carry_in, carry_out;
       rg.at(k, u, j, first, last, carry_in, carry_out);
       if (first) {
+        // a new piece: its initial state (given, carried or zero) is published
+        // for y_inter(k) and written, times exp(lam_end(k)), for b_intra(k)
         b = (int)(u / hpp);
         h = (int)(u % hpp) * 2 + hl;
         Dh = p.D ? p.D[h] : 0.f;
@@ -701,47 +677,129 @@ __global__ void __launch_bounds__(THREADS, 1)
         } else if (p.init) {
           src = p.init + ((int64_t)b * p.H + h) * NS * P;
         }
-        if (src && !*abort_flag) {
-          const float4* s4 = reinterpret_cast<const float4*>(src + (int64_t)r * P);
+        if (src && *abort_flag) src = nullptr;
+        ctl.wait(LAMRDY0 + (int)(k & 3), (uint32_t)((k >> 2) & 1));
+        const float dec = ex2(tab((int)(k & 3), hl, 0)[T - 1]);
 #pragma unroll
-          for (int i = 0; i < P / 4; ++i) {
-            const float4 v = s4[i];
-            s[4 * i] = v.x;
-            s[4 * i + 1] = v.y;
-            s[4 * i + 2] = v.z;
-            s[4 * i + 3] = v.w;
+        for (int c = 0; c < 2; ++c) {
+          uint32_t v[32];
+          if (src) {
+            const float4* s4 = reinterpret_cast<const float4*>(src + (int64_t)r * P + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 f = s4[i];
+              v[4 * i] = __float_as_uint(f.x);
+              v[4 * i + 1] = __float_as_uint(f.y);
+              v[4 * i + 2] = __float_as_uint(f.z);
+              v[4 * i + 3] = __float_as_uint(f.w);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
           }
-        } else {
-#pragma unroll
-          for (int i = 0; i < P; ++i) s[i] = 0.f;
+          publish_half(c, v);
+          scale_back(c, v, dec);
         }
-        publish_state();  // the state before this piece's first sub-chunk
+        fence_async_smem();
+        mbar_arrive(&bar[STATEFULL]);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar[BIREADY]);
       }
       const int slot = (int)(k & 3), pi = (int)(k & 1), st = (int)(k & 1);
-      bool ok = ctl.wait(LAMRDY0 + slot, (uint32_t)((k >> 2) & 1));
-      if (ok) ok = ctl.wait(BIFULL, (uint32_t)(k & 1));
-      tc_fence_after();
       const float* lj = tab(slot, hl, 0);
-      // state: s(k) = exp(lam_end) s(k-1) + b_intra(k)
-      const float dec = ex2(lj[T - 1]);
-      const float2 dec2 = make_float2(dec, dec);
+      // ---- P = S (.) L of this head into SP[1-pi], columns 64 hl .. +63
+      {
+        bool ok = ctl.wait(LAMRDY0 + slot, (uint32_t)((k >> 2) & 1));
+        if (ok) ok = ctl.wait(SFULL, (uint32_t)(k & 1));
+        (void)ok;
+        tc_fence_after();
+        const uint32_t tS = tmem + lq + TM_SP + 128 * pi, tP = tmem + lq + TM_SP + 128 * (1 - pi) + 64 * hl;
+        const float lam_t = lj[r];
+        const float* ec = tab(slot, hl, 1);
+        auto make_block = [&](int kb, const uint32_t* rv, uint32_t* pk) {
+          if (kb < q) {
+            // below the diagonal block: exp(lam_t - lam_s) = 2^(lt - l_end(kb)) * ec[s]
+            const float4* ec4 = reinterpret_cast<const float4*>(ec);
+            const float rowf = ex2(lam_t - lj[32 * kb + 31]);
+            const float2 rf2 = make_float2(rowf, rowf);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lq + TM_BI + 64 * hl + 32 * c, v);
-        tmem_wait_ld();
+            for (int v = 0; v < 8; ++v) {
+              const float4 c = ec4[8 * kb + v];
+              const float2 a0 = mul2(mul2(make_float2(__uint_as_float(rv[4 * v]), __uint_as_float(rv[4 * v + 1])),
+                                          make_float2(c.x, c.y)),
+                                     rf2);
+              const float2 a1 = mul2(mul2(make_float2(__uint_as_float(rv[4 * v + 2]), __uint_as_float(rv[4 * v + 3])),
+                                          make_float2(c.z, c.w)),
+                                     rf2);
+              pk[2 * v] = pack_bf16(a0.x, a0.y);
+              pk[2 * v + 1] = pack_bf16(a1.x, a1.y);
+            }
+          } else if (kb == q) {
+            // diagonal block: direct decays, clamped at 0 above the diagonal and then zeroed
+            const float4* lj4 = reinterpret_cast<const float4*>(lj);
+            const int rl = r - 32 * kb;
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float2 o = fma2(dec2, make_float2(s[32 * c + i], s[32 * c + i + 1]),
-                                make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])));
-          s[32 * c + i] = o.x;
-          s[32 * c + i + 1] = o.y;
+            for (int v = 0; v < 8; ++v) {
+              const float4 l = lj4[8 * kb + v];
+              float e0 = ex2(fminf(lam_t - l.x, 0.f)), e1 = ex2(fminf(lam_t - l.y, 0.f));
+              float e2 = ex2(fminf(lam_t - l.z, 0.f)), e3 = ex2(fminf(lam_t - l.w, 0.f));
+              if constexpr (XDT) {
+                const float4 fx = reinterpret_cast<const float4*>(tab(slot, hl, 2))[8 * kb + v];
+                e0 *= fx.x;
+                e1 *= fx.y;
+                e2 *= fx.z;
+                e3 *= fx.w;
+              }
+              const float f0 = (4 * v + 0 <= rl) ? __uint_as_float(rv[4 * v + 0]) * e0 : 0.f;
+              const float f1 = (4 * v + 1 <= rl) ? __uint_as_float(rv[4 * v + 1]) * e1 : 0.f;
+              const float f2 = (4 * v + 2 <= rl) ? __uint_as_float(rv[4 * v + 2]) * e2 : 0.f;
+              const float f3 = (4 * v + 3 <= rl) ? __uint_as_float(rv[4 * v + 3]) * e3 : 0.f;
+              pk[2 * v] = pack_bf16(f0, f1);
+              pk[2 * v + 1] = pack_bf16(f2, f3);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = 0u;
+          }
+        };
+#pragma unroll 1
+        for (int kb = 0; kb < 4; kb += 2) {
+          uint32_t r0[32], r1[32], pk[16];
+          // warp-uniform: only blocks on or below the diagonal block are read
+          if (kb <= q) tmem_ld32(tS + 32 * kb, r0);
+          if (kb + 1 <= q) tmem_ld32(tS + 32 * (kb + 1), r1);
+          tmem_wait_ld();
+          make_block(kb, r0, pk);
+          tmem_st16(tP + 16 * kb, pk);
+          make_block(kb + 1, r1, pk);
+          tmem_st16(tP + 16 * (kb + 1), pk);
         }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar[PFULL]);
       }
-      tc_fence_before();
-      mbar_arrive(&bar[BIEMPTY]);
+      // ---- state: the MMA left s(k) = exp(lam_end) s(k-1) + b_intra(k) in TMEM
+      bool ok = ctl.wait(BIFULL, (uint32_t)(k & 1));
+      tc_fence_after();
       if (!last) {
-        publish_state();  // y_inter(k) has completed (BIFULL covers it): the buffer is free
+        // publish bf16 s(k) for y_inter(k+1) (y_inter(k) has completed: BIFULL
+        // covers it) and write exp(lam_end(k+1)) s(k) back for b_intra(k+1)
+        ctl.wait(LAMRDY0 + (int)((k + 1) & 3), (uint32_t)(((k + 1) >> 2) & 1));
+        const float dec = ex2(tab((int)((k + 1) & 3), hl, 0)[T - 1]);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tSt + 32 * c, v);
+          tmem_wait_ld();
+          publish_half(c, v);
+          scale_back(c, v, dec);
+        }
+        fence_async_smem();
+        mbar_arrive(&bar[STATEFULL]);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar[BIREADY]);
       } else {
         // end of a piece: the sequence's final state, or the carry of a head piece
         float* dst = nullptr;
@@ -749,19 +807,29 @@ __global__ void __launch_bounds__(THREADS, 1)
           dst = p.carry + ((int64_t)blockIdx.x * 2 + hl) * NS * P;
         else if (p.final_state)
           dst = p.final_state + ((int64_t)b * p.H + h) * NS * P;
-        if (dst) {
-          float4* d4 = reinterpret_cast<float4*>(dst + (int64_t)r * P);
 #pragma unroll
-          for (int i = 0; i < P / 4; ++i) d4[i] = make_float4(s[4 * i], s[4 * i + 1], s[4 * i + 2], s[4 * i + 3]);
+        for (int c = 0; c < 2; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tSt + 32 * c, v);
+          tmem_wait_ld();
+          if (dst) {
+            float4* d4 = reinterpret_cast<float4*>(dst + (int64_t)r * P + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                  __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          }
         }
+        tc_fence_before();
         if (carry_out) {
           __threadfence();
-          named_sync(4, EPIT);
+          named_sync(2, EPIT);
           if (et == 0 && p.withhold != 2) st_release(p.carry_flag + blockIdx.x, 1);
         }
       }
-      // y_t = y_intra + exp(lam_t) y_inter + D x_t, written over this head's x
-      // row (each thread reads and writes only its own row) and stored by TMA
+      // ---- y_t = y_intra + exp(lam_t) y_inter + D x_t, written over this head's
+      // x row (each thread reads and writes only its own row); the producer
+      // stores the tile once all 128 rows are staged
       if (ok) ok = ctl.wait(YFULL, (uint32_t)(k & 1));
       tc_fence_after();
       const float etl = ex2(lj[r]);
@@ -794,18 +862,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(&bar[YEMPTY]);
-      fence_async_smem();
-      named_sync(2 + hl, T);  // this head's 128 rows are staged
-      if (r == 0) {
-        if (!*abort_flag) {
-          tma_store_4d(&map_y, sm + OFF_X + st * 2 * TILE + hl * TILE, 0, h, j * T, b);
-          tma_store_commit();
-          tma_store_wait_read0();
-        }
-        mbar_arrive(&bar[XEMPTY0 + st]);
-      }
+      fence_async_smem();  // the y rows are visible to the store (async proxy)
+      mbar_arrive(&bar[YSTAGED0 + hl]);
     }
-    if (r == 0) tma_store_wait0();  // the y tiles are in global memory before the CTA exits
   }
 
   tc_fence_before();

@@ -32,7 +32,8 @@
 //
 // TMEM (512 columns): two 128-column regions SP[0], SP[1] take turns -- S(k)
 // goes to SP[k&1], P(k) to SP[1-(k&1)], y_intra(k) back to SP[k&1] -- so S of
-// the next sub-chunk starts while this one's outputs are being read; y_inter
+// the next sub-chunk (issued once y_intra(k), the reader of P(k), completed)
+// runs while this one's outputs are being read; y_inter
 // has 128 columns, and the running fp32 state of both heads lives in the last
 // 128 (after b_intra(k) it holds s(k); the head warps read it, publish its
 // bf16 copy for y_inter(k+1), and write exp(lam_end(k+1)) s(k) back for the
@@ -445,8 +446,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int pi = (int)(k & 1);
         const uint32_t tS = tmem + TM_SP + 128 * pi, tP = tmem + TM_SP + 128 * (1 - pi);
         const uint32_t ph = (uint32_t)(k & 1), php = (uint32_t)((k - 1) & 1);
-        // S(k) into SP[pi] (its last reader, y_intra(k-1), was issued before)
+        // S(k) into SP[pi], over P(k-1): the y_intra(k-1) MMAs read their A
+        // operand there, and MMAs into different accumulators carry no
+        // read-before-write order, so S(k) waits until they have completed
         if (ok) ok = ctl.wait(BCFULL, ph);
+        if (ok && k > 0) ok = ctl.wait(YFULL, php);
         if (ok) {
           tc_fence_after();
 #pragma unroll

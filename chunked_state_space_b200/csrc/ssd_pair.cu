@@ -77,7 +77,7 @@ constexpr uint32_t OFF_TAB = 12 * TILE;          // float tables [slot 4][head 2
 constexpr uint32_t TAB_BYTES = 4 * 2 * 3 * T * 4;
 constexpr uint32_t OFF_WTOT = OFF_TAB + TAB_BYTES;  // scan partials [head 2][warp 2]
 constexpr uint32_t OFF_BAR = OFF_WTOT + 64;
-constexpr uint32_t NBAR = 18;
+constexpr uint32_t NBAR = 20;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
@@ -94,9 +94,11 @@ enum {
   STATEFULL = 7,  // bf16 state published (256)
   YEMPTY = 8,     // y_inter read (256)
   XFULL0 = 9,     // [stage] x tiles landed (tx)
-  YSTAGED0 = 11,  // [head] 128 y rows of the head staged in its x tile (128)
-  LAMRDY0 = 13,   // [slot 4] tables written (64 aux threads)
-  DRAIN = 17
+  YSTAGED0 = 11,  // [stage][head] 128 y rows of the head staged in its x tile (128); one barrier per
+                  // stage, so the head warps cannot complete a second phase before the producer has
+                  // seen the first (the stage is reloaded only after the producer stored its y)
+  LAMRDY0 = 15,   // [slot 4] tables written (64 aux threads)
+  DRAIN = 19
 };
 constexpr int AUX = 64, HEADT = 128, EPIT = 256;
 constexpr int W_TMA = 0, W_MMA = 1;
@@ -304,10 +306,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&bar[BIREADY], EPIT);
     mbar_init(&bar[STATEFULL], EPIT);
     mbar_init(&bar[YEMPTY], EPIT);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar[XFULL0 + i], 1);
-      mbar_init(&bar[YSTAGED0 + i], HEADT);
-    }
+    for (int i = 0; i < 2; ++i) mbar_init(&bar[XFULL0 + i], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&bar[YSTAGED0 + i], HEADT);
     for (int i = 0; i < 4; ++i) mbar_init(&bar[LAMRDY0 + i], AUX);
     mbar_init(&bar[DRAIN], 1);
     fence_mbar_init();
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint64_t t_last = globaltimer_ns();
       while ((kb < K || kx < K || ky < K) && !*abort_flag) {
         bool progress = false;
-        if (ky < K && mbar_test_wait(&bar[YSTAGED0 + hy], (uint32_t)(ky & 1))) {
+        if (ky < K && mbar_test_wait(&bar[YSTAGED0 + 2 * (ky & 1) + hy], (uint32_t)((ky >> 1) & 1))) {
           int b, h0, g, t0;
           coords(ky, b, h0, g, t0);
           tma_store_4d(&map_y, sm + OFF_X + (ky & 1) * 2 * TILE + hy * TILE, 0, h0 + hy, t0, b);
@@ -867,7 +867,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       mbar_arrive(&bar[YEMPTY]);
       fence_async_smem();  // the y rows are visible to the store (async proxy)
-      mbar_arrive(&bar[YSTAGED0 + hl]);
+      mbar_arrive(&bar[YSTAGED0 + 2 * st + hl]);
     }
   }
 

@@ -309,11 +309,12 @@ def ssd_vertical_workspace_size(dims: Dims, n_layers: int, vblock: int) -> int:
 
 
 def ssd_vertical_fwd(x0, layers: Sequence[dict], states: Sequence[torch.Tensor], vblock: int, chunk: int = 256,
-                     rms_eps: float = 1e-6, y_out=None, workspace=None, stream=None, input_dt: bool = False):
+                     rms_eps: float = 1e-6, y_out=None, workspace=None, stream=None, input_dt: bool = False,
+                     one_head: bool = False):
     """Depth-first multi-layer schedule.  layers[l] has dt, A, B, C and optionally D;
     states[l] ([B,H,N,P] f32) holds layer l's initial state and receives its final state."""
     n = len(layers)
-    dims = make_dims(x0, layers[0]["B"], chunk, input_dt)
+    dims = make_dims(x0, layers[0]["B"], chunk, input_dt, one_head)
     _contig(x0, *[t for p in layers for t in (p["dt"], p["A"], p["B"], p["C"], p.get("D"))], *states)
     if y_out is None:
         y_out = torch.empty_like(x0)

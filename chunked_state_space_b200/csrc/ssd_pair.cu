@@ -18,17 +18,20 @@
 //                                                           MMA accumulates onto the scaled state)
 // (with the dt-scaled input every column s of P and row s of X' also carries dt_s).
 //
-// Warp roles (384 threads): warp 0 runs every TMA transfer -- loads of x (two
-// stages, both heads), B and C (one buffer), L2 prefetches, and the stores of
-// finished y tiles; warp 1 owns TMEM and issues the MMAs in the order S,
-// y_inter, b_intra, y_intra; warps 2-3 load dt, scan lam and write X'; warps
-// 4-7 / 8-11 are the warps of head a / b (warp w owns TMEM lane quarter w % 4,
-// one thread per row): they turn S into that head's P, then update its state
-// and finish its y.  The two heads' masks thus run side by side, two warps
-// per SM sub-partition.  The x tile of a head is also where its y tile is
-// staged for the TMA store: each thread reads its own x row and overwrites it
-// with its y row; the producer stores the tile once all 128 rows are staged,
-// so no head warp waits for a store.
+// Warp roles (384 threads): lane 0 of warp 0 issues the TMA loads -- x (two
+// stages, both heads), B and C (one buffer) -- and L2 prefetches, and never
+// blocks; lane 1 of warp 0 stores finished y tiles (the two lanes diverge and
+// each runs while the other waits); warp 1
+// owns TMEM and issues the MMAs in the order S, y_inter, b_intra, y_intra;
+// warps 2-3 load dt, scan lam and write X'; warps 4-7 / 8-11 are the warps of
+// head a / b (warp w owns TMEM lane quarter w % 4, one thread per row): they
+// turn S into that head's P, then update its state and finish its y.  The two
+// heads' masks thus run side by side, two warps per SM sub-partition.  The x
+// tile of a head is also where its y tile is staged for the TMA store: each
+// thread reads its own x row and overwrites it with its y row; the store lane
+// stores the tile once all 128 rows are staged and, once the store has read
+// both heads' tiles, frees the x stage for the next load.  No head warp waits
+// for a store, and no load waits behind one.
 //
 // TMEM (512 columns): two 128-column regions SP[0], SP[1] take turns -- S(k)
 // goes to SP[k&1], P(k) to SP[1-(k&1)], y_intra(k) back to SP[k&1] -- so S of
@@ -77,7 +80,7 @@ constexpr uint32_t OFF_TAB = 12 * TILE;          // float tables [slot 4][head 2
 constexpr uint32_t TAB_BYTES = 4 * 2 * 3 * T * 4;
 constexpr uint32_t OFF_WTOT = OFF_TAB + TAB_BYTES;  // scan partials [head 2][warp 2]
 constexpr uint32_t OFF_BAR = OFF_WTOT + 64;
-constexpr uint32_t NBAR = 20;
+constexpr uint32_t NBAR = 22;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
@@ -95,10 +98,11 @@ enum {
   YEMPTY = 8,     // y_inter read (256)
   XFULL0 = 9,     // [stage] x tiles landed (tx)
   YSTAGED0 = 11,  // [stage][head] 128 y rows of the head staged in its x tile (128); one barrier per
-                  // stage, so the head warps cannot complete a second phase before the producer has
-                  // seen the first (the stage is reloaded only after the producer stored its y)
+                  // stage, so the head warps cannot complete a second phase before the store lane has
+                  // seen the first (the stage is reloaded only after its y was stored)
   LAMRDY0 = 15,   // [slot 4] tables written (64 aux threads)
-  DRAIN = 19
+  DRAIN = 19,
+  XEMPTY0 = 20    // [stage] both y tiles stored from the stage and read (store lane, 1)
 };
 constexpr int AUX = 64, HEADT = 128, EPIT = 256;
 constexpr int W_TMA = 0, W_MMA = 1;
@@ -260,17 +264,6 @@ __device__ __forceinline__ void st_release(int* p, int v) {
 }
 
 
-// Wait until at most `n` bulk store groups of this thread are still reading
-// shared memory (n = 0, 1 or 2).
-__device__ __forceinline__ void store_wait_read(int n) {
-  if (n <= 0)
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-  else if (n == 1)
-    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-  else
-    asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory");
-}
-
 template <bool XDT>
 __global__ void __launch_bounds__(THREADS, 1)
     k_ssd_pair(Params p, const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
@@ -306,7 +299,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&bar[BIREADY], EPIT);
     mbar_init(&bar[STATEFULL], EPIT);
     mbar_init(&bar[YEMPTY], EPIT);
-    for (int i = 0; i < 2; ++i) mbar_init(&bar[XFULL0 + i], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[XFULL0 + i], 1);
+      mbar_init(&bar[XEMPTY0 + i], 1);
+    }
     for (int i = 0; i < 4; ++i) mbar_init(&bar[YSTAGED0 + i], HEADT);
     for (int i = 0; i < 4; ++i) mbar_init(&bar[LAMRDY0 + i], AUX);
     mbar_init(&bar[DRAIN], 1);
@@ -334,10 +330,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == W_TMA) {
     // ------------------------------------------------------------ TMA producer
-    // Three queues polled in turn: y stores (head a then b of sub-chunk ky, once
-    // its 128 rows are staged), B/C of sub-chunk kb (one buffer, free once
-    // y_inter and b_intra of kb-1 completed), x of sub-chunk kx (two stages, free
-    // once both heads' y tiles of kx-2 have been read by their stores).
+    // Two queues polled in turn: B/C of sub-chunk kb (one buffer, free once
+    // y_inter and b_intra of kb-1 completed) and x of sub-chunk kx (two stages,
+    // free once the store warp has stored both heads' y tiles of kx-2).
     if (lane == 0) {
       constexpr int kPrefetch = 3;
       auto prefetch = [&](int64_t k) {
@@ -353,41 +348,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       };
       for (int64_t k = 0; k < kPrefetch; ++k) prefetch(k);
       const bool loads = p.withhold != 1;
-      int64_t kb = 0, kx = 0, ky = 0, pf = kPrefetch;
-      int hy = 0;          // next head to store of sub-chunk ky
-      int64_t groups = 0;  // store groups committed (one per head tile)
+      int64_t kb = 0, kx = 0, pf = kPrefetch;
       uint32_t idle = 0;
       uint64_t t_last = globaltimer_ns();
-      while ((kb < K || kx < K || ky < K) && !*abort_flag) {
+      while ((kb < K || kx < K) && !*abort_flag) {
         bool progress = false;
-        if (ky < K && mbar_test_wait(&bar[YSTAGED0 + 2 * (ky & 1) + hy], (uint32_t)((ky >> 1) & 1))) {
-          int b, h0, g, t0;
-          coords(ky, b, h0, g, t0);
-          tma_store_4d(&map_y, sm + OFF_X + (ky & 1) * 2 * TILE + hy * TILE, 0, h0 + hy, t0, b);
-          tma_store_commit();
-          ++groups;
-          if (++hy == 2) {
-            hy = 0;
-            ++ky;
-          }
-          progress = true;
-        }
-        // x(kx) reuses the stage of x(kx-2): both y tiles of kx-2 must have been
-        // stored (issued) and read; groups issued after them may stay in flight
-        if (kx < K && kx <= kb + 1 && (kx < 2 || ky > kx - 2)) {
-          if (kx >= 2) store_wait_read((int)(groups - 2 * (kx - 1)));
-          int b, h0, g, t0;
-          coords(kx, b, h0, g, t0);
-          const int st = (int)(kx & 1);
-          uint8_t* dst = sm + OFF_X + st * 2 * TILE;
-          if (loads) {
-            mbar_arrive_expect_tx(&bar[XFULL0 + st], 2 * TILE);
-            tma_load_4d(dst, &map_x, &bar[XFULL0 + st], 0, h0, t0, b);
-            tma_load_4d(dst + TILE, &map_x, &bar[XFULL0 + st], 0, h0 + 1, t0, b);
-          }
-          ++kx;
-          progress = true;
-        }
         if (kb < K && (kb < 1 || mbar_test_wait(&bar[BIFULL], (kb - 1) & 1))) {
           int b, h0, g, t0;
           coords(kb, b, h0, g, t0);
@@ -400,6 +365,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           ++kb;
           if (pf < kb + kPrefetch) prefetch(pf++);
+          progress = true;
+        }
+        if (kx < K && kx <= kb + 1 &&
+            (kx < 2 || mbar_test_wait(&bar[XEMPTY0 + (kx & 1)], (uint32_t)(((kx - 2) >> 1) & 1)))) {
+          int b, h0, g, t0;
+          coords(kx, b, h0, g, t0);
+          const int st = (int)(kx & 1);
+          uint8_t* dst = sm + OFF_X + st * 2 * TILE;
+          if (loads) {
+            mbar_arrive_expect_tx(&bar[XFULL0 + st], 2 * TILE);
+            tma_load_4d(dst, &map_x, &bar[XFULL0 + st], 0, h0, t0, b);
+            tma_load_4d(dst + TILE, &map_x, &bar[XFULL0 + st], 0, h0 + 1, t0, b);
+          }
+          ++kx;
           progress = true;
         }
         if (progress) {
@@ -415,9 +394,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           __nanosleep(32);
         }
       }
-      // every load issued must land and every store complete before the CTA
-      // may exit (bounded: valid tiles land unless the device is wedged)
-      tma_store_wait0();
+      // every load issued must land before the CTA may exit (bounded: valid
+      // tiles land unless the device is wedged)
       if (loads) {
         const uint64_t t0 = globaltimer_ns();
         if (kb > 0)
@@ -427,6 +405,27 @@ __global__ void __launch_bounds__(THREADS, 1)
           while (!mbar_try_wait(&bar[XFULL0 + (k & 1)], (k >> 1) & 1) && globaltimer_ns() - t0 < 1000000000ull) {
           }
       }
+    }
+    if (lane == 1) {
+      // ---------------------------------------------------------- y stores
+      // head a then head b of each sub-chunk once its 128 rows are staged;
+      // then wait until both stores have read the stage and free it for x(k+2)
+      for (int64_t k = 0; k < K; ++k) {
+        int b, h0, g, t0;
+        coords(k, b, h0, g, t0);
+        const int st = (int)(k & 1);
+#pragma unroll 1
+        for (int hy = 0; hy < 2; ++hy) {
+          const bool ok = ctl.wait(YSTAGED0 + 2 * st + hy, (uint32_t)((k >> 1) & 1));
+          if (ok) {
+            tma_store_4d(&map_y, sm + OFF_X + st * 2 * TILE + hy * TILE, 0, h0 + hy, t0, b);
+            tma_store_commit();
+          }
+        }
+        tma_store_wait_read0();
+        mbar_arrive(&bar[XEMPTY0 + st]);
+      }
+      tma_store_wait0();  // the y tiles are in global memory before the CTA exits
     }
   } else if (warp == W_MMA) {
     // ------------------------------------------------------------ MMA issuer

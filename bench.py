@@ -266,8 +266,8 @@ def main():
                          "batch, heads and sizes instead of the scan")
     ap.add_argument("--unfused", action="store_true",
                     help="time the four step kernels (ssd_scan_fwd_unfused) instead of the fused kernel")
-    ap.add_argument("--one-head", action="store_true",
-                    help="the one-head-per-CTA fused kernel even where the two-head kernel applies (comparison)")
+    ap.add_argument("--two-heads", action="store_true",
+                    help="the fused kernel with two heads of a group per CTA (SSD_FLAG_TWO_HEADS_PER_CTA; comparison)")
     ap.add_argument("--no-extras", action="store_true",
                     help="layer stacks: skip the horizontal and graph-replay figures (sweeps)")
     args = ap.parse_args()
@@ -307,7 +307,7 @@ def main():
     d = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
     y = torch.empty_like(d["x"])
     fin = torch.empty((wl.batch, wl.nheads, wl.dstate, wl.headdim), dtype=torch.float32, device=dev)
-    dims = ssd.make_dims(d["x"], d["B"], wl.chunk, args.input_dt, args.one_head)
+    dims = ssd.make_dims(d["x"], d["B"], wl.chunk, args.input_dt, args.two_heads)
     ws = torch.empty(max(ssd.ssd_scan_workspace_size(dims), 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     torch.cuda.synchronize(dev)
@@ -315,7 +315,7 @@ def main():
     def step():
         ssd.ssd_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init"], chunk=wl.chunk, y=y,
                          final_state=fin, workspace=ws, stream=stream, input_dt=args.input_dt,
-                         one_head=args.one_head, unfused=args.unfused)
+                         two_heads=args.two_heads, unfused=args.unfused)
 
     if args.strided:  # x, B, C as views of one fused projection output
         HP, GN = wl.nheads * wl.headdim, wl.ngroups * wl.dstate
@@ -330,7 +330,7 @@ def main():
         def step():  # noqa: F811
             ssd.ssd_scan_fwd_strided(xv, d["dt"], d["A"], bv, cv, d["D"], d["init"], chunk=wl.chunk, y=y,
                                      final_state=fin, stream=stream, input_dt=args.input_dt,
-                                     one_head=args.one_head)
+                                     two_heads=args.two_heads)
 
     path, kernels_per_step = ssd.ssd_scan_path(dims)
     if args.unfused:
@@ -393,7 +393,7 @@ def main():
                    "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk,
                    "state_dtype": "f32", "path": path, "parallelism": f"dp{world} (independent batches per rank)",
                    "variant": (("input_dt " if args.input_dt else "") + ("strided " if args.strided else "") +
-                               ("one_head" if args.one_head else "")).strip() or "plain",
+                               ("two_heads" if args.two_heads else "")).strip() or "plain",
                    "l2": ("512 MB L2 flush between steps (inputs fit in L2); per-step events exclude it"
                           if flush is not None else
                           f"inputs larger than L2 ({algorithmic_bytes(wl) / 1e9:.2f} GB per rank); no flush")},

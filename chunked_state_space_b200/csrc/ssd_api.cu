@@ -24,7 +24,7 @@ size_t io_size(int io) { return io == SSD_BF16 ? 2 : 4; }
 
 ssd_status validate_dims(const ssd_dims* d) {
   if (!d) return SSD_ERR_INVALID_ARG;
-  if ((d->flags & ~(SSD_FLAG_INPUT_DT | SSD_FLAG_ONE_HEAD_PER_CTA)) != 0) return SSD_ERR_INVALID_ARG;
+  if ((d->flags & ~(SSD_FLAG_INPUT_DT | SSD_FLAG_TWO_HEADS_PER_CTA)) != 0) return SSD_ERR_INVALID_ARG;
   if (d->io_dtype != SSD_F32 && d->io_dtype != SSD_BF16) return SSD_ERR_DTYPE;
   if (d->batch < 1 || d->seqlen < 1 || d->nheads < 1 || d->headdim < 1 || d->dstate < 1 || d->ngroups < 1 ||
       d->chunk < 1)
@@ -57,7 +57,7 @@ Problem make_problem(const ssd_dims* d) {
   p.lddt = p.H;
   p.ldbc = p.G * p.N;
   p.input_dt = (d->flags & SSD_FLAG_INPUT_DT) ? 1 : 0;
-  p.single_head = (d->flags & SSD_FLAG_ONE_HEAD_PER_CTA) ? 1 : 0;
+  p.two_heads = (d->flags & SSD_FLAG_TWO_HEADS_PER_CTA) ? 1 : 0;
   return p;
 }
 

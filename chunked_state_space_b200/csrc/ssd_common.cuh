@@ -30,7 +30,7 @@ struct Problem {
   // lddt = H, ldbc = G*N.  Only the fused tensor-core kernel reads them.
   int64_t ldx, lddt, ldbc, ldy;
   int input_dt;     // SSD_FLAG_INPUT_DT: the input term is dt_t B_t x_t^T
-  int single_head;  // SSD_FLAG_ONE_HEAD_PER_CTA: never the two-head kernel
+  int two_heads;    // SSD_FLAG_TWO_HEADS_PER_CTA: the two-head kernel where it applies
 };
 
 template <typename T>

@@ -57,6 +57,7 @@
 // on every barrier it arrives on, so no barrier phase is left half-counted and
 // no copy is in flight when the CTA exits.
 #include "ssd_common.cuh"
+#include "ssd_split.cuh"
 #include "tma.cuh"
 #include "umma.cuh"
 
@@ -64,6 +65,9 @@ namespace ssd {
 namespace pair {
 
 using namespace umma;
+using split::Range;
+using split::ld_acquire;
+using split::st_release;
 
 constexpr int T = 128;   // tokens per sub-chunk
 constexpr int P = 64;    // head dim
@@ -123,62 +127,6 @@ struct Params {
   float* carry;            // [nctas][2][NS][P] end states of head pieces, or NULL (no split)
   int* carry_flag;         // [nctas], zeroed before the launch
   int withhold;            // self-test of the bounded waits: 1 = no TMA loads, 2 = no carries published
-};
-
-// The sub-chunks of CTA c: [lo, hi) of the concatenated list, run in the order
-// head piece of the last sequence (if the range ends inside it), whole
-// sequences, tail piece of the first sequence (if the range starts inside it).
-struct Range {
-  int64_t lo, hi;
-  int nsub;
-  int64_t u_lo, u_hi;  // first and last sequence touched
-  int j_lo, j_hi;      // start of the first piece, end (exclusive) of the last piece
-  int head_len;        // sub-chunks of the leading head piece (0 if none)
-  int tail_len;        // sub-chunks of the trailing tail piece (0 if none)
-  int64_t full_first;  // first whole sequence
-  __device__ void init(int64_t total, int nctas, int c, int ns) {
-    nsub = ns;
-    lo = total * c / nctas;
-    hi = total * (c + 1) / nctas;
-    u_lo = lo / ns;
-    j_lo = (int)(lo % ns);
-    u_hi = (hi - 1) / ns;
-    j_hi = (int)((hi - 1) % ns) + 1;
-    head_len = (u_hi > u_lo && j_hi < ns) ? j_hi : 0;
-    tail_len = j_lo > 0 ? ns - j_lo : 0;
-    full_first = j_lo > 0 ? u_lo + 1 : u_lo;
-  }
-  __device__ int64_t count() const { return hi - lo; }
-  // sequence, sub-chunk, and piece boundaries of the k-th sub-chunk this CTA runs
-  __device__ void at(int64_t k, int64_t& u, int& j, bool& first, bool& last, bool& carry_in,
-                     bool& carry_out) const {
-    if (k < head_len) {
-      u = u_hi;
-      j = (int)k;
-      first = (k == 0);
-      last = (k == head_len - 1);
-      carry_in = false;
-      carry_out = last;
-      return;
-    }
-    const int64_t kk = k - head_len;
-    const int64_t nfull_sub = count() - head_len - tail_len;
-    if (kk < nfull_sub) {
-      u = full_first + kk / nsub;
-      j = (int)(kk % nsub);
-      first = (j == 0);
-      last = (j == nsub - 1);
-      carry_in = carry_out = false;
-      return;
-    }
-    const int64_t kt = kk - nfull_sub;
-    u = u_lo;
-    j = j_lo + (int)kt;
-    first = (kt == 0);
-    last = (j == nsub - 1);
-    carry_in = first;
-    carry_out = false;
-  }
 };
 
 struct Ctl {
@@ -253,16 +201,6 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
 __device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
-
-__device__ __forceinline__ int ld_acquire(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release(int* p, int v) {
-  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
 
 template <bool XDT>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -887,36 +825,14 @@ bool pair_supported(const Problem& p) {
          p.B * p.H < (1ll << 31);
 }
 
-static int sm_count() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cached[dev] = n;
-  }
-  return cached[dev];
-}
-
-// CTAs of the split schedule: one per SM, never more than the head pairs (a
-// range is then at least one whole sequence long, so no piece needs a carry in
-// and a carry out at once).
-int pair_split_ctas(const Problem& p) {
-  const int64_t npairs = p.B * p.H / 2;
-  const int64_t n = sm_count();
-  return (int)(npairs < n ? npairs : n);
-}
+// CTAs of the split schedule: one per SM, never more than the head pairs.
+int pair_split_ctas(const Problem& p) { return split::ctas(p.B * p.H / 2); }
 
 // Workspace of the split schedule: the carries [ctas][2][N][P] f32 and their
 // flags, or 0 when every CTA runs whole sequences anyway.
 size_t pair_workspace_bytes(const Problem& p) {
   if (!pair_supported(p)) return 0;
-  const int64_t npairs = p.B * p.H / 2;
-  const int ctas = pair_split_ctas(p);
-  if (ctas >= npairs) return 0;  // one whole sequence per CTA
-  const size_t carry = (size_t)ctas * 2 * pair::NS * pair::P * sizeof(float);
-  return carry + (size_t)((ctas * sizeof(int) + 255) / 256 * 256);
+  return split::workspace_bytes(p.B * p.H / 2, (size_t)2 * pair::NS * pair::P);
 }
 
 // withhold: 0 normal; 1 issue no TMA loads (self-test of the bounded waits);

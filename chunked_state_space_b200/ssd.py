@@ -125,16 +125,16 @@ def _io_code(t: torch.Tensor) -> int:
 
 
 FLAG_INPUT_DT = 1        # SSD_FLAG_INPUT_DT: the input term is dt_t B_t x_t^T
-FLAG_ONE_HEAD_PER_CTA = 2  # SSD_FLAG_ONE_HEAD_PER_CTA: never the two-head kernel
+FLAG_TWO_HEADS_PER_CTA = 2  # SSD_FLAG_TWO_HEADS_PER_CTA: the two-head kernel where it applies
 
 
 def make_dims(x: torch.Tensor, Bm: torch.Tensor, chunk: int, input_dt: bool = False,
-              one_head: bool = False) -> Dims:
+              two_heads: bool = False) -> Dims:
     if x.dim() != 4 or Bm.dim() != 4:
         raise SSDError(2, "x must be [B,L,H,P] and B/C [B,L,G,N]")
     Bz, L, H, P = x.shape
     G, N = Bm.shape[2], Bm.shape[3]
-    flags = (FLAG_INPUT_DT if input_dt else 0) | (FLAG_ONE_HEAD_PER_CTA if one_head else 0)
+    flags = (FLAG_INPUT_DT if input_dt else 0) | (FLAG_TWO_HEADS_PER_CTA if two_heads else 0)
     return Dims(Bz, L, H, P, N, G, int(chunk), _io_code(x), flags)
 
 
@@ -169,12 +169,12 @@ def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]):
 
 def ssd_scan_fwd(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, y=None, final_state=None,
                  workspace=None, stream=None, want_final: bool = True, unfused: bool = False, input_dt: bool = False,
-                 one_head: bool = False):
+                 two_heads: bool = False):
     """y, final_state = scan(x, dt, A, B, C, D, init_state) with chunk size `chunk`.
     input_dt: the input term is dt_t B_t x_t^T (tensor-core path).
-    one_head: the one-head-per-CTA fused kernel even where the two-head one applies."""
+    two_heads: the fused kernel with two heads of a group per CTA where it applies."""
     _contig(x, dt, A, Bm, Cm, D, init_state, y, final_state)
-    dims = make_dims(x, Bm, chunk, input_dt, one_head)
+    dims = make_dims(x, Bm, chunk, input_dt, two_heads)
     if y is None:
         y = torch.empty_like(x)
     if final_state is None and want_final:
@@ -221,7 +221,7 @@ def ssd_scan_fwd_host(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 25
 
 
 def ssd_scan_fwd_strided(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, y=None, final_state=None,
-                         stream=None, want_final: bool = True, input_dt: bool = False, one_head: bool = False):
+                         stream=None, want_final: bool = True, input_dt: bool = False, two_heads: bool = False):
     """ssd_scan_fwd on strided views (tensor-core path): x [B,L,H,P], dt [B,L,H],
     B/C [B,L,G,N] and y may have any batch and token strides as long as each
     token's heads (groups) are dense, e.g. slices of one fused projection output.
@@ -232,7 +232,7 @@ def ssd_scan_fwd_strided(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int =
         if tuple(t.stride()[2:]) != inner:
             raise SSDError(2, "each token's heads/groups must be dense")
     _contig(A, D, init_state, final_state)
-    dims = make_dims(x, Bm, chunk, input_dt, one_head)
+    dims = make_dims(x, Bm, chunk, input_dt, two_heads)
     if y is None:
         y = torch.empty(x.shape, dtype=x.dtype, device=x.device)
     if final_state is None and want_final:
@@ -310,11 +310,11 @@ def ssd_vertical_workspace_size(dims: Dims, n_layers: int, vblock: int) -> int:
 
 def ssd_vertical_fwd(x0, layers: Sequence[dict], states: Sequence[torch.Tensor], vblock: int, chunk: int = 256,
                      rms_eps: float = 1e-6, y_out=None, workspace=None, stream=None, input_dt: bool = False,
-                     one_head: bool = False):
+                     two_heads: bool = False):
     """Depth-first multi-layer schedule.  layers[l] has dt, A, B, C and optionally D;
     states[l] ([B,H,N,P] f32) holds layer l's initial state and receives its final state."""
     n = len(layers)
-    dims = make_dims(x0, layers[0]["B"], chunk, input_dt, one_head)
+    dims = make_dims(x0, layers[0]["B"], chunk, input_dt, two_heads)
     _contig(x0, *[t for p in layers for t in (p["dt"], p["A"], p["B"], p["C"], p.get("D"))], *states)
     if y_out is None:
         y_out = torch.empty_like(x0)
@@ -388,22 +388,23 @@ def ssd_selftest_fused_trace(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: i
 
 
 def ssd_selftest_timeout(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, stream=None,
-                         one_head: bool = False) -> None:
-    """Diagnostic: launch the fused kernel (the two-head one where it applies,
-    unless one_head) with its TMA loads withheld, so its bounded waits run out;
-    read the outcome with ssd_read_device_status."""
-    dims = make_dims(x, Bm, chunk, one_head=one_head)
+                         two_heads: bool = False) -> None:
+    """Diagnostic: launch the fused kernel (the two-head one with two_heads, where
+    it applies) with its TMA loads withheld, so its bounded waits run out; read
+    the outcome with ssd_read_device_status."""
+    dims = make_dims(x, Bm, chunk, two_heads=two_heads)
     y = torch.empty_like(x)
     fin = torch.empty((dims.batch, dims.nheads, dims.dstate, dims.headdim), dtype=torch.float32, device=x.device)
     _check(lib().ssd_selftest_timeout(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D),
                                       _ptr(init_state), _ptr(y), _ptr(fin), _stream(stream)), "ssd_selftest_timeout")
 
 
-def ssd_selftest_carry_timeout(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, stream=None) -> None:
-    """Diagnostic: launch the two-head kernel with its split schedule but with no
-    carry ever published, so every wait for one runs out; read the outcome with
-    ssd_read_device_status."""
-    dims = make_dims(x, Bm, chunk)
+def ssd_selftest_carry_timeout(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, stream=None,
+                               two_heads: bool = False) -> None:
+    """Diagnostic: launch the fused kernel (the two-head one with two_heads) with
+    its split schedule but with no carry ever published, so every wait for one
+    runs out; read the outcome with ssd_read_device_status."""
+    dims = make_dims(x, Bm, chunk, two_heads=two_heads)
     y = torch.empty_like(x)
     fin = torch.empty((dims.batch, dims.nheads, dims.dstate, dims.headdim), dtype=torch.float32, device=x.device)
     ws = _workspace(ssd_scan_workspace_size(dims), x.device, None)

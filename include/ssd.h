@@ -94,11 +94,14 @@ typedef struct ssd_dims {
  * tensor-core path takes the shape, and by ssd_step; every other entry point
  * (and ssd_scan_fwd on the CUDA-core path) returns SSD_ERR_UNSUPPORTED.
  *
- * SSD_FLAG_ONE_HEAD_PER_CTA: run the one-head-per-CTA fused kernel even where
- * the two-head kernel takes the shape (same results within rounding; for
- * comparing the two kernels).  Changes nothing on other paths.
+ * SSD_FLAG_TWO_HEADS_PER_CTA: run the fused scan with two heads of a group per
+ * CTA (they share their B and C tiles, S = C B^T and the state products) where
+ * the shape allows it (an even number of heads per group); same results within
+ * rounding.  Kept for comparison: on B200 it measured slower than the default
+ * one-head kernel (its per-row CUDA-core work has half the warps per head).
+ * Changes nothing on other paths.
  */
-typedef enum { SSD_FLAG_INPUT_DT = 1, SSD_FLAG_ONE_HEAD_PER_CTA = 2 } ssd_flags;
+typedef enum { SSD_FLAG_INPUT_DT = 1, SSD_FLAG_TWO_HEADS_PER_CTA = 2 } ssd_flags;
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* ssd_status_string(ssd_status s);
@@ -183,11 +186,12 @@ ssd_status ssd_scan_fwd_host(const ssd_dims* d, const void* x, const float* dt, 
  * Which implementation ssd_scan_fwd uses for `d`: *path = SSD_PATH_CUDA_CORES
  * (four CUDA-core step kernels), SSD_PATH_TENSOR_STEPS (four step kernels,
  * steps 2 and 4 on tcgen05 tensor cores), SSD_PATH_FUSED (one tensor-core
- * kernel, one (batch, head) sequence per CTA) or SSD_PATH_FUSED_PAIR (one
- * tensor-core kernel, two heads of a group per CTA sharing their B and C
- * tiles; with the workspace of ssd_scan_workspace_size it cuts the
- * concatenated sequences into equal ranges, one persistent CTA per SM, and
- * hands the state across range boundaries through the workspace);
+ * kernel) or SSD_PATH_FUSED_PAIR (one tensor-core kernel, two heads of a
+ * group per CTA sharing their B and C tiles; SSD_FLAG_TWO_HEADS_PER_CTA).
+ * With the workspace of ssd_scan_workspace_size and more sequences (pairs)
+ * than SMs, the fused kernels cut the concatenated sequences into equal
+ * ranges, one persistent CTA per SM, and hand the state across range
+ * boundaries through the workspace; otherwise a CTA runs whole sequences;
  * *kernels = kernel launches per call.  Either output pointer may be NULL.
  * Errors: as ssd_scan_workspace_size.
  */

@@ -62,8 +62,8 @@ ssd_status ssd_selftest_fused_trace(const ssd_dims* d, const void* x, const floa
 
 /*
  * ssd_selftest_timeout exercises the bounded waits of ssd_scan_fwd's fused
- * tensor-core kernel (the two-head kernel where it takes the shape, unless
- * d->flags has SSD_FLAG_ONE_HEAD_PER_CTA; else the one-head kernel): same
+ * tensor-core kernel (the two-head kernel when d->flags has
+ * SSD_FLAG_TWO_HEADS_PER_CTA and it takes the shape, else the one-head kernel): same
  * arguments and validation as ssd_scan_fwd (the problem must be one a fused
  * kernel takes, else SSD_ERR_UNSUPPORTED), but
  * the kernel issues none of its TMA loads, so every wait on them gives up
@@ -78,13 +78,14 @@ ssd_status ssd_selftest_timeout(const ssd_dims* d, const void* x, const float* d
                                 void* stream);
 
 /*
- * ssd_selftest_carry_timeout exercises the one wait of the two-head fused
- * kernel that is not on a barrier of its own CTA: in its split schedule a CTA
+ * ssd_selftest_carry_timeout exercises the one wait of the fused kernels
+ * that is not on a barrier of their own CTA: in the split schedule a CTA
  * whose range starts inside a sequence waits for the previous CTA to publish
  * that sequence's state (the page's inter-chunk recursion, "分块推理…" §2.2,
  * handed across CTAs).  Same arguments and validation as ssd_scan_fwd plus
- * the workspace; the problem must be one the two-head kernel splits (even
- * heads per group, more head pairs than SMs; else SSD_ERR_UNSUPPORTED).  No
+ * the workspace; the problem must be one the fused kernel (the two-head one
+ * with SSD_FLAG_TWO_HEADS_PER_CTA) splits: more sequences (pairs) than SMs,
+ * else SSD_ERR_UNSUPPORTED.  No
  * carry is ever published, so those waits give up after about two seconds;
  * the launch returns SSD_OK and the following ssd_read_device_status(stream)
  * returns SSD_ERR_TIMEOUT.  y and final_state are left undefined; nothing

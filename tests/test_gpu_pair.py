@@ -1,16 +1,17 @@
-"""The two-heads-per-CTA fused kernel (SSD_PATH_FUSED_PAIR) against the fp64
-oracle.
+"""The fused kernels' split schedule and the two-heads-per-CTA kernel
+(SSD_FLAG_TWO_HEADS_PER_CTA, path SSD_PATH_FUSED_PAIR) against the fp64 oracle.
 
-Two heads of one group share a CTA, their B/C tiles and S = C B^T.  With the
-caller's workspace and more head pairs than SMs the kernel cuts the
-concatenated sequences into equal ranges, one persistent CTA per SM, and a
-CTA that starts inside a sequence takes its initial state from the CTA before
-it (the inter-chunk recursion of "分块推理…" §2.2 handed across CTAs).  These
-cases cover one pair, ragged and one-token sequences, several pairs per
-group, the dt-scaled input, and the split schedule with many range
-boundaries; each is compared with the oracle at the bf16 tolerance, and the
-split schedule bitwise with the whole-sequence schedule (same arithmetic,
-the carry passes through memory in fp32)."""
+With the caller's workspace and more sequences (pairs) than SMs, a fused
+kernel cuts the concatenated sequences into equal ranges, one persistent CTA
+per SM, and a CTA that starts inside a sequence takes its initial state from
+the CTA before it (the inter-chunk recursion of "分块推理…" §2.2 handed across
+CTAs).  In the two-head kernel two heads of one group share a CTA, their B/C
+tiles and S = C B^T.  The cases cover one pair, ragged and one-token
+sequences, several pairs per group, the dt-scaled input, and the split
+schedule with many range boundaries for both kernels; each is compared with
+the oracle at the bf16 tolerance, and the split schedule bitwise with the
+whole-sequence schedule (same arithmetic, the carry passes through memory in
+fp32)."""
 import pytest
 import torch
 
@@ -40,14 +41,14 @@ def test_pair_kernel_matches_oracle(over, input_dt):
     wl = inputs.custom("mamba2_130m_layer", **over)
     host = inputs.generate(wl)
     dev = device_inputs(host)
-    assert ssd.ssd_scan_path(ssd.make_dims(dev["x"], dev["B"], wl.chunk, input_dt))[0] == "fused_pair"
-    y, fin = _scan(dev, wl, input_dt=input_dt)
+    assert ssd.ssd_scan_path(ssd.make_dims(dev["x"], dev["B"], wl.chunk, input_dt, True))[0] == "fused_pair"
+    y, fin = _scan(dev, wl, input_dt=input_dt, two_heads=True)
     y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host), input_dt=input_dt)
     assert rel_err(to_np64(y), y_ref) <= TOL["bf16"]
     assert rel_err(to_np64(fin), f_ref) <= TOL["bf16"]
-    # the one-head kernel on the same inputs (both are checked against the oracle)
-    assert ssd.ssd_scan_path(ssd.make_dims(dev["x"], dev["B"], wl.chunk, input_dt, True))[0] == "fused"
-    y1, f1 = _scan(dev, wl, input_dt=input_dt, one_head=True)
+    # the default one-head kernel on the same inputs (both checked against the oracle)
+    assert ssd.ssd_scan_path(ssd.make_dims(dev["x"], dev["B"], wl.chunk, input_dt))[0] == "fused"
+    y1, f1 = _scan(dev, wl, input_dt=input_dt)
     assert rel_err(to_np64(y1), y_ref) <= TOL["bf16"]
     assert rel_err(to_np64(f1), f_ref) <= TOL["bf16"]
 
@@ -57,13 +58,14 @@ def test_pair_kernel_matches_oracle(over, input_dt):
     dict(batch=1, seqlen=1000, nheads=300, ngroups=2),                # 150 pairs of 8 sub-chunks
     dict(batch=3, seqlen=640, nheads=100, ngroups=5, init_var=0.1),   # 150 pairs, 20 heads per group
 ])
-def test_split_schedule_matches_oracle_and_whole_sequences(over):
+@pytest.mark.parametrize("two_heads", [False, True])
+def test_split_schedule_matches_oracle_and_whole_sequences(over, two_heads):
     wl = inputs.custom("mamba2_130m_layer", **over)
     host = inputs.generate(wl)
     dev = device_inputs(host)
-    dims = ssd.make_dims(dev["x"], dev["B"], wl.chunk)
-    assert ssd.ssd_scan_path(dims)[0] == "fused_pair"
-    y, fin = _scan(dev, wl)
+    dims = ssd.make_dims(dev["x"], dev["B"], wl.chunk, two_heads=two_heads)
+    assert ssd.ssd_scan_path(dims)[0] == ("fused_pair" if two_heads else "fused")
+    y, fin = _scan(dev, wl, two_heads=two_heads)
     y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host))
     ey, ef = rel_err(to_np64(y), y_ref), rel_err(to_np64(fin), f_ref)
     assert ey <= TOL["bf16"], ey
@@ -72,32 +74,34 @@ def test_split_schedule_matches_oracle_and_whole_sequences(over):
     # there every CTA runs whole sequences.  The split must give the same
     # bits (a wrong or late carry changes whole sequences by O(1)).
     ys, fs = ssd.ssd_scan_fwd_strided(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
-                                      chunk=wl.chunk)
+                                      chunk=wl.chunk, two_heads=two_heads)
     torch.cuda.synchronize()
     assert torch.equal(ys, y)
     assert torch.equal(fs, fin)
 
 
-def test_split_schedule_repeatable_and_workspace_reused():
+@pytest.mark.parametrize("two_heads", [False, True])
+def test_split_schedule_repeatable_and_workspace_reused(two_heads):
     """Back-to-back calls on one workspace (the carry flags are reset by each
     call) give identical results."""
     wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=300, nheads=160, ngroups=1, init_var=0.1)
     dev = device_inputs(inputs.generate(wl))
-    dims = ssd.make_dims(dev["x"], dev["B"], wl.chunk)
+    dims = ssd.make_dims(dev["x"], dev["B"], wl.chunk, two_heads=two_heads)
     ws = torch.empty(ssd.ssd_scan_workspace_size(dims), dtype=torch.uint8, device="cuda")
     ws.fill_(0xFF)  # contents need not be initialised
-    outs = [_scan(dev, wl, workspace=ws) for _ in range(3)]
+    outs = [_scan(dev, wl, workspace=ws, two_heads=two_heads) for _ in range(3)]
     for y, f in outs[1:]:
         assert torch.equal(y, outs[0][0]) and torch.equal(f, outs[0][1])
 
 
-def test_long_sequences_repeat_bitwise():
-    """Long runs on one CTA per sequence pair (512 sub-chunks each) give the same
-    bits every time: a race between the kernel's roles (a buffer reused before
-    its last reader finished) shows up as run-to-run differences."""
+@pytest.mark.parametrize("two_heads", [False, True])
+def test_long_sequences_repeat_bitwise(two_heads):
+    """Long runs (512 sub-chunks per sequence) give the same bits every time: a
+    race between a kernel's roles (a buffer reused before its last reader
+    finished) shows up as run-to-run differences."""
     wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=65536, nheads=2, ngroups=1, init_var=0.1)
     dev = device_inputs(inputs.generate(wl))
-    outs = [_scan(dev, wl) for _ in range(4)]
+    outs = [_scan(dev, wl, two_heads=two_heads) for _ in range(4)]
     for y, f in outs[1:]:
         assert torch.equal(y, outs[0][0]) and torch.equal(f, outs[0][1])
     # and the same bits when the sequence is cut into blocks with the state carried
@@ -107,7 +111,7 @@ def test_long_sequences_repeat_bitwise():
     for k0 in range(0, wl.seqlen, V):
         sl = lambda t: t[:, k0:k0 + V].contiguous()
         yk, _ = ssd.ssd_scan_fwd(sl(dev["x"]), sl(dev["dt"]), dev["A"], sl(dev["B"]), sl(dev["C"]), dev["D"], st,
-                                 chunk=wl.chunk, final_state=st)
+                                 chunk=wl.chunk, final_state=st, two_heads=two_heads)
         y_blk[:, k0:k0 + V] = yk
     torch.cuda.synchronize()
     assert torch.equal(y_blk, outs[0][0])

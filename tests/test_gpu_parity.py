@@ -115,8 +115,8 @@ def _decay_regime(host, regime):
 
 @pytest.mark.parametrize("regime", ["A_zero", "dt_zero", "strong", "mixed"])
 @pytest.mark.parametrize("input_dt", [False, True])
-@pytest.mark.parametrize("one_head", [False, True])
-def test_fused_decay_extremes(regime, input_dt, one_head):
+@pytest.mark.parametrize("two_heads", [False, True])
+def test_fused_decay_extremes(regime, input_dt, two_heads):
     """Both fused tensor-core kernels at the ends of the decay range, against the
     oracle: a == 1 over whole 128-token sub-chunks (the off-diagonal factors stay
     1), and |dt*A| = 64 per token (every factor below the diagonal underflows to
@@ -124,10 +124,10 @@ def test_fused_decay_extremes(regime, input_dt, one_head):
     wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=700, nheads=4, ngroups=2, init_var=0.1)
     host = _decay_regime(inputs.generate(wl), regime)
     dev = device_inputs(host)
-    path = ssd.ssd_scan_path(ssd.make_dims(dev["x"], dev["B"], wl.chunk, input_dt, one_head))[0]
-    assert path == ("fused" if one_head else "fused_pair")
+    path = ssd.ssd_scan_path(ssd.make_dims(dev["x"], dev["B"], wl.chunk, input_dt, two_heads))[0]
+    assert path == ("fused_pair" if two_heads else "fused")
     y, fin = ssd.ssd_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
-                              chunk=wl.chunk, input_dt=input_dt, one_head=one_head)
+                              chunk=wl.chunk, input_dt=input_dt, two_heads=two_heads)
     torch.cuda.synchronize()
     y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host), input_dt=input_dt)
     ey, ef = rel_err(to_np64(y), y_ref), rel_err(to_np64(fin), f_ref)

@@ -22,10 +22,9 @@ SSD_OK = 0
 SSD_ERR_TIMEOUT = 8
 
 
-@pytest.mark.parametrize("one_head", [False, True])
-def test_withheld_loads_time_out_and_context_survives(one_head):
-    """Both fused kernels: the two-head one (default for this shape) and the
-    one-head one."""
+@pytest.mark.parametrize("two_heads", [False, True])
+def test_withheld_loads_time_out_and_context_survives(two_heads):
+    """Both fused kernels: the one-head one (default) and the two-head one."""
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     wl = inputs.custom("mamba2_130m_layer", batch=1, seqlen=512, nheads=2)
     host = inputs.generate(wl)
@@ -34,7 +33,7 @@ def test_withheld_loads_time_out_and_context_survives(one_head):
 
     t0 = time.monotonic()
     ssd.ssd_selftest_timeout(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
-                             chunk=wl.chunk, one_head=one_head)
+                             chunk=wl.chunk, two_heads=two_heads)
     status = ssd.ssd_read_device_status()  # synchronises the stream
     elapsed = time.monotonic() - t0
     assert status == SSD_ERR_TIMEOUT
@@ -43,7 +42,7 @@ def test_withheld_loads_time_out_and_context_survives(one_head):
 
     # the context is intact: a normal scan right after matches the oracle
     y, fin = ssd.ssd_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
-                              chunk=wl.chunk)
+                              chunk=wl.chunk, two_heads=two_heads)
     torch.cuda.synchronize()
     assert ssd.ssd_read_device_status() == SSD_OK
     y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host))
@@ -51,8 +50,9 @@ def test_withheld_loads_time_out_and_context_survives(one_head):
     assert rel_err(to_np64(fin), f_ref) <= TOL["bf16"]
 
 
-def test_carry_wait_times_out_and_context_survives():
-    """The two-head kernel's split schedule with no carry ever published: every
+@pytest.mark.parametrize("two_heads", [False, True])
+def test_carry_wait_times_out_and_context_survives(two_heads):
+    """A fused kernel's split schedule with no carry ever published: every
     CTA that starts inside a sequence gives up waiting for its predecessor's
     state after about two seconds; the host reads SSD_ERR_TIMEOUT, and a normal
     scan (with its carries) then matches the oracle in the same context."""
@@ -62,14 +62,14 @@ def test_carry_wait_times_out_and_context_survives():
     assert ssd.ssd_read_device_status() == SSD_OK
     t0 = time.monotonic()
     ssd.ssd_selftest_carry_timeout(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
-                                   chunk=wl.chunk)
+                                   chunk=wl.chunk, two_heads=two_heads)
     status = ssd.ssd_read_device_status()
     elapsed = time.monotonic() - t0
     assert status == SSD_ERR_TIMEOUT
     assert elapsed < 30.0, elapsed
     assert ssd.ssd_read_device_status() == SSD_OK
     y, fin = ssd.ssd_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
-                              chunk=wl.chunk)
+                              chunk=wl.chunk, two_heads=two_heads)
     torch.cuda.synchronize()
     assert ssd.ssd_read_device_status() == SSD_OK
     y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host))

@@ -2,13 +2,9 @@
 // of "分块推理：解锁循环模型并行计算，实现长序列高效处理" §2.1-§2.2 in one pass, with the
 // inter-chunk state carried on chip.
 //
-// A CTA walks 128-token sub-chunks j of (batch, head) sequences (a Q = 256
-// chunk is two of them: the page's intra/inter split applied once more inside
-// the chunk, which is exact by its §2.3).  With a workspace and more sequences
-// than SMs, the sequences are cut into equal ranges, one persistent CTA per SM
-// (ssd_split.cuh: a CTA runs its head piece first and hands that piece's end
-// state to the next CTA, which needs it only for the tail piece it runs
-// last); otherwise each CTA runs one whole sequence.  Per
+// One CTA owns one (batch, head) sequence and walks it in 128-token
+// sub-chunks j (a Q = 256 chunk is two of them: the page's intra/inter split
+// applied once more inside the chunk, which is exact by its §2.3).  Per
 // sub-chunk, with lam the in-sub-chunk cumulative sum of dt*A:
 //   S       = C_j B_j^T                                   (tcgen05, 128x128x128)
 //   P       = S (.) exp(lam_t - lam_s) [s <= t]  -> bf16 in TMEM, columns 0-63
@@ -31,7 +27,6 @@
 // raises g_device_status and the roles drain without further waits.
 #include <atomic>
 
-#include "ssd_split.cuh"
 #include "ssd_tc.cuh"
 #include "tma.cuh"
 #include "umma.cuh"
@@ -71,10 +66,6 @@ struct Params {
   int mode;
   int64_t L;
   int H, G, nsub;
-  int64_t total;  // whole scan: B * H * nsub, the concatenated sub-chunks
-  int nctas;      // whole scan: CTAs the sub-chunks are split over
-  float* carry;   // [nctas][NS][P] end states of head pieces, or NULL
-  int* carry_flag;  // [nctas], zeroed before the launch
   int64_t nc, Q;         // chunking of the step kernels
   const float* lam_in;   // step-1 log-decay sums [B,H,nc,Q] (step modes)
   const float* dt;
@@ -90,9 +81,8 @@ struct Params {
   int64_t sy;
   unsigned long long* trace;  // diagnostics: per-sub-chunk event clocks of CTA 0, then
                               // [start ns, end ns, SM] of every CTA; or NULL
-  int withhold_loads;         // self-test of the timeout path: 1 = issue no TMA loads, so
-                              // every wait on them runs out; 2 = publish no carries
-                              // (0 in every other launch)
+  int withhold_loads;         // self-test of the timeout path: issue no TMA loads, so
+                              // every wait on them runs out (0 in every other launch)
 };
 
 // Trace events (clock64 of CTA 0), one row of kTraceEvents per sub-chunk.
@@ -209,38 +199,17 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool chunked = p.mode != MODE_SCAN;
-  // step modes: one CTA per (batch, head, chunk); whole scan: the CTA's range
-  const int64_t bh_c = chunked ? (int64_t)blockIdx.x / p.nc : 0;
+  const int64_t bh = chunked ? (int64_t)blockIdx.x / p.nc : (int64_t)blockIdx.x;
   const int64_t cidx = chunked ? (int64_t)blockIdx.x % p.nc : 0;   // chunk of this CTA (step modes)
-  const int t_base = (int)(cidx * p.Q);                          // first token of this CTA (step modes)
-  const int64_t cslot = bh_c * p.nc + cidx;                      // [B,H,nc] index (step modes)
-  split::Range rg;
-  if (!chunked) rg.init(p.total, p.nctas, blockIdx.x, p.nsub);
-  const int nsub = chunked ? (int)ceil_div(min((int64_t)p.Q, p.L - t_base), (int64_t)T) : (int)rg.count();
-  // (batch, head), first token and piece boundaries of this CTA's j-th sub-chunk
-  struct At {
-    int b, h, t0;
-    bool first, last, carry_in, carry_out;
-  };
-  auto at = [&](int j) {
-    At a;
-    if (chunked) {
-      a.b = (int)(bh_c / p.H);
-      a.h = (int)(bh_c % p.H);
-      a.t0 = t_base + j * T;
-      a.first = (j == 0);
-      a.last = (j == nsub - 1);
-      a.carry_in = a.carry_out = false;
-    } else {
-      int64_t u;
-      int jj;
-      rg.at(j, u, jj, a.first, a.last, a.carry_in, a.carry_out);
-      a.b = (int)(u / p.H);
-      a.h = (int)(u % p.H);
-      a.t0 = jj * T;
-    }
-    return a;
-  };
+  const int b = (int)(bh / p.H), h = (int)(bh % p.H);
+  const int g = h / (p.H / p.G);
+  const int t_base = (int)(cidx * p.Q);                          // first token of this CTA
+  const int nsub = chunked ? (int)ceil_div(min((int64_t)p.Q, p.L - t_base), (int64_t)T) : p.nsub;
+  const int64_t cslot = bh * p.nc + cidx;                       // [B,H,nc] index (step modes)
+  const float* init_ptr = chunked ? (p.mode == MODE_CHUNK_SCAN ? p.init + cslot * NS * P : nullptr)
+                                  : (p.init ? p.init + bh * NS * P : nullptr);
+  float* final_ptr = chunked ? (p.mode == MODE_CHUNK_STATE ? p.final_state + cslot * NS * P : nullptr)
+                             : (p.final_state ? p.final_state + bh * NS * P : nullptr);
   unsigned long long* const trace = (p.trace && blockIdx.x == 0) ? p.trace : nullptr;
   auto mark = [&](int j, int ev) {
     if (trace) trace[j * kTraceEvents + ev] = clock64();
@@ -287,25 +256,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       constexpr int kPrefetch = 3;
       auto prefetch = [&](int jp) {
         if (jp >= nsub) return;
-        const At w = at(jp);
-        const int g = w.h / (p.H / p.G);
-        tma_prefetch_4d(&map_x, 0, w.h, w.t0, w.b);
-        tma_prefetch_4d(&map_b, 0, g, w.t0, w.b);
-        tma_prefetch_4d(&map_b, 64, g, w.t0, w.b);
-        tma_prefetch_4d(&map_c, 0, g, w.t0, w.b);
-        tma_prefetch_4d(&map_c, 64, g, w.t0, w.b);
+        const int tp = t_base + jp * T;
+        tma_prefetch_4d(&map_x, 0, h, tp, b);
+        tma_prefetch_4d(&map_b, 0, g, tp, b);
+        tma_prefetch_4d(&map_b, 64, g, tp, b);
+        tma_prefetch_4d(&map_c, 0, g, tp, b);
+        tma_prefetch_4d(&map_c, 64, g, tp, b);
       };
       for (int jp = 0; jp < kPrefetch; ++jp) prefetch(jp);
-      const int nload = p.withhold_loads == 1 ? 0 : nsub;
+      const int nload = nsub & (p.withhold_loads - 1);  // 0 or nsub (withhold_loads is 0 or 1)
       for (int j = 0; j < nload; ++j) {
         const int st = j & 1;
         prefetch(j + kPrefetch);
         if (j >= 2 && !ctl.wait(EMPTY0 + st, ((j >> 1) + 1) & 1)) break;
         uint8_t* sx = sm + st * STAGE;
-        const At w = at(j);
-        const int g = w.h / (p.H / p.G), t0 = w.t0, b = w.b;
+        const int t0 = t_base + j * T;
         mbar_arrive_expect_tx(&bar[FULL0 + st], TX_BYTES);
-        tma_load_4d(sx + OFF_X, &map_x, &bar[FULL0 + st], 0, w.h, t0, b);
+        tma_load_4d(sx + OFF_X, &map_x, &bar[FULL0 + st], 0, h, t0, b);
         tma_load_4d(sx + OFF_B, &map_b, &bar[FULL0 + st], 0, g, t0, b);
         tma_load_4d(sx + OFF_B + TILE, &map_b, &bar[FULL0 + st], 64, g, t0, b);
         tma_load_4d(sx + OFF_C, &map_c, &bar[FULL0 + st], 0, g, t0, b);
@@ -410,24 +377,20 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp < 4) {
     // ------------------------------------------------------------ dt, lam, decay factors, X'
     const int a = threadIdx.x;  // 0..63 (warps 0-1)
-    // dt and A of the j-th sub-chunk (read only by the whole scan)
-    auto load_dt = [&](int j, float& d0, float& d1, float& Aj) {
-      d0 = d1 = Aj = 0.f;
-      if (chunked || j >= nsub) return;
-      const At w = at(j);
-      const float* dtb = p.dt + (int64_t)w.b * p.sdt + w.h;
-      const int64_t t0 = (int64_t)w.t0 + 2 * a;
-      Aj = p.A[w.h];
-      d0 = (t0 < p.L) ? dtb[t0 * p.lddt] : 0.f;
-      d1 = (t0 + 1 < p.L) ? dtb[(t0 + 1) * p.lddt] : 0.f;
+    const float Ah = chunked ? 0.f : p.A[h];  // A (and dt) are read only by the whole scan
+    const float* dtb = p.dt + (int64_t)b * p.sdt + h;
+    auto load_dt = [&](int j, float& d0, float& d1) {
+      const int64_t t0 = (int64_t)j * T + 2 * a;
+      d0 = (!chunked && j < nsub && t0 < p.L) ? dtb[t0 * p.lddt] : 0.f;
+      d1 = (!chunked && j < nsub && t0 + 1 < p.L) ? dtb[(t0 + 1) * p.lddt] : 0.f;
     };
     const float* lamc = chunked ? p.lam_in + cslot * p.Q : nullptr;
-    float d0, d1, Ah;
-    load_dt(0, d0, d1, Ah);
+    float d0, d1;
+    load_dt(0, d0, d1);
     for (int j = 0; j < nsub; ++j) {
       const int st = j & 1, slot = j & 3;
-      float n0, n1, An;
-      load_dt(j + 1, n0, n1, An);  // one sub-chunk ahead
+      float n0, n1;
+      load_dt(j + 1, n0, n1);  // one sub-chunk ahead
       // inclusive scan of dt*A over the 128 tokens (two per thread)
       const float l0 = d0 * Ah, l1 = d1 * Ah;
       float v = l0 + l1;
@@ -471,7 +434,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (a == 0) mark(j, EV_LAM_READY);
       d0 = n0;
       d1 = n1;
-      Ah = An;
       // X'_j = diag(exp(lam_end - lam_t)) X_j, rows a and a + 64, into buffer j & 1
       // (free once the products of sub-chunk j - 2 have completed and its y tile,
       // staged in the same buffer, has been read by the TMA store)
@@ -591,13 +553,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int q = warp & 3;
     const int r = q * 32 + lane;  // state row n and output row t
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+    const float Dh = p.D ? p.D[h] : 0.f;
     // x row of the sub-chunk, loaded before waiting for its products (it is in L2
     // from the TMA load; the wait hides the latency)
+    const __nv_bfloat16* xg = p.x + (int64_t)b * p.sx + (int64_t)h * P;
     auto load_x = [&](int j, uint4* xv) {
-      const At w = at(j < nsub ? j : nsub - 1);
-      const int64_t tg = (int64_t)w.t0 + r;
+      const int64_t tg = (int64_t)t_base + (int64_t)j * T + r;
       if (j < nsub && tg < p.L) {
-        const __nv_bfloat16* xg = p.x + (int64_t)w.b * p.sx + (int64_t)w.h * P;
         const uint4* src = reinterpret_cast<const uint4*>(xg + tg * p.ldx);
 #pragma unroll
         for (int c = 0; c < 8; ++c) xv[c] = src[c];
@@ -608,68 +570,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     };
     uint4 xcur[8];
     float s[P];
-    // the state before the first sub-chunk of a piece: the previous CTA's carry
-    // (waited for), the caller's initial state, or zero
-    auto load_init = [&](const At& w) {
-      const float* src = nullptr;
-      if (chunked) {
-        src = (p.mode == MODE_CHUNK_SCAN) ? p.init + cslot * NS * P : nullptr;
-      } else if (w.carry_in) {
-        const int* flag = p.carry_flag + (blockIdx.x - 1);
-        if (split::ld_acquire(flag) == 0) {
-          const uint64_t t0 = globaltimer_ns();
-          bool done = false;
-          while (!done && !*abort_flag) {
-            __nanosleep(256);
-            done = split::ld_acquire(flag) != 0;
-            if (!done && globaltimer_ns() - t0 > 2000000000ull) {
-              *abort_flag = 1;
-              atomicExch(&g_device_status, 2);
-              break;
-            }
-          }
-        }
-        if (!*abort_flag) src = p.carry + (int64_t)(blockIdx.x - 1) * NS * P;
-      } else if (p.init) {
-        src = p.init + ((int64_t)w.b * p.H + w.h) * NS * P;
-      }
-      if (src) {
-        const float4* s4 = reinterpret_cast<const float4*>(src + (int64_t)r * P);
+    if (init_ptr) {
+      const float4* src = reinterpret_cast<const float4*>(init_ptr + (int64_t)r * P);
 #pragma unroll
-        for (int i = 0; i < P / 4; ++i) {
-          const float4 v = s4[i];
-          s[4 * i] = v.x; s[4 * i + 1] = v.y; s[4 * i + 2] = v.z; s[4 * i + 3] = v.w;
-        }
-      } else {
+      for (int i = 0; i < P / 4; ++i) {
+        const float4 v = src[i];
+        s[4 * i] = v.x; s[4 * i + 1] = v.y; s[4 * i + 2] = v.z; s[4 * i + 3] = v.w;
+      }
+    } else {
 #pragma unroll
-        for (int i = 0; i < P; ++i) s[i] = 0.f;
-      }
-    };
-    // the state after the last sub-chunk of a piece: the sequence's final
-    // state, the carry of a head piece (published with a release flag), or the
-    // chunk state of the chunk-state step
-    auto store_end = [&](const At& w) {
-      float* dst = nullptr;
-      if (chunked)
-        dst = (p.mode == MODE_CHUNK_STATE) ? p.final_state + cslot * NS * P : nullptr;
-      else if (w.carry_out)
-        dst = p.carry + (int64_t)blockIdx.x * NS * P;
-      else if (p.final_state)
-        dst = p.final_state + ((int64_t)w.b * p.H + w.h) * NS * P;
-      if (dst) {
-        float4* d4 = reinterpret_cast<float4*>(dst + (int64_t)r * P);
-#pragma unroll
-        for (int i = 0; i < P / 4; ++i) d4[i] = make_float4(s[4 * i], s[4 * i + 1], s[4 * i + 2], s[4 * i + 3]);
-      }
-      if (w.carry_out) {
-        __threadfence();
-        named_sync(3, T);
-        if (r == 0 && p.withhold_loads != 2) split::st_release(p.carry_flag + blockIdx.x, 1);
-      }
-    };
-    At cur = at(0);
-    float Dh = p.D ? p.D[cur.h] : 0.f, Dh_next = Dh;
-    load_init(cur);
+      for (int i = 0; i < P; ++i) s[i] = 0.f;
+    }
     const uint32_t sPrev = sbase + OFF_PREV;
     auto publish_state = [&]() {
 #pragma unroll
@@ -687,7 +598,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     publish_state();
     for (int j = 0; j < nsub; ++j) {
       const int buf = j & 1;
-      cur = at(j);
       load_x(j, xcur);
       bool ok = ctl.wait(CFULL0 + buf, (j >> 1) & 1);
       if (ok) ok = ctl.wait(LAMRDY0 + (j & 3), (j >> 2) & 1);      // acquire lam of this sub-chunk
@@ -711,17 +621,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           s[32 * c + i + 1] = o.y;
         }
       }
-      if (!cur.last) {
-        if (ok) publish_state();
-      } else {
-        store_end(cur);
-        if (j + 1 < nsub) {  // a new piece starts: its own initial state and D
-          const At nx = at(j + 1);
-          load_init(nx);
-          Dh_next = p.D ? p.D[nx.h] : 0.f;
-          if (ok) publish_state();
-        }
-      }
+      if (ok) publish_state();
       if (r == 0) mark(j, EV_STATE_PUB);
       // y_t = y_intra + exp(lam_t) y_inter + D x_t, staged as a 128-B-swizzled tile
       // in the X' buffer of this sub-chunk (free: its products have completed) and
@@ -759,16 +659,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       named_sync(2, T);  // the 128 rows are staged
       if (r == 0) {
         if (p.y) {
-          tma_store_4d(&map_y, sm + OFF_XP + buf * TILE, 0, cur.h, cur.t0, cur.b);
+          tma_store_4d(&map_y, sm + OFF_XP + buf * TILE, 0, h, t_base + j * T, b);
           tma_store_commit();
           tma_store_wait_read0();
         }
         mbar_arrive(&bar[YFREE0 + buf]);
       }
       if (r == 0) mark(j, EV_EPI_DONE);
-      Dh = Dh_next;
     }
     if (r == 0) tma_store_wait0();  // the y tiles are in global memory before the CTA exits
+    if (final_ptr) {
+      float4* dst = reinterpret_cast<float4*>(final_ptr + (int64_t)r * P);
+#pragma unroll
+      for (int i = 0; i < P / 4; ++i) dst[i] = make_float4(s[4 * i], s[4 * i + 1], s[4 * i + 2], s[4 * i + 3]);
+    }
   }
 
   tc_fence_before();
@@ -793,23 +697,13 @@ int fused_kernels_per_call(const Problem&) { return 1; }
 
 bool uses_pair_kernel(const Problem& p) { return p.two_heads && pair_supported(p); }
 
-// Workspace of the one-head kernel's split schedule: one carry [N][P] f32 per
-// CTA and the flags, or 0 when every CTA runs one whole sequence anyway.
-size_t fused_workspace_bytes(const Problem& p) {
-  if (!fused_supported(p)) return 0;
-  return split::workspace_bytes(p.B * p.H, (size_t)fused::NS * fused::P);
-}
-
-// The step modes read and write only the caller's step tensors; the whole scan
-// keeps the running state on chip and needs a workspace only for the carries
-// between CTAs of its split schedule.
-size_t tc_workspace_bytes(const Problem& p) {
-  return uses_pair_kernel(p) ? pair_workspace_bytes(p) : fused_workspace_bytes(p);
-}
+// The one-head kernel keeps the running state on chip (whole scan) or reads and
+// writes only the caller's step tensors (step modes): no workspace.  The
+// two-head kernel needs one for the carries of its split schedule.
+size_t tc_workspace_bytes(const Problem& p) { return uses_pair_kernel(p) ? pair_workspace_bytes(p) : 0; }
 
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
-                               void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads = 0,
-                               void* workspace = nullptr, size_t workspace_bytes = 0);
+                               void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads = 0);
 
 cudaError_t launch_fused_traced(const Problem& p, const float* init, float* final_state, unsigned long long* trace,
                                 cudaStream_t st) {
@@ -821,18 +715,10 @@ cudaError_t launch_fused_withheld(const Problem& p, const float* init, float* fi
   return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, nullptr, st, 1);
 }
 
-cudaError_t launch_fused_carry_withheld(const Problem& p, const float* init, float* final_state, void* workspace,
-                                        size_t workspace_bytes, cudaStream_t st) {
-  if (uses_pair_kernel(p)) return launch_pair(p, init, final_state, workspace, workspace_bytes, st, 2);
-  return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, nullptr, st, 2, workspace,
-                     workspace_bytes);
-}
-
 cudaError_t launch_fused(const Problem& p, const float* init, float* final_state, void* workspace,
                          size_t workspace_bytes, cudaStream_t st) {
   if (uses_pair_kernel(p)) return launch_pair(p, init, final_state, workspace, workspace_bytes, st, 0);
-  return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, nullptr, st, 0, workspace,
-                     workspace_bytes);
+  return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, nullptr, st);
 }
 
 // Step 2 on tensor cores: one CTA per (batch, head, chunk), zero start, the
@@ -848,8 +734,7 @@ cudaError_t launch_chunk_scan_tc(const Problem& p, const float* lam, const float
 }
 
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
-                               void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads,
-                               void* workspace, size_t workspace_bytes) {
+                               void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads) {
   using namespace fused;
   // every pointer the mode reads must be present (the step entry points pass
   // only the tensors of their step)
@@ -898,22 +783,6 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   kp.sy = p.sy;
   kp.trace = trace;
   kp.withhold_loads = withhold_loads;
-  // whole scan: split over one persistent CTA per SM when a workspace for the
-  // carries is given (and useful), else one CTA per sequence
-  kp.total = p.B * p.H * (int64_t)kp.nsub;
-  kp.nctas = (int)(p.B * p.H);
-  kp.carry = nullptr;
-  kp.carry_flag = nullptr;
-  if (mode == MODE_SCAN && !trace) {
-    const size_t need = fused_workspace_bytes(p);
-    if (need > 0 && workspace && workspace_bytes >= need) {
-      kp.nctas = split::ctas(p.B * p.H);
-      kp.carry = static_cast<float*>(workspace);
-      kp.carry_flag = reinterpret_cast<int*>(static_cast<char*>(workspace) + (size_t)kp.nctas * NS * P * sizeof(float));
-      cudaError_t e = cudaMemsetAsync(kp.carry_flag, 0, (size_t)kp.nctas * sizeof(int), st);
-      if (e != cudaSuccess) return e;
-    }
-  }
   // the shared-memory opt-in once per device (not stream work; keeps launches
   // free of other API calls, e.g. inside a CUDA graph capture)
   static std::atomic<unsigned long long> attr_set{0};
@@ -928,7 +797,7 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
     if (e != cudaSuccess) return e;
     attr_set.fetch_or(bit);
   }
-  const int64_t ctas = mode == fused::MODE_SCAN ? (int64_t)kp.nctas : p.B * p.H * p.nc;
+  const int64_t ctas = mode == fused::MODE_SCAN ? p.B * p.H : p.B * p.H * p.nc;
   if (p.input_dt && mode == fused::MODE_SCAN)
     k_ssd_fused<true><<<(unsigned)ctas, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
   else

@@ -210,7 +210,7 @@ extern "C" ssd_status ssd_selftest_timeout(const ssd_dims* d, const void* x, con
   return cuda_status(launch_fused_withheld(p, init_state, final_state, static_cast<cudaStream_t>(stream)));
 }
 
-// Carry path of the fused kernels: the split schedule of ssd_scan_fwd with no
+// Carry path of the two-head kernel: the split schedule of ssd_scan_fwd with no
 // carry ever published, so every CTA that starts inside a sequence waits for
 // its predecessor's state until its bounded wait runs out (about two seconds),
 // records SSD_ERR_TIMEOUT and drains; nothing faults.
@@ -224,10 +224,10 @@ extern "C" ssd_status ssd_selftest_carry_timeout(const ssd_dims* d, const void* 
   s = validate_scan_args(d, x, dt, A, Bm, Cm, D, init_state, y, final_state);
   if (s != SSD_OK) return s;
   Problem p = make_problem(d);
-  if (!fused_supported(p) || tc_workspace_bytes(p) == 0) return SSD_ERR_UNSUPPORTED;
-  if (!workspace || workspace_bytes < tc_workspace_bytes(p)) return SSD_ERR_WORKSPACE;
+  if (!uses_pair_kernel(p) || pair_workspace_bytes(p) == 0) return SSD_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < pair_workspace_bytes(p)) return SSD_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0) return SSD_ERR_ALIGN;
   p.x = x; p.dt = dt; p.A = A; p.Bm = Bm; p.Cm = Cm; p.D = D; p.y = y;
-  return cuda_status(launch_fused_carry_withheld(p, init_state, final_state, workspace, workspace_bytes,
-                                                 static_cast<cudaStream_t>(stream)));
+  return cuda_status(
+      launch_pair(p, init_state, final_state, workspace, workspace_bytes, static_cast<cudaStream_t>(stream), 2));
 }

@@ -29,10 +29,6 @@ cudaError_t launch_chunk_scan_tc(const Problem& p, const float* lam, const float
 // (NULL / too small) every CTA runs whole sequences.
 cudaError_t launch_fused(const Problem& p, const float* init, float* final_state, void* workspace,
                          size_t workspace_bytes, cudaStream_t st);
-// The same launch with no carry ever published (self-test of the carry wait).
-cudaError_t launch_fused_carry_withheld(const Problem& p, const float* init, float* final_state, void* workspace,
-                                        size_t workspace_bytes, cudaStream_t st);
-size_t fused_workspace_bytes(const Problem& p);
 // withhold: 0 normal; 1 no TMA loads; 2 no carries published (self-tests of the bounded waits)
 cudaError_t launch_pair(const Problem& p, const float* init, float* final_state, void* workspace,
                         size_t workspace_bytes, cudaStream_t st, int withhold);

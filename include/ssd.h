@@ -188,10 +188,11 @@ ssd_status ssd_scan_fwd_host(const ssd_dims* d, const void* x, const float* dt, 
  * steps 2 and 4 on tcgen05 tensor cores), SSD_PATH_FUSED (one tensor-core
  * kernel) or SSD_PATH_FUSED_PAIR (one tensor-core kernel, two heads of a
  * group per CTA sharing their B and C tiles; SSD_FLAG_TWO_HEADS_PER_CTA).
- * With the workspace of ssd_scan_workspace_size and more sequences (pairs)
- * than SMs, the fused kernels cut the concatenated sequences into equal
- * ranges, one persistent CTA per SM, and hand the state across range
- * boundaries through the workspace; otherwise a CTA runs whole sequences;
+ * The one-head kernel runs one (batch, head) sequence per CTA.  The two-head
+ * kernel, given the workspace of ssd_scan_workspace_size and more head pairs
+ * than SMs, cuts the concatenated sequences into equal ranges, one persistent
+ * CTA per SM, and hands the state across range boundaries through the
+ * workspace; otherwise it runs whole sequences;
  * *kernels = kernel launches per call.  Either output pointer may be NULL.
  * Errors: as ssd_scan_workspace_size.
  */

@@ -78,14 +78,14 @@ ssd_status ssd_selftest_timeout(const ssd_dims* d, const void* x, const float* d
                                 void* stream);
 
 /*
- * ssd_selftest_carry_timeout exercises the one wait of the fused kernels
- * that is not on a barrier of their own CTA: in the split schedule a CTA
+ * ssd_selftest_carry_timeout exercises the one wait of the two-head fused
+ * kernel that is not on a barrier of its own CTA: in its split schedule a CTA
  * whose range starts inside a sequence waits for the previous CTA to publish
  * that sequence's state (the page's inter-chunk recursion, "分块推理…" §2.2,
  * handed across CTAs).  Same arguments and validation as ssd_scan_fwd plus
- * the workspace; the problem must be one the fused kernel (the two-head one
- * with SSD_FLAG_TWO_HEADS_PER_CTA) splits: more sequences (pairs) than SMs,
- * else SSD_ERR_UNSUPPORTED.  No
+ * the workspace; d->flags must request the two-head kernel
+ * (SSD_FLAG_TWO_HEADS_PER_CTA) and the problem be one it splits (even heads per
+ * group, more head pairs than SMs), else SSD_ERR_UNSUPPORTED.  No
  * carry is ever published, so those waits give up after about two seconds;
  * the launch returns SSD_OK and the following ssd_read_device_status(stream)
  * returns SSD_ERR_TIMEOUT.  y and final_state are left undefined; nothing

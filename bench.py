@@ -266,6 +266,9 @@ def main():
                          "batch, heads and sizes instead of the scan")
     ap.add_argument("--unfused", action="store_true",
                     help="time the four step kernels (ssd_scan_fwd_unfused) instead of the fused kernel")
+    ap.add_argument("--split", default="batch", choices=["batch", "sequence"],
+                    help="with N > 1 ranks: each rank scans its own batch (batch), or every rank holds one token "
+                         "segment of every sequence of one batch and the states are handed across ranks (sequence)")
     ap.add_argument("--two-heads", action="store_true",
                     help="the fused kernel with two heads of a group per CTA (SSD_FLAG_TWO_HEADS_PER_CTA; comparison)")
     ap.add_argument("--no-extras", action="store_true",
@@ -298,6 +301,8 @@ def main():
         return run_stack(args, wl, dev, rank, world)
     if args.decode:
         return run_decode(args, wl, dev, rank, world)
+    if args.split == "sequence":
+        return run_sequence_split(args, wl, dev, rank, world)
     host = inputs.generate(wl, seed=rank_seed(rank))  # each rank: its own independent batch
     pinned = {}
     for k, v in host.items():
@@ -406,6 +411,55 @@ def main():
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_sequence_split(args, wl, dev, rank, world):
+    """Sequence (context) parallelism: one batch of the workload, every rank
+    holding tokens [r L/N, (r+1) L/N) of every sequence.  A step is
+    seqshard.ssd_scan_fwd_seqshard: a scan of the segment from zero, one
+    all-gather of (end state, segment log-decay) over NCCL, and a scan of the
+    segment from the carried state.  Total work is fixed (strong scaling)."""
+    import torch
+    import torch.distributed as dist
+    from chunked_state_space_b200 import inputs, seqshard, ssd
+    if world == 1 and not dist.is_initialized():
+        import datetime
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29517")
+        dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    host = inputs.generate(wl, seed=0)  # the same batch on every rank
+    t0, t1 = rank * wl.seqlen // world, (rank + 1) * wl.seqlen // world
+    to = lambda v: (torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16 else
+                    torch.from_numpy(v))
+    seg = {k: to(v[:, t0:t1]).contiguous().to(dev) if k in ("x", "dt", "B", "C") else to(v).to(dev)
+           for k, v in host.items()}
+    del host
+    dims = ssd.make_dims(seg["x"], seg["B"], wl.chunk)
+    ws = torch.empty(max(ssd.ssd_scan_workspace_size(dims), 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        seqshard.ssd_scan_fwd_seqshard(seg["x"], seg["dt"], seg["A"], seg["B"], seg["C"], seg["D"], seg["init"],
+                                       chunk=wl.chunk, workspace=ws, stream=stream)
+
+    per_step, ms_total, clk = timed_steps(step, args, stream, dev, dev.index, world)
+    ms = ms_total / args.steps
+    line = {
+        "metric": METRIC, "value": wl.batch * wl.seqlen / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "seqlen": wl.seqlen, "nheads": wl.nheads,
+                   "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk,
+                   "parallelism": f"sp{world} (token segments per rank, states handed across ranks)",
+                   "l2": f"inputs larger than L2 ({algorithmic_bytes(wl) / world / 1e9:.2f} GB per rank); no flush"},
+        "clocks": clk, "gpu_launches": 2 * args.steps,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist.is_initialized():
         dist.destroy_process_group()
     return 0
 

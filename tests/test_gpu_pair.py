@@ -115,3 +115,25 @@ def test_long_sequences_repeat_bitwise(two_heads):
     torch.cuda.synchronize()
     assert torch.equal(y_blk, outs[0][0])
     assert torch.equal(st, outs[0][1])
+
+
+def test_sequence_shard_single_rank_equals_scan():
+    """seqshard on one rank (NCCL, world size 1): the carried state is the
+    caller's initial state, so the result is the plain scan's, bitwise."""
+    import datetime
+    import os
+    import torch.distributed as dist
+    from chunked_state_space_b200 import seqshard
+    wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=700, nheads=4, ngroups=2, init_var=0.1)
+    dev = device_inputs(inputs.generate(wl))
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29531")
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        y, fin = seqshard.ssd_scan_fwd_seqshard(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"],
+                                                dev["init"], chunk=wl.chunk)
+        y0, f0 = _scan(dev, wl)
+        assert torch.equal(y, y0) and torch.equal(fin, f0)
+    finally:
+        dist.destroy_process_group()

@@ -12,6 +12,11 @@ Functions and the passages they follow (page titles as published):
   per-token dt, B, C: "告别Transformer的二次方噩梦…" §2.1).
 * ``scan_chunked``     -- the chunk decomposition with its intermediates
   (by_intra, b_intra, b(c), by_inter; same page §2.1-§2.2).
+* ``scan_recurrence_vdecay`` / ``scan_chunked_vdecay`` -- the same with a
+  vector-valued decay, one rate per state channel (the diagonal A of the
+  selective scan, "告别Transformer的二次方噩梦…" §2.1; per-channel decays as in
+  the recurrences of "分块推理…" §6): the token recurrence and its chunk
+  decomposition.
 * ``round_bf16``, ``rmsnorm_bf16`` -- storage rounding and the layer-to-layer
   normalisation of the multi-layer stack (a reading; the page's §3 only says
   that layer l's output feeds layer l+1).
@@ -58,6 +63,10 @@ class _Oracle:
         lib.oracle_scan_recurrence.argtypes = [_I] * 6 + [_P] * 9 + [ctypes.c_int]
         lib.oracle_scan_chunked.restype = None
         lib.oracle_scan_chunked.argtypes = [_I] * 7 + [_P] * 14 + [ctypes.c_int]
+        lib.oracle_scan_recurrence_vdecay.restype = None
+        lib.oracle_scan_recurrence_vdecay.argtypes = [_I] * 6 + [_P] * 9
+        lib.oracle_scan_chunked_vdecay.restype = None
+        lib.oracle_scan_chunked_vdecay.argtypes = [_I] * 7 + [_P] * 9
         lib.oracle_round_bf16.restype = None
         lib.oracle_round_bf16.argtypes = [_I, _P, _P]
         lib.oracle_rmsnorm_bf16.restype = None
@@ -136,6 +145,33 @@ def scan_chunked(x, dt, A, Bm, Cm, Q, D=None, init=None, o: Optional[_Oracle] = 
                               _ptr(out["prev_states"]), _ptr(out["y_intra"]), _ptr(out["y_inter"]),
                               _ptr(out["y"]), _ptr(out["final"]), int(bool(input_dt)))
     return out
+
+
+def scan_recurrence_vdecay(x, dt, Av, Bm, Cm, D=None, init=None, o: Optional[_Oracle] = None):
+    """Token recurrence with a per-channel decay a_t[n] = exp(dt_t Av[h, n]), Av [H, N].
+    Returns (y [B,L,H,P], final [B,H,N,P])."""
+    o = o or load()
+    x, dt, Av, Bm, Cm, D, init = map(_f64, (x, dt, Av, Bm, Cm, D, init))
+    Bz, L, H, P, N, G = _dims(x, Bm)
+    assert Av.shape == (H, N)
+    y = np.empty((Bz, L, H, P))
+    fin = np.empty((Bz, H, N, P))
+    o.lib.oracle_scan_recurrence_vdecay(Bz, L, H, P, N, G, _ptr(x), _ptr(dt), _ptr(Av), _ptr(Bm), _ptr(Cm),
+                                        _ptr(D), _ptr(init), _ptr(y), _ptr(fin))
+    return y, fin
+
+
+def scan_chunked_vdecay(x, dt, Av, Bm, Cm, Q, D=None, init=None, o: Optional[_Oracle] = None):
+    """Chunk decomposition of the per-channel-decay scan.  Returns (y, final)."""
+    o = o or load()
+    x, dt, Av, Bm, Cm, D, init = map(_f64, (x, dt, Av, Bm, Cm, D, init))
+    Bz, L, H, P, N, G = _dims(x, Bm)
+    assert Av.shape == (H, N)
+    y = np.empty((Bz, L, H, P))
+    fin = np.empty((Bz, H, N, P))
+    o.lib.oracle_scan_chunked_vdecay(Bz, L, H, P, N, G, Q, _ptr(x), _ptr(dt), _ptr(Av), _ptr(Bm), _ptr(Cm),
+                                     _ptr(D), _ptr(init), _ptr(y), _ptr(fin))
+    return y, fin
 
 
 def round_bf16(a, o: Optional[_Oracle] = None) -> np.ndarray:

@@ -30,9 +30,9 @@
  *    the intra mask is L_ts = prod_{r=s+1..t} a_r for s <= t, 0 otherwise;
  *    the chunk-local state weights are prod_{r=s+1..c1-1} a_r.
  *
- * Every pinned function is checked in tests/test_oracle.py against closed
- * forms, brute-force double sums, invariants and hand-worked values; none is
- * "parity unpinned".
+ * Every pinned function is checked in tests/test_oracle.py (the vector-decay
+ * variant in tests/test_oracle_vdecay.py) against closed forms, brute-force
+ * double sums, invariants and hand-worked values; none is "parity unpinned".
  *
  * Layouts (all row-major, contiguous):
  *   x, y        [B, L, H, P]     dt [B, L, H]      A, D [H]
@@ -190,6 +190,132 @@ void oracle_scan_chunked(int64_t Bz, int64_t L, int64_t H, int64_t P, int64_t N,
     }
     if (final_state) memcpy(final_state + (b * H + h) * N * P, prev, sizeof(double) * N * P);
     free(prev); free(bin); free(a); free(yi); free(ye);
+  }
+}
+
+/*
+ * The recurrence with a vector-valued decay, one rate per state channel n --
+ * the diagonal state matrix of the selective scan ([P3] §2.1: A is diagonal)
+ * and the per-channel decay of the recurrences [P1] §6 names alongside Mamba
+ * (RWKV, xLSTM):
+ *   a_t[n] = exp(dt[b,t,h] * Av[h,n])
+ *   h_t[n,:] = a_t[n] h_{t-1}[n,:] + B[b,t,g,n] x[b,t,h,:]
+ *   y_t = C[b,t,g,:]^T h_t + D[h] x[b,t,h,:]
+ * Av: [H, N].  With Av[h,n] the same for every n this is oracle_scan_recurrence.
+ */
+void oracle_scan_recurrence_vdecay(int64_t Bz, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G,
+                                   const double* x, const double* dt, const double* Av,
+                                   const double* Bm, const double* Cm, const double* D,
+                                   const double* init, double* y, double* final_state) {
+  const int64_t hpg = H / G;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < Bz * H; ++bh) {
+    const int64_t b = bh / H, h = bh % H, g = h / hpg;
+    double* st = (double*)malloc(sizeof(double) * N * P);
+    if (init)
+      memcpy(st, init + (b * H + h) * N * P, sizeof(double) * N * P);
+    else
+      memset(st, 0, sizeof(double) * N * P);
+    const double d = D ? D[h] : 0.0;
+    for (int64_t t = 0; t < L; ++t) {
+      const double dtv = dt[(b * L + t) * H + h];
+      const double* xt = x + IX4(b, t, h, 0, L, H, P);
+      const double* bt = Bm + IX4(b, t, g, 0, L, G, N);
+      const double* ct = Cm + IX4(b, t, g, 0, L, G, N);
+      double* yt = y + IX4(b, t, h, 0, L, H, P);
+      for (int64_t n = 0; n < N; ++n) {
+        const double a = exp(dtv * Av[h * N + n]);
+        double* row = st + n * P;
+        for (int64_t p = 0; p < P; ++p) row[p] = a * row[p] + bt[n] * xt[p];
+      }
+      for (int64_t p = 0; p < P; ++p) yt[p] = d * xt[p];
+      for (int64_t n = 0; n < N; ++n)
+        for (int64_t p = 0; p < P; ++p) yt[p] += ct[n] * st[n * P + p];
+    }
+    if (final_state) memcpy(final_state + (b * H + h) * N * P, st, sizeof(double) * N * P);
+    free(st);
+  }
+}
+
+/*
+ * The chunk decomposition of [P1] §2.1-§2.2 for the vector-valued decay: the
+ * scalar products of a over token ranges become products per state channel,
+ * so the intra-chunk term no longer factors into (C B^T) (.) L and is summed
+ * channel by channel.  Chunk c covers tokens [c0, c1):
+ *   by_intra[t]   = sum_{s=c0..t} sum_n C_t[n] L_ts[n] B_s[n] x_s,  L_ts[n] = prod_{r=s+1..t} a_r[n]
+ *   b_intra(c)    = per channel n: sum_{s=c0..c1-1} (prod_{r=s+1..c1-1} a_r[n]) B_s[n] x_s^T
+ *   b(c)[n,:]     = b_intra(c)[n,:] + (prod_{r=c0..c1-1} a_r[n]) b(c-1)[n,:],  b(-1) = init
+ *   by_inter[t]   = sum_n (prod_{r=c0..t} a_r[n]) C_t[n] b(c-1)[n,:]
+ *   y[t]          = by_intra[t] + by_inter[t] + D_h x_t ;  final = b(nc-1)
+ * Decays are products of a_r[n] = exp(dt_r Av[h,n]), formed literally.
+ */
+void oracle_scan_chunked_vdecay(int64_t Bz, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G,
+                                int64_t Q, const double* x, const double* dt, const double* Av,
+                                const double* Bm, const double* Cm, const double* D, const double* init,
+                                double* y, double* final_state) {
+  const int64_t hpg = H / G;
+  const int64_t nc = (L + Q - 1) / Q;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < Bz * H; ++bh) {
+    const int64_t b = bh / H, h = bh % H, g = h / hpg;
+    const double d = D ? D[h] : 0.0;
+    double* prev = (double*)malloc(sizeof(double) * N * P);
+    double* bin = (double*)malloc(sizeof(double) * N * P);
+    double* a = (double*)malloc(sizeof(double) * Q * N); /* a[i * N + n] */
+    double* w = (double*)malloc(sizeof(double) * N);
+    if (init)
+      memcpy(prev, init + (b * H + h) * N * P, sizeof(double) * N * P);
+    else
+      memset(prev, 0, sizeof(double) * N * P);
+    for (int64_t c = 0; c < nc; ++c) {
+      const int64_t c0 = c * Q, c1 = (c0 + Q < L) ? c0 + Q : L, len = c1 - c0;
+      for (int64_t i = 0; i < len; ++i)
+        for (int64_t n = 0; n < N; ++n) a[i * N + n] = exp(dt[(b * L + c0 + i) * H + h] * Av[h * N + n]);
+      for (int64_t i = 0; i < len; ++i) {
+        const int64_t t = c0 + i;
+        const double* ct = Cm + IX4(b, t, g, 0, L, G, N);
+        double* yt = y + IX4(b, t, h, 0, L, H, P);
+        const double* xt = x + IX4(b, t, h, 0, L, H, P);
+        for (int64_t p = 0; p < P; ++p) yt[p] = d * xt[p];
+        /* by_intra: walk s from t down to c0, carrying L_ts[n] */
+        for (int64_t n = 0; n < N; ++n) w[n] = 1.0;
+        for (int64_t j = i; j >= 0; --j) {
+          if (j < i)
+            for (int64_t n = 0; n < N; ++n) w[n] *= a[(j + 1) * N + n];
+          const int64_t s = c0 + j;
+          const double* bs = Bm + IX4(b, s, g, 0, L, G, N);
+          const double* xs = x + IX4(b, s, h, 0, L, H, P);
+          double k = 0.0;
+          for (int64_t n = 0; n < N; ++n) k += ct[n] * w[n] * bs[n];
+          for (int64_t p = 0; p < P; ++p) yt[p] += k * xs[p];
+        }
+        /* by_inter: inclusive per-channel decay times C_t[n] b(c-1)[n,:] */
+        for (int64_t n = 0; n < N; ++n) {
+          double dl = 1.0;
+          for (int64_t j = 0; j <= i; ++j) dl *= a[j * N + n];
+          for (int64_t p = 0; p < P; ++p) yt[p] += dl * ct[n] * prev[n * P + p];
+        }
+      }
+      /* chunk-local state from a zero start, then the recursion */
+      memset(bin, 0, sizeof(double) * N * P);
+      for (int64_t j = 0; j < len; ++j) {
+        const int64_t s = c0 + j;
+        const double* bs = Bm + IX4(b, s, g, 0, L, G, N);
+        const double* xs = x + IX4(b, s, h, 0, L, H, P);
+        for (int64_t n = 0; n < N; ++n) {
+          double wn = 1.0;
+          for (int64_t r = j + 1; r < len; ++r) wn *= a[r * N + n];
+          for (int64_t p = 0; p < P; ++p) bin[n * P + p] += wn * bs[n] * xs[p];
+        }
+      }
+      for (int64_t n = 0; n < N; ++n) {
+        double Ac = 1.0;
+        for (int64_t j = 0; j < len; ++j) Ac *= a[j * N + n];
+        for (int64_t p = 0; p < P; ++p) prev[n * P + p] = bin[n * P + p] + Ac * prev[n * P + p];
+      }
+    }
+    if (final_state) memcpy(final_state + (b * H + h) * N * P, prev, sizeof(double) * N * P);
+    free(prev); free(bin); free(a); free(w);
   }
 }
 

@@ -14,6 +14,7 @@ import pytest
 
 import oracle
 from test_oracle import _read_golden, brute_force, rand_problem, rel
+import test_oracle_vdecay as vd
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "ssd_oracle.c")
 
@@ -40,6 +41,18 @@ MUTANTS = {
     "lam_missing_A": ("if (i < len) s += dt[(b * L + c0 + i) * H + h] * A[h];",
                       "if (i < len) s += dt[(b * L + c0 + i) * H + h];"),
     "rms_count": ("ss / (double)F", "ss / (double)(F - 1)"),
+    "vdecay_channel_reversed": ("const double a = exp(dtv * Av[h * N + n]);",
+                                "const double a = exp(dtv * Av[h * N + (N - 1 - n)]);"),
+    "vdecay_decay_dropped": ("for (int64_t p = 0; p < P; ++p) row[p] = a * row[p] + bt[n] * xt[p];",
+                             "for (int64_t p = 0; p < P; ++p) row[p] = row[p] + bt[n] * xt[p];"),
+    "vdecay_chunked_mask_shift": ("for (int64_t n = 0; n < N; ++n) w[n] *= a[(j + 1) * N + n];",
+                                  "for (int64_t n = 0; n < N; ++n) w[n] *= a[j * N + n];"),
+    "vdecay_chunked_inter_exclusive": ("for (int64_t j = 0; j <= i; ++j) dl *= a[j * N + n];",
+                                       "for (int64_t j = 0; j < i; ++j) dl *= a[j * N + n];"),
+    "vdecay_chunked_state_weight_shift": ("for (int64_t r = j + 1; r < len; ++r) wn *= a[r * N + n];",
+                                          "for (int64_t r = j; r < len; ++r) wn *= a[r * N + n];"),
+    "vdecay_recursion_decay_dropped": ("prev[n * P + p] = bin[n * P + p] + Ac * prev[n * P + p];",
+                                       "prev[n * P + p] = bin[n * P + p] + prev[n * P + p];"),
     "bf16_truncates": ("nearbyint(ldexp(m, 8))", "trunc(ldexp(m, 8))"),
 }
 
@@ -123,6 +136,38 @@ def _pins(o):
         out = oracle.rmsnorm_bf16(a, 0.0, o=o)
         return out[0, 0, 1, 2] == -3.46875  # bf16(-sqrt(12)) worked by hand: sqrt(12) = 3.4641...
     check("rmsnorm_one_hot", rms)
+
+    gv = vd._read_golden("vector_decay.txt")
+
+    def golden_vdecay():
+        Lv, Nv = 3, 2
+        args_v = (gv["x"].reshape(1, Lv, 1, 1), gv["dt"].reshape(1, Lv, 1), gv["Av"].reshape(1, Nv),
+                  gv["B"].reshape(1, Lv, 1, Nv), gv["C"].reshape(1, Lv, 1, Nv))
+        y, f = oracle.scan_recurrence_vdecay(*args_v, gv["D"], gv["h0"].reshape(1, 1, Nv, 1), o=o)
+        return np.allclose(y.ravel(), gv["y"], atol=1e-12) and np.allclose(f.ravel(), gv["final"], atol=1e-12)
+    check("golden_vdecay", golden_vdecay)
+
+    pv = vd.problem(Bz=1, L=17, H=2, P=2, N=3, G=1, seed=5)
+
+    def vdecay_chunked():
+        y, f = oracle.scan_recurrence_vdecay(*pv, o=o)
+        for Q in (1, 4, 16):
+            yc, fc = oracle.scan_chunked_vdecay(*pv[:5], Q, pv[5], pv[6], o=o)
+            if not (rel(yc, y) < 1e-12 and rel(fc, f) < 1e-12):
+                return False
+        return True
+    check("vdecay_chunked_vs_recurrence", vdecay_chunked)
+
+    def vdecay_golden_chunked():
+        Lv, Nv = 3, 2
+        args_v = (gv["x"].reshape(1, Lv, 1, 1), gv["dt"].reshape(1, Lv, 1), gv["Av"].reshape(1, Nv),
+                  gv["B"].reshape(1, Lv, 1, Nv), gv["C"].reshape(1, Lv, 1, Nv))
+        for Q in (2, 3):
+            y, f = oracle.scan_chunked_vdecay(*args_v, Q, gv["D"], gv["h0"].reshape(1, 1, Nv, 1), o=o)
+            if not (np.allclose(y.ravel(), gv["y"], atol=1e-12) and np.allclose(f.ravel(), gv["final"], atol=1e-12)):
+                return False
+        return True
+    check("vdecay_golden_chunked", vdecay_golden_chunked)
 
     def bf16():
         v = np.array([1.0 + 3 * 2.0 ** -9, -(1.0 + 2.0 ** -8 + 2.0 ** -10)])

@@ -6,5 +6,6 @@
 #include "ssd_pair.cu"
 #include "ssd_api.cu"
 #include "ssd_noalloc.cu"
+#include "ssd_vdecay.cu"
 #include "ssd_hostio.cu"
 #include "ssd_selftest.cu"

@@ -28,7 +28,7 @@ EXPORTED = ["ssd_status_string", "ssd_version", "ssd_scan_workspace_size", "ssd_
             "ssd_read_device_status", "ssd_selftest_umma", "ssd_scan_path", "ssd_step",
             "ssd_selftest_fused_trace", "ssd_scan_fwd_noalloc",
             "ssd_selftest_timeout", "ssd_scan_fwd_host", "ssd_scan_fwd_host_workspace_size",
-            "ssd_scan_fwd_strided", "ssd_selftest_carry_timeout"]
+            "ssd_scan_fwd_strided", "ssd_selftest_carry_timeout", "ssd_scan_fwd_vdecay"]
 
 
 class SSDError(RuntimeError):
@@ -86,6 +86,7 @@ def lib() -> ctypes.CDLL:
         "ssd_selftest_fused_trace": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_int64, _P]),
         "ssd_selftest_timeout": (ctypes.c_int, [D] + [_P] * 10),
         "ssd_selftest_carry_timeout": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_size_t, _P]),
+        "ssd_scan_fwd_vdecay": (ctypes.c_int, [D] + [_P] * 10),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -186,6 +187,23 @@ def ssd_scan_fwd(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, y=
     s = fn(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D), _ptr(init_state), _ptr(y),
            _ptr(final_state), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check(s, "ssd_scan_fwd_unfused" if unfused else "ssd_scan_fwd")
+    return y, final_state
+
+
+def ssd_scan_fwd_vdecay(x, dt, Av, Bm, Cm, D=None, init_state=None, y=None, final_state=None, stream=None,
+                        want_final: bool = True):
+    """y, final_state of the scan with a per-channel decay a_t[n] = exp(dt_t Av[h, n]),
+    Av [H, N] f32 (token recurrence on CUDA cores; fp32 or bf16 io)."""
+    _contig(x, dt, Av, Bm, Cm, D, init_state, y, final_state)
+    dims = make_dims(x, Bm, 1)
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None and want_final:
+        final_state = torch.empty((dims.batch, dims.nheads, dims.dstate, dims.headdim), dtype=torch.float32,
+                                  device=x.device)
+    _check(lib().ssd_scan_fwd_vdecay(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(Av), _ptr(Bm), _ptr(Cm), _ptr(D),
+                                     _ptr(init_state), _ptr(y), _ptr(final_state), _stream(stream)),
+           "ssd_scan_fwd_vdecay")
     return y, final_state
 
 

@@ -336,6 +336,26 @@ ssd_status ssd_step(const ssd_dims* d, const void* x, const float* dt, const flo
                     const void* Cm, const float* D, float* state, void* y, void* stream);
 
 /*
+ * The scan with a vector-valued decay: one decay rate per state channel n in
+ * place of the per-head scalar -- the diagonal state matrix of the selective
+ * scan ("告别Transformer的二次方噩梦…" §2.1) and the per-channel decays of the
+ * recurrences "分块推理…" §6 names (RWKV, xLSTM):
+ *     a_t[n] = exp(dt[b,t,h] * Av[h,n])
+ *     h_t[n,:] = a_t[n] h_{t-1}[n,:] + Bm[b,t,g,n] x[b,t,h,:]
+ *     y_t = Cm[b,t,g,:]^T h_t + D[h] x[b,t,h,:]
+ *   Av: [H, N] f32 (non-positive); every other argument, layout and error as
+ *   ssd_scan_fwd (fp32 or bf16 io), without a workspace; d->flags must be 0
+ *   (else SSD_ERR_UNSUPPORTED).  Pointers need their element's natural
+ *   alignment only.  Runs the token recurrence on CUDA cores (fp32 state):
+ *   with channel-dependent decays the chunked form's intra-chunk term no
+ *   longer factors into (C B^T) (.) L.  With Av[h,n] equal over n the result
+ *   is ssd_scan_fwd's up to rounding.
+ */
+ssd_status ssd_scan_fwd_vdecay(const ssd_dims* d, const void* x, const float* dt, const float* Av, const void* Bm,
+                               const void* Cm, const float* D, const float* init_state, void* y,
+                               float* final_state, void* stream);
+
+/*
  * Read and clear the device status word that bounded waits inside the
  * kernels set (synchronises `stream`).  Returns SSD_OK or SSD_ERR_TIMEOUT.
  */

@@ -215,3 +215,15 @@ def test_noalloc_rejects_sizes_beyond_its_buffer(lib):
     assert lib.ssd_scan_fwd_noalloc(ctypes.byref(d), *ptrs, None) == 5
     # a size that fits passes validation; a NULL x is still refused first
     assert lib.ssd_scan_fwd_noalloc(ctypes.byref(dims()), None, *ptrs[1:], None) == 1
+
+
+def test_vdecay_entry_rejects(lib):
+    d = dims(chunk=1)
+    ptrs = [ctypes.c_void_p(BASE + k * GB) for k in (0, 2, 3, 4, 5, 6, 7, 8, 9)]  # x dt Av B C D init y final
+    assert lib.ssd_scan_fwd_vdecay(ctypes.byref(dims(chunk=1, flags=1)), *ptrs, None) == 5  # no flags
+    assert lib.ssd_scan_fwd_vdecay(ctypes.byref(d), ptrs[0], ptrs[1], None, *ptrs[3:], None) == 1  # NULL Av
+    assert lib.ssd_scan_fwd_vdecay(ctypes.byref(d), ptrs[0], ptrs[1], ctypes.c_void_p(BASE + 2 * GB + 2),
+                                   *ptrs[3:], None) == 4  # Av misaligned
+    # y overlapping Av [H, N]
+    assert lib.ssd_scan_fwd_vdecay(ctypes.byref(d), *ptrs[:7], ctypes.c_void_p(BASE + 3 * GB + 16), ptrs[8],
+                                   None) == 1

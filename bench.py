@@ -577,13 +577,14 @@ def run_stack(args, wl, dev, rank, world):
     states = [torch.zeros((wl.batch, wl.nheads, wl.dstate, wl.headdim), dtype=torch.float32, device=dev)
               for _ in range(wl.n_layers)]
     y = torch.empty_like(x0)
-    dims = ssd.make_dims(x0, layers[0]["B"], wl.chunk)
+    th = args.two_heads
+    dims = ssd.make_dims(x0, layers[0]["B"], wl.chunk, two_heads=th)
     ws = torch.empty(ssd.ssd_vertical_workspace_size(dims, wl.n_layers, wl.vblock), dtype=torch.uint8, device=dev)
     torch.cuda.synchronize(dev)
 
     def vertical():
         ssd.ssd_vertical_fwd(x0, layers, states, vblock=wl.vblock, chunk=wl.chunk, rms_eps=eps, y_out=y,
-                             workspace=ws, stream=stream)
+                             workspace=ws, stream=stream, two_heads=th)
 
     per_step, ms_total, clk = timed_steps(vertical, args, stream, dev, local, world)
     ms_per_step = ms_total / args.steps
@@ -605,7 +606,7 @@ def run_stack(args, wl, dev, rank, world):
         x = x0
         for l, p in enumerate(layers):
             ssd.ssd_scan_fwd(x, p["dt"], p["A"], p["B"], p["C"], p["D"], states[l], chunk=wl.chunk, y=y,
-                             final_state=states[l], stream=stream)
+                             final_state=states[l], stream=stream, two_heads=th)
             if l + 1 < wl.n_layers:
                 ssd.ssd_rmsnorm(y, eps, out=xh, stream=stream)
                 x = xh
@@ -625,12 +626,12 @@ def run_stack(args, wl, dev, rank, world):
         side.wait_stream(stream)
         with torch.cuda.stream(side):
             ssd.ssd_vertical_fwd(x0, layers, states, vblock=wl.vblock, chunk=wl.chunk, rms_eps=eps, y_out=y,
-                                 workspace=ws, stream=side)
+                                 workspace=ws, stream=side, two_heads=th)
         stream.wait_stream(side)
         torch.cuda.synchronize(dev)
         with torch.cuda.graph(g, stream=side):
             ssd.ssd_vertical_fwd(x0, layers, states, vblock=wl.vblock, chunk=wl.chunk, rms_eps=eps, y_out=y,
-                                 workspace=ws, stream=side)
+                                 workspace=ws, stream=side, two_heads=th)
         torch.cuda.synchronize(dev)
         _, g_total, _ = timed_steps(g.replay, hs, stream, dev, local, world)
         graph_ms = g_total / hs.steps
@@ -677,6 +678,7 @@ def run_stack(args, wl, dev, rank, world):
         "config": {"workload": wl.name, "batch": wl.batch, "seqlen": wl.seqlen, "nheads": wl.nheads,
                    "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk,
                    "n_layers": wl.n_layers, "vblock": wl.vblock, "schedule": "vertical (ssd_vertical_fwd)",
+                   "kernel": "two heads per CTA" if th else "one head per CTA",
                    "horizontal_ms_per_step": h_ms, "vertical_graph_ms_per_step": graph_ms,
                    "vertical_host_enqueue_ms": host_ms,
                    "parallelism": f"dp{world} (independent batches per rank)",

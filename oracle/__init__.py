@@ -17,9 +17,10 @@ Functions and the passages they follow (page titles as published):
   selective scan, "告别Transformer的二次方噩梦…" §2.1; per-channel decays as in
   the recurrences of "分块推理…" §6): the token recurrence and its chunk
   decomposition.
-* ``round_bf16``, ``rmsnorm_bf16`` -- storage rounding and the layer-to-layer
-  normalisation of the multi-layer stack (a reading; the page's §3 only says
-  that layer l's output feeds layer l+1).
+* ``round_bf16``, ``rmsnorm``, ``rmsnorm_bf16`` -- storage rounding and the
+  layer-to-layer normalisation of the multi-layer stack, unrounded (as a
+  fused implementation feeds it) and stored in bf16 (a reading; the page's §3
+  only says that layer l's output feeds layer l+1).
 * ``stack_horizontal`` / ``stack_vertical`` -- the two multi-layer schedules
   of §3.1 and §3.2 of the same page.
 
@@ -71,6 +72,8 @@ class _Oracle:
         lib.oracle_round_bf16.argtypes = [_I, _P, _P]
         lib.oracle_rmsnorm_bf16.restype = None
         lib.oracle_rmsnorm_bf16.argtypes = [_I, _I, _P, ctypes.c_double, _P]
+        lib.oracle_rmsnorm.restype = None
+        lib.oracle_rmsnorm.argtypes = [_I, _I, _P, ctypes.c_double, _P]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         self.lib = lib
@@ -179,6 +182,16 @@ def round_bf16(a, o: Optional[_Oracle] = None) -> np.ndarray:
     a = _f64(a)
     out = np.empty_like(a)
     o.lib.oracle_round_bf16(a.size, _ptr(a), _ptr(out))
+    return out
+
+
+def rmsnorm(a, eps: float, o: Optional[_Oracle] = None) -> np.ndarray:
+    """RMS-normalise each token of a [B, L, H, P] array over its H*P features (fp64, unrounded)."""
+    o = o or load()
+    a = _f64(a)
+    Bz, L, H, P = a.shape
+    out = np.empty_like(a)
+    o.lib.oracle_rmsnorm(Bz * L, H * P, _ptr(a), eps, _ptr(out))
     return out
 
 

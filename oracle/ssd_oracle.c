@@ -339,15 +339,25 @@ void oracle_round_bf16(int64_t n, const double* in, double* out) {
  * H*P features of a token, no learned weight):
  *   out[r, :] = bf16( in[r, :] / sqrt(mean_f in[r, f]^2 + eps) )
  */
-void oracle_rmsnorm_bf16(int64_t rows, int64_t F, const double* in, double eps, double* out) {
+/* RMS normalisation of each row of F features: v / sqrt(mean(v^2) + eps), in
+ * fp64 and unrounded (a fused implementation never stores the normalised
+ * row, so no storage rounding happens between the layers). */
+void oracle_rmsnorm(int64_t rows, int64_t F, const double* in, double eps, double* out) {
 #pragma omp parallel for schedule(static)
   for (int64_t r = 0; r < rows; ++r) {
     const double* v = in + r * F;
     double ss = 0.0;
     for (int64_t f = 0; f < F; ++f) ss += v[f] * v[f];
     const double inv = 1.0 / sqrt(ss / (double)F + eps);
-    for (int64_t f = 0; f < F; ++f) out[r * F + f] = round_bf16(v[f] * inv);
+    for (int64_t f = 0; f < F; ++f) out[r * F + f] = v[f] * inv;
   }
+}
+
+/* The same, stored in bf16 (the layer input a separate normalisation pass writes). */
+void oracle_rmsnorm_bf16(int64_t rows, int64_t F, const double* in, double eps, double* out) {
+  oracle_rmsnorm(rows, F, in, eps, out);
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < rows * F; ++i) out[i] = round_bf16(out[i]);
 }
 
 #ifdef _OPENMP

@@ -337,6 +337,31 @@ def test_rmsnorm_closed_forms():
     assert np.all(oracle.rmsnorm_bf16(np.zeros((1, 1, H, P)), 1e-6) == 0)
 
 
+def test_rmsnorm_unrounded_closed_forms():
+    H, P = 3, 4
+    F = H * P
+    # one-hot row: v / sqrt(v^2 / F + eps), here with eps = 0.25 worked by hand:
+    # v = -7.5 -> v^2 / F = 56.25 / 12 = 4.6875, + 0.25 = 4.9375
+    a = np.zeros((1, 1, H, P))
+    a[0, 0, 1, 2] = -7.5
+    out = oracle.rmsnorm(a, 0.25)
+    assert abs(out[0, 0, 1, 2] - (-7.5 / math.sqrt(4.9375))) < 1e-15
+    assert np.count_nonzero(out) == 1
+    # eps = 0: every row has mean square exactly one, signs kept, scale-free
+    rng = np.random.default_rng(15)
+    b = rng.standard_normal((2, 5, H, P))
+    o1 = oracle.rmsnorm(b, 0.0)
+    np.testing.assert_allclose(np.mean(o1.reshape(10, F) ** 2, axis=1), 1.0, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(oracle.rmsnorm(b * 1024.0, 0.0), o1, rtol=1e-14, atol=0)
+    np.testing.assert_array_equal(np.sign(o1), np.sign(b))
+    # one row's features are normalised together, rows independently
+    two = np.concatenate([b[:, :1], 3.0 * b[:, :1]], axis=1)
+    o2 = oracle.rmsnorm(two, 0.0)
+    np.testing.assert_allclose(o2[:, 0], o2[:, 1], rtol=1e-14, atol=0)
+    # the stored form is this one rounded to bf16
+    np.testing.assert_array_equal(oracle.round_bf16(oracle.rmsnorm(b, 1e-6)), oracle.rmsnorm_bf16(b, 1e-6))
+
+
 # ---------------------------------------------------------------- multi-layer schedules
 
 def _layers(n_layers, Bz, L, H, P, N, G, seed):

@@ -41,6 +41,8 @@ MUTANTS = {
     "lam_missing_A": ("if (i < len) s += dt[(b * L + c0 + i) * H + h] * A[h];",
                       "if (i < len) s += dt[(b * L + c0 + i) * H + h];"),
     "rms_count": ("ss / (double)F", "ss / (double)(F - 1)"),
+    "rms_eps_dropped": ("const double inv = 1.0 / sqrt(ss / (double)F + eps);",
+                        "const double inv = 1.0 / sqrt(ss / (double)F);"),
     "vdecay_channel_reversed": ("const double a = exp(dtv * Av[h * N + n]);",
                                 "const double a = exp(dtv * Av[h * N + (N - 1 - n)]);"),
     "vdecay_decay_dropped": ("for (int64_t p = 0; p < P; ++p) row[p] = a * row[p] + bt[n] * xt[p];",
@@ -136,6 +138,13 @@ def _pins(o):
         out = oracle.rmsnorm_bf16(a, 0.0, o=o)
         return out[0, 0, 1, 2] == -3.46875  # bf16(-sqrt(12)) worked by hand: sqrt(12) = 3.4641...
     check("rmsnorm_one_hot", rms)
+
+    def rms_eps():
+        a = np.zeros((1, 1, 3, 4))
+        a[0, 0, 1, 2] = -7.5
+        out = oracle.rmsnorm(a, 0.25, o=o)
+        return abs(out[0, 0, 1, 2] - (-7.5 / math.sqrt(4.9375))) < 1e-15  # 56.25 / 12 + 0.25 = 4.9375
+    check("rmsnorm_eps", rms_eps)
 
     gv = vd._read_golden("vector_decay.txt")
 

@@ -597,19 +597,33 @@ def run_stack(args, wl, dev, rank, world):
     tokens = wl.batch * wl.seqlen * world
     value = tokens / (ms_per_step * 1e-3)
     nblk = -(-wl.seqlen // wl.vblock)
-    launches = nblk * (2 * wl.n_layers - 1)
+    # one scan launch per (block, layer); the two-head kernel adds a norm pass per
+    # (block, layer boundary), the one-head kernel has the norm fused
+    launches = nblk * ((2 * wl.n_layers - 1) if th else wl.n_layers)
 
-    # horizontal schedule: layer by layer over the whole sequence
+    # horizontal schedule: layer by layer over the whole sequence (the same
+    # arithmetic as the vertical one: the norm fused, or its own pass)
     xh = torch.empty_like(x0)
+    xh2 = None if th else torch.empty_like(x0)
+    ss = [torch.empty(x0.shape[:3], dtype=torch.float32, device=dev) for _ in range(2)]
 
     def horizontal():
         x = x0
         for l, p in enumerate(layers):
-            ssd.ssd_scan_fwd(x, p["dt"], p["A"], p["B"], p["C"], p["D"], states[l], chunk=wl.chunk, y=y,
-                             final_state=states[l], stream=stream, two_heads=th)
-            if l + 1 < wl.n_layers:
-                ssd.ssd_rmsnorm(y, eps, out=xh, stream=stream)
-                x = xh
+            last = l + 1 == wl.n_layers
+            if th:
+                ssd.ssd_scan_fwd(x, p["dt"], p["A"], p["B"], p["C"], p["D"], states[l], chunk=wl.chunk, y=y,
+                                 final_state=states[l], stream=stream, two_heads=th)
+                if not last:
+                    ssd.ssd_rmsnorm(y, eps, out=xh, stream=stream)
+                    x = xh
+            else:
+                yl = y if last else (xh if l % 2 == 0 else xh2)
+                ssd.ssd_scan_fwd_normed(x, ss[(l + 1) % 2] if l > 0 else None, p["dt"], p["A"], p["B"], p["C"],
+                                        p["D"], states[l], chunk=wl.chunk, rms_eps=eps, y=yl,
+                                        ss_out=None if last else ss[l % 2], want_sums=not last,
+                                        final_state=states[l], stream=stream)
+                x = yl
 
     hs = argparse.Namespace(steps=max(2, args.steps // 2), warmup=args.warmup)
     h_ms = graph_ms = None
@@ -687,9 +701,11 @@ def run_stack(args, wl, dev, rank, world):
                                "d2h_bytes_per_step": d2h},
         "gpu_launches": launches * args.steps,
         "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
-                     "traffic": None, "kernel": "whole step (k_ssd_fused per block and layer, k_rmsnorm between)",
-                     "algorithmic_bytes": f"{wl.n_layers} x one layer's scan bytes; the RMS norm traffic between "
-                                          "layers is not counted",
+                     "traffic": None,
+                     "kernel": ("whole step (k_ssd_pair per block and layer, k_rmsnorm between)" if th else
+                                "whole step (k_ssd_fused per block and layer, the RMS norm fused in)"),
+                     "algorithmic_bytes": f"{wl.n_layers} x one layer's scan bytes; the RMS norm's sums of squares "
+                                          "(and with two heads per CTA its own pass) are not counted",
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else
                      "fallback 6650 GB/s"},
     }

@@ -217,6 +217,36 @@ ssd_status ssd_scan_fwd(const ssd_dims* d, const void* x, const float* dt, const
   return run_unfused(p, init_state, final_state, static_cast<char*>(workspace), st);
 }
 
+ssd_status ssd_scan_fwd_normed(const ssd_dims* d, const void* x, const float* ss_in, float rms_eps,
+                               const float* dt, const float* A, const void* Bm, const void* Cm,
+                               const float* D, const float* init_state, void* y, float* ss_out,
+                               float* final_state, void* stream) {
+  ssd_status s = validate_dims(d);
+  if (s != SSD_OK) return s;
+  if (d->flags & ~SSD_FLAG_INPUT_DT) return SSD_ERR_UNSUPPORTED;  // the one-head kernel only
+  s = validate_scan_args(d, x, dt, A, Bm, Cm, D, init_state, y, final_state);
+  if (s != SSD_OK) return s;
+  Problem p = make_problem(d);
+  if (!fused_supported(p)) return SSD_ERR_UNSUPPORTED;
+  if (!(rms_eps >= 0.0f)) return SSD_ERR_INVALID_ARG;
+  if ((ss_in && !aligned16(ss_in)) || (ss_out && !aligned16(ss_out))) return SSD_ERR_ALIGN;
+  const size_t es = io_size(d->io_dtype);
+  const size_t act = es * (size_t)p.B * p.L * p.H * p.P, sums = sizeof(float) * (size_t)p.B * p.L * p.H;
+  const Range rx = range_of(x, act), ry = range_of(y, act);
+  if (ss_in && (overlaps(range_of(ss_in, sums), rx) || overlaps(range_of(ss_in, sums), ry)))
+    return SSD_ERR_INVALID_ARG;
+  if (ss_out && (overlaps(range_of(ss_out, sums), rx) || overlaps(range_of(ss_out, sums), ry) ||
+                 (ss_in && overlaps(range_of(ss_out, sums), range_of(ss_in, sums)))))
+    return SSD_ERR_INVALID_ARG;
+  p.x = x; p.dt = dt; p.A = A; p.Bm = Bm; p.Cm = Cm; p.D = D; p.y = y;
+  NormIO nio;
+  nio.ss_in = ss_in;
+  nio.ss_out = ss_out;
+  nio.batch_stride = p.L * p.H;
+  nio.eps = rms_eps;
+  return cuda_status(launch_fused_normed(p, init_state, final_state, nio, static_cast<cudaStream_t>(stream)));
+}
+
 ssd_status ssd_scan_fwd_strided(const ssd_dims* d, const void* x, int64_t x_bstride, int64_t x_tstride,
                                 const float* dt, int64_t dt_bstride, int64_t dt_tstride, const float* A, const void* Bm,
                                 const void* Cm, int64_t bc_bstride, int64_t bc_tstride, const float* D,
@@ -323,7 +353,8 @@ ssd_status ssd_rmsnorm(int64_t rows, int64_t features, int32_t io_dtype, const v
 }
 
 // Vertical (depth-first) schedule.  Workspace: the single-layer workspace of
-// a V-token slice, then two activation buffers [B, V, H, P] (io dtype).
+// a V-token slice, then the activation blocks [B, V, H, P] (io dtype) and, for
+// the fused RMS norm, their per-(token, head) sums of squares [B, V, H] f32.
 ssd_status ssd_vertical_workspace_size(const ssd_dims* d, int32_t n_layers, int64_t vblock, size_t* bytes) {
   if (!bytes) return SSD_ERR_INVALID_ARG;
   ssd_status s = validate_dims(d);
@@ -337,7 +368,8 @@ ssd_status ssd_vertical_workspace_size(const ssd_dims* d, int32_t n_layers, int6
   const size_t act = align_up(io_size(d->io_dtype) * (size_t)d->batch * dv.seqlen * d->nheads * d->headdim);
   // the wavefront schedule keeps two activation blocks per layer boundary
   const size_t nact = n_layers > 2 ? 2 * (size_t)(n_layers - 1) : 2;
-  *bytes = align_up(one) + nact * act;
+  const size_t sums = align_up(sizeof(float) * (size_t)d->batch * dv.seqlen * d->nheads);
+  *bytes = align_up(one) + nact * (act + sums);
   return SSD_OK;
 }
 
@@ -415,9 +447,12 @@ static ssd_status vertical_wavefront(const ssd_dims* d_, int32_t n_layers, int64
   ssd_scan_workspace_size(&dv, &one);
   const size_t es = io_size(d_->io_dtype);
   const size_t act = align_up(es * (size_t)d_->batch * V * d_->nheads * d_->headdim);
+  const size_t sums = align_up(sizeof(float) * (size_t)d_->batch * V * d_->nheads);
   char* ring = static_cast<char*>(workspace) + align_up(one);
-  // input buffer of layer l (1 <= l < n_layers) for blocks of parity q
-  auto in_buf = [&](int l, int64_t q) { return ring + ((size_t)(l - 1) * 2 + (size_t)q) * act; };
+  // input buffer of layer l (1 <= l < n_layers) for blocks of parity q, and its
+  // rows' per-(token, head) sums of squares
+  auto in_buf = [&](int l, int64_t q) { return ring + ((size_t)(l - 1) * 2 + (size_t)q) * (act + sums); };
+  auto in_sums = [&](int l, int64_t q) { return reinterpret_cast<float*>(in_buf(l, q) + act); };
   const int64_t HP = full.H * full.P;
 
   // fork: every layer stream starts after the work already on `st`
@@ -473,9 +508,18 @@ static ssd_status vertical_wavefront(const ssd_dims* d_, int32_t n_layers, int64
         p.y = in_buf(l + 1, k & 1);
         p.sy = Vk * HP;
       }
-      s = cuda_status(launch_fused(p, states[l], states[l], nullptr, 0, sl));
-      if (s == SSD_OK && !last)
-        s = cuda_status(launch_rmsnorm(d_->batch * Vk, HP, d_->io_dtype, p.y, rms_eps, p.y, sl));
+      if (uses_pair_kernel(p)) {  // the two-head kernel: the norm as its own pass
+        s = cuda_status(launch_fused(p, states[l], states[l], nullptr, 0, sl));
+        if (s == SSD_OK && !last)
+          s = cuda_status(launch_rmsnorm(d_->batch * Vk, HP, d_->io_dtype, p.y, rms_eps, p.y, sl));
+      } else {  // the norm fused: sums out of layer l, scales into layer l+1
+        NormIO nio;
+        nio.ss_in = l > 0 ? in_sums(l, k & 1) : nullptr;
+        nio.ss_out = last ? nullptr : in_sums(l + 1, k & 1);
+        nio.batch_stride = Vk * full.H;
+        nio.eps = rms_eps;
+        s = cuda_status(launch_fused_normed(p, states[l], states[l], nio, sl));
+      }
       if (s != SSD_OK) break;
       e = cudaEventRecord(pool->out[l], sl);
       if (e == cudaSuccess && l > 0) e = cudaEventRecord(pool->freed[2 * l + (k & 1)], sl);

@@ -47,8 +47,10 @@ constexpr uint32_t OFF_XP = 2 * STAGE;         // X' (two buffers)
 constexpr uint32_t OFF_PREV = OFF_XP + 2 * TILE;  // bf16 state, MN-major [n][p]
 constexpr uint32_t OFF_LAM = OFF_PREV + TILE;  // float [4][128]
 constexpr uint32_t OFF_ECOL = OFF_LAM + 4 * T * 4;  // float [4][128]
-constexpr uint32_t OFF_DTS = OFF_ECOL + 4 * T * 4;   // float [4][128]: the input term's dt (1 without the flag)
-constexpr uint32_t OFF_WTOT = OFF_DTS + 4 * T * 4;
+constexpr uint32_t OFF_DTS = OFF_ECOL + 4 * T * 4;   // float [4][128]: the input term's column factor
+                                                     // (dt_s, times r_s with the normalised input)
+constexpr uint32_t OFF_RN = OFF_DTS + 4 * T * 4;     // float [4][128]: r_t of the normalised input
+constexpr uint32_t OFF_WTOT = OFF_RN + 4 * T * 4;
 constexpr uint32_t OFF_BAR = OFF_WTOT + 64;
 constexpr uint32_t NBAR = 20;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
@@ -79,6 +81,13 @@ struct Params {
   int64_t sx, ldx;    // batch and token strides of x
   __nv_bfloat16* y;
   int64_t sy;
+  // RMS-normalised input (layer stacks): the input rows are the previous
+  // layer's stored y, and each token t enters as r_t x_t with
+  // r_t = 1 / sqrt(sum over heads of ss_in[b, t, h] / (H P) + eps)
+  const float* ss_in;   // [B][L][H] sums of squares of the input rows per (token, head), or NULL
+  float* ss_out;        // [B][L][H] sums of squares of this call's stored (bf16) y rows, or NULL
+  int64_t sss;          // batch stride of ss_in and ss_out (floats)
+  float norm_eps, inv_feat;  // eps, 1 / (H P)
   unsigned long long* trace;  // diagnostics: per-sub-chunk event clocks of CTA 0, then
                               // [start ns, end ns, SM] of every CTA; or NULL
   int withhold_loads;         // self-test of the timeout path: issue no TMA loads, so
@@ -177,9 +186,11 @@ __device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
 
-// XDT: the dt-scaled input variant, a separate instantiation so that the plain
-// scan carries none of its per-column factors.
-template <bool XDT>
+// XDT: the dt-scaled input variant; NORM: a layer of a stack with the RMS norm
+// fused (input scaled from ss_in when given, sums of squares to ss_out when
+// given).  Separate instantiations, so that the plain scan carries none of
+// their per-column factors and sums.
+template <bool XDT, bool NORM>
 __global__ void __launch_bounds__(THREADS, 1)
     k_ssd_fused(Params p, const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
                 const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_y) {
@@ -191,6 +202,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   float* lamb = reinterpret_cast<float*>(sm + OFF_LAM);
   float* ecolb = reinterpret_cast<float*>(sm + OFF_ECOL);
   float* dtsb = reinterpret_cast<float*>(sm + OFF_DTS);
+  float* rnb = reinterpret_cast<float*>(sm + OFF_RN);
+  constexpr bool CF = XDT || NORM;  // the input term has a factor per column s
   float* wtot = reinterpret_cast<float*>(sm + OFF_WTOT);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
@@ -385,12 +398,89 @@ __global__ void __launch_bounds__(THREADS, 1)
       d1 = (!chunked && j < nsub && t0 + 1 < p.L) ? dtb[(t0 + 1) * p.lddt] : 0.f;
     };
     const float* lamc = chunked ? p.lam_in + cslot * p.Q : nullptr;
-    float d0, d1;
+    // r of tokens 2a, 2a+1 of sub-chunk j from the H per-head sums of squares
+    // of the previous layer's stored y (0 past L).  A token's H sums are
+    // contiguous.  With H % 4 == 0 the first 32 of them (8 float4 per token)
+    // are loaded one sub-chunk ahead into registers (issue_rn) and summed when
+    // needed (finish_rn), so the trip to L2 overlaps a whole iteration; sums
+    // past the first 32 heads, and rows with H % 4 != 0, are loaded when needed.
+    const bool vec = (p.H & 3) == 0;
+    float4 pv[8], pw[8];
+    auto rn_row = [&](int j, int k) { return p.ss_in + (int64_t)b * p.sss + ((int64_t)j * T + 2 * a + k) * p.H; };
+    auto issue_rn = [&](int j) {
+      const int64_t t0 = (int64_t)j * T + 2 * a;
+      const bool use = p.ss_in && vec && j < nsub;
+      const float4* q0 = use ? reinterpret_cast<const float4*>(rn_row(j, 0)) : nullptr;
+      const float4* q1 = use ? reinterpret_cast<const float4*>(rn_row(j, 1)) : nullptr;
+      const int n4 = p.H >> 2;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        pv[i] = (use && i < n4 && t0 < p.L) ? q0[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        pw[i] = (use && i < n4 && t0 + 1 < p.L) ? q1[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    auto finish_rn = [&](int j, float& r0, float& r1) {
+      if (!p.ss_in) {  // the stack's first layer: its input is used as is
+        r0 = r1 = 1.f;
+        return;
+      }
+      const int64_t t0 = (int64_t)j * T + 2 * a;
+      const bool in0 = t0 < p.L, in1 = t0 + 1 < p.L;
+      float s0 = 0.f, s1 = 0.f;
+      if (vec) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {  // the prefetched first 32 heads
+          s0 += (pv[i].x + pv[i].y) + (pv[i].z + pv[i].w);
+          s1 += (pw[i].x + pw[i].y) + (pw[i].z + pw[i].w);
+        }
+        const float4* q0 = reinterpret_cast<const float4*>(rn_row(j, 0));
+        const float4* q1 = reinterpret_cast<const float4*>(rn_row(j, 1));
+        const int n4 = p.H >> 2;
+        for (int i0 = 8; i0 < n4; i0 += 8) {  // heads past the first 32
+          float4 v[8], w[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const bool ok = i0 + i < n4;
+            v[i] = (ok && in0) ? q0[i0 + i] : make_float4(0.f, 0.f, 0.f, 0.f);
+            w[i] = (ok && in1) ? q1[i0 + i] : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            s0 += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+            s1 += (w[i].x + w[i].y) + (w[i].z + w[i].w);
+          }
+        }
+      } else {
+        const float* q = rn_row(j, 0);
+        for (int i0 = 0; i0 < p.H; i0 += 16) {
+          float v[16], w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const bool ok = i0 + i < p.H;
+            v[i] = (ok && in0) ? q[i0 + i] : 0.f;
+            w[i] = (ok && in1) ? q[p.H + i0 + i] : 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            s0 += v[i];
+            s1 += w[i];
+          }
+        }
+      }
+      r0 = in0 ? rsqrtf(s0 * p.inv_feat + p.norm_eps) : 0.f;
+      r1 = in1 ? rsqrtf(s1 * p.inv_feat + p.norm_eps) : 0.f;
+    };
+    float d0, d1;  // dt of the next sub-chunk to be tabled (tokens 2a, 2a+1)
     load_dt(0, d0, d1);
-    for (int j = 0; j < nsub; ++j) {
-      const int st = j & 1, slot = j & 3;
+    if constexpr (NORM) issue_rn(0);
+    // The tables of sub-chunk jt into slot jt & 3 (lam, the column decays and
+    // factors, r), then LAMRDY; dt and the norm sums of jt + 1 are requested on
+    // the way.  The loop below runs them one sub-chunk ahead of X', so the
+    // mask never waits for the X' of the sub-chunk before it.
+    auto tables = [&](int jt) {
+      const int slot = jt & 3;
       float n0, n1;
-      load_dt(j + 1, n0, n1);  // one sub-chunk ahead
+      load_dt(jt + 1, n0, n1);
       // inclusive scan of dt*A over the 128 tokens (two per thread)
       const float l0 = d0 * Ah, l1 = d1 * Ah;
       float v = l0 + l1;
@@ -405,8 +495,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       float lam1 = v + pre;       // token 2a+1
       float lam0 = lam1 - l1;     // token 2a
       if (chunked) {              // step modes: sub-chunk-local sums from step 1's output
-        const float* ls = lamc + j * T;
-        const float base0 = (j == 0) ? 0.f : ls[-1];
+        const float* ls = lamc + jt * T;
+        const float base0 = (jt == 0) ? 0.f : ls[-1];
         lam0 = ls[2 * a] - base0;
         lam1 = ls[2 * a + 1] - base0;
       }
@@ -416,9 +506,24 @@ __global__ void __launch_bounds__(THREADS, 1)
       float* dts = dtsb + slot * T;
       lj[2 * a] = lam0 * kLog2e;
       lj[2 * a + 1] = lam1 * kLog2e;
-      if constexpr (XDT) {  // the input term's factor per column: dt_s
-        dts[2 * a] = d0;
-        dts[2 * a + 1] = d1;
+      // the input term's factor per column s: dt_s (dt-scaled input) times r_s
+      // (normalised input)
+      float cf0 = 1.f, cf1 = 1.f;
+      if constexpr (XDT) {
+        cf0 = d0;
+        cf1 = d1;
+      }
+      if constexpr (NORM) {
+        float rn0, rn1;
+        finish_rn(jt, rn0, rn1);
+        rnb[slot * T + 2 * a] = rn0;
+        rnb[slot * T + 2 * a + 1] = rn1;
+        cf0 *= rn0;
+        cf1 *= rn1;
+      }
+      if constexpr (CF) {
+        dts[2 * a] = cf0;
+        dts[2 * a + 1] = cf1;
       }
       named_sync(1, AUX);
       // decay from each column s to the last column of its 32-block (times the
@@ -426,14 +531,25 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float lr = lj[(2 * a) | 31];
       ec[2 * a] = ex2(lr - lj[2 * a]);
       ec[2 * a + 1] = ex2(lr - lj[2 * a + 1]);
-      if constexpr (XDT) {
-        ec[2 * a] *= d0;
-        ec[2 * a + 1] *= d1;
+      if constexpr (CF) {
+        ec[2 * a] *= cf0;
+        ec[2 * a + 1] *= cf1;
       }
       mbar_arrive(&bar[LAMRDY0 + slot]);
-      if (a == 0) mark(j, EV_LAM_READY);
+      if (a == 0) mark(jt, EV_LAM_READY);
       d0 = n0;
       d1 = n1;
+      if constexpr (NORM) issue_rn(jt + 1);  // in flight until the next tables
+    };
+    tables(0);
+    for (int j = 0; j < nsub; ++j) {
+      const int st = j & 1, slot = j & 3;
+      // Slot (j + 1) & 3 last held sub-chunk j - 3, whose readers (its mask,
+      // epilogue and X') are done: this loop waited for its products and its y
+      // store in iteration j - 1.
+      if (j + 1 < nsub) tables(j + 1);
+      const float* lj = lamb + slot * T;
+      const float* dts = dtsb + slot * T;
       // X'_j = diag(exp(lam_end - lam_t)) X_j, rows a and a + 64, into buffer j & 1
       // (free once the products of sub-chunk j - 2 have completed and its y tile,
       // staged in the same buffer, has been read by the TMA store)
@@ -448,7 +564,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int rr = 0; rr < 2; ++rr) {
           const int row = a + 64 * rr;
           float w = ex2(lam_end - lj[row]);
-          if constexpr (XDT) w *= dts[row];
+          if constexpr (CF) w *= dts[row];
           uint4 v4[8];
 #pragma unroll
           for (int c = 0; c < 8; ++c) v4[c] = src[swz128(row, c * 8) >> 4];
@@ -511,7 +627,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const float4 l = lj4[8 * kb + v];
             float e0 = ex2(fminf(lam_t - l.x, 0.f)), e1 = ex2(fminf(lam_t - l.y, 0.f));
             float e2 = ex2(fminf(lam_t - l.z, 0.f)), e3 = ex2(fminf(lam_t - l.w, 0.f));
-            if constexpr (XDT) {  // the columns' input factors
+            if constexpr (CF) {  // the columns' input factors
               const float4 fx = dt4[8 * kb + v];
               e0 *= fx.x; e1 *= fx.y; e2 *= fx.z; e3 *= fx.w;
             }
@@ -630,6 +746,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       // masking warps' shared-memory loads in the same memory pipe.
       const float et = ex2(lj[r]);
       const uint32_t ystage = sbase + OFF_XP + buf * TILE;
+      // the skip term sees the input as the scan does: r_t x_t when normalised
+      float Dt = Dh;
+      if constexpr (NORM) Dt *= rnb[(j & 3) * T + r];
+      float ss = 0.f;  // sum of squares of the stored (bf16) y row
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t yi[16], ye[16];
@@ -646,12 +766,21 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int i = 0; i < 4; ++i) {
             const int k0 = h2 * 8 + 2 * i;
             const float2 xf = bf2_to_f2(xu[i]);
-            float2 yo = fma2(make_float2(Dh, Dh), xf, make_float2(__uint_as_float(yi[k0]), __uint_as_float(yi[k0 + 1])));
+            float2 yo = fma2(make_float2(Dt, Dt), xf, make_float2(__uint_as_float(yi[k0]), __uint_as_float(yi[k0 + 1])));
             yo = fma2(make_float2(et, et), make_float2(__uint_as_float(ye[k0]), __uint_as_float(ye[k0 + 1])), yo);
             o[i] = pack_bf16(yo.x, yo.y);
+            if constexpr (NORM) {
+              const float2 q = bf2_to_f2(o[i]);
+              ss = fmaf(q.x, q.x, ss);
+              ss = fmaf(q.y, q.y, ss);
+            }
           }
           sts128(ystage + swz128(r, 8 * cc), ov);
         }
+      }
+      if (NORM && p.ss_out) {  // this head's share of the next layer's RMS norm
+        const int64_t tg = (int64_t)t_base + (int64_t)j * T + r;
+        if (tg < p.L) p.ss_out[(int64_t)b * p.sss + tg * p.H + h] = ss;
       }
       tc_fence_before();
       mbar_arrive(&bar[TEMPTY0 + buf]);
@@ -703,7 +832,8 @@ bool uses_pair_kernel(const Problem& p) { return p.two_heads && pair_supported(p
 size_t tc_workspace_bytes(const Problem& p) { return uses_pair_kernel(p) ? pair_workspace_bytes(p) : 0; }
 
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
-                               void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads = 0);
+                               void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads = 0,
+                               const NormIO* norm = nullptr);
 
 cudaError_t launch_fused_traced(const Problem& p, const float* init, float* final_state, unsigned long long* trace,
                                 cudaStream_t st) {
@@ -721,6 +851,15 @@ cudaError_t launch_fused(const Problem& p, const float* init, float* final_state
   return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, nullptr, st);
 }
 
+// One layer of a stack with the RMS norm between layers fused in (one head per
+// CTA): the input rows are normalised on the fly from the previous layer's
+// per-(token, head) sums of squares, and this layer's sums are written for
+// the next (either may be absent).
+cudaError_t launch_fused_normed(const Problem& p, const float* init, float* final_state, const NormIO& norm,
+                                cudaStream_t st) {
+  return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, nullptr, st, 0, &norm);
+}
+
 // Step 2 on tensor cores: one CTA per (batch, head, chunk), zero start, the
 // chunk's end state written to states[b,h,c].
 cudaError_t launch_chunk_state_tc(const Problem& p, const float* lam, float* states, cudaStream_t st) {
@@ -734,7 +873,8 @@ cudaError_t launch_chunk_scan_tc(const Problem& p, const float* lam, const float
 }
 
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
-                               void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads) {
+                               void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads,
+                               const NormIO* norm) {
   using namespace fused;
   // every pointer the mode reads must be present (the step entry points pass
   // only the tensors of their step)
@@ -783,6 +923,11 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   kp.sy = p.sy;
   kp.trace = trace;
   kp.withhold_loads = withhold_loads;
+  kp.ss_in = (norm && mode == MODE_SCAN) ? norm->ss_in : nullptr;
+  kp.ss_out = (norm && mode == MODE_SCAN) ? norm->ss_out : nullptr;
+  kp.sss = norm ? norm->batch_stride : 0;
+  kp.norm_eps = norm ? norm->eps : 0.f;
+  kp.inv_feat = 1.0f / (float)(p.H * P);
   // the shared-memory opt-in once per device (not stream work; keeps launches
   // free of other API calls, e.g. inside a CUDA graph capture)
   static std::atomic<unsigned long long> attr_set{0};
@@ -791,17 +936,24 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   if (e != cudaSuccess) return e;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set.load() & bit)) {
-    e = cudaFuncSetAttribute(k_ssd_fused<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(k_ssd_fused<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    const void* fns[4] = {(const void*)k_ssd_fused<false, false>, (const void*)k_ssd_fused<true, false>,
+                          (const void*)k_ssd_fused<false, true>, (const void*)k_ssd_fused<true, true>};
+    for (int i = 0; i < 4 && e == cudaSuccess; ++i)
+      e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set.fetch_or(bit);
   }
   const int64_t ctas = mode == fused::MODE_SCAN ? p.B * p.H : p.B * p.H * p.nc;
-  if (p.input_dt && mode == fused::MODE_SCAN)
-    k_ssd_fused<true><<<(unsigned)ctas, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+  const bool xdt = p.input_dt && mode == fused::MODE_SCAN, nrm = kp.ss_in != nullptr || kp.ss_out != nullptr;
+  const dim3 grid((unsigned)ctas);
+  if (xdt && nrm)
+    k_ssd_fused<true, true><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+  else if (xdt)
+    k_ssd_fused<true, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+  else if (nrm)
+    k_ssd_fused<false, true><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
   else
-    k_ssd_fused<false><<<(unsigned)ctas, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+    k_ssd_fused<false, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
   return cudaGetLastError();
 }
 

@@ -42,14 +42,12 @@
 // bf16 copy for y_inter(k+1), and write exp(lam_end(k+1)) s(k) back for the
 // b_intra(k+1) MMA to accumulate onto).
 //
-// Work split: the (batch, head pair) sequences are concatenated into one list
-// of sub-chunks and cut into equal ranges, one per CTA (persistent launch of
-// at most one CTA per SM).  A range holds at most a tail piece of one
-// sequence, whole sequences, and a head piece of the next.  A CTA runs its
-// head piece first and publishes that piece's end state (the page's §2.2
-// recursion: the carry is b(c-1) of the next chunk) to a workspace slot; the
-// next CTA needs it only for its tail piece, which it runs last.  Without a
-// workspace every CTA runs whole sequences.
+// Work split (csrc/ssd_split.cuh): with a workspace and at least as many
+// (batch, head pair) sequences as SMs, one persistent CTA per SM runs
+// (segment, sequence) items round-robin, numbered segment-major; a segment
+// after the first starts from the end state its predecessor published to the
+// sequence's workspace slot (the page's §2.2 recursion: the carry is b(c-1)
+// of the next chunk).  Without a workspace every CTA runs whole sequences.
 //
 // Every wait is bounded (about one second); a wait that gives up raises the
 // device status word, and every role then runs its loop to the end without
@@ -65,7 +63,7 @@ namespace ssd {
 namespace pair {
 
 using namespace umma;
-using split::Range;
+using split::Rounds;
 using split::ld_acquire;
 using split::st_release;
 
@@ -114,8 +112,8 @@ constexpr int W_TMA = 0, W_MMA = 1;
 struct Params {
   int64_t L;
   int H, G, nsub;   // nsub = ceil(L / T)
-  int64_t npairs;   // B * H / 2
-  int64_t total;    // npairs * nsub (sub-chunks of all sequences)
+  int64_t npairs;   // B * H / 2: the sequences of the schedule
+  int nseg;         // segments per sequence
   int nctas;
   const float* dt;
   int64_t sdt, lddt;
@@ -124,8 +122,8 @@ struct Params {
   const float* init;
   float* final_state;
   const __nv_bfloat16* x;  // only its layout is used here (TMA maps); kept for completeness
-  float* carry;            // [nctas][2][NS][P] end states of head pieces, or NULL (no split)
-  int* carry_flag;         // [nctas], zeroed before the launch
+  float* carry;            // [npairs][2][NS][P] end state of the last finished segment, or NULL
+  int* carry_flag;         // [npairs] segments whose end state is published, zeroed before the launch
   int withhold;            // self-test of the bounded waits: 1 = no TMA loads, 2 = no carries published
 };
 
@@ -221,8 +219,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hpp = p.H / 2;  // head pairs per batch
-  Range rg;
-  rg.init(p.total, p.nctas, blockIdx.x, p.nsub);
+  Rounds rg;
+  rg.init(p.npairs, p.nsub, p.nseg, p.nctas, blockIdx.x);
   const int64_t K = rg.count();
 
   if (warp == W_MMA) tmem_alloc(tmem_slot, TMEM_COLS);
@@ -257,9 +255,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   auto coords = [&](int64_t k, int& b, int& h0, int& g, int& t0) {
     int64_t u;
-    int j;
+    int j, r;
     bool f, l, ci, co;
-    rg.at(k, u, j, f, l, ci, co);
+    rg.at(k, u, j, r, f, l, ci, co);
     b = (int)(u / hpp);
     h0 = (int)(u % hpp) * 2;
     g = h0 / (p.H / p.G);
@@ -447,9 +445,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         return;
       }
       int64_t u;
-      int j;
+      int j, r;
       bool f, l, ci, co;
-      rg.at(k, u, j, f, l, ci, co);
+      rg.at(k, u, j, r, f, l, ci, co);
       const int b = (int)(u / hpp), h0 = (int)(u % hpp) * 2;
       const float* dtb = p.dt + (int64_t)b * p.sdt + h0;
       const int64_t t0 = (int64_t)j * T + 2 * a;
@@ -588,9 +586,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     int64_t u = -1;
     int b = 0, h = 0;
     for (int64_t k = 0; k < K; ++k) {
-      int j;
+      int j, seg;
       bool first, last, carry_in, carry_out;
-      rg.at(k, u, j, first, last, carry_in, carry_out);
+      rg.at(k, u, j, seg, first, last, carry_in, carry_out);
       if (first) {
         // a new piece: its initial state (given, carried or zero) is published
         // for y_inter(k) and written, times exp(lam_end(k)), for b_intra(k)
@@ -599,22 +597,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         Dh = p.D ? p.D[h] : 0.f;
         const float* src = nullptr;
         if (carry_in) {
-          // the previous CTA publishes this sequence's state at our first
-          // sub-chunk (its head piece, which it ran first); wait for it
-          const int* flag = p.carry_flag + (blockIdx.x - 1);
-          if (ld_acquire(flag) == 0) {
+          // segment seg - 1 of this sequence (an item at least one round
+          // earlier, normally finished) publishes its end state; wait for it
+          const int* flag = p.carry_flag + u;
+          if (ld_acquire(flag) < seg) {
             const uint64_t t0 = globaltimer_ns();
             bool done = false;
             while (!done && !*abort_flag) {
               __nanosleep(256);
-              done = ld_acquire(flag) != 0;
+              done = ld_acquire(flag) >= seg;
               if (!done && globaltimer_ns() - t0 > 2000000000ull) {
                 ctl.give_up();
                 break;
               }
             }
           }
-          src = p.carry + ((int64_t)(blockIdx.x - 1) * 2 + hl) * NS * P;
+          src = p.carry + (u * 2 + hl) * NS * P;
         } else if (p.init) {
           src = p.init + ((int64_t)b * p.H + h) * NS * P;
         }
@@ -742,10 +740,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_before();
         mbar_arrive(&bar[BIREADY]);
       } else {
-        // end of a piece: the sequence's final state, or the carry of a head piece
+        // end of a segment: the sequence's final state, or the carry of the next
+        // segment (the slot was read at this segment's start)
         float* dst = nullptr;
         if (carry_out)
-          dst = p.carry + ((int64_t)blockIdx.x * 2 + hl) * NS * P;
+          dst = p.carry + (u * 2 + hl) * NS * P;
         else if (p.final_state)
           dst = p.final_state + ((int64_t)b * p.H + h) * NS * P;
 #pragma unroll
@@ -765,7 +764,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (carry_out) {
           __threadfence();
           named_sync(2, EPIT);
-          if (et == 0 && p.withhold != 2) st_release(p.carry_flag + blockIdx.x, 1);
+          if (et == 0 && p.withhold != 2) st_release(p.carry_flag + u, seg + 1);
         }
       }
       // ---- y_t = y_intra + exp(lam_t) y_inter + D x_t, written over this head's
@@ -825,14 +824,27 @@ bool pair_supported(const Problem& p) {
          p.B * p.H < (1ll << 31);
 }
 
-// CTAs of the split schedule: one per SM, never more than the head pairs.
-int pair_split_ctas(const Problem& p) { return split::ctas(p.B * p.H / 2); }
+// Segments per sequence (csrc/ssd_split.cuh), or the count a self-test set.
+static int g_segments_override = 0;
+void set_pair_segments(int nseg) { g_segments_override = nseg > 0 ? nseg : 0; }
+static int pair_segments(const Problem& p) {
+  const int nsub = (int)ceil_div(p.L, (int64_t)pair::T);
+  if (g_segments_override > 0) return (nsub % g_segments_override == 0) ? g_segments_override : 1;
+  return split::segments(p.B * p.H / 2, nsub, split::sm_count());
+}
 
-// Workspace of the split schedule: the carries [ctas][2][N][P] f32 and their
-// flags, or 0 when every CTA runs whole sequences anyway.
+// CTAs of the segmented schedule: one per SM, never more than the items.
+int pair_split_ctas(const Problem& p) {
+  const int64_t items = p.B * p.H / 2 * pair_segments(p);
+  const int n = split::sm_count();
+  return (int)(items < n ? items : n);
+}
+
+// Workspace of the segmented schedule: one carry slot [2][N][P] f32 per head
+// pair and their flags, or 0 when the sequences run whole.
 size_t pair_workspace_bytes(const Problem& p) {
   if (!pair_supported(p)) return 0;
-  return split::workspace_bytes(p.B * p.H / 2, (size_t)2 * pair::NS * pair::P);
+  return split::workspace_bytes(p.B * p.H / 2, pair_segments(p), (size_t)2 * pair::NS * pair::P);
 }
 
 // withhold: 0 normal; 1 issue no TMA loads (self-test of the bounded waits);
@@ -857,7 +869,6 @@ cudaError_t launch_pair(const Problem& p, const float* init, float* final_state,
   kp.G = (int)p.G;
   kp.nsub = (int)ceil_div(p.L, T);
   kp.npairs = p.B * p.H / 2;
-  kp.total = kp.npairs * kp.nsub;
   kp.dt = p.dt;
   kp.sdt = p.sdt;
   kp.lddt = p.lddt;
@@ -869,14 +880,16 @@ cudaError_t launch_pair(const Problem& p, const float* init, float* final_state,
   kp.withhold = withhold;
   const size_t need = pair_workspace_bytes(p);
   if (need > 0 && workspace && workspace_bytes >= need) {
+    kp.nseg = pair_segments(p);
     kp.nctas = pair_split_ctas(p);
     kp.carry = static_cast<float*>(workspace);
     kp.carry_flag = reinterpret_cast<int*>(static_cast<char*>(workspace) +
-                                           (size_t)kp.nctas * 2 * NS * P * sizeof(float));
-    cudaError_t e = cudaMemsetAsync(kp.carry_flag, 0, (size_t)kp.nctas * sizeof(int), st);
+                                           (size_t)kp.npairs * 2 * NS * P * sizeof(float));
+    cudaError_t e = cudaMemsetAsync(kp.carry_flag, 0, (size_t)kp.npairs * sizeof(int), st);
     if (e != cudaSuccess) return e;
   } else {
-    kp.nctas = (int)kp.npairs;  // whole sequences
+    kp.nseg = 1;                // whole sequences, one CTA each
+    kp.nctas = (int)kp.npairs;
     kp.carry = nullptr;
     kp.carry_flag = nullptr;
   }

@@ -210,9 +210,9 @@ extern "C" ssd_status ssd_selftest_timeout(const ssd_dims* d, const void* x, con
   return cuda_status(launch_fused_withheld(p, init_state, final_state, static_cast<cudaStream_t>(stream)));
 }
 
-// Carry path of the two-head kernel: the split schedule of ssd_scan_fwd with no
-// carry ever published, so every CTA that starts inside a sequence waits for
-// its predecessor's state until its bounded wait runs out (about two seconds),
+// Carry path of the two-head kernel: the segmented schedule of ssd_scan_fwd with
+// no carry ever published, so every segment after the first waits for its
+// predecessor's state until its bounded wait runs out (about two seconds),
 // records SSD_ERR_TIMEOUT and drains; nothing faults.
 extern "C" ssd_status ssd_selftest_carry_timeout(const ssd_dims* d, const void* x, const float* dt, const float* A,
                                                  const void* Bm, const void* Cm, const float* D,
@@ -230,4 +230,12 @@ extern "C" ssd_status ssd_selftest_carry_timeout(const ssd_dims* d, const void* 
   p.x = x; p.dt = dt; p.A = A; p.Bm = Bm; p.Cm = Cm; p.D = D; p.y = y;
   return cuda_status(
       launch_pair(p, init_state, final_state, workspace, workspace_bytes, static_cast<cudaStream_t>(stream), 2));
+}
+
+// Segments per sequence of the two-head kernel's schedule for the following
+// launches of this process (0 restores the choice from the shape).
+extern "C" ssd_status ssd_selftest_set_segments(int nseg) {
+  if (nseg < 0) return SSD_ERR_INVALID_ARG;
+  ssd::set_pair_segments(nseg);
+  return SSD_OK;
 }

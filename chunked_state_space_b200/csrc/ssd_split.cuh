@@ -1,13 +1,18 @@
-// Split schedule shared by the fused scan kernels: the sequences (units) of a
-// launch are concatenated into one list of 128-token sub-chunks and cut into
-// equal ranges, one per persistent CTA.  When there are at least as many
-// units as CTAs, a range is at least one unit long, so it holds at most a
-// tail piece of one unit, whole units, and a head piece of the next.  The CTA
-// runs its head piece first and publishes that piece's end state (the carry:
-// the page's inter-chunk recursion handed across CTAs, "分块推理…" §2.2) to a
-// workspace slot with a release flag; the next CTA needs it only for its tail
-// piece, which it runs last.  With one unit per CTA this is the plain
-// one-sequence-per-CTA launch.
+// Segment-round schedule of the persistent fused scan kernels.  Every
+// sequence (unit) of the launch is cut into nseg equal segments of
+// seg = nsub / nseg 128-token sub-chunks; the (segment r, sequence q) work
+// items are numbered segment-major, v = r * nseq + q, and persistent CTA c
+// runs the items c, c + G, c + 2G, ... in that order (G CTAs, one per SM).
+// A segment after the first starts from the end state of the segment before
+// it: the page's inter-chunk recursion ("分块推理…" §2.2: b(c) from b(c-1))
+// handed across CTAs through a workspace slot per sequence and a flag that
+// counts the segments of the sequence whose end state has been published.
+// With nseq >= G the item a segment waits for (v - nseq) lies at least one
+// round earlier, so in the steady state the carry is there when it is needed.
+// Numbering the items segment-major keeps the CTAs of one round on the same
+// segment of neighbouring sequences: the heads of one batch then walk the
+// same tokens together and read each B/C tile from DRAM once, the rest from
+// L2.  With nseg = 1 the schedule runs whole sequences, round-robin.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -16,59 +21,35 @@
 namespace ssd {
 namespace split {
 
-// The sub-chunks of CTA c: [lo, hi) of the concatenated list, run in the order
-// head piece of the last sequence (if the range ends inside it), whole
-// sequences, tail piece of the first sequence (if the range starts inside it).
-struct Range {
-  int64_t lo, hi;
-  int nsub;
-  int64_t u_lo, u_hi;  // first and last sequence touched
-  int j_lo, j_hi;      // start of the first piece, end (exclusive) of the last piece
-  int head_len;        // sub-chunks of the leading head piece (0 if none)
-  int tail_len;        // sub-chunks of the trailing tail piece (0 if none)
-  int64_t full_first;  // first whole sequence
-  __device__ void init(int64_t total, int nctas, int c, int ns) {
-    nsub = ns;
-    lo = total * c / nctas;
-    hi = total * (c + 1) / nctas;
-    u_lo = lo / ns;
-    j_lo = (int)(lo % ns);
-    u_hi = (hi - 1) / ns;
-    j_hi = (int)((hi - 1) % ns) + 1;
-    head_len = (u_hi > u_lo && j_hi < ns) ? j_hi : 0;
-    tail_len = j_lo > 0 ? ns - j_lo : 0;
-    full_first = j_lo > 0 ? u_lo + 1 : u_lo;
+struct Rounds {
+  int64_t nseq;   // sequences of the launch
+  int nseg, seg;  // segments per sequence, sub-chunks per segment
+  int G, c;       // CTAs of the launch, this CTA
+  int64_t items;  // work items of this CTA
+  __device__ void init(int64_t nseq_, int nsub, int nseg_, int G_, int c_) {
+    nseq = nseq_;
+    nseg = nseg_;
+    seg = nsub / nseg_;
+    G = G_;
+    c = c_;
+    const int64_t all = nseq * nseg;
+    items = all > c ? (all - c + G - 1) / G : 0;
   }
-  __device__ int64_t count() const { return hi - lo; }
-  // sequence, sub-chunk, and piece boundaries of the k-th sub-chunk this CTA runs
-  __device__ void at(int64_t k, int64_t& u, int& j, bool& first, bool& last, bool& carry_in,
+  __device__ int64_t count() const { return items * seg; }
+  // sequence u, sub-chunk j, segment r, and segment boundaries of the k-th
+  // sub-chunk this CTA runs
+  __device__ void at(int64_t k, int64_t& u, int& j, int& r, bool& first, bool& last, bool& carry_in,
                      bool& carry_out) const {
-    if (k < head_len) {
-      u = u_hi;
-      j = (int)k;
-      first = (k == 0);
-      last = (k == head_len - 1);
-      carry_in = false;
-      carry_out = last;
-      return;
-    }
-    const int64_t kk = k - head_len;
-    const int64_t nfull_sub = count() - head_len - tail_len;
-    if (kk < nfull_sub) {
-      u = full_first + kk / nsub;
-      j = (int)(kk % nsub);
-      first = (j == 0);
-      last = (j == nsub - 1);
-      carry_in = carry_out = false;
-      return;
-    }
-    const int64_t kt = kk - nfull_sub;
-    u = u_lo;
-    j = j_lo + (int)kt;
-    first = (kt == 0);
-    last = (j == nsub - 1);
-    carry_in = first;
-    carry_out = false;
+    const int64_t i = k / seg;
+    const int o = (int)(k - i * seg);
+    const int64_t v = c + i * G;
+    r = (int)(v / nseq);
+    u = v - (int64_t)r * nseq;
+    j = r * seg + o;
+    first = (o == 0);
+    last = (o == seg - 1);
+    carry_in = first && r > 0;
+    carry_out = last && r < nseg - 1;
   }
 };
 
@@ -94,20 +75,32 @@ inline int sm_count() {
   return cached[dev];
 }
 
-// CTAs of a split launch over `units` sequences: one per SM, never more than
-// the units (so no range lies strictly inside one unit).
-inline int ctas(int64_t units) {
-  const int64_t n = sm_count();
-  return (int)(units < n ? units : n);
+// Segments per sequence for `nseq` sequences of `nsub` sub-chunks on G CTAs:
+// the divisor of nsub that minimises rounds x (segment length + the carry's
+// cost, about one and a half sub-chunks of traffic), among those that keep
+// every carry at least one round back (nseq >= G); 1 otherwise.
+inline int segments(int64_t nseq, int nsub, int G) {
+  if (nseq < G || nsub <= 1) return 1;
+  int best = 1;
+  double best_cost = 0;
+  for (int n = 1; n <= nsub; ++n) {
+    if (nsub % n) continue;
+    const int64_t rounds = (nseq * n + G - 1) / G;
+    const double cost = (double)rounds * ((double)(nsub / n) + (n > 1 ? 1.5 : 0.0));
+    if (n == 1 || cost < best_cost) {
+      best = n;
+      best_cost = cost;
+    }
+  }
+  return best;
 }
 
-// Workspace of a split launch: `slot_floats` per CTA for the carry, then one
-// int flag per CTA (zeroed before every launch); 0 when every CTA runs whole
-// units anyway.
-inline size_t workspace_bytes(int64_t units, size_t slot_floats) {
-  const int n = ctas(units);
-  if (n >= units) return 0;
-  return (size_t)n * slot_floats * sizeof(float) + (size_t)((n * sizeof(int) + 255) / 256 * 256);
+// Workspace of a segmented launch: one carry slot of `slot_floats` per
+// sequence, then one int flag per sequence (zeroed before every launch); 0
+// when the sequences run whole.
+inline size_t workspace_bytes(int64_t nseq, int nseg, size_t slot_floats) {
+  if (nseg <= 1) return 0;
+  return (size_t)nseq * slot_floats * sizeof(float) + (size_t)((nseq * sizeof(int) + 255) / 256 * 256);
 }
 
 }  // namespace split

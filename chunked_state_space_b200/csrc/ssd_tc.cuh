@@ -24,11 +24,30 @@ size_t pair_workspace_bytes(const Problem& p);
 
 cudaError_t launch_chunk_state_tc(const Problem& p, const float* lam, float* states, cudaStream_t st);
 cudaError_t launch_chunk_scan_tc(const Problem& p, const float* lam, const float* prev, cudaStream_t st);
+// Segments per sequence of the two-head kernel's schedule: 0 = chosen from
+// the shape (the default), n > 0 = n wherever n divides the sub-chunks
+// (self-tests of the carries).
+void set_pair_segments(int nseg);
 // The whole scan in one launch.  With a workspace of pair_workspace_bytes
-// the two-head kernel splits sequences evenly across the SMs; without one
-// (NULL / too small) every CTA runs whole sequences.
+// the two-head kernel runs segments of the sequences round-robin on one
+// persistent CTA per SM; without one (NULL / too small) every CTA runs whole
+// sequences.
 cudaError_t launch_fused(const Problem& p, const float* init, float* final_state, void* workspace,
                          size_t workspace_bytes, cudaStream_t st);
+// The RMS norm between the layers of a stack, fused into the one-head kernel:
+// ss_in holds, per (batch, token, head), the sum of squares of the input row
+// (the previous layer's stored y), from which each token's scale
+// r_t = 1 / sqrt(sum_h ss_in / (H P) + eps) is applied on the fly; ss_out
+// receives the same sums for this call's stored y.  Both [B][L][H] f32 with
+// token stride H and batch stride batch_stride; either may be NULL.
+struct NormIO {
+  const float* ss_in;
+  float* ss_out;
+  int64_t batch_stride;
+  float eps;
+};
+cudaError_t launch_fused_normed(const Problem& p, const float* init, float* final_state, const NormIO& norm,
+                                cudaStream_t st);
 // withhold: 0 normal; 1 no TMA loads; 2 no carries published (self-tests of the bounded waits)
 cudaError_t launch_pair(const Problem& p, const float* init, float* final_state, void* workspace,
                         size_t workspace_bytes, cudaStream_t st, int withhold);

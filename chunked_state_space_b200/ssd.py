@@ -28,7 +28,8 @@ EXPORTED = ["ssd_status_string", "ssd_version", "ssd_scan_workspace_size", "ssd_
             "ssd_read_device_status", "ssd_selftest_umma", "ssd_scan_path", "ssd_step",
             "ssd_selftest_fused_trace", "ssd_scan_fwd_noalloc",
             "ssd_selftest_timeout", "ssd_scan_fwd_host", "ssd_scan_fwd_host_workspace_size",
-            "ssd_scan_fwd_strided", "ssd_selftest_carry_timeout", "ssd_scan_fwd_vdecay"]
+            "ssd_scan_fwd_strided", "ssd_selftest_carry_timeout", "ssd_scan_fwd_vdecay",
+            "ssd_selftest_set_segments", "ssd_scan_fwd_normed"]
 
 
 class SSDError(RuntimeError):
@@ -86,6 +87,8 @@ def lib() -> ctypes.CDLL:
         "ssd_selftest_fused_trace": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_int64, _P]),
         "ssd_selftest_timeout": (ctypes.c_int, [D] + [_P] * 10),
         "ssd_selftest_carry_timeout": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_size_t, _P]),
+        "ssd_selftest_set_segments": (ctypes.c_int, [ctypes.c_int]),
+        "ssd_scan_fwd_normed": (ctypes.c_int, [D, _P, _P, ctypes.c_float] + [_P] * 10),
         "ssd_scan_fwd_vdecay": (ctypes.c_int, [D] + [_P] * 10),
     }
     for name, (res, args) in sig.items():
@@ -188,6 +191,28 @@ def ssd_scan_fwd(x, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, y=
            _ptr(final_state), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check(s, "ssd_scan_fwd_unfused" if unfused else "ssd_scan_fwd")
     return y, final_state
+
+
+def ssd_scan_fwd_normed(x, ss_in, dt, A, Bm, Cm, D=None, init_state=None, chunk: int = 256, rms_eps: float = 1e-6,
+                        y=None, ss_out=None, want_sums: bool = True, final_state=None, want_final: bool = True,
+                        stream=None, input_dt: bool = False):
+    """One layer of a stack with the RMS norm between layers fused: x is the
+    previous layer's stored y and ss_in [B,L,H] f32 its per-(token, head) sums
+    of squares (None: x used as is).  Returns (y, ss_out [B,L,H] f32 of this
+    layer's stored y or None, final_state)."""
+    _contig(x, ss_in, dt, A, Bm, Cm, D, init_state, y, ss_out, final_state)
+    dims = make_dims(x, Bm, chunk, input_dt)
+    if y is None:
+        y = torch.empty_like(x)
+    if ss_out is None and want_sums:
+        ss_out = torch.empty(x.shape[:3], dtype=torch.float32, device=x.device)
+    if final_state is None and want_final:
+        final_state = torch.empty((dims.batch, dims.nheads, dims.dstate, dims.headdim), dtype=torch.float32,
+                                  device=x.device)
+    _check(lib().ssd_scan_fwd_normed(ctypes.byref(dims), _ptr(x), _ptr(ss_in), float(rms_eps), _ptr(dt), _ptr(A),
+                                     _ptr(Bm), _ptr(Cm), _ptr(D), _ptr(init_state), _ptr(y), _ptr(ss_out),
+                                     _ptr(final_state), _stream(stream)), "ssd_scan_fwd_normed")
+    return y, ss_out, final_state
 
 
 def ssd_scan_fwd_vdecay(x, dt, Av, Bm, Cm, D=None, init_state=None, y=None, final_state=None, stream=None,
@@ -430,3 +455,9 @@ def ssd_selftest_carry_timeout(x, dt, A, Bm, Cm, D=None, init_state=None, chunk:
                                             _ptr(D), _ptr(init_state), _ptr(y), _ptr(fin), _ptr(ws),
                                             ws.numel() * ws.element_size(), _stream(stream)),
            "ssd_selftest_carry_timeout")
+
+
+def ssd_selftest_set_segments(nseg: int) -> None:
+    """Segments per sequence of the two-head kernel's schedule for the
+    following launches (0 = chosen from the shape)."""
+    _check(lib().ssd_selftest_set_segments(int(nseg)), "ssd_selftest_set_segments")

@@ -280,10 +280,32 @@ ssd_status ssd_rmsnorm(int64_t rows, int64_t features, int32_t io_dtype, const v
                        void* out, void* stream);
 
 /*
+ * One layer of a stack with the layer-to-layer RMS norm fused into the scan
+ * (the normalisation of ssd_rmsnorm, but the normalised input is never
+ * stored): the scan of x'_t = r_t x_t with
+ *   r_t = 1 / sqrt(sum_h ss_in[b,t,h] / (H P) + rms_eps),
+ * where x is the previous layer's stored y and ss_in[b,t,h] = sum_p x[b,t,h,p]^2
+ * (as the previous call wrote to its ss_out).  The skip term is D_h x'_t.
+ *   x, dt, A, Bm, Cm, D, init_state, y, final_state: as ssd_scan_fwd;
+ *   ss_in [B,L,H] f32 or NULL (x is used as is: the stack's first layer);
+ *   ss_out [B,L,H] f32 or NULL: ss_out[b,t,h] = sum_p y[b,t,h,p]^2 over the
+ *   stored (io dtype) values of this call's y, for the next layer.
+ * Takes the one-head tensor-core kernel only (bf16, P = 64, N = 128, Q a
+ * multiple of 128; flags 0 or SSD_FLAG_INPUT_DT), else SSD_ERR_UNSUPPORTED.
+ * ss_in, ss_out 16-byte aligned, not overlapping x, y or each other; no
+ * workspace.  Layers chained through it give the results of ssd_vertical_fwd
+ * with vblock >= L bitwise.
+ */
+ssd_status ssd_scan_fwd_normed(const ssd_dims* d, const void* x, const float* ss_in, float rms_eps,
+                               const float* dt, const float* A, const void* Bm, const void* Cm,
+                               const float* D, const float* init_state, void* y, float* ss_out,
+                               float* final_state, void* stream);
+
+/*
  * Bytes of workspace ssd_vertical_fwd needs for `d`, `n_layers` and the
  * vertical block length `vblock` (V): the single-block scan scratch plus two
  * V-token activation blocks per layer boundary ([B,V,H,P] io each; at least
- * two).
+ * two) and their per-(token, head) sums of squares ([B,V,H] f32 each).
  */
 ssd_status ssd_vertical_workspace_size(const ssd_dims* d, int32_t n_layers, int64_t vblock,
                                        size_t* bytes);
@@ -298,9 +320,15 @@ ssd_status ssd_vertical_workspace_size(const ssd_dims* d, int32_t n_layers, int6
  *   states: HOST array of n_layers DEVICE pointers [B,H,N,P] f32: the initial
  *   state of each layer on entry, its final state on return (in place).
  *   y_out: the last layer's output [B,L,H,P] io.
- * Layer l+1's input is ssd_rmsnorm(y_l) (eps = rms_eps), stored in io dtype.
+ * Layer l+1's input is y_l RMS-normalised over its H*P features (eps =
+ * rms_eps).  With the one-head fused kernel the norm is fused: layer l writes
+ * y_l and its per-(token, head) sums of squares, layer l+1 scales its input
+ * rows on the fly (ssd_scan_fwd_normed), and no normalised copy is stored;
+ * otherwise (SSD_FLAG_TWO_HEADS_PER_CTA, other shapes) layer l+1's input is
+ * ssd_rmsnorm(y_l), stored in io dtype.
  * When V is a multiple of Q the result is bitwise equal to running the layers
- * one after another over the whole sequence (the §3.1 horizontal schedule).
+ * one after another over the whole sequence (the §3.1 horizontal schedule):
+ * ssd_scan_fwd_normed per layer, or ssd_scan_fwd and ssd_rmsnorm.
  * Execution: with more than one layer and a problem the fused tensor-core
  * kernel takes, the (block, layer) launches run as a wavefront: layer l on a
  * stream of its own, block k of layer l after block k of layer l-1, so

@@ -79,13 +79,14 @@ ssd_status ssd_selftest_timeout(const ssd_dims* d, const void* x, const float* d
 
 /*
  * ssd_selftest_carry_timeout exercises the one wait of the two-head fused
- * kernel that is not on a barrier of its own CTA: in its split schedule a CTA
- * whose range starts inside a sequence waits for the previous CTA to publish
- * that sequence's state (the page's inter-chunk recursion, "分块推理…" §2.2,
- * handed across CTAs).  Same arguments and validation as ssd_scan_fwd plus
- * the workspace; d->flags must request the two-head kernel
- * (SSD_FLAG_TWO_HEADS_PER_CTA) and the problem be one it splits (even heads per
- * group, more head pairs than SMs), else SSD_ERR_UNSUPPORTED.  No
+ * kernel that is not on a barrier of its own CTA: in its segmented schedule a
+ * segment after the first waits for the CTA that ran the segment before it to
+ * publish that sequence's state (the page's inter-chunk recursion, "分块推理…"
+ * §2.2, handed across CTAs).  Same arguments and validation as ssd_scan_fwd
+ * plus the workspace; d->flags must request the two-head kernel
+ * (SSD_FLAG_TWO_HEADS_PER_CTA) and the problem be one it segments (even heads
+ * per group, and more than one segment per sequence, chosen from the shape or
+ * set by ssd_selftest_set_segments), else SSD_ERR_UNSUPPORTED.  No
  * carry is ever published, so those waits give up after about two seconds;
  * the launch returns SSD_OK and the following ssd_read_device_status(stream)
  * returns SSD_ERR_TIMEOUT.  y and final_state are left undefined; nothing
@@ -95,6 +96,17 @@ ssd_status ssd_selftest_carry_timeout(const ssd_dims* d, const void* x, const fl
                                       const void* Bm, const void* Cm, const float* D, const float* init_state,
                                       void* y, float* final_state, void* workspace, size_t workspace_bytes,
                                       void* stream);
+
+/*
+ * ssd_selftest_set_segments sets how many segments the two-head kernel cuts
+ * each sequence into for the following launches of this process (host state,
+ * not thread-safe): nseg > 0 wherever nseg divides the sequence's 128-token
+ * sub-chunks (else whole sequences), 0 = chosen from the shape (the default).
+ * With fewer head pairs than SMs a forced segmentation puts a segment and its
+ * predecessor in the same round, so the later one waits for the earlier one:
+ * correct, slower.  Returns SSD_ERR_INVALID_ARG for nseg < 0.
+ */
+ssd_status ssd_selftest_set_segments(int nseg);
 
 #ifdef __cplusplus
 }

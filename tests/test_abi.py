@@ -148,8 +148,22 @@ def test_vertical_rejects(lib):
         assert lib.ssd_vertical_workspace_size(ctypes.byref(d), layers, 512, ctypes.byref(m)) == 0
         sizes[layers] = m.value
     assert sizes[1] == sizes[2] and sizes[2] >= one.value + 2 * act
-    assert sizes[24] - sizes[3] == 2 * (24 - 3) * act
+    sums = 2 * 512 * 4 * 4  # B * V * H f32: the blocks' per-(token, head) sums of squares (fused norm)
+    assert sizes[24] - sizes[3] == 2 * (24 - 3) * (act + sums)
     assert lib.ssd_vertical_fwd(ctypes.byref(d), 2, 512, 1e-6, None, *([None] * 6), None, None, 0, None) == 1
+
+
+def test_normed_entry_rejects(lib):
+    """ssd_scan_fwd_normed takes the one-head tensor-core kernel only and checks
+    its arguments before anything touches the device (no GPU needed)."""
+    f = lib.ssd_scan_fwd_normed
+    eps = ctypes.c_float(1e-6)
+    d = dims()
+    assert f(ctypes.byref(d), *([None] * 2), eps, *([None] * 10)) == 1          # NULL x, dt, ...
+    assert f(ctypes.byref(dims(flags=2)), *([None] * 2), eps, *([None] * 10)) == 5  # two heads per CTA
+    assert f(ctypes.byref(dims(flags=4)), *([None] * 2), eps, *([None] * 10)) == 1  # unknown flag bit
+    assert f(None, *([None] * 2), eps, *([None] * 10)) == 1
+    assert f(ctypes.byref(dims(seqlen=0)), *([None] * 2), eps, *([None] * 10)) == 2
 
 
 def test_host_io_entry_rejects(lib):

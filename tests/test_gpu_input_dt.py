@@ -49,17 +49,25 @@ def test_vertical_input_dt_equals_horizontal():
     zeros = lambda: [torch.zeros((wl.batch, wl.nheads, wl.dstate, wl.headdim), device="cuda") for _ in range(n_layers)]
     st_v = zeros()
     yv = ssd.ssd_vertical_fwd(x0, layers, st_v, vblock=V, chunk=wl.chunk, rms_eps=eps, input_dt=True)
+    # horizontal: layer by layer, the norm fused (dt-scaled and normalised input together)
     st_h = zeros()
-    x = x0
+    x, ss, ys = x0, None, []
     for l, p in enumerate(layers):
-        y, _ = ssd.ssd_scan_fwd(x, p["dt"], p["A"], p["B"], p["C"], p["D"], st_h[l], chunk=wl.chunk,
-                                final_state=st_h[l], input_dt=True)
-        if l + 1 < n_layers:
-            x = ssd.ssd_rmsnorm(y, eps)
+        y, ss, _ = ssd.ssd_scan_fwd_normed(x, ss, p["dt"], p["A"], p["B"], p["C"], p["D"], st_h[l], chunk=wl.chunk,
+                                           rms_eps=eps, final_state=st_h[l], input_dt=True)
+        ys.append(y)
+        x = y
     torch.cuda.synchronize()
-    assert torch.equal(yv, y)
+    assert torch.equal(yv, ys[-1])
     for a, b in zip(st_v, st_h):
         assert torch.equal(a, b)
+    # the last layer teacher-forced: the oracle's dt-scaled scan of the previous
+    # GPU layer's y, RMS-normalised by the oracle
+    host_last = inputs.generate(wl, layer=n_layers - 1, names=("dt", "A", "B", "C", "D"))
+    f = inputs.to_f64
+    y_ref, _ = oracle.scan_recurrence(oracle.rmsnorm(to_np64(ys[-2]), eps), f(host_last["dt"]), f(host_last["A"]),
+                                      f(host_last["B"]), f(host_last["C"]), f(host_last["D"]), None, input_dt=True)
+    assert rel_err(to_np64(ys[-1]), y_ref) <= TOL["bf16"]
 
 
 @pytest.mark.parametrize("name,over", [

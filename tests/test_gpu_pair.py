@@ -1,16 +1,19 @@
 """The two-heads-per-CTA fused kernel (SSD_FLAG_TWO_HEADS_PER_CTA, path
-SSD_PATH_FUSED_PAIR) and its split schedule against the fp64 oracle.
+SSD_PATH_FUSED_PAIR) and its segmented schedule against the fp64 oracle.
 
 Two heads of one group share a CTA, their B/C tiles and S = C B^T.  With the
-caller's workspace and more head pairs than SMs the kernel cuts the
-concatenated sequences into equal ranges, one persistent CTA per SM, and a
-CTA that starts inside a sequence takes its initial state from the CTA before
-it (the inter-chunk recursion of "分块推理…" §2.2 handed across CTAs).  The
-cases cover one pair, ragged and one-token sequences, several pairs per group,
-the dt-scaled input, and the split schedule with many range boundaries; each
-is compared with the oracle at the bf16 tolerance, and the split schedule
-bitwise with the whole-sequence schedule (same arithmetic, the carry passes
-through memory in fp32)."""
+caller's workspace the kernel can cut every sequence into segments and run the
+(segment, sequence) items round-robin on one persistent CTA per SM; a segment
+after the first takes its initial state from the CTA that ran the segment
+before it (the inter-chunk recursion of "分块推理…" §2.2 handed across CTAs).
+The cases cover one pair, ragged and one-token sequences, several pairs per
+group, the dt-scaled input, and the segmented schedule with the shape's own
+segment count and with forced counts (down to one sub-chunk per segment, and
+segments whose predecessor runs in the same round); each is compared with the
+oracle at the bf16 tolerance, and the segmented schedule bitwise with whole
+sequences (same arithmetic, the carry passes through memory in fp32)."""
+import contextlib
+
 import pytest
 import torch
 
@@ -52,43 +55,57 @@ def test_pair_kernel_matches_oracle(over, input_dt):
     assert rel_err(to_np64(f1), f_ref) <= TOL["bf16"]
 
 
-@pytest.mark.parametrize("over", [
-    dict(batch=2, seqlen=300, nheads=160, ngroups=1, init_var=0.1),   # 160 pairs of 3 sub-chunks: ~1 per CTA
-    dict(batch=1, seqlen=1000, nheads=300, ngroups=2),                # 150 pairs of 8 sub-chunks
-    dict(batch=3, seqlen=640, nheads=100, ngroups=5, init_var=0.1),   # 150 pairs, 20 heads per group
+@contextlib.contextmanager
+def segments(n):
+    ssd.ssd_selftest_set_segments(n)
+    try:
+        yield
+    finally:
+        ssd.ssd_selftest_set_segments(0)
+
+
+@pytest.mark.parametrize("over,nseg", [
+    (dict(batch=2, seqlen=300, nheads=160, ngroups=1, init_var=0.1), 3),   # 160 pairs, one sub-chunk per segment
+    (dict(batch=1, seqlen=1000, nheads=300, ngroups=2), 0),                 # 150 pairs, the shape's own choice
+    (dict(batch=1, seqlen=1000, nheads=300, ngroups=2), 8),                 # ragged last segment of one sub-chunk
+    (dict(batch=3, seqlen=640, nheads=100, ngroups=5, init_var=0.1), 5),    # 150 pairs, 20 heads per group
+    (dict(batch=1, seqlen=2048, nheads=8, ngroups=1, init_var=0.1), 16),    # 4 pairs: predecessors in the same round
+    (dict(batch=8, seqlen=4096, nheads=80, ngroups=1), 0),                  # 320 pairs of 32 sub-chunks
 ])
-@pytest.mark.parametrize("two_heads", [True])
-def test_split_schedule_matches_oracle_and_whole_sequences(over, two_heads):
+def test_segmented_schedule_matches_oracle_and_whole_sequences(over, nseg):
     wl = inputs.custom("mamba2_130m_layer", **over)
     host = inputs.generate(wl)
     dev = device_inputs(host)
-    dims = ssd.make_dims(dev["x"], dev["B"], wl.chunk, two_heads=two_heads)
-    assert ssd.ssd_scan_path(dims)[0] == ("fused_pair" if two_heads else "fused")
-    y, fin = _scan(dev, wl, two_heads=two_heads)
-    y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host))
-    ey, ef = rel_err(to_np64(y), y_ref), rel_err(to_np64(fin), f_ref)
-    assert ey <= TOL["bf16"], ey
-    assert ef <= TOL["bf16"], ef
+    dims = ssd.make_dims(dev["x"], dev["B"], wl.chunk, two_heads=True)
+    assert ssd.ssd_scan_path(dims)[0] == "fused_pair"
+    with segments(nseg):
+        assert ssd.ssd_scan_workspace_size(dims) > 0  # the schedule is segmented
+        y, fin = _scan(dev, wl, two_heads=True)
+    if wl.batch * wl.nheads * wl.seqlen <= 2 ** 21:
+        y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host))
+        ey, ef = rel_err(to_np64(y), y_ref), rel_err(to_np64(fin), f_ref)
+        assert ey <= TOL["bf16"], ey
+        assert ef <= TOL["bf16"], ef
     # The carries themselves: the strided entry point has no workspace, so
-    # there every CTA runs whole sequences.  The split must give the same
+    # there every CTA runs whole sequences.  The segments must give the same
     # bits (a wrong or late carry changes whole sequences by O(1)).
     ys, fs = ssd.ssd_scan_fwd_strided(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
-                                      chunk=wl.chunk, two_heads=two_heads)
+                                      chunk=wl.chunk, two_heads=True)
     torch.cuda.synchronize()
     assert torch.equal(ys, y)
     assert torch.equal(fs, fin)
 
 
-@pytest.mark.parametrize("two_heads", [True])
-def test_split_schedule_repeatable_and_workspace_reused(two_heads):
+def test_segmented_schedule_repeatable_and_workspace_reused():
     """Back-to-back calls on one workspace (the carry flags are reset by each
     call) give identical results."""
     wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=300, nheads=160, ngroups=1, init_var=0.1)
     dev = device_inputs(inputs.generate(wl))
-    dims = ssd.make_dims(dev["x"], dev["B"], wl.chunk, two_heads=two_heads)
-    ws = torch.empty(ssd.ssd_scan_workspace_size(dims), dtype=torch.uint8, device="cuda")
-    ws.fill_(0xFF)  # contents need not be initialised
-    outs = [_scan(dev, wl, workspace=ws, two_heads=two_heads) for _ in range(3)]
+    dims = ssd.make_dims(dev["x"], dev["B"], wl.chunk, two_heads=True)
+    with segments(3):
+        ws = torch.empty(ssd.ssd_scan_workspace_size(dims), dtype=torch.uint8, device="cuda")
+        ws.fill_(0xFF)  # contents need not be initialised
+        outs = [_scan(dev, wl, workspace=ws, two_heads=True) for _ in range(3)]
     for y, f in outs[1:]:
         assert torch.equal(y, outs[0][0]) and torch.equal(f, outs[0][1])
 

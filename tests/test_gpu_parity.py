@@ -257,23 +257,41 @@ def _stack_layers(wl, n_layers):
     return layers_host, [device_inputs(h) for h in layers_host]
 
 
-def _horizontal_gpu(x0, layers, states, wl, eps):
+def _horizontal_normed(x0, layers, states, wl, eps):
+    """The layer-major schedule through the public one-layer call with the norm
+    fused (ssd_scan_fwd_normed): every layer's y and the sums of squares it
+    passes on.  Returns (ys, sums) with sums[l] the input sums of layer l."""
+    ys, sums = [], [None]
     x = x0
-    y = None
     for l, p in enumerate(layers):
-        y, _ = ssd.ssd_scan_fwd(x, p["dt"], p["A"], p["B"], p["C"], p["D"], states[l], chunk=wl.chunk,
-                                final_state=states[l])
-        if l + 1 < len(layers):
-            x = ssd.ssd_rmsnorm(y, eps)
+        y, ss, _ = ssd.ssd_scan_fwd_normed(x, sums[-1], p["dt"], p["A"], p["B"], p["C"], p["D"], states[l],
+                                           chunk=wl.chunk, rms_eps=eps, final_state=states[l],
+                                           want_sums=l + 1 < len(layers))
+        ys.append(y)
+        sums.append(ss)
+        x = y
     torch.cuda.synchronize()
-    return y
+    return ys, sums[:-1]
+
+
+def _normed_input(y_prev, eps, b, h, tok_block=4096):
+    """The input layer l+1 sees, for batch b and head h: the previous layer's
+    stored y RMS-normalised over each token's H*P features (oracle.rmsnorm,
+    fp64, unrounded: the fused path never stores it), in token blocks."""
+    L = y_prev.shape[1]
+    out = np.empty((L, y_prev.shape[3]))
+    for t0 in range(0, L, tok_block):
+        out[t0:t0 + tok_block] = oracle.rmsnorm(to_np64(y_prev[b:b + 1, t0:t0 + tok_block]), eps)[0, :, h]
+    return out
 
 
 @pytest.mark.parametrize("L,V", [(1024, 256), (1000, 256), (1000, 300)])
 def test_vertical_small(L, V):
-    """3-layer stack: vertical == horizontal (bitwise when V % Q == 0), every
-    layer teacher-forced against the oracle on its own bf16 input (5e-3), and
-    the end-to-end output within the bound of _check_end_to_end."""
+    """3-layer stack with the RMS norm fused between layers: vertical ==
+    horizontal (bitwise when V % Q == 0), every layer teacher-forced against
+    the oracle on its own input (the previous GPU layer's y, normalised by the
+    oracle; 5e-3), the sums of squares each layer passes on, and the end-to-end
+    output within the bound of _check_end_to_end."""
     wl = inputs.custom("stack24_vertical", batch=2, seqlen=L, nheads=4)
     n_layers, eps = 3, 1e-6
     host_layers, dev_layers = _stack_layers(wl, n_layers)
@@ -283,14 +301,7 @@ def test_vertical_small(L, V):
                     for _ in range(n_layers)]
     st_v, st_h = zero(), zero()
     yv = ssd.ssd_vertical_fwd(x0, dev_layers, st_v, vblock=V, chunk=wl.chunk, rms_eps=eps)
-    xs, ys = [x0], []
-    for l, p in enumerate(dev_layers):
-        y, _ = ssd.ssd_scan_fwd(xs[-1], p["dt"], p["A"], p["B"], p["C"], p["D"], st_h[l], chunk=wl.chunk,
-                                final_state=st_h[l])
-        ys.append(y)
-        if l + 1 < n_layers:
-            xs.append(ssd.ssd_rmsnorm(y, eps))
-    torch.cuda.synchronize()
+    ys, sums = _horizontal_normed(x0, dev_layers, st_h, wl, eps)
     if V % wl.chunk == 0:
         assert torch.equal(yv, ys[-1])
         for a, b in zip(st_v, st_h):
@@ -298,11 +309,44 @@ def test_vertical_small(L, V):
     f = inputs.to_f64
     layers64 = [dict(dt=f(h["dt"]), A=f(h["A"]), B=f(h["B"]), C=f(h["C"]), D=f(h["D"])) for h in host_layers]
     for l, p in enumerate(layers64):
-        y_ref, f_ref = oracle.scan_recurrence(to_np64(xs[l]), p["dt"], p["A"], p["B"], p["C"], p["D"], None)
+        x_in = f(x0h) if l == 0 else oracle.rmsnorm(to_np64(ys[l - 1]), eps)
+        y_ref, f_ref = oracle.scan_recurrence(x_in, p["dt"], p["A"], p["B"], p["C"], p["D"], None)
         assert rel_err(to_np64(ys[l]), y_ref) <= TOL["bf16"], ("layer", l)
         assert rel_err(to_np64(st_h[l]), f_ref) <= TOL["bf16"], ("state", l)
         assert rel_err(to_np64(st_v[l]), f_ref) <= TOL["bf16"], ("vertical state", l)
+        if l > 0:  # the sums layer l read: over the P values of the stored y_{l-1}
+            ss_ref = np.sum(to_np64(ys[l - 1]) ** 2, axis=-1)
+            assert rel_err(to_np64(sums[l]), ss_ref) <= 1e-5, ("sums", l)
     _check_end_to_end(f(x0h), layers64, eps, to_np64(yv), tag=f"3-layer stack L={L} V={V}")
+
+
+def test_vertical_two_heads_keeps_the_norm_pass():
+    """With two heads per CTA the stack keeps the norm as its own pass
+    (ssd_rmsnorm between layers, the normalised input stored in bf16): vertical
+    == that horizontal schedule bitwise, and the last layer teacher-forced
+    against the oracle on the stored input."""
+    wl = inputs.custom("stack24_vertical", batch=2, seqlen=1024, nheads=4)
+    n_layers, eps, V = 3, 1e-6, 256
+    host_layers, dev_layers = _stack_layers(wl, n_layers)
+    x0 = to_dev(inputs.generate(wl, names=("x",))["x"])
+    zero = lambda: [torch.zeros((wl.batch, wl.nheads, wl.dstate, wl.headdim), device="cuda")
+                    for _ in range(n_layers)]
+    st_v, st_h = zero(), zero()
+    yv = ssd.ssd_vertical_fwd(x0, dev_layers, st_v, vblock=V, chunk=wl.chunk, rms_eps=eps, two_heads=True)
+    xs, y = [x0], None
+    for l, p in enumerate(dev_layers):
+        y, _ = ssd.ssd_scan_fwd(xs[-1], p["dt"], p["A"], p["B"], p["C"], p["D"], st_h[l], chunk=wl.chunk,
+                                final_state=st_h[l], two_heads=True)
+        if l + 1 < n_layers:
+            xs.append(ssd.ssd_rmsnorm(y, eps))
+    torch.cuda.synchronize()
+    assert torch.equal(yv, y)
+    for a, b in zip(st_v, st_h):
+        assert torch.equal(a, b)
+    f = inputs.to_f64
+    h = host_layers[-1]
+    y_ref, _ = oracle.scan_recurrence(to_np64(xs[-1]), f(h["dt"]), f(h["A"]), f(h["B"]), f(h["C"]), f(h["D"]), None)
+    assert rel_err(to_np64(y), y_ref) <= TOL["bf16"]
 
 
 def _check_end_to_end(x0, layers64, eps, y_end, tag="stack"):
@@ -348,12 +392,14 @@ def _stack_sensitivity(x0, layers64, eps, rel, seed=0):
 
 @pytest.mark.slow
 def test_stack24_vertical_full():
-    """The 24-layer stack at full size.
+    """The 24-layer stack at full size (RMS norm fused between layers).
 
-    1. vertical == horizontal bitwise on the GPU (V % Q == 0);
+    1. vertical == horizontal bitwise on the GPU (V % Q == 0), the horizontal
+       schedule run layer by layer through ssd_scan_fwd_normed;
     2. every layer, teacher-forced: the GPU's y_l and final state for a sampled
-       (batch, head) over the whole sequence match the oracle run on the GPU's
-       own bf16 input x_l (5e-3), and x_{l+1} is the RMS-normalised y_l;
+       (batch, head) over the whole sequence match the oracle run on the input
+       the layer sees (y_{l-1} of the GPU, RMS-normalised by the oracle; 5e-3),
+       and the sums of squares passed on are those of the stored y_l;
     3. end to end on a prefix against the oracle's stack, within the bound of
        _check_end_to_end.
     """
@@ -366,16 +412,9 @@ def test_stack24_vertical_full():
     st_v = zero(wl.batch)
     yv = ssd.ssd_vertical_fwd(x0, dev_layers, st_v, vblock=V, chunk=wl.chunk, rms_eps=eps)
     torch.cuda.synchronize()
-    # horizontal schedule, keeping every layer's input and output
+    # horizontal schedule, keeping every layer's output and the sums it passes on
     st_h = zero(wl.batch)
-    xs, ys = [x0], []
-    for l, p in enumerate(dev_layers):
-        y, _ = ssd.ssd_scan_fwd(xs[-1], p["dt"], p["A"], p["B"], p["C"], p["D"], st_h[l], chunk=wl.chunk,
-                                final_state=st_h[l])
-        ys.append(y)
-        if l + 1 < n_layers:
-            xs.append(ssd.ssd_rmsnorm(y, eps))
-    torch.cuda.synchronize()
+    ys, sums = _horizontal_normed(x0, dev_layers, st_h, wl, eps)
     assert torch.equal(yv, ys[-1])
     for a, b in zip(st_v, st_h):
         assert torch.equal(a, b)
@@ -383,7 +422,8 @@ def test_stack24_vertical_full():
     rng = np.random.default_rng(2)
     samp = [(int(rng.integers(wl.batch)), int(rng.integers(wl.nheads))) for _ in range(n_layers)]
     f = inputs.to_f64
-    xo = np.stack([to_np64(xs[l][b, :, h]) for l, (b, h) in enumerate(samp)], axis=1)[None]
+    xo = np.stack([to_np64(x0[b, :, h]) if l == 0 else _normed_input(ys[l - 1], eps, b, h)
+                   for l, (b, h) in enumerate(samp)], axis=1)[None]
     dto = np.stack([f(host_layers[l]["dt"][b, :, h]) for l, (b, h) in enumerate(samp)], axis=1)[None]
     Bo = np.stack([f(host_layers[l]["B"][b, :, 0]) for l, (b, h) in enumerate(samp)], axis=1)[None]
     Co = np.stack([f(host_layers[l]["C"][b, :, 0]) for l, (b, h) in enumerate(samp)], axis=1)[None]
@@ -393,11 +433,10 @@ def test_stack24_vertical_full():
     for l, (b, h) in enumerate(samp):
         assert rel_err(to_np64(ys[l][b, :, h]), y_ref[0, :, l]) <= TOL["bf16"], ("layer", l)
         assert rel_err(to_np64(st_h[l][b, h]), f_ref[0, l]) <= TOL["bf16"], ("state", l)
-    for l in range(n_layers - 1):
+    for l in range(1, n_layers):
         tok = slice(0, 4096)
-        ref = oracle.rmsnorm_bf16(to_np64(ys[l][:1, tok]), eps)
-        got = to_np64(xs[l + 1][:1, tok])
-        assert np.max(np.abs(got - ref)) <= 2.0 ** -7 * np.max(np.abs(ref)), ("rmsnorm", l)
+        ss_ref = np.sum(to_np64(ys[l - 1][:1, tok]) ** 2, axis=-1)
+        assert rel_err(to_np64(sums[l][:1, tok]), ss_ref) <= 1e-5, ("sums", l)
     # 3. end to end on a prefix (batch 0, 1024 tokens); the prefix is causal, so
     # it equals the first 1024 tokens of the full run
     Lp = 1024

@@ -52,25 +52,29 @@ def test_withheld_loads_time_out_and_context_survives(two_heads):
 
 @pytest.mark.parametrize("two_heads", [True])
 def test_carry_wait_times_out_and_context_survives(two_heads):
-    """The two-head kernel's split schedule with no carry ever published: every
-    CTA that starts inside a sequence gives up waiting for its predecessor's
-    state after about two seconds; the host reads SSD_ERR_TIMEOUT, and a normal
-    scan (with its carries) then matches the oracle in the same context."""
+    """The two-head kernel's segmented schedule with no carry ever published:
+    every segment after the first gives up waiting for its predecessor's state
+    after about two seconds; the host reads SSD_ERR_TIMEOUT, and a normal scan
+    (with its carries) then matches the oracle in the same context."""
     wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=300, nheads=160, ngroups=1, init_var=0.1)
     host = inputs.generate(wl)
     dev = device_inputs(host)
     assert ssd.ssd_read_device_status() == SSD_OK
-    t0 = time.monotonic()
-    ssd.ssd_selftest_carry_timeout(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
-                                   chunk=wl.chunk, two_heads=two_heads)
-    status = ssd.ssd_read_device_status()
-    elapsed = time.monotonic() - t0
-    assert status == SSD_ERR_TIMEOUT
-    assert elapsed < 30.0, elapsed
-    assert ssd.ssd_read_device_status() == SSD_OK
-    y, fin = ssd.ssd_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
-                              chunk=wl.chunk, two_heads=two_heads)
-    torch.cuda.synchronize()
+    ssd.ssd_selftest_set_segments(3)
+    try:
+        t0 = time.monotonic()
+        ssd.ssd_selftest_carry_timeout(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
+                                       chunk=wl.chunk, two_heads=two_heads)
+        status = ssd.ssd_read_device_status()
+        elapsed = time.monotonic() - t0
+        assert status == SSD_ERR_TIMEOUT
+        assert elapsed < 30.0, elapsed
+        assert ssd.ssd_read_device_status() == SSD_OK
+        y, fin = ssd.ssd_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
+                                  chunk=wl.chunk, two_heads=two_heads)
+        torch.cuda.synchronize()
+    finally:
+        ssd.ssd_selftest_set_segments(0)
     assert ssd.ssd_read_device_status() == SSD_OK
     y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host))
     assert rel_err(to_np64(y), y_ref) <= TOL["bf16"]

@@ -278,6 +278,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       };
       for (int jp = 0; jp < kPrefetch; ++jp) prefetch(jp);
       const int nload = nsub & (p.withhold_loads - 1);  // 0 or nsub (withhold_loads is 0 or 1)
+      int issued = 0;
       for (int j = 0; j < nload; ++j) {
         const int st = j & 1;
         prefetch(j + kPrefetch);
@@ -290,10 +291,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_load_4d(sx + OFF_B + TILE, &map_b, &bar[FULL0 + st], 64, g, t0, b);
         tma_load_4d(sx + OFF_C, &map_c, &bar[FULL0 + st], 0, g, t0, b);
         tma_load_4d(sx + OFF_C + TILE, &map_c, &bar[FULL0 + st], 64, g, t0, b);
+        issued = j + 1;
         mark(j, EV_LOADS);
       }
-      // drain: the last loads of each stage must land before the CTA may exit
-      for (int j = (nload > 2 ? nload - 2 : 0); j < nload; ++j) {
+      // drain: the last loads issued to each stage must land before the CTA may
+      // exit (also after an early exit from the loop)
+      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) {
         uint64_t* fb = &bar[FULL0 + (j & 1)];
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(fb, (j >> 1) & 1) && globaltimer_ns() - t0 < 1000000000ull) {

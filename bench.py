@@ -503,7 +503,7 @@ def run_decode(args, wl, dev, rank, world):
                    "l2": "512 MB L2 flush between steps (the state fits in L2); per-step events exclude it"},
         "clocks": clk, "gpu_launches": args.steps,
         "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
-                     "traffic": None, "kernel": "k_ssd_step_v4", "bytes_per_launch": nbytes,
+                     "traffic": None, "kernel": "k_ssd_step_bulk", "bytes_per_launch": nbytes,
                      "peak_source": peak_src},
     }
     if rank == 0:

@@ -5,14 +5,14 @@
 // the mode a model runs in when it generates with a state cache.
 //
 // HBM-bound on the fp32 state: every call reads and writes N*P*4 bytes per
-// (batch, head).  One block per (batch, head).  The vector kernel (P % 4 == 0,
-// 16-byte aligned state) gives thread (c, r) the four columns 4c..4c+3 of
-// state rows r, r + R, ... (R = 256 / (P/4)): 128-bit loads and stores, all
-// of a thread's rows loaded before any is written back, so a block keeps its
-// whole 32 KB state tile in flight.  The scalar kernel covers every other
-// shape.  a = exp(dt A) is evaluated once per warp and broadcast.  y is
-// reduced over r in shared memory in a fixed order (deterministic).
+// (batch, head).  One block per (batch, head).  The staged kernel (P % 4 ==
+// 0, N <= 128, 16-byte aligned state) copies the block's state tile into
+// shared memory with one bulk copy and updates it from there (below); the
+// scalar kernel covers every other shape.  a = exp(dt A) is evaluated once per
+// warp and broadcast.  y is reduced over the state rows in shared memory in a
+// fixed order (deterministic).
 #include "ssd_common.cuh"
+#include "umma.cuh"
 
 namespace ssd {
 
@@ -55,53 +55,80 @@ __global__ void __launch_bounds__(256) k_ssd_step(const T* __restrict__ x, const
   }
 }
 
-// 128-bit form: P % 4 == 0, state 16-byte aligned, N <= 128.  Thread (c, r):
-// columns 4c..4c+3, rows r + R k for k < N / R (R = 4 * 256 / P rows per pass).
+// Staged form (P % 4 == 0, N <= 128, state 16-byte aligned): thread 0 brings
+// the block's whole state tile [N][P] f32 (at most 32 KB) into shared memory
+// with one bulk copy while the others load B, C, dt, A and x; the 256 threads
+// then update the tile from shared memory and write it back with 128-bit
+// stores.  A block holds 37 KB of shared memory and few registers, so six run
+// per SM and the whole state of a 2.7B-shaped layer is in flight at once.
 template <typename T>
-__global__ void __launch_bounds__(256) k_ssd_step_v4(const T* __restrict__ x, const float* __restrict__ dt,
-                                                     const float* __restrict__ A, const T* __restrict__ Bm,
-                                                     const T* __restrict__ Cm, const float* __restrict__ D,
-                                                     float* __restrict__ state, T* __restrict__ y, int H, int G, int N,
-                                                     int P, int input_dt) {
+__global__ void __launch_bounds__(256) k_ssd_step_bulk(const T* __restrict__ x, const float* __restrict__ dt,
+                                                       const float* __restrict__ A, const T* __restrict__ Bm,
+                                                       const T* __restrict__ Cm, const float* __restrict__ D,
+                                                       float* __restrict__ state, T* __restrict__ y, int H, int G,
+                                                       int N, int P, int input_dt) {
+  using namespace umma;
+  extern __shared__ __align__(128) float tile[];  // [N][P]
   __shared__ float4 part[256];
-  constexpr int kMaxRows = 16;  // N <= 128 rows over at least R = 16 rows per pass (P <= 64)
+  __shared__ float sb[128], sc[128];  // B and C of the token, one entry per state row
+  __shared__ __align__(8) uint64_t bar;
   const int bh = blockIdx.x;
   const int b = bh / H, h = bh % H;
   const int g = h / (H / G);
   const int C4 = P / 4, R = 256 / C4;
   const int tid = threadIdx.x, lane = tid & 31;
   const int c = tid % C4, r = tid / C4;
-  const float dtv = dt[bh];
-  float a = 0.f;
-  if (lane == 0) a = expf(dtv * A[h]);
-  a = __shfl_sync(0xffffffffu, a, 0);
-  float xp[4], xin[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    xp[i] = to_f32(x[(int64_t)bh * P + 4 * c + i]);
-    xin[i] = input_dt ? dtv * xp[i] : xp[i];
+  float* st = state + (int64_t)bh * N * P;
+  const uint32_t bytes = (uint32_t)(N * P) * 4u;
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&bar, bytes);
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(tile)),
+        "l"(st), "r"(bytes), "r"(smem_u32(&bar))
+        : "memory");
   }
   const T* bg = Bm + ((int64_t)b * G + g) * N;
   const T* cg = Cm + ((int64_t)b * G + g) * N;
-  float4* st4 = reinterpret_cast<float4*>(state + (int64_t)bh * N * P);
-  float4 v[kMaxRows];
-  // rows of this thread; threads past the last full pass (r >= R, when C4
-  // does not divide 256) own none
-  const int nk = r < R ? (N - r + R - 1) / R : 0;
+  float bt = 0.f, ct = 0.f;
+  if (tid < N) {
+    bt = to_f32(bg[tid]);
+    ct = to_f32(cg[tid]);
+  }
+  const float dtv = dt[bh];
+  const float Ah = lane == 0 ? A[h] : 0.f;
+  float xp[4];
 #pragma unroll
-  for (int k = 0; k < kMaxRows; ++k)
-    if (k < nk) v[k] = st4[(int64_t)(r + k * R) * C4 + c];
+  for (int i = 0; i < 4; ++i) xp[i] = to_f32(x[(int64_t)bh * P + 4 * c + i]);
+  float a = 0.f;
+  if (lane == 0) a = expf(dtv * Ah);
+  a = __shfl_sync(0xffffffffu, a, 0);
+  float xin[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) xin[i] = input_dt ? dtv * xp[i] : xp[i];
+  if (tid < N) {
+    sb[tid] = bt;
+    sc[tid] = ct;
+  }
+  __syncthreads();  // sb, sc and the initialised barrier are visible to all
+  if (!mbar_wait(&bar, 0)) {  // bounded: the copy of valid memory lands unless the device is wedged
+    if (tid == 0) atomicExch(&g_device_status, 2);
+    return;
+  }
+  const float4* t4 = reinterpret_cast<const float4*>(tile);
+  float4* st4 = reinterpret_cast<float4*>(st);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-  for (int k = 0; k < kMaxRows; ++k) {
-    if (k < nk) {
-      const int n = r + k * R;
-      const float bn = to_f32(bg[n]), cn = to_f32(cg[n]);
+  if (r < R) {
+    for (int n = r; n < N; n += R) {
+      const float4 v = t4[n * C4 + c];
+      const float bn = sb[n], cn = sc[n];
       float4 o;
-      o.x = fmaf(a, v[k].x, bn * xin[0]);
-      o.y = fmaf(a, v[k].y, bn * xin[1]);
-      o.z = fmaf(a, v[k].z, bn * xin[2]);
-      o.w = fmaf(a, v[k].w, bn * xin[3]);
+      o.x = fmaf(a, v.x, bn * xin[0]);
+      o.y = fmaf(a, v.y, bn * xin[1]);
+      o.z = fmaf(a, v.z, bn * xin[2]);
+      o.w = fmaf(a, v.w, bn * xin[3]);
       st4[(int64_t)n * C4 + c] = o;
       acc.x = fmaf(cn, o.x, acc.x);
       acc.y = fmaf(cn, o.y, acc.y);
@@ -119,8 +146,7 @@ __global__ void __launch_bounds__(256) k_ssd_step_v4(const T* __restrict__ x, co
       s += (i == 0) ? q.x : (i == 1) ? q.y : (i == 2) ? q.z : q.w;
     }
     const float d = D ? D[h] : 0.f;
-    const float xv = to_f32(x[(int64_t)bh * P + tid]);
-    y[(int64_t)bh * P + tid] = from_f32<T>(s + d * xv);
+    y[(int64_t)bh * P + tid] = from_f32<T>(s + d * to_f32(x[(int64_t)bh * P + tid]));
   }
 }
 
@@ -128,12 +154,13 @@ cudaError_t launch_ssd_step(const Problem& p, float* state, cudaStream_t st) {
   const int P = (int)p.P;
   if (P % 4 == 0 && (reinterpret_cast<uintptr_t>(state) & 15u) == 0 && p.N <= 128) {
     const int threads = 256;  // (P/4) columns x (1024/P) rows per pass
+    const size_t tile = sizeof(float) * (size_t)p.N * P;  // <= 32 KB
     if (p.io == SSD_BF16)
-      k_ssd_step_v4<__nv_bfloat16><<<(unsigned)(p.B * p.H), threads, 0, st>>>(
+      k_ssd_step_bulk<__nv_bfloat16><<<(unsigned)(p.B * p.H), threads, tile, st>>>(
           (const __nv_bfloat16*)p.x, p.dt, p.A, (const __nv_bfloat16*)p.Bm, (const __nv_bfloat16*)p.Cm, p.D, state,
           (__nv_bfloat16*)p.y, (int)p.H, (int)p.G, (int)p.N, P, p.input_dt);
     else
-      k_ssd_step_v4<float><<<(unsigned)(p.B * p.H), threads, 0, st>>>(
+      k_ssd_step_bulk<float><<<(unsigned)(p.B * p.H), threads, tile, st>>>(
           (const float*)p.x, p.dt, p.A, (const float*)p.Bm, (const float*)p.Cm, p.D, state, (float*)p.y, (int)p.H,
           (int)p.G, (int)p.N, P, p.input_dt);
     return cudaGetLastError();

@@ -16,7 +16,7 @@ pytestmark = pytest.mark.gpu
     ("tiny_f32", dict(batch=1, seqlen=20, nheads=3, ngroups=1, headdim=5, dstate=7, init_var=0.3)),
     ("mamba2_130m_layer", dict(batch=2, seqlen=24, nheads=4, ngroups=2, init_var=0.1)),
     ("mamba2_2p7b_layer", dict(seqlen=6)),
-    # 128-bit kernel with 3 column groups (256 threads do not split evenly) and with 1
+    # staged kernel with 3 column groups (256 threads do not split evenly) and with 1
     ("tiny_f32", dict(batch=2, seqlen=12, nheads=2, ngroups=1, headdim=12, dstate=100, init_var=0.3)),
     ("mamba2_130m_layer", dict(batch=1, seqlen=10, nheads=2, ngroups=1, headdim=4, dstate=128, init_var=0.1)),
 ])
@@ -59,7 +59,7 @@ def test_decode_continues_a_prefill():
 
 def test_decode_state_view_not_16_byte_aligned():
     """A state that is only 4-byte aligned (a view one float into a buffer) takes
-    the scalar kernel and gives the same results as the 128-bit kernel."""
+    the scalar kernel and gives the same results as the staged kernel."""
     wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=8, nheads=4, ngroups=2, init_var=0.1)
     host = inputs.generate(wl)
     dev = device_inputs(host)

@@ -309,38 +309,71 @@ cudaError_t launch_chunk_scan_simt(const Problem& p, const float* lam, const flo
 
 // ---------------------------------------------------------------------------
 // RMS normalisation of each row of `features` values, fp32 arithmetic,
-// deterministic block reduction.  One block of 256 threads per row; in and
-// out may alias (every read of a row happens before the reduction barrier).
+// deterministic warp reduction.  One warp per row, eight rows per block (a
+// block per row left most of its threads idle and made the launch thousands
+// of tiny blocks long); with bf16 rows of a multiple of 8 values, 16-byte
+// loads and stores.  in and out may alias: a lane reads each of its values
+// before it writes it.
 template <typename T>
-__global__ void __launch_bounds__(256) k_rmsnorm(const T* in, float eps, T* out, int64_t F) {
-  __shared__ float red[8];
-  const int64_t r = blockIdx.x;
+__global__ void __launch_bounds__(256) k_rmsnorm(const T* in, float eps, T* out, int64_t rows, int64_t F) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (r >= rows) return;
   const T* v = in + r * F;
   T* o = out + r * F;
+  const bool vec = sizeof(T) == 2 && (F & 7) == 0 && ((reinterpret_cast<uintptr_t>(in) | reinterpret_cast<uintptr_t>(out)) & 15) == 0;
   float ss = 0.f;
-  for (int64_t f = threadIdx.x; f < F; f += 256) {
-    const float a = to_f32(v[f]);
-    ss = fmaf(a, a, ss);
+  if (vec) {
+    const uint4* v4 = reinterpret_cast<const uint4*>(v);
+    for (int64_t f = lane; f < F / 8; f += 32) {
+      const uint4 q = v4[f];
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float a = __uint_as_float(w[i] << 16), c = __uint_as_float(w[i] & 0xFFFF0000u);
+        ss = fmaf(a, a, ss);
+        ss = fmaf(c, c, ss);
+      }
+    }
+  } else {
+    for (int64_t f = lane; f < F; f += 32) {
+      const float a = to_f32(v[f]);
+      ss = fmaf(a, a, ss);
+    }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  float tot = 0.f;
+  const float inv = 1.0f / sqrtf(ss / (float)F + eps);
+  if (vec) {
+    const uint4* v4 = reinterpret_cast<const uint4*>(v);
+    uint4* o4 = reinterpret_cast<uint4*>(o);
+    for (int64_t f = lane; f < F / 8; f += 32) {
+      const uint4 q = v4[f];
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+      uint32_t z[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) tot += red[i];
-  const float inv = 1.0f / sqrtf(tot / (float)F + eps);
-  for (int64_t f = threadIdx.x; f < F; f += 256) o[f] = from_f32<T>(to_f32(v[f]) * inv);
+      for (int i = 0; i < 4; ++i) {
+        const float a = __uint_as_float(w[i] << 16) * inv, c = __uint_as_float(w[i] & 0xFFFF0000u) * inv;
+        const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(a));
+        const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(c));
+        z[i] = lo | (hi << 16);
+      }
+      o4[f] = make_uint4(z[0], z[1], z[2], z[3]);
+    }
+  } else {
+    for (int64_t f = lane; f < F; f += 32) o[f] = from_f32<T>(to_f32(v[f]) * inv);
+  }
 }
 
 cudaError_t launch_rmsnorm(int64_t rows, int64_t features, int io, const void* in, float eps, void* out,
                            cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
+  const unsigned blocks = (unsigned)((rows + 7) / 8);
   if (io == SSD_BF16)
-    k_rmsnorm<__nv_bfloat16><<<(unsigned)rows, 256, 0, st>>>((const __nv_bfloat16*)in, eps,
-                                                             (__nv_bfloat16*)out, features);
+    k_rmsnorm<__nv_bfloat16><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)in, eps, (__nv_bfloat16*)out, rows,
+                                                     features);
   else
-    k_rmsnorm<float><<<(unsigned)rows, 256, 0, st>>>((const float*)in, eps, (float*)out, features);
+    k_rmsnorm<float><<<blocks, 256, 0, st>>>((const float*)in, eps, (float*)out, rows, features);
   return cudaGetLastError();
 }
 

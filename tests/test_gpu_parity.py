@@ -183,15 +183,24 @@ def test_steps_match_oracle_intermediates(case):
     assert rel_err(to_np64(y), ref["y"]) <= tol
 
 
-def test_rmsnorm_matches_oracle():
+@pytest.mark.parametrize("shape,dtype", [
+    ((2, 37, 24, 64), torch.bfloat16),   # 74 rows (not a multiple of 8), 16-byte vectors
+    ((1, 5, 3, 5), torch.bfloat16),      # 15 features: the scalar path
+    ((2, 9, 4, 16), torch.float32),
+])
+def test_rmsnorm_matches_oracle(shape, dtype):
     rng = np.random.default_rng(0)
-    a = rng.standard_normal((2, 37, 24, 64)).astype(np.float32) * 3.0
-    t = torch.from_numpy(a).cuda().to(torch.bfloat16)
+    a = rng.standard_normal(shape).astype(np.float32) * 3.0
+    t = torch.from_numpy(a).cuda().to(dtype)
     out = ssd.ssd_rmsnorm(t, 1e-6)
     torch.cuda.synchronize()
-    ref = oracle.rmsnorm_bf16(to_np64(t), 1e-6)
-    # both round to bf16: compare within one bf16 ulp of the normalised values
-    assert np.max(np.abs(to_np64(out) - ref)) <= 2.0 ** -7 * np.max(np.abs(ref))
+    if dtype == torch.bfloat16:
+        ref = oracle.rmsnorm_bf16(to_np64(t), 1e-6)
+        # both round to bf16: compare within one bf16 ulp of the normalised values
+        assert np.max(np.abs(to_np64(out) - ref)) <= 2.0 ** -7 * np.max(np.abs(ref))
+    else:
+        ref = oracle.rmsnorm(to_np64(t), 1e-6)
+        assert np.max(np.abs(to_np64(out) - ref)) <= 1e-5 * np.max(np.abs(ref))
     # in place
     t2 = t.clone()
     ssd.ssd_rmsnorm(t2, 1e-6, out=t2)

@@ -85,7 +85,7 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {
-    "ssd_fused": ("ssd_fused.cu", "ssd_common.cuh", "ssd_tc.cuh", "tma.cuh", "umma.cuh"),
+    "ssd_fused": ("ssd_fused.cu", "ssd_split.cuh", "ssd_common.cuh", "ssd_tc.cuh", "tma.cuh", "umma.cuh"),
     "ssd_pair": ("ssd_pair.cu", "ssd_common.cuh", "ssd_tc.cuh", "tma.cuh", "umma.cuh"),
 }
 PATH_KERNEL = {"fused": "ssd_fused", "fused_pair": "ssd_pair"}

@@ -27,6 +27,7 @@
 // raises g_device_status and the roles drain without further waits.
 #include <atomic>
 
+#include "ssd_split.cuh"
 #include "ssd_tc.cuh"
 #include "tma.cuh"
 #include "umma.cuh"
@@ -69,7 +70,8 @@ struct Params {
   int64_t L;
   int H, G, nsub;
   int64_t nc, Q;         // chunking of the step kernels
-  const float* lam_in;   // step-1 log-decay sums [B,H,nc,Q] (step modes)
+  const float* lam_in;   // step-1 log-decay sums [B,H,nc,Q] (step modes), or NULL: the
+                         // kernel scans dt itself from the chunk's first token
   const float* dt;
   int64_t sdt, lddt;  // batch and token strides of dt
   int input_dt;       // the input term is dt_t B_t x_t^T
@@ -90,6 +92,7 @@ struct Params {
   float norm_eps, inv_feat;  // eps, 1 / (H P)
   unsigned long long* trace;  // diagnostics: per-sub-chunk event clocks of CTA 0, then
                               // [start ns, end ns, SM] of every CTA; or NULL
+  float* seg_decay;           // chunk-state mode: [B,H,nc] total log-decay of each chunk, or NULL
   int withhold_loads;         // self-test of the timeout path: issue no TMA loads, so
                               // every wait on them runs out (0 in every other launch)
 };
@@ -186,11 +189,13 @@ __device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
 
+// LEAN: the chunk-state mode reduced to what a chunk's end state needs (x and
+// B tiles, X', b_intra, the state recursion): no C, no S, no mask, no y.
 // XDT: the dt-scaled input variant; NORM: a layer of a stack with the RMS norm
 // fused (input scaled from ss_in when given, sums of squares to ss_out when
 // given).  Separate instantiations, so that the plain scan carries none of
 // their per-column factors and sums.
-template <bool XDT, bool NORM>
+template <bool XDT, bool NORM, bool LEAN>
 __global__ void __launch_bounds__(THREADS, 1)
     k_ssd_fused(Params p, const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
                 const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_y) {
@@ -243,7 +248,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&bar[FULL0 + i], 1);
       mbar_init(&bar[EMPTY0 + i], 1);
       mbar_init(&bar[SFULL0 + i], 1);
-      mbar_init(&bar[PFULL0 + i], T + AUX);
+      mbar_init(&bar[PFULL0 + i], LEAN ? AUX : T + AUX);
       mbar_init(&bar[CFULL0 + i], 1);
       mbar_init(&bar[TEMPTY0 + i], T);
       mbar_init(&bar[YFREE0 + i], 1);
@@ -273,8 +278,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_prefetch_4d(&map_x, 0, h, tp, b);
         tma_prefetch_4d(&map_b, 0, g, tp, b);
         tma_prefetch_4d(&map_b, 64, g, tp, b);
-        tma_prefetch_4d(&map_c, 0, g, tp, b);
-        tma_prefetch_4d(&map_c, 64, g, tp, b);
+        if (!LEAN) {
+          tma_prefetch_4d(&map_c, 0, g, tp, b);
+          tma_prefetch_4d(&map_c, 64, g, tp, b);
+        }
       };
       for (int jp = 0; jp < kPrefetch; ++jp) prefetch(jp);
       const int nload = nsub & (p.withhold_loads - 1);  // 0 or nsub (withhold_loads is 0 or 1)
@@ -285,12 +292,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (j >= 2 && !ctl.wait(EMPTY0 + st, ((j >> 1) + 1) & 1)) break;
         uint8_t* sx = sm + st * STAGE;
         const int t0 = t_base + j * T;
-        mbar_arrive_expect_tx(&bar[FULL0 + st], TX_BYTES);
+        mbar_arrive_expect_tx(&bar[FULL0 + st], LEAN ? 3 * TILE : TX_BYTES);
         tma_load_4d(sx + OFF_X, &map_x, &bar[FULL0 + st], 0, h, t0, b);
         tma_load_4d(sx + OFF_B, &map_b, &bar[FULL0 + st], 0, g, t0, b);
         tma_load_4d(sx + OFF_B + TILE, &map_b, &bar[FULL0 + st], 64, g, t0, b);
-        tma_load_4d(sx + OFF_C, &map_c, &bar[FULL0 + st], 0, g, t0, b);
-        tma_load_4d(sx + OFF_C + TILE, &map_c, &bar[FULL0 + st], 64, g, t0, b);
+        if (!LEAN) {
+          tma_load_4d(sx + OFF_C, &map_c, &bar[FULL0 + st], 0, g, t0, b);
+          tma_load_4d(sx + OFF_C + TILE, &map_c, &bar[FULL0 + st], 64, g, t0, b);
+        }
         issued = j + 1;
         mark(j, EV_LOADS);
       }
@@ -325,7 +334,31 @@ __global__ void __launch_bounds__(THREADS, 1)
       int js = 0, jc = 0;
       uint32_t idle = 0;
       uint64_t t_last = globaltimer_ns();
-      while (jc < nsub) {
+      if constexpr (LEAN) {
+        // b_intra of each sub-chunk once X' is written (PFULL: the aux warps
+        // alone) and the epilogue has read b_intra of jc-2 from the buffer
+        for (; jc < nsub; ++jc) {
+          const int st = jc & 1, buf = jc & 1;
+          bool ok = ctl.wait(PFULL0 + st, (jc >> 1) & 1);
+          if (ok && jc >= 2) ok = ctl.wait(TEMPTY0 + buf, ((jc >> 1) + 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t base = tmem + buf * 256;
+          const uint64_t cB = desc_advance(dBmn, st * STAGE), cXp = desc_advance(dXp, st * TILE);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ss(base + 192, desc_advance(cB, ks * 2048), desc_advance(cXp, ks * 2048), idB, ks > 0);
+          mma_commit(&bar[CFULL0 + buf]);
+          mma_commit(&bar[EMPTY0 + st]);
+        }
+        (void)idS;
+        (void)idY;
+        (void)dPrev;
+        (void)dX;
+        (void)dBk;
+        (void)js;
+      }
+      while (!LEAN && jc < nsub) {
         bool progress = false;
         if (jc < js && mbar_test_wait(&bar[PFULL0 + (jc & 1)], (jc >> 1) & 1) &&
             mbar_test_wait(&bar[STATEFULL], jc & 1)) {
@@ -393,14 +426,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp < 4) {
     // ------------------------------------------------------------ dt, lam, decay factors, X'
     const int a = threadIdx.x;  // 0..63 (warps 0-1)
-    const float Ah = chunked ? 0.f : p.A[h];  // A (and dt) are read only by the whole scan
+    // lam comes from dt (whole scan, and step modes without a step-1 output)
+    // or from step 1's output (lamc)
+    const float* lamc = (chunked && p.lam_in) ? p.lam_in + cslot * p.Q : nullptr;
+    const float Ah = lamc ? 0.f : p.A[h];
     const float* dtb = p.dt + (int64_t)b * p.sdt + h;
     auto load_dt = [&](int j, float& d0, float& d1) {
-      const int64_t t0 = (int64_t)j * T + 2 * a;
-      d0 = (!chunked && j < nsub && t0 < p.L) ? dtb[t0 * p.lddt] : 0.f;
-      d1 = (!chunked && j < nsub && t0 + 1 < p.L) ? dtb[(t0 + 1) * p.lddt] : 0.f;
+      const int64_t t0 = (int64_t)t_base + (int64_t)j * T + 2 * a;
+      d0 = (!lamc && j < nsub && t0 < p.L) ? dtb[t0 * p.lddt] : 0.f;
+      d1 = (!lamc && j < nsub && t0 + 1 < p.L) ? dtb[(t0 + 1) * p.lddt] : 0.f;
     };
-    const float* lamc = chunked ? p.lam_in + cslot * p.Q : nullptr;
     // r of tokens 2a, 2a+1 of sub-chunk j from the H per-head sums of squares
     // of the previous layer's stored y (0 past L).  A token's H sums are
     // contiguous.  With H % 4 == 0 the first 32 of them (8 float4 per token)
@@ -497,7 +532,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float pre = (warp == 1) ? wtot[0] : 0.f;
       float lam1 = v + pre;       // token 2a+1
       float lam0 = lam1 - l1;     // token 2a
-      if (chunked) {              // step modes: sub-chunk-local sums from step 1's output
+      if (lamc) {                 // step modes: sub-chunk-local sums from step 1's output
         const float* ls = lamc + jt * T;
         const float base0 = (jt == 0) ? 0.f : ls[-1];
         lam0 = ls[2 * a] - base0;
@@ -558,7 +593,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // staged in the same buffer, has been read by the TMA store)
       bool ok = ctl.wait(FULL0 + st, (j >> 1) & 1);
       if (ok && j >= 2) ok = ctl.wait(CFULL0 + st, ((j - 2) >> 1) & 1);
-      if (ok && j >= 2) ok = ctl.wait(YFREE0 + st, ((j - 2) >> 1) & 1);  // y(j-2) staged here is stored
+      if (!LEAN && ok && j >= 2) ok = ctl.wait(YFREE0 + st, ((j - 2) >> 1) & 1);  // y(j-2) staged here is stored
       if (ok) {
         const float lam_end = lj[T - 1];  // log2 units
         const uint4* src = reinterpret_cast<const uint4*>(sm + st * STAGE + OFF_X);
@@ -590,6 +625,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ P = S (.) L
+    if constexpr (!LEAN) {  // (the lean mode has no S and no mask)
     const int q = warp & 3;          // TMEM lane quarter = 32-row block
     const int row = q * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
@@ -667,6 +703,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive(&bar[PFULL0 + buf]);
       if (q == 3 && lane == 0) mark(j, EV_MASK_DONE);
     }
+    }
   } else {
     // ------------------------------------------------------------ y, state, final
     const int q = warp & 3;
@@ -714,10 +751,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       fence_async_smem();
       mbar_arrive(&bar[STATEFULL]);
     };
-    publish_state();
+    if (!LEAN) publish_state();
+    float lam_sum = 0.f;  // log2 of the chunk's total decay (lean chunk-state mode)
     for (int j = 0; j < nsub; ++j) {
       const int buf = j & 1;
-      load_x(j, xcur);
+      if (!LEAN) load_x(j, xcur);
       bool ok = ctl.wait(CFULL0 + buf, (j >> 1) & 1);
       if (ok) ok = ctl.wait(LAMRDY0 + (j & 3), (j >> 2) & 1);      // acquire lam of this sub-chunk
       tc_fence_after();
@@ -739,6 +777,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           s[32 * c + i] = o.x;
           s[32 * c + i + 1] = o.y;
         }
+      }
+      if constexpr (LEAN) {  // only the state: release the buffer and go on
+        tc_fence_before();
+        mbar_arrive(&bar[TEMPTY0 + buf]);
+        lam_sum += lam_end;
+        continue;
       }
       if (ok) publish_state();
       if (r == 0) mark(j, EV_STATE_PUB);
@@ -800,6 +844,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (r == 0) mark(j, EV_EPI_DONE);
     }
     if (r == 0) tma_store_wait0();  // the y tiles are in global memory before the CTA exits
+    if (LEAN && p.seg_decay && r == 0) p.seg_decay[cslot] = lam_sum * 0.6931471805599453f;  // log2 -> ln
     if (final_ptr) {
       float4* dst = reinterpret_cast<float4*>(final_ptr + (int64_t)r * P);
 #pragma unroll
@@ -825,18 +870,71 @@ bool fused_supported(const Problem& p) {
 
 bool tc_supported(const Problem& p) { return fused_supported(p) && p.B * p.H * p.nc < (1ll << 31); }
 
-int fused_kernels_per_call(const Problem&) { return 1; }
 
 bool uses_pair_kernel(const Problem& p) { return p.two_heads && pair_supported(p); }
 
-// The one-head kernel keeps the running state on chip (whole scan) or reads and
-// writes only the caller's step tensors (step modes): no workspace.  The
-// two-head kernel needs one for the carries of its split schedule.
-size_t tc_workspace_bytes(const Problem& p) { return uses_pair_kernel(p) ? pair_workspace_bytes(p) : 0; }
+// Segments for problems with fewer (batch, head) sequences than SMs: one CTA
+// per sequence would leave SMs idle, so every sequence is cut into nseg
+// segments of Qseg tokens and the scan runs in three launches (the page's
+// chunk decomposition one level up, "分块推理…" §2.1-§2.2, with a segment as the
+// chunk): the lean kernel forms each segment's end state from a zero start and
+// its total log-decay, k_state_passing combines them in order into each
+// segment's start state (and the final state), and the full kernel scans every
+// segment from its start state.  Chosen only where a cost model of rounds of
+// CTAs (a lean segment costing about a third of a full one) predicts a gain.
+struct SegPlan {
+  int nseg;      // 1: whole sequences in one launch
+  int64_t qseg;  // segment length in tokens (a multiple of 128)
+};
+static int g_fused_segments = 0;  // forced by a self-test (0: the cost model decides)
+void set_fused_segments(int nseg) { g_fused_segments = nseg > 0 ? nseg : 0; }
+static SegPlan seg_plan(const Problem& p) {
+  SegPlan plan{1, 0};
+  if (uses_pair_kernel(p) || !fused_supported(p)) return plan;
+  const int64_t nsub = ceil_div(p.L, (int64_t)fused::T), bh = p.B * p.H;
+  const int64_t nsm = split::sm_count();
+  auto make = [&](int64_t n) {
+    const int64_t seg = ceil_div(nsub, n);
+    return SegPlan{(int)ceil_div(nsub, seg), seg * fused::T};
+  };
+  if (g_fused_segments > 0) {
+    const SegPlan f = make(g_fused_segments);
+    return (f.nseg > 1 && bh * f.nseg < (1ll << 31)) ? f : plan;
+  }
+  if (bh >= nsm || nsub < 8) return plan;
+  const double plain = (double)ceil_div(bh, nsm) * (double)(nsub + 2);
+  double best = 0.9 * plain;
+  for (int64_t n = 2; n <= 64 && n <= nsub / 4; ++n) {
+    const SegPlan c = make(n);
+    const double seg = (double)(c.qseg / fused::T), rounds = (double)ceil_div(bh * c.nseg, nsm);
+    const double cost = rounds * (seg + 2.0) + rounds * (0.35 * seg + 1.5) + 1.0;
+    if (c.nseg > 1 && cost < best) {
+      best = cost;
+      plan = c;
+    }
+  }
+  return plan;
+}
+static size_t seg_workspace_bytes(const Problem& p, const SegPlan& plan) {
+  if (plan.nseg <= 1) return 0;
+  const size_t states = sizeof(float) * (size_t)p.B * p.H * plan.nseg * p.N * p.P;
+  return (states + 255) / 256 * 256 + sizeof(float) * (size_t)p.B * p.H * plan.nseg;
+}
+
+// Kernel launches of one fused call: three for the segmented form.
+int fused_kernels_per_call(const Problem& p) { return seg_plan(p).nseg > 1 ? 3 : 1; }
+
+// The one-head kernel keeps the running state on chip; its segmented form
+// (above) needs the segments' states and decays.  The two-head kernel needs
+// room for the carries of its split schedule.
+size_t tc_workspace_bytes(const Problem& p) {
+  if (uses_pair_kernel(p)) return pair_workspace_bytes(p);
+  return seg_workspace_bytes(p, seg_plan(p));
+}
 
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
                                void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads = 0,
-                               const NormIO* norm = nullptr);
+                               const NormIO* norm = nullptr, float* seg_decay = nullptr);
 
 cudaError_t launch_fused_traced(const Problem& p, const float* init, float* final_state, unsigned long long* trace,
                                 cudaStream_t st) {
@@ -851,6 +949,24 @@ cudaError_t launch_fused_withheld(const Problem& p, const float* init, float* fi
 cudaError_t launch_fused(const Problem& p, const float* init, float* final_state, void* workspace,
                          size_t workspace_bytes, cudaStream_t st) {
   if (uses_pair_kernel(p)) return launch_pair(p, init, final_state, workspace, workspace_bytes, st, 0);
+  const SegPlan plan = seg_plan(p);
+  const size_t need = seg_workspace_bytes(p, plan);
+  if (plan.nseg > 1 && workspace && workspace_bytes >= need) {
+    Problem ps = p;  // segments as the chunks of the step modes
+    ps.Q = plan.qseg;
+    ps.nc = plan.nseg;
+    float* states = static_cast<float*>(workspace);
+    float* decays = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                             (sizeof(float) * (size_t)p.B * p.H * plan.nseg * p.N * p.P + 255) /
+                                                 256 * 256);
+    cudaError_t e = launch_segment_states(ps, states, decays, st);
+    if (e != cudaSuccess) return e;
+    Problem pc = ps;  // the combine reads one decay per segment
+    pc.Q = 1;
+    e = launch_state_passing(pc, states, decays, init, states, final_state, st);
+    if (e != cudaSuccess) return e;
+    return launch_segment_scan(ps, states, st);
+  }
   return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, nullptr, st);
 }
 
@@ -861,6 +977,18 @@ cudaError_t launch_fused(const Problem& p, const float* init, float* final_state
 cudaError_t launch_fused_normed(const Problem& p, const float* init, float* final_state, const NormIO& norm,
                                 cudaStream_t st) {
   return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, nullptr, st, 0, &norm);
+}
+
+// Segments of long sequences (p.Q = the segment length, a multiple of 128):
+// the end state of every segment from a zero start and the segment's total
+// log-decay, with the lean kernel (dt scanned in the kernel) ...
+cudaError_t launch_segment_states(const Problem& p, float* states, float* seg_decay, cudaStream_t st) {
+  return launch_mode(p, fused::MODE_CHUNK_STATE, nullptr, nullptr, states, nullptr, nullptr, st, 0, nullptr,
+                     seg_decay);
+}
+// ... and each segment's outputs from its start state prev[b,h,c].
+cudaError_t launch_segment_scan(const Problem& p, const float* prev, cudaStream_t st) {
+  return launch_mode(p, fused::MODE_CHUNK_SCAN, nullptr, prev, nullptr, p.y, nullptr, st);
 }
 
 // Step 2 on tensor cores: one CTA per (batch, head, chunk), zero start, the
@@ -877,14 +1005,14 @@ cudaError_t launch_chunk_scan_tc(const Problem& p, const float* lam, const float
 
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
                                void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads,
-                               const NormIO* norm) {
+                               const NormIO* norm, float* seg_decay) {
   using namespace fused;
   // every pointer the mode reads must be present (the step entry points pass
   // only the tensors of their step)
   if (!p.x || !p.Bm) return cudaErrorInvalidValue;
   if (mode == MODE_SCAN && (!p.dt || !p.A || !p.Cm || !y)) return cudaErrorInvalidValue;
-  if (mode == MODE_CHUNK_STATE && (!lam || !final_state)) return cudaErrorInvalidValue;
-  if (mode == MODE_CHUNK_SCAN && (!lam || !init || !p.Cm || !y)) return cudaErrorInvalidValue;
+  if (mode == MODE_CHUNK_STATE && (!final_state || (!lam && (!p.dt || !p.A)))) return cudaErrorInvalidValue;
+  if (mode == MODE_CHUNK_SCAN && (!init || !p.Cm || !y || (!lam && (!p.dt || !p.A)))) return cudaErrorInvalidValue;
   // the chunk-state mode never uses C: its C tiles are read from B (valid memory)
   const void* cptr = (mode == MODE_CHUNK_STATE) ? p.Bm : p.Cm;
   CUtensorMap mx, mb, mc, my;
@@ -926,6 +1054,7 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   kp.sy = p.sy;
   kp.trace = trace;
   kp.withhold_loads = withhold_loads;
+  kp.seg_decay = seg_decay;
   kp.ss_in = (norm && mode == MODE_SCAN) ? norm->ss_in : nullptr;
   kp.ss_out = (norm && mode == MODE_SCAN) ? norm->ss_out : nullptr;
   kp.sss = norm ? norm->batch_stride : 0;
@@ -939,24 +1068,32 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   if (e != cudaSuccess) return e;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set.load() & bit)) {
-    const void* fns[4] = {(const void*)k_ssd_fused<false, false>, (const void*)k_ssd_fused<true, false>,
-                          (const void*)k_ssd_fused<false, true>, (const void*)k_ssd_fused<true, true>};
-    for (int i = 0; i < 4 && e == cudaSuccess; ++i)
+    const void* fns[6] = {(const void*)k_ssd_fused<false, false, false>, (const void*)k_ssd_fused<true, false, false>,
+                          (const void*)k_ssd_fused<false, true, false>, (const void*)k_ssd_fused<true, true, false>,
+                          (const void*)k_ssd_fused<false, false, true>, (const void*)k_ssd_fused<true, false, true>};
+    for (int i = 0; i < 6 && e == cudaSuccess; ++i)
       e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set.fetch_or(bit);
   }
   const int64_t ctas = mode == fused::MODE_SCAN ? p.B * p.H : p.B * p.H * p.nc;
-  const bool xdt = p.input_dt && mode == fused::MODE_SCAN, nrm = kp.ss_in != nullptr || kp.ss_out != nullptr;
+  // the dt-scaled input whenever dt is read here (the whole scan, and the step
+  // modes without a step-1 output); lean: the chunk-state mode of segments
+  const bool xdt = p.input_dt && (mode == fused::MODE_SCAN || !lam), nrm = kp.ss_in != nullptr || kp.ss_out != nullptr;
+  const bool lean = mode == fused::MODE_CHUNK_STATE && seg_decay != nullptr;
   const dim3 grid((unsigned)ctas);
-  if (xdt && nrm)
-    k_ssd_fused<true, true><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+  if (lean && xdt)
+    k_ssd_fused<true, false, true><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+  else if (lean)
+    k_ssd_fused<false, false, true><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+  else if (xdt && nrm)
+    k_ssd_fused<true, true, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
   else if (xdt)
-    k_ssd_fused<true, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+    k_ssd_fused<true, false, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
   else if (nrm)
-    k_ssd_fused<false, true><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+    k_ssd_fused<false, true, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
   else
-    k_ssd_fused<false, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+    k_ssd_fused<false, false, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
   return cudaGetLastError();
 }
 

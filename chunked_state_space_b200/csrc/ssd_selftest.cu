@@ -237,5 +237,6 @@ extern "C" ssd_status ssd_selftest_carry_timeout(const ssd_dims* d, const void* 
 extern "C" ssd_status ssd_selftest_set_segments(int nseg) {
   if (nseg < 0) return SSD_ERR_INVALID_ARG;
   ssd::set_pair_segments(nseg);
+  ssd::set_fused_segments(nseg);
   return SSD_OK;
 }

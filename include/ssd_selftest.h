@@ -102,6 +102,9 @@ ssd_status ssd_selftest_carry_timeout(const ssd_dims* d, const void* x, const fl
  * each sequence into for the following launches of this process (host state,
  * not thread-safe): nseg > 0 wherever nseg divides the sequence's 128-token
  * sub-chunks (else whole sequences), 0 = chosen from the shape (the default).
+ * It also forces the one-head kernel's segmented form (three launches: the
+ * segments' end states, their combine, the segments' scans) with about nseg
+ * segments of whole sub-chunks, whatever the problem's size.
  * With fewer head pairs than SMs a forced segmentation puts a segment and its
  * predecessor in the same round, so the later one waits for the earlier one:
  * correct, slower.  Returns SSD_ERR_INVALID_ARG for nseg < 0.

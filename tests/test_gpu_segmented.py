@@ -1,0 +1,70 @@
+"""The one-head kernel's segmented form for problems with fewer (batch, head)
+sequences than SMs: the segments' end states from a zero start (the lean
+kernel: x, B, X', b_intra and the state recursion only), their ordered
+combine into each segment's start state (the chunk decomposition of
+"分块推理…" §2.1-§2.2 with a segment as the chunk), and the full scan of every
+segment from its start state.  Compared with the fp64 oracle; the segment
+boundaries fall inside the page's Q-token chunks and at ragged ends."""
+import contextlib
+
+import pytest
+import torch
+
+import oracle
+from chunked_state_space_b200 import inputs, ssd
+from gpu_util import TOL, device_inputs, oracle_args, rel_err, to_np64
+
+pytestmark = pytest.mark.gpu
+
+
+@contextlib.contextmanager
+def segments(n):
+    ssd.ssd_selftest_set_segments(n)
+    try:
+        yield
+    finally:
+        ssd.ssd_selftest_set_segments(0)
+
+
+def _run(dev, wl, input_dt=False):
+    y, fin = ssd.ssd_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
+                              chunk=wl.chunk, input_dt=input_dt)
+    torch.cuda.synchronize()
+    return y, fin
+
+
+@pytest.mark.parametrize("over,nseg", [
+    (dict(batch=2, seqlen=4096, nheads=24, ngroups=1, init_var=0.1), 0),   # the 130M layer: the cost model's choice
+    (dict(batch=1, seqlen=1000, nheads=4, ngroups=2, init_var=0.1), 3),    # ragged: 8 sub-chunks in 3 segments
+    (dict(batch=2, seqlen=2048, nheads=6, ngroups=3), 16),                 # one sub-chunk per segment
+    (dict(batch=1, seqlen=300, nheads=2, ngroups=1, chunk=128, init_var=0.1), 2),  # Q = 128, short last segment
+])
+@pytest.mark.parametrize("input_dt", [False, True])
+def test_segmented_scan_matches_oracle(over, nseg, input_dt):
+    wl = inputs.custom("mamba2_130m_layer", **over)
+    host = inputs.generate(wl)
+    dev = device_inputs(host)
+    with segments(nseg):
+        dims = ssd.make_dims(dev["x"], dev["B"], wl.chunk, input_dt)
+        path, kernels = ssd.ssd_scan_path(dims)
+        assert path == "fused" and kernels == 3  # the segmented form
+        y, fin = _run(dev, wl, input_dt)
+    y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host), input_dt=input_dt)
+    assert rel_err(to_np64(y), y_ref) <= TOL["bf16"]
+    assert rel_err(to_np64(fin), f_ref) <= TOL["bf16"]
+    assert ssd.ssd_read_device_status() == 0
+
+
+def test_segmented_and_whole_sequences_agree():
+    """The same problem through the segmented form and through one CTA per
+    sequence (the strided entry point has no workspace): equal to within the
+    bf16 rounding of the start states the segmented form hands over."""
+    wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=4096, nheads=24, ngroups=1, init_var=0.1)
+    dev = device_inputs(inputs.generate(wl))
+    y, fin = _run(dev, wl)
+    assert ssd.ssd_scan_path(ssd.make_dims(dev["x"], dev["B"], wl.chunk))[1] == 3
+    ys, fs = ssd.ssd_scan_fwd_strided(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
+                                      chunk=wl.chunk)
+    torch.cuda.synchronize()
+    assert rel_err(to_np64(y), to_np64(ys)) <= 5e-3
+    assert rel_err(to_np64(fin), to_np64(fs)) <= 1e-4

@@ -329,6 +329,29 @@ def test_vertical_small(L, V):
     _check_end_to_end(f(x0h), layers64, eps, to_np64(yv), tag=f"3-layer stack L={L} V={V}")
 
 
+@pytest.mark.parametrize("nheads,seqlen", [(6, 1000), (36, 300)])
+def test_normed_scan_chains_two_layers(nheads, seqlen):
+    """ssd_scan_fwd_normed on head counts that are not a multiple of 4 (the
+    scalar sums path) and above 32 (sums past the prefetched first 32 heads),
+    with a ragged sequence: layer 1's y against the oracle on the input it sees
+    (layer 0's stored y, normalised by the oracle), and the sums layer 0 passes
+    on against those of its stored y."""
+    wl = inputs.custom("stack24_vertical", batch=2, seqlen=seqlen, nheads=nheads, ngroups=2)
+    host_layers, dev_layers = _stack_layers(wl, 2)
+    x0h = inputs.generate(wl, names=("x",))["x"]
+    x0 = to_dev(x0h)
+    states = [torch.zeros((wl.batch, wl.nheads, wl.dstate, wl.headdim), device="cuda") for _ in range(2)]
+    eps = 1e-6
+    ys, sums = _horizontal_normed(x0, dev_layers, states, wl, eps)
+    np.testing.assert_allclose(to_np64(sums[1]), np.sum(to_np64(ys[0]) ** 2, axis=-1), rtol=1e-5, atol=0)
+    f = inputs.to_f64
+    h = host_layers[1]
+    y_ref, f_ref = oracle.scan_recurrence(oracle.rmsnorm(to_np64(ys[0]), eps), f(h["dt"]), f(h["A"]), f(h["B"]),
+                                          f(h["C"]), f(h["D"]), None)
+    assert rel_err(to_np64(ys[1]), y_ref) <= TOL["bf16"]
+    assert rel_err(to_np64(states[1]), f_ref) <= TOL["bf16"]
+
+
 def test_vertical_two_heads_keeps_the_norm_pass():
     """With two heads per CTA the stack keeps the norm as its own pass
     (ssd_rmsnorm between layers, the normalised input stored in bf16): vertical

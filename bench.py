@@ -102,17 +102,19 @@ def kernel_source_hash(kernel: str = "ssd_fused") -> str:
     return h.hexdigest()[:16]
 
 
-def traffic_from_profile(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources; else None."""
+def traffic_from_profile(kernel: str, wl=None):
+    """DRAM bytes per step of a workload from the committed ncu summary
+    (profiles/traffic.json, keyed "kernel/workload"), if it was taken on the
+    current kernel sources at this workload's sizes; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     try:
         with open(path) as f:
             t = json.load(f)
-        ent = t.get(kernel)
-        if ent and ent.get("source_hash") == kernel_source_hash(kernel):
+        ent = t.get(f"{kernel}/{wl.name}" if wl is not None else kernel)
+        if ent and ent.get("source_hash") == kernel_source_hash(kernel) and (
+                wl is None or ent.get("shape") == [wl.batch, wl.seqlen, wl.nheads]):
             return float(ent["dram_bytes_per_launch"])
     except Exception:
         return None
@@ -256,6 +258,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--batch", type=int, default=None, help="override the batch size (profiling runs)")
+    ap.add_argument("--seqlen", type=int, default=None, help="override the sequence length (profiling runs)")
     ap.add_argument("--vblock", type=int, default=None, help="override the vertical block V (layer stacks)")
     ap.add_argument("--input-dt", action="store_true",
                     help="the dt-scaled input variant (SSD_FLAG_INPUT_DT)")
@@ -292,11 +295,8 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    wl = inputs.WORKLOADS[args.workload]
-    if args.batch:
-        wl = inputs.custom(wl.name, batch=args.batch)
-    if args.vblock:
-        wl = inputs.custom(wl.name, batch=wl.batch, vblock=args.vblock)
+    over = {k: v for k, v in (("batch", args.batch), ("seqlen", args.seqlen), ("vblock", args.vblock)) if v}
+    wl = inputs.custom(args.workload, **over) if over else inputs.WORKLOADS[args.workload]
     if wl.n_layers > 1:
         return run_stack(args, wl, dev, rank, world)
     if args.decode:
@@ -376,13 +376,19 @@ def main():
     e2e_value = tokens / (e2e_ms * 1e-3)
 
     hbm_peak, tc_peak, tc_sust, peak_src = load_peaks()
-    kernel_ms = statistics.mean(per_step) if path in ssd.FUSED_PATHS and kernels_per_step == 1 else None
+    # the fused path: one launch, or the segmented form's three (lean pass,
+    # combine, full pass), timed together as one step
+    kernel_ms = statistics.mean(per_step) if path in ssd.FUSED_PATHS and not args.unfused else None
     roofline = None
     if kernel_ms is not None:
         kname = PATH_KERNEL[path]
+        label = "k_" + kname
+        if kernels_per_step > 1:
+            label += (" segmented form, whole step: lean pass (k_ssd_fused<.., LEAN>), k_state_passing, "
+                      "full pass (k_ssd_fused)")
         ach = algorithmic_bytes(wl) / (kernel_ms * 1e-3) / 1e9
         roofline = {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
-                    "traffic": traffic_from_profile(kname), "kernel": "k_" + kname,
+                    "traffic": traffic_from_profile(kname, wl), "kernel": label,
                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else
                     "fallback 6650 GB/s",
                     "tensor_tflops": algorithmic_flops(wl) / (kernel_ms * 1e-3) / 1e12,

@@ -77,8 +77,15 @@ struct Params {
   int input_dt;       // the input term is dt_t B_t x_t^T
   const float* A;
   const float* D;
-  const float* init;
-  float* final_state;
+  const float* init;         // whole-sequence CTAs: [B*H][N][P] initial states, or NULL
+  float* final_state;        // whole-sequence CTAs: [B*H][N][P] final states, or NULL
+  const float* chunk_init;   // chunk-scan CTAs: [slots][N][P] start state of each chunk
+  float* chunk_final;        // chunk-state CTAs: [slots][N][P] end state of each chunk
+  // Grid layout: the first `whole` CTAs scan sequences 0..whole-1 whole (step
+  // modes with whole > 0 are mixed grids); the rest run the step mode over
+  // sequences seq0, seq0+1, ..., one CTA per chunk, chunk slot
+  // (sequence - seq0) * nc + chunk.
+  int64_t whole, seq0;
   const __nv_bfloat16* x;
   int64_t sx, ldx;    // batch and token strides of x
   __nv_bfloat16* y;
@@ -216,17 +223,18 @@ __global__ void __launch_bounds__(THREADS, 1)
   Ctl ctl{bar, abort_flag};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool chunked = p.mode != MODE_SCAN;
-  const int64_t bh = chunked ? (int64_t)blockIdx.x / p.nc : (int64_t)blockIdx.x;
-  const int64_t cidx = chunked ? (int64_t)blockIdx.x % p.nc : 0;   // chunk of this CTA (step modes)
+  const bool chunked = p.mode != MODE_SCAN && (int64_t)blockIdx.x >= p.whole;
+  const int64_t cb = (int64_t)blockIdx.x - p.whole;                // chunk CTA index (step modes)
+  const int64_t bh = chunked ? p.seq0 + cb / p.nc : (int64_t)blockIdx.x;
+  const int64_t cidx = chunked ? cb % p.nc : 0;                    // chunk of this CTA (step modes)
   const int b = (int)(bh / p.H), h = (int)(bh % p.H);
   const int g = h / (p.H / p.G);
   const int t_base = (int)(cidx * p.Q);                          // first token of this CTA
   const int nsub = chunked ? (int)ceil_div(min((int64_t)p.Q, p.L - t_base), (int64_t)T) : p.nsub;
-  const int64_t cslot = bh * p.nc + cidx;                       // [B,H,nc] index (step modes)
-  const float* init_ptr = chunked ? (p.mode == MODE_CHUNK_SCAN ? p.init + cslot * NS * P : nullptr)
+  const int64_t cslot = (bh - p.seq0) * p.nc + cidx;            // chunk slot (step modes)
+  const float* init_ptr = chunked ? (p.mode == MODE_CHUNK_SCAN ? p.chunk_init + cslot * NS * P : nullptr)
                                   : (p.init ? p.init + bh * NS * P : nullptr);
-  float* final_ptr = chunked ? (p.mode == MODE_CHUNK_STATE ? p.final_state + cslot * NS * P : nullptr)
+  float* final_ptr = chunked ? (p.mode == MODE_CHUNK_STATE ? p.chunk_final + cslot * NS * P : nullptr)
                              : (p.final_state ? p.final_state + bh * NS * P : nullptr);
   unsigned long long* const trace = (p.trace && blockIdx.x == 0) ? p.trace : nullptr;
   auto mark = [&](int j, int ev) {
@@ -873,52 +881,92 @@ bool tc_supported(const Problem& p) { return fused_supported(p) && p.B * p.H * p
 
 bool uses_pair_kernel(const Problem& p) { return p.two_heads && pair_supported(p); }
 
-// Segments for problems with fewer (batch, head) sequences than SMs: one CTA
-// per sequence would leave SMs idle, so every sequence is cut into nseg
-// segments of Qseg tokens and the scan runs in three launches (the page's
-// chunk decomposition one level up, "分块推理…" §2.1-§2.2, with a segment as the
-// chunk): the lean kernel forms each segment's end state from a zero start and
-// its total log-decay, k_state_passing combines them in order into each
-// segment's start state (and the final state), and the full kernel scans every
-// segment from its start state.  Chosen only where a cost model of rounds of
-// CTAs (a lean segment costing about a third of a full one) predicts a gain.
+// Segments, where one CTA per (batch, head) sequence would leave SMs idle:
+// with fewer sequences than SMs, or with B*H = q*SMs + r sequences whose last
+// r run as a partial round of CTAs while the other SMs have nothing left.
+// The first `whole` sequences run whole (one CTA each); every later one is
+// cut into nseg segments of qseg tokens (the page's chunk decomposition one
+// level up, "分块推理…" §2.1-§2.2, with a segment as the chunk).  Three launches:
+// the lean kernel forms each segment's end state from a zero start and its
+// total log-decay, k_state_passing combines them in order into each
+// segment's start state (and the sequence's final state), and the full
+// kernel runs the whole sequences first and then every segment from its
+// start state, so the short segment CTAs fill the SMs that the last whole
+// ones leave free.  Chosen only where a cost model of CTA rounds (a lean
+// segment costing about a third of a full one) predicts a gain.
 struct SegPlan {
-  int nseg;      // 1: whole sequences in one launch
-  int64_t qseg;  // segment length in tokens (a multiple of 128)
+  int nseg;       // 1: whole sequences in one launch
+  int64_t qseg;   // segment length in tokens (a multiple of 128)
+  int64_t whole;  // sequences 0..whole-1 run whole; the rest are segmented
 };
-static int g_fused_segments = 0;  // forced by a self-test (0: the cost model decides)
-void set_fused_segments(int nseg) { g_fused_segments = nseg > 0 ? nseg : 0; }
+static int g_fused_segments = 0;         // forced by a self-test (0: the cost model decides)
+static int64_t g_fused_whole = 0;        // sequences run whole when the segment count is forced
+void set_fused_segments(int nseg) { set_fused_split(nseg, 0); }
+void set_fused_split(int nseg, int64_t whole) {
+  g_fused_segments = nseg > 0 ? nseg : 0;
+  g_fused_whole = whole > 0 ? whole : 0;
+}
+
+// Finish time, in sub-chunk periods, of `nw` CTAs of cost w followed by `ns`
+// CTAs of cost s on `nsm` SMs, each CTA starting on the SM that frees first
+// (CTAs start in grid order).
+static double makespan(int64_t nsm, int64_t nw, double w, int64_t ns, double s) {
+  const int64_t q = nw / nsm, r = nw % nsm;  // r SMs run one more whole CTA
+  const double t0 = q * w, t1 = t0 + w;
+  const int64_t a = nsm - r;                // SMs free at t0
+  if (r == 0) return t0 + (double)ceil_div(ns, nsm) * s;
+  // segments first go to the a SMs free at t0, until those pass t1 ...
+  const int64_t m = (int64_t)std::ceil(w / s);
+  if (ns <= a * m) return std::max(t1, t0 + (double)ceil_div(ns, a) * s);
+  // ... then to every SM in turn, the r SMs free at t1 first
+  const int64_t n2 = ns - a * m, k = n2 / nsm, e = n2 % nsm;
+  return std::max(t0 + (m + k + (e > r ? 1 : 0)) * s, t1 + (k + (e > 0 ? 1 : 0)) * s);
+}
+
 static SegPlan seg_plan(const Problem& p) {
-  SegPlan plan{1, 0};
-  if (uses_pair_kernel(p) || !fused_supported(p)) return plan;
   const int64_t nsub = ceil_div(p.L, (int64_t)fused::T), bh = p.B * p.H;
+  SegPlan plan{1, 0, bh};
+  if (uses_pair_kernel(p) || !fused_supported(p)) return plan;
   const int64_t nsm = split::sm_count();
-  auto make = [&](int64_t n) {
+  auto make = [&](int64_t n, int64_t whole) {
     const int64_t seg = ceil_div(nsub, n);
-    return SegPlan{(int)ceil_div(nsub, seg), seg * fused::T};
+    return SegPlan{(int)ceil_div(nsub, seg), seg * fused::T, whole};
   };
   if (g_fused_segments > 0) {
-    const SegPlan f = make(g_fused_segments);
-    return (f.nseg > 1 && bh * f.nseg < (1ll << 31)) ? f : plan;
+    const SegPlan f = make(g_fused_segments, std::min(g_fused_whole, bh - 1));
+    const bool ok = f.nseg > 1 && (bh - f.whole) * f.nseg < (1ll << 31) && (f.whole == 0 || bh - f.whole < 65536);
+    return ok ? f : plan;
   }
-  if (bh >= nsm || nsub < 8) return plan;
-  const double plain = (double)ceil_div(bh, nsm) * (double)(nsub + 2);
-  double best = 0.9 * plain;
+  if (nsub < 8) return plan;
+  // cost in sub-chunk periods: a CTA costs its sub-chunks plus about two of
+  // pipeline fill and drain; a lean segment about 0.35 of a full one, plus
+  // one period for the combine launch
+  const double w = (double)(nsub + 2);
+  const double plain = (double)ceil_div(bh, nsm) * w;
+  const int64_t whole = bh >= nsm ? bh - bh % nsm : 0;  // full rounds stay whole
+  if (whole == bh) return plan;
+  const double gain = whole > 0 ? 0.95 : 0.9;
+  double best = gain * plain;
   for (int64_t n = 2; n <= 64 && n <= nsub / 4; ++n) {
-    const SegPlan c = make(n);
-    const double seg = (double)(c.qseg / fused::T), rounds = (double)ceil_div(bh * c.nseg, nsm);
-    const double cost = rounds * (seg + 2.0) + rounds * (0.35 * seg + 1.5) + 1.0;
-    if (c.nseg > 1 && cost < best) {
+    const SegPlan c = make(n, whole);
+    const int64_t segs = (bh - whole) * c.nseg;
+    const double seg = (double)(c.qseg / fused::T);
+    const double cost = makespan(nsm, whole, w, segs, seg + 2.0) +
+                        (double)ceil_div(segs, nsm) * (0.35 * seg + 1.5) + 1.0;
+    if (c.nseg > 1 && segs < (1ll << 31) && cost < best) {
       best = cost;
       plan = c;
     }
   }
   return plan;
 }
+static size_t seg_states_bytes(const Problem& p, const SegPlan& plan) {
+  const size_t states = sizeof(float) * (size_t)(p.B * p.H - plan.whole) * plan.nseg * p.N * p.P;
+  return (states + 255) / 256 * 256;
+}
 static size_t seg_workspace_bytes(const Problem& p, const SegPlan& plan) {
   if (plan.nseg <= 1) return 0;
-  const size_t states = sizeof(float) * (size_t)p.B * p.H * plan.nseg * p.N * p.P;
-  return (states + 255) / 256 * 256 + sizeof(float) * (size_t)p.B * p.H * plan.nseg;
+  return seg_states_bytes(p, plan) + sizeof(float) * (size_t)(p.B * p.H - plan.whole) * plan.nseg;
 }
 
 // Kernel launches of one fused call: three for the segmented form.
@@ -932,9 +980,19 @@ size_t tc_workspace_bytes(const Problem& p) {
   return seg_workspace_bytes(p, seg_plan(p));
 }
 
+// The grid of a launch: `whole` leading CTAs scan whole sequences from init
+// to final_state; the step-mode CTAs cover the chunks of sequences seq0 on,
+// reading start states from chunk_init or writing end states to chunk_final.
+struct GridSplit {
+  int64_t whole = 0, seq0 = 0;
+  const float* init = nullptr;
+  float* final_state = nullptr;
+};
+
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
                                void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads = 0,
-                               const NormIO* norm = nullptr, float* seg_decay = nullptr);
+                               const NormIO* norm = nullptr, float* seg_decay = nullptr,
+                               const GridSplit& split = GridSplit());
 
 cudaError_t launch_fused_traced(const Problem& p, const float* init, float* final_state, unsigned long long* trace,
                                 cudaStream_t st) {
@@ -955,17 +1013,24 @@ cudaError_t launch_fused(const Problem& p, const float* init, float* final_state
     Problem ps = p;  // segments as the chunks of the step modes
     ps.Q = plan.qseg;
     ps.nc = plan.nseg;
+    const int64_t w = plan.whole, NP = p.N * p.P;
     float* states = static_cast<float*>(workspace);
-    float* decays = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                             (sizeof(float) * (size_t)p.B * p.H * plan.nseg * p.N * p.P + 255) /
-                                                 256 * 256);
-    cudaError_t e = launch_segment_states(ps, states, decays, st);
+    float* decays = reinterpret_cast<float*>(static_cast<char*>(workspace) + seg_states_bytes(p, plan));
+    cudaError_t e = launch_segment_states(ps, w, states, decays, st);
     if (e != cudaSuccess) return e;
-    Problem pc = ps;  // the combine reads one decay per segment
+    // the combine reads one decay per segment, over the segmented sequences
+    // only (with whole > 0 as one batch of B*H - whole heads, fewer than
+    // 65536 by the plan)
+    Problem pc = ps;
     pc.Q = 1;
-    e = launch_state_passing(pc, states, decays, init, states, final_state, st);
+    if (w > 0) {
+      pc.B = 1;
+      pc.H = p.B * p.H - w;
+    }
+    e = launch_state_passing(pc, states, decays, init ? init + w * NP : nullptr, states,
+                             final_state ? final_state + w * NP : nullptr, st);
     if (e != cudaSuccess) return e;
-    return launch_segment_scan(ps, states, st);
+    return launch_segment_scan(ps, w, states, init, final_state, st);
   }
   return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, nullptr, st);
 }
@@ -979,16 +1044,27 @@ cudaError_t launch_fused_normed(const Problem& p, const float* init, float* fina
   return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, nullptr, st, 0, &norm);
 }
 
-// Segments of long sequences (p.Q = the segment length, a multiple of 128):
-// the end state of every segment from a zero start and the segment's total
+// Segments of long sequences (p.Q = the segment length, a multiple of 128;
+// sequences `whole` on, slot (sequence - whole) * nc + segment): the end
+// state of every segment from a zero start and the segment's total
 // log-decay, with the lean kernel (dt scanned in the kernel) ...
-cudaError_t launch_segment_states(const Problem& p, float* states, float* seg_decay, cudaStream_t st) {
+cudaError_t launch_segment_states(const Problem& p, int64_t whole, float* states, float* seg_decay,
+                                  cudaStream_t st) {
+  GridSplit sp;
+  sp.seq0 = whole;
   return launch_mode(p, fused::MODE_CHUNK_STATE, nullptr, nullptr, states, nullptr, nullptr, st, 0, nullptr,
-                     seg_decay);
+                     seg_decay, sp);
 }
-// ... and each segment's outputs from its start state prev[b,h,c].
-cudaError_t launch_segment_scan(const Problem& p, const float* prev, cudaStream_t st) {
-  return launch_mode(p, fused::MODE_CHUNK_SCAN, nullptr, prev, nullptr, p.y, nullptr, st);
+// ... and the outputs: sequences 0..whole-1 whole (from init, to
+// final_state), then every segment from its start state prev[slot].
+cudaError_t launch_segment_scan(const Problem& p, int64_t whole, const float* prev, const float* init,
+                                float* final_state, cudaStream_t st) {
+  GridSplit sp;
+  sp.whole = whole;
+  sp.seq0 = whole;
+  sp.init = init;
+  sp.final_state = final_state;
+  return launch_mode(p, fused::MODE_CHUNK_SCAN, nullptr, prev, nullptr, p.y, nullptr, st, 0, nullptr, nullptr, sp);
 }
 
 // Step 2 on tensor cores: one CTA per (batch, head, chunk), zero start, the
@@ -1005,7 +1081,7 @@ cudaError_t launch_chunk_scan_tc(const Problem& p, const float* lam, const float
 
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
                                void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads,
-                               const NormIO* norm, float* seg_decay) {
+                               const NormIO* norm, float* seg_decay, const GridSplit& split) {
   using namespace fused;
   // every pointer the mode reads must be present (the step entry points pass
   // only the tensors of their step)
@@ -1045,8 +1121,15 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   kp.input_dt = p.input_dt;
   kp.A = p.A;
   kp.D = p.D;
-  kp.init = init;
-  kp.final_state = final_state;
+  // whole-sequence CTAs take init / final_state; the step modes' CTAs their
+  // chunk states (mixed grids: both)
+  const bool step_mode = mode != MODE_SCAN;
+  kp.init = step_mode ? split.init : init;
+  kp.final_state = step_mode ? split.final_state : final_state;
+  kp.chunk_init = mode == MODE_CHUNK_SCAN ? init : nullptr;
+  kp.chunk_final = mode == MODE_CHUNK_STATE ? final_state : nullptr;
+  kp.whole = step_mode ? split.whole : 0;
+  kp.seq0 = step_mode ? split.seq0 : 0;
   kp.x = static_cast<const __nv_bfloat16*>(p.x);
   kp.sx = p.sx;
   kp.ldx = p.ldx;
@@ -1076,7 +1159,9 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
     if (e != cudaSuccess) return e;
     attr_set.fetch_or(bit);
   }
-  const int64_t ctas = mode == fused::MODE_SCAN ? p.B * p.H : p.B * p.H * p.nc;
+  const int64_t ctas = mode == fused::MODE_SCAN ? p.B * p.H : kp.whole + (p.B * p.H - kp.seq0) * p.nc;
+  if (kp.whole < 0 || kp.whole > kp.seq0 || kp.seq0 > p.B * p.H || ctas <= 0 || ctas >= (1ll << 31))
+    return cudaErrorInvalidValue;
   // the dt-scaled input whenever dt is read here (the whole scan, and the step
   // modes without a step-1 output); lean: the chunk-state mode of segments
   const bool xdt = p.input_dt && (mode == fused::MODE_SCAN || !lam), nrm = kp.ss_in != nullptr || kp.ss_out != nullptr;

@@ -240,3 +240,11 @@ extern "C" ssd_status ssd_selftest_set_segments(int nseg) {
   ssd::set_fused_segments(nseg);
   return SSD_OK;
 }
+
+// The one-head kernel's segmented form for the following launches: the first
+// `whole` sequences whole, every later one in about nseg segments.
+extern "C" ssd_status ssd_selftest_set_split(int nseg, int64_t whole) {
+  if (nseg < 0 || whole < 0) return SSD_ERR_INVALID_ARG;
+  ssd::set_fused_split(nseg, whole);
+  return SSD_OK;
+}

@@ -28,12 +28,16 @@ cudaError_t launch_chunk_scan_tc(const Problem& p, const float* lam, const float
 // the shape (the default), n > 0 = n wherever n divides the sub-chunks
 // (self-tests of the carries).
 void set_pair_segments(int nseg);
-// Segments per sequence of the one-head kernel's segmented form for problems
-// with fewer sequences than SMs: 0 = chosen by its cost model, n > 0 = about
-// n segments whatever the size (self-tests).
+// Segments per sequence of the one-head kernel's segmented form (problems
+// with fewer sequences than SMs, or the last partial round of sequences):
+// 0 = chosen by its cost model, n > 0 = about n segments whatever the size,
+// with the first `whole` sequences run whole (self-tests).
 void set_fused_segments(int nseg);
-cudaError_t launch_segment_states(const Problem& p, float* states, float* seg_decay, cudaStream_t st);
-cudaError_t launch_segment_scan(const Problem& p, const float* prev, cudaStream_t st);
+void set_fused_split(int nseg, int64_t whole);
+cudaError_t launch_segment_states(const Problem& p, int64_t whole, float* states, float* seg_decay,
+                                  cudaStream_t st);
+cudaError_t launch_segment_scan(const Problem& p, int64_t whole, const float* prev, const float* init,
+                                float* final_state, cudaStream_t st);
 // The whole scan in one launch.  With a workspace of pair_workspace_bytes
 // the two-head kernel runs segments of the sequences round-robin on one
 // persistent CTA per SM; without one (NULL / too small) every CTA runs whole

@@ -111,6 +111,22 @@ ssd_status ssd_selftest_carry_timeout(const ssd_dims* d, const void* x, const fl
  */
 ssd_status ssd_selftest_set_segments(int nseg);
 
+/*
+ * ssd_selftest_set_split forces the one-head kernel's segmented form for the
+ * following launches of this process (host state, not thread-safe), in its
+ * mixed layout: the first `whole` (batch, head) sequences (in batch-major
+ * order) are scanned whole by one CTA each, from the caller's initial state
+ * to its final state, and every later sequence is cut into about nseg
+ * segments of whole 128-token sub-chunks (end states, combine, segment
+ * scans).  whole is clamped to B*H - 1; nseg = 0 restores the cost model's
+ * choice (which uses this layout when B*H exceeds a whole number of rounds
+ * of CTAs on the SMs by a partial round).  The two-head kernel is not
+ * affected.  Returns SSD_ERR_INVALID_ARG for nseg < 0 or whole < 0.
+ * Same arithmetic as the default path: results equal one CTA per sequence
+ * up to the rounding of the segments' combine.
+ */
+ssd_status ssd_selftest_set_split(int nseg, int64_t whole);
+
 #ifdef __cplusplus
 }
 #endif

@@ -264,6 +264,8 @@ def main():
                     help="the dt-scaled input variant (SSD_FLAG_INPUT_DT)")
     ap.add_argument("--strided", action="store_true",
                     help="x, B, C as column slices of one fused [B, L, H*P + 2*G*N] tensor (ssd_scan_fwd_strided)")
+    ap.add_argument("--vdecay", action="store_true",
+                    help="the scan with a vector-valued decay (one rate per state channel) on the workload's shapes")
     ap.add_argument("--decode", action="store_true",
                     help="time the decode step ssd_step (one token per call, state in place) at the workload's "
                          "batch, heads and sizes instead of the scan")
@@ -301,6 +303,8 @@ def main():
         return run_stack(args, wl, dev, rank, world)
     if args.decode:
         return run_decode(args, wl, dev, rank, world)
+    if args.vdecay:
+        return run_vdecay(args, wl, dev, rank, world)
     if args.split == "sequence":
         return run_sequence_split(args, wl, dev, rank, world)
     host = inputs.generate(wl, seed=rank_seed(rank))  # each rank: its own independent batch
@@ -515,6 +519,107 @@ def run_decode(args, wl, dev, rank, world):
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def run_vdecay(args, wl, dev, rank, world):
+    """The scan with a vector-valued decay, one rate per state channel
+    (ssd_scan_fwd_vdecay, a_t[n] = exp(dt_t Av[h, n])), on the workload's
+    shapes.  The token recurrence on CUDA cores: per state entry and token a
+    product b x, a fused multiply-add a h + b x and one into y (5 flops), so the
+    roofline is the fp32 pipe: SMs x 128 lanes x 2 flops x the SM clock."""
+    import torch
+    from chunked_state_space_b200 import inputs, ssd
+    Bz, L, H, P, N = wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.dstate
+    host = inputs.generate(wl, seed=rank_seed(rank))
+    host["Av"] = inputs.generate(wl, seed=rank_seed(rank), names=("Av",))["Av"]
+
+    def to_t(v):
+        return torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16 else torch.from_numpy(v)
+
+    pinned = {k: to_t(v).pin_memory() for k, v in host.items()}
+    del host
+    d = {k: v.to(dev) for k, v in pinned.items()}
+    y = torch.empty_like(d["x"])
+    fin = torch.empty_like(d["init"])
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev) if l2_resident(wl) else None
+
+    def step():
+        ssd.ssd_scan_fwd_vdecay(d["x"], d["dt"], d["Av"], d["B"], d["C"], d["D"], d["init"], y=y, final_state=fin,
+                                stream=stream)
+
+    per_step, ms_total, clk = timed_steps(step, args, stream, dev, dev.index, world, flush)
+    ms = ms_total / args.steps
+    tokens = Bz * L * world
+    # end to end: pinned host inputs to the device, the scan, y and the final state back, every step
+    h_y = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    h_fin = torch.empty(fin.shape, dtype=fin.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = y.numel() * y.element_size() + fin.numel() * fin.element_size()
+
+    def e2e_step():
+        for k, v in pinned.items():
+            d[k].copy_(v, non_blocking=True)
+        step()
+        h_y.copy_(y, non_blocking=True)
+        h_fin.copy_(fin, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(max(args.e2e_steps, 1)):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / max(args.e2e_steps, 1), dev)
+    flops = 5.0 * N * P * Bz * L * H
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = clk.get("sm_max_mhz") or 1965
+    peak = sms * 128 * 2 * mhz * 1e6 / 1e12
+    ach = flops / (statistics.mean(per_step) * 1e-3) / 1e12
+    line = {
+        "metric": "SSD scan tokens/s with a vector-valued decay (ssd_scan_fwd_vdecay, one rate per state channel)",
+        "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if wl.io == "f32" else "bf16 io, f32 state", "data": "synthetic",
+        "config": {"workload": wl.name + " vector decay", "batch": Bz, "seqlen": L, "nheads": H, "headdim": P,
+                   "dstate": N, "ngroups": wl.ngroups, "decay": "Av[h, n] = -exp(U[0, ln 16]) per (head, channel)",
+                   "l2": ("512 MB L2 flush between steps (inputs fit in L2); per-step events exclude it"
+                          if flush is not None else
+                          f"inputs larger than L2 ({algorithmic_bytes(wl) / 1e9:.2f} GB per rank); no flush")},
+        "clocks": clk, "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                               "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "alu", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                     "traffic": None, "kernel": "k_ssd_scan_vdecay64",
+                     "flops_per_launch": flops,
+                     "peak_source": f"{sms} SMs x 128 fp32 lanes x 2 flops x {mhz} MHz (unit counts, max SM clock)"},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_vdecay(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline_vdecay(wl):
+    """The oracle's per-channel-decay recurrence on one sequence of the
+    workload (all heads, full length), as it stands."""
+    import oracle
+    from chunked_state_space_b200 import inputs
+    one = inputs.custom(wl.name, batch=1)
+    host = inputs.generate(one, seed=1000)
+    av = inputs.generate(one, seed=1000, names=("Av",))["Av"]
+    args = [inputs.to_f64(host[k]) for k in ("x", "dt")] + [av.astype(np.float64)] + \
+        [inputs.to_f64(host[k]) for k in ("B", "C", "D", "init")]
+    del host
+    t0 = time.perf_counter()
+    oracle.scan_recurrence_vdecay(*args)
+    el = time.perf_counter() - t0
+    return {"value": wl.seqlen / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"1 of {wl.batch} sequences, full length {wl.seqlen}, all {wl.nheads} heads "
+                      f"(fp64 per-channel-decay token recurrence); {el:.1f} s"}
 
 
 def timed_steps(step, args, stream, dev, local, world, flush=None):

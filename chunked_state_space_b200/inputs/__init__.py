@@ -38,7 +38,7 @@ _SRC = os.path.join(_HERE, "ssdgen.c")
 _LIB_PATH = os.path.join(_HERE, "libssdgen.so")
 
 # tensor ids used in the stream keys
-TENSOR_IDS = {"x": 0, "dt": 1, "A": 2, "B": 3, "C": 4, "D": 5, "init": 6}
+TENSOR_IDS = {"x": 0, "dt": 1, "A": 2, "B": 3, "C": 4, "D": 5, "init": 6, "Av": 7}
 
 NORMAL, UNIFORM, SOFTPLUS_NORMAL, NEG_EXP_UNIFORM, CONSTANT = 0, 1, 2, 3, 4
 
@@ -149,6 +149,8 @@ def tensor_spec(wl: Workload, name: str):
         return (Bz, L, H), "f32", SOFTPLUS_NORMAL, wl.dt_shift, 1.0
     if name == "A":
         return (H,), "f32", NEG_EXP_UNIFORM, 0.0, math.log(16.0)
+    if name == "Av":  # the vector-valued decay's rates: one per (head, state channel), as A per head
+        return (H, N), "f32", NEG_EXP_UNIFORM, 0.0, math.log(16.0)
     if name in ("B", "C"):
         return (Bz, L, G, N), wl.io, NORMAL, 0.0, bc_std
     if name == "D":

@@ -30,6 +30,8 @@ def _av(H, N, seed, equal=False):
     ("tiny_f32", dict(batch=1, seqlen=1, nheads=2)),
     ("tiny_f32", dict(batch=1, seqlen=45, nheads=3, ngroups=3, headdim=5, dstate=7, init_var=0.3)),
     ("mamba2_130m_layer", dict(batch=2, seqlen=700, nheads=4, ngroups=2, init_var=0.1)),
+    ("tiny_f32", dict(batch=1, seqlen=100, nheads=2, headdim=64, dstate=64, init_var=0.3)),  # P 64, fp32 io
+    ("mamba2_130m_layer", dict(batch=1, seqlen=37, nheads=3, ngroups=3, dstate=48)),        # P 64, N 48
     ("mamba2_130m_layer", dict(batch=1, seqlen=257, nheads=2, headdim=12, dstate=100, init_var=0.1)),
 ])
 @pytest.mark.parametrize("equal", [False, True])

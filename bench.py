@@ -603,22 +603,29 @@ def run_vdecay(args, wl, dev, rank, world):
     return 0
 
 
-def cpu_baseline_vdecay(wl):
-    """The oracle's per-channel-decay recurrence on one sequence of the
-    workload (all heads, full length), as it stands."""
+def cpu_baseline_vdecay(wl, target_s: float = 10.0):
+    """The oracle's per-channel-decay recurrence, as it stands, on whole
+    sequences of the workload (all heads, full length) one after another until
+    about `target_s` seconds of CPU work, or the whole batch."""
     import oracle
     from chunked_state_space_b200 import inputs
     one = inputs.custom(wl.name, batch=1)
-    host = inputs.generate(one, seed=1000)
-    av = inputs.generate(one, seed=1000, names=("Av",))["Av"]
-    args = [inputs.to_f64(host[k]) for k in ("x", "dt")] + [av.astype(np.float64)] + \
-        [inputs.to_f64(host[k]) for k in ("B", "C", "D", "init")]
-    del host
-    t0 = time.perf_counter()
-    oracle.scan_recurrence_vdecay(*args)
-    el = time.perf_counter() - t0
-    return {"value": wl.seqlen / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"1 of {wl.batch} sequences, full length {wl.seqlen}, all {wl.nheads} heads "
+    av = inputs.generate(one, seed=1000, names=("Av",))["Av"].astype(np.float64)
+    tokens, el, nb = 0, 0.0, 0
+    for b in range(wl.batch):
+        host = inputs.generate(one, seed=1000 + b)
+        args = [inputs.to_f64(host[k]) for k in ("x", "dt")] + [av] + \
+            [inputs.to_f64(host[k]) for k in ("B", "C", "D", "init")]
+        del host
+        t0 = time.perf_counter()
+        oracle.scan_recurrence_vdecay(*args)
+        el += time.perf_counter() - t0
+        tokens += wl.seqlen
+        nb += 1
+        if el >= target_s:
+            break
+    return {"value": tokens / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{nb} of {wl.batch} sequences, full length {wl.seqlen}, all {wl.nheads} heads "
                       f"(fp64 per-channel-decay token recurrence); {el:.1f} s"}
 
 

@@ -85,7 +85,8 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {
-    "ssd_fused": ("ssd_fused.cu", "ssd_split.cuh", "ssd_common.cuh", "ssd_tc.cuh", "tma.cuh", "umma.cuh"),
+    "ssd_fused": ("ssd_fused.cu", "ssd_lean.cu", "ssd_split.cuh", "ssd_common.cuh", "ssd_tc.cuh", "tma.cuh",
+                  "umma.cuh"),
     "ssd_pair": ("ssd_pair.cu", "ssd_common.cuh", "ssd_tc.cuh", "tma.cuh", "umma.cuh"),
 }
 PATH_KERNEL = {"fused": "ssd_fused", "fused_pair": "ssd_pair"}
@@ -380,15 +381,15 @@ def main():
     e2e_value = tokens / (e2e_ms * 1e-3)
 
     hbm_peak, tc_peak, tc_sust, peak_src = load_peaks()
-    # the fused path: one launch, or the segmented form's three (lean pass,
-    # combine, full pass), timed together as one step
+    # the fused path: one launch, or the segmented form's three (segment end
+    # states, combine, full pass), timed together as one step
     kernel_ms = statistics.mean(per_step) if path in ssd.FUSED_PATHS and not args.unfused else None
     roofline = None
     if kernel_ms is not None:
         kname = PATH_KERNEL[path]
         label = "k_" + kname
         if kernels_per_step > 1:
-            label += (" segmented form, whole step: lean pass (k_ssd_fused<.., LEAN>), k_state_passing, "
+            label += (" segmented form, whole step: segment end states (k_ssd_segment_states), k_state_passing, "
                       "full pass (k_ssd_fused)")
         ach = algorithmic_bytes(wl) / (kernel_ms * 1e-3) / 1e9
         roofline = {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,

@@ -3,6 +3,7 @@
 #include "ssd_simt.cu"
 #include "ssd_step.cu"
 #include "ssd_fused.cu"
+#include "ssd_lean.cu"
 #include "ssd_pair.cu"
 #include "ssd_api.cu"
 #include "ssd_noalloc.cu"

@@ -83,9 +83,11 @@ struct Params {
   float* chunk_final;        // chunk-state CTAs: [slots][N][P] end state of each chunk
   // Grid layout: the first `whole` CTAs scan sequences 0..whole-1 whole (step
   // modes with whole > 0 are mixed grids); the rest run the step mode over
-  // sequences seq0, seq0+1, ..., one CTA per chunk, chunk slot
-  // (sequence - seq0) * nc + chunk.
-  int64_t whole, seq0;
+  // the nseq sequences seq0, seq0+1, ..., one CTA per chunk, sequence-fastest
+  // (CTAs that run together read the same tokens of neighbouring heads: whole
+  // rows of x, shared tiles of B and C), chunk slot (sequence - seq0) * nc +
+  // chunk.
+  int64_t whole, seq0, nseq;
   const __nv_bfloat16* x;
   int64_t sx, ldx;    // batch and token strides of x
   __nv_bfloat16* y;
@@ -99,7 +101,6 @@ struct Params {
   float norm_eps, inv_feat;  // eps, 1 / (H P)
   unsigned long long* trace;  // diagnostics: per-sub-chunk event clocks of CTA 0, then
                               // [start ns, end ns, SM] of every CTA; or NULL
-  float* seg_decay;           // chunk-state mode: [B,H,nc] total log-decay of each chunk, or NULL
   int withhold_loads;         // self-test of the timeout path: issue no TMA loads, so
                               // every wait on them runs out (0 in every other launch)
 };
@@ -196,13 +197,11 @@ __device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
 
-// LEAN: the chunk-state mode reduced to what a chunk's end state needs (x and
-// B tiles, X', b_intra, the state recursion): no C, no S, no mask, no y.
 // XDT: the dt-scaled input variant; NORM: a layer of a stack with the RMS norm
 // fused (input scaled from ss_in when given, sums of squares to ss_out when
 // given).  Separate instantiations, so that the plain scan carries none of
 // their per-column factors and sums.
-template <bool XDT, bool NORM, bool LEAN>
+template <bool XDT, bool NORM>
 __global__ void __launch_bounds__(THREADS, 1)
     k_ssd_fused(Params p, const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
                 const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_y) {
@@ -225,8 +224,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool chunked = p.mode != MODE_SCAN && (int64_t)blockIdx.x >= p.whole;
   const int64_t cb = (int64_t)blockIdx.x - p.whole;                // chunk CTA index (step modes)
-  const int64_t bh = chunked ? p.seq0 + cb / p.nc : (int64_t)blockIdx.x;
-  const int64_t cidx = chunked ? cb % p.nc : 0;                    // chunk of this CTA (step modes)
+  const int64_t bh = chunked ? p.seq0 + cb % p.nseq : (int64_t)blockIdx.x;
+  const int64_t cidx = chunked ? cb / p.nseq : 0;                  // chunk of this CTA (step modes)
   const int b = (int)(bh / p.H), h = (int)(bh % p.H);
   const int g = h / (p.H / p.G);
   const int t_base = (int)(cidx * p.Q);                          // first token of this CTA
@@ -256,7 +255,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&bar[FULL0 + i], 1);
       mbar_init(&bar[EMPTY0 + i], 1);
       mbar_init(&bar[SFULL0 + i], 1);
-      mbar_init(&bar[PFULL0 + i], LEAN ? AUX : T + AUX);
+      mbar_init(&bar[PFULL0 + i], T + AUX);
       mbar_init(&bar[CFULL0 + i], 1);
       mbar_init(&bar[TEMPTY0 + i], T);
       mbar_init(&bar[YFREE0 + i], 1);
@@ -286,10 +285,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_prefetch_4d(&map_x, 0, h, tp, b);
         tma_prefetch_4d(&map_b, 0, g, tp, b);
         tma_prefetch_4d(&map_b, 64, g, tp, b);
-        if (!LEAN) {
-          tma_prefetch_4d(&map_c, 0, g, tp, b);
-          tma_prefetch_4d(&map_c, 64, g, tp, b);
-        }
+        tma_prefetch_4d(&map_c, 0, g, tp, b);
+        tma_prefetch_4d(&map_c, 64, g, tp, b);
       };
       for (int jp = 0; jp < kPrefetch; ++jp) prefetch(jp);
       const int nload = nsub & (p.withhold_loads - 1);  // 0 or nsub (withhold_loads is 0 or 1)
@@ -300,14 +297,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (j >= 2 && !ctl.wait(EMPTY0 + st, ((j >> 1) + 1) & 1)) break;
         uint8_t* sx = sm + st * STAGE;
         const int t0 = t_base + j * T;
-        mbar_arrive_expect_tx(&bar[FULL0 + st], LEAN ? 3 * TILE : TX_BYTES);
+        mbar_arrive_expect_tx(&bar[FULL0 + st], TX_BYTES);
         tma_load_4d(sx + OFF_X, &map_x, &bar[FULL0 + st], 0, h, t0, b);
         tma_load_4d(sx + OFF_B, &map_b, &bar[FULL0 + st], 0, g, t0, b);
         tma_load_4d(sx + OFF_B + TILE, &map_b, &bar[FULL0 + st], 64, g, t0, b);
-        if (!LEAN) {
-          tma_load_4d(sx + OFF_C, &map_c, &bar[FULL0 + st], 0, g, t0, b);
-          tma_load_4d(sx + OFF_C + TILE, &map_c, &bar[FULL0 + st], 64, g, t0, b);
-        }
+        tma_load_4d(sx + OFF_C, &map_c, &bar[FULL0 + st], 0, g, t0, b);
+        tma_load_4d(sx + OFF_C + TILE, &map_c, &bar[FULL0 + st], 64, g, t0, b);
         issued = j + 1;
         mark(j, EV_LOADS);
       }
@@ -342,31 +337,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       int js = 0, jc = 0;
       uint32_t idle = 0;
       uint64_t t_last = globaltimer_ns();
-      if constexpr (LEAN) {
-        // b_intra of each sub-chunk once X' is written (PFULL: the aux warps
-        // alone) and the epilogue has read b_intra of jc-2 from the buffer
-        for (; jc < nsub; ++jc) {
-          const int st = jc & 1, buf = jc & 1;
-          bool ok = ctl.wait(PFULL0 + st, (jc >> 1) & 1);
-          if (ok && jc >= 2) ok = ctl.wait(TEMPTY0 + buf, ((jc >> 1) + 1) & 1);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t base = tmem + buf * 256;
-          const uint64_t cB = desc_advance(dBmn, st * STAGE), cXp = desc_advance(dXp, st * TILE);
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            mma_ss(base + 192, desc_advance(cB, ks * 2048), desc_advance(cXp, ks * 2048), idB, ks > 0);
-          mma_commit(&bar[CFULL0 + buf]);
-          mma_commit(&bar[EMPTY0 + st]);
-        }
-        (void)idS;
-        (void)idY;
-        (void)dPrev;
-        (void)dX;
-        (void)dBk;
-        (void)js;
-      }
-      while (!LEAN && jc < nsub) {
+      while (jc < nsub) {
         bool progress = false;
         if (jc < js && mbar_test_wait(&bar[PFULL0 + (jc & 1)], (jc >> 1) & 1) &&
             mbar_test_wait(&bar[STATEFULL], jc & 1)) {
@@ -601,7 +572,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // staged in the same buffer, has been read by the TMA store)
       bool ok = ctl.wait(FULL0 + st, (j >> 1) & 1);
       if (ok && j >= 2) ok = ctl.wait(CFULL0 + st, ((j - 2) >> 1) & 1);
-      if (!LEAN && ok && j >= 2) ok = ctl.wait(YFREE0 + st, ((j - 2) >> 1) & 1);  // y(j-2) staged here is stored
+      if (ok && j >= 2) ok = ctl.wait(YFREE0 + st, ((j - 2) >> 1) & 1);  // y(j-2) staged here is stored
       if (ok) {
         const float lam_end = lj[T - 1];  // log2 units
         const uint4* src = reinterpret_cast<const uint4*>(sm + st * STAGE + OFF_X);
@@ -633,7 +604,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ P = S (.) L
-    if constexpr (!LEAN) {  // (the lean mode has no S and no mask)
     const int q = warp & 3;          // TMEM lane quarter = 32-row block
     const int row = q * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
@@ -711,7 +681,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive(&bar[PFULL0 + buf]);
       if (q == 3 && lane == 0) mark(j, EV_MASK_DONE);
     }
-    }
   } else {
     // ------------------------------------------------------------ y, state, final
     const int q = warp & 3;
@@ -759,11 +728,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       fence_async_smem();
       mbar_arrive(&bar[STATEFULL]);
     };
-    if (!LEAN) publish_state();
-    float lam_sum = 0.f;  // log2 of the chunk's total decay (lean chunk-state mode)
+    publish_state();
     for (int j = 0; j < nsub; ++j) {
       const int buf = j & 1;
-      if (!LEAN) load_x(j, xcur);
+      load_x(j, xcur);
       bool ok = ctl.wait(CFULL0 + buf, (j >> 1) & 1);
       if (ok) ok = ctl.wait(LAMRDY0 + (j & 3), (j >> 2) & 1);      // acquire lam of this sub-chunk
       tc_fence_after();
@@ -785,12 +753,6 @@ __global__ void __launch_bounds__(THREADS, 1)
           s[32 * c + i] = o.x;
           s[32 * c + i + 1] = o.y;
         }
-      }
-      if constexpr (LEAN) {  // only the state: release the buffer and go on
-        tc_fence_before();
-        mbar_arrive(&bar[TEMPTY0 + buf]);
-        lam_sum += lam_end;
-        continue;
       }
       if (ok) publish_state();
       if (r == 0) mark(j, EV_STATE_PUB);
@@ -852,7 +814,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (r == 0) mark(j, EV_EPI_DONE);
     }
     if (r == 0) tma_store_wait0();  // the y tiles are in global memory before the CTA exits
-    if (LEAN && p.seg_decay && r == 0) p.seg_decay[cslot] = lam_sum * 0.6931471805599453f;  // log2 -> ln
     if (final_ptr) {
       float4* dst = reinterpret_cast<float4*>(final_ptr + (int64_t)r * P);
 #pragma unroll
@@ -887,13 +848,13 @@ bool uses_pair_kernel(const Problem& p) { return p.two_heads && pair_supported(p
 // The first `whole` sequences run whole (one CTA each); every later one is
 // cut into nseg segments of qseg tokens (the page's chunk decomposition one
 // level up, "分块推理…" §2.1-§2.2, with a segment as the chunk).  Three launches:
-// the lean kernel forms each segment's end state from a zero start and its
-// total log-decay, k_state_passing combines them in order into each
+// k_ssd_segment_states (csrc/ssd_lean.cu) forms each segment's end state from
+// a zero start and its total log-decay, k_state_passing combines them in order into each
 // segment's start state (and the sequence's final state), and the full
 // kernel runs the whole sequences first and then every segment from its
 // start state, so the short segment CTAs fill the SMs that the last whole
-// ones leave free.  Chosen only where a cost model of CTA rounds (a lean
-// segment costing about a third of a full one) predicts a gain.
+// ones leave free.  Chosen only where a cost model of CTA rounds (a segment's
+// end state costing about a third of its full scan) predicts a gain.
 struct SegPlan {
   int nseg;       // 1: whole sequences in one launch
   int64_t qseg;   // segment length in tokens (a multiple of 128)
@@ -939,7 +900,7 @@ static SegPlan seg_plan(const Problem& p) {
   }
   if (nsub < 8) return plan;
   // cost in sub-chunk periods: a CTA costs its sub-chunks plus about two of
-  // pipeline fill and drain; a lean segment about 0.35 of a full one, plus
+  // pipeline fill and drain; a segment's end state about 0.35 of its scan, plus
   // one period for the combine launch
   const double w = (double)(nsub + 2);
   const double plain = (double)ceil_div(bh, nsm) * w;
@@ -991,8 +952,7 @@ struct GridSplit {
 
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
                                void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads = 0,
-                               const NormIO* norm = nullptr, float* seg_decay = nullptr,
-                               const GridSplit& split = GridSplit());
+                               const NormIO* norm = nullptr, const GridSplit& split = GridSplit());
 
 cudaError_t launch_fused_traced(const Problem& p, const float* init, float* final_state, unsigned long long* trace,
                                 cudaStream_t st) {
@@ -1044,19 +1004,10 @@ cudaError_t launch_fused_normed(const Problem& p, const float* init, float* fina
   return launch_mode(p, fused::MODE_SCAN, nullptr, init, final_state, p.y, nullptr, st, 0, &norm);
 }
 
-// Segments of long sequences (p.Q = the segment length, a multiple of 128;
-// sequences `whole` on, slot (sequence - whole) * nc + segment): the end
-// state of every segment from a zero start and the segment's total
-// log-decay, with the lean kernel (dt scanned in the kernel) ...
-cudaError_t launch_segment_states(const Problem& p, int64_t whole, float* states, float* seg_decay,
-                                  cudaStream_t st) {
-  GridSplit sp;
-  sp.seq0 = whole;
-  return launch_mode(p, fused::MODE_CHUNK_STATE, nullptr, nullptr, states, nullptr, nullptr, st, 0, nullptr,
-                     seg_decay, sp);
-}
-// ... and the outputs: sequences 0..whole-1 whole (from init, to
-// final_state), then every segment from its start state prev[slot].
+// The outputs of the segmented form: sequences 0..whole-1 whole (from init,
+// to final_state), then every segment of the later sequences from its start
+// state prev[slot] (the segments' end states come from
+// launch_segment_states, csrc/ssd_lean.cu).
 cudaError_t launch_segment_scan(const Problem& p, int64_t whole, const float* prev, const float* init,
                                 float* final_state, cudaStream_t st) {
   GridSplit sp;
@@ -1064,7 +1015,7 @@ cudaError_t launch_segment_scan(const Problem& p, int64_t whole, const float* pr
   sp.seq0 = whole;
   sp.init = init;
   sp.final_state = final_state;
-  return launch_mode(p, fused::MODE_CHUNK_SCAN, nullptr, prev, nullptr, p.y, nullptr, st, 0, nullptr, nullptr, sp);
+  return launch_mode(p, fused::MODE_CHUNK_SCAN, nullptr, prev, nullptr, p.y, nullptr, st, 0, nullptr, sp);
 }
 
 // Step 2 on tensor cores: one CTA per (batch, head, chunk), zero start, the
@@ -1081,7 +1032,7 @@ cudaError_t launch_chunk_scan_tc(const Problem& p, const float* lam, const float
 
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
                                void* y, unsigned long long* trace, cudaStream_t st, int withhold_loads,
-                               const NormIO* norm, float* seg_decay, const GridSplit& split) {
+                               const NormIO* norm, const GridSplit& split) {
   using namespace fused;
   // every pointer the mode reads must be present (the step entry points pass
   // only the tensors of their step)
@@ -1130,6 +1081,7 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   kp.chunk_final = mode == MODE_CHUNK_STATE ? final_state : nullptr;
   kp.whole = step_mode ? split.whole : 0;
   kp.seq0 = step_mode ? split.seq0 : 0;
+  kp.nseq = p.B * p.H - kp.seq0;
   kp.x = static_cast<const __nv_bfloat16*>(p.x);
   kp.sx = p.sx;
   kp.ldx = p.ldx;
@@ -1137,7 +1089,6 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   kp.sy = p.sy;
   kp.trace = trace;
   kp.withhold_loads = withhold_loads;
-  kp.seg_decay = seg_decay;
   kp.ss_in = (norm && mode == MODE_SCAN) ? norm->ss_in : nullptr;
   kp.ss_out = (norm && mode == MODE_SCAN) ? norm->ss_out : nullptr;
   kp.sss = norm ? norm->batch_stride : 0;
@@ -1151,10 +1102,9 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   if (e != cudaSuccess) return e;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set.load() & bit)) {
-    const void* fns[6] = {(const void*)k_ssd_fused<false, false, false>, (const void*)k_ssd_fused<true, false, false>,
-                          (const void*)k_ssd_fused<false, true, false>, (const void*)k_ssd_fused<true, true, false>,
-                          (const void*)k_ssd_fused<false, false, true>, (const void*)k_ssd_fused<true, false, true>};
-    for (int i = 0; i < 6 && e == cudaSuccess; ++i)
+    const void* fns[4] = {(const void*)k_ssd_fused<false, false>, (const void*)k_ssd_fused<true, false>,
+                          (const void*)k_ssd_fused<false, true>, (const void*)k_ssd_fused<true, true>};
+    for (int i = 0; i < 4 && e == cudaSuccess; ++i)
       e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set.fetch_or(bit);
@@ -1163,22 +1113,17 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   if (kp.whole < 0 || kp.whole > kp.seq0 || kp.seq0 > p.B * p.H || ctas <= 0 || ctas >= (1ll << 31))
     return cudaErrorInvalidValue;
   // the dt-scaled input whenever dt is read here (the whole scan, and the step
-  // modes without a step-1 output); lean: the chunk-state mode of segments
+  // modes without a step-1 output)
   const bool xdt = p.input_dt && (mode == fused::MODE_SCAN || !lam), nrm = kp.ss_in != nullptr || kp.ss_out != nullptr;
-  const bool lean = mode == fused::MODE_CHUNK_STATE && seg_decay != nullptr;
   const dim3 grid((unsigned)ctas);
-  if (lean && xdt)
-    k_ssd_fused<true, false, true><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
-  else if (lean)
-    k_ssd_fused<false, false, true><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
-  else if (xdt && nrm)
-    k_ssd_fused<true, true, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+  if (xdt && nrm)
+    k_ssd_fused<true, true><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
   else if (xdt)
-    k_ssd_fused<true, false, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+    k_ssd_fused<true, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
   else if (nrm)
-    k_ssd_fused<false, true, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+    k_ssd_fused<false, true><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
   else
-    k_ssd_fused<false, false, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
+    k_ssd_fused<false, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
   return cudaGetLastError();
 }
 

@@ -120,18 +120,34 @@ def test_long_sequences_repeat_bitwise(two_heads):
     outs = [_scan(dev, wl, two_heads=two_heads) for _ in range(4)]
     for y, f in outs[1:]:
         assert torch.equal(y, outs[0][0]) and torch.equal(f, outs[0][1])
-    # and the same bits when the sequence is cut into blocks with the state carried
+    # and the same bits when the sequence is cut into blocks with the state
+    # carried.  With one head per CTA this holds for one CTA per sequence (the
+    # strided entry point, no workspace): the segmented form that the
+    # workspace entry picks for 4 sequences forms segment end states with
+    # their own roundings, so its blocks agree with the whole run to bf16
+    # precision (checked below), not bit for bit.
+    if two_heads:
+        whole = lambda x, dt, B, C, st: ssd.ssd_scan_fwd(x, dt, dev["A"], B, C, dev["D"], st, chunk=wl.chunk,
+                                                         final_state=st, two_heads=True)
+        ref = outs[0]
+    else:
+        whole = lambda x, dt, B, C, st: ssd.ssd_scan_fwd_strided(x, dt, dev["A"], B, C, dev["D"], st,
+                                                                 chunk=wl.chunk, final_state=st)
+        st0 = dev["init"].clone()
+        ref = (whole(dev["x"], dev["dt"], dev["B"], dev["C"], st0)[0], st0)
     V = 2048
     y_blk = torch.empty_like(dev["x"])
     st = dev["init"].clone()
     for k0 in range(0, wl.seqlen, V):
         sl = lambda t: t[:, k0:k0 + V].contiguous()
-        yk, _ = ssd.ssd_scan_fwd(sl(dev["x"]), sl(dev["dt"]), dev["A"], sl(dev["B"]), sl(dev["C"]), dev["D"], st,
-                                 chunk=wl.chunk, final_state=st, two_heads=two_heads)
+        yk, _ = whole(sl(dev["x"]), sl(dev["dt"]), sl(dev["B"]), sl(dev["C"]), st)
         y_blk[:, k0:k0 + V] = yk
     torch.cuda.synchronize()
-    assert torch.equal(y_blk, outs[0][0])
-    assert torch.equal(st, outs[0][1])
+    assert torch.equal(y_blk, ref[0])
+    assert torch.equal(st, ref[1])
+    if not two_heads:  # the segmented whole run against the blocks
+        assert rel_err(to_np64(outs[0][0]), to_np64(y_blk)) <= 5e-3
+        assert rel_err(to_np64(outs[0][1]), to_np64(st)) <= 2e-3
 
 
 def test_sequence_shard_single_rank_equals_scan():

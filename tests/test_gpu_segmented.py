@@ -57,17 +57,27 @@ def test_segmented_scan_matches_oracle(over, nseg, input_dt):
 
 def test_segmented_and_whole_sequences_agree():
     """The same problem through the segmented form and through one CTA per
-    sequence (the strided entry point has no workspace): equal to within the
-    bf16 rounding of the start states the segmented form hands over."""
+    sequence (the strided entry point has no workspace).  Both stay within
+    the bf16 bound of the oracle; against each other they differ by bf16
+    roundings: a segment's end state takes each input row x_s once rounded
+    to bf16 after its decay to the segment's end is folded in, the one-CTA
+    scan rounds it after the decay to its 128-token tile's end only, so the
+    two sums carry different roundings of the same terms (2^-9 relative
+    each)."""
     wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=4096, nheads=24, ngroups=1, init_var=0.1)
-    dev = device_inputs(inputs.generate(wl))
+    host = inputs.generate(wl)
+    dev = device_inputs(host)
     y, fin = _run(dev, wl)
     assert ssd.ssd_scan_path(ssd.make_dims(dev["x"], dev["B"], wl.chunk))[1] == 3
     ys, fs = ssd.ssd_scan_fwd_strided(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
                                       chunk=wl.chunk)
     torch.cuda.synchronize()
+    y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host))
+    for got_y, got_f in ((y, fin), (ys, fs)):
+        assert rel_err(to_np64(got_y), y_ref) <= TOL["bf16"]
+        assert rel_err(to_np64(got_f), f_ref) <= TOL["bf16"]
     assert rel_err(to_np64(y), to_np64(ys)) <= 5e-3
-    assert rel_err(to_np64(fin), to_np64(fs)) <= 1e-4
+    assert rel_err(to_np64(fin), to_np64(fs)) <= 2e-3
 
 
 @contextlib.contextmanager

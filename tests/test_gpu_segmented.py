@@ -1,6 +1,6 @@
 """The one-head kernel's segmented form for problems with fewer (batch, head)
-sequences than SMs: the segments' end states from a zero start (the lean
-kernel: x, B, X', b_intra and the state recursion only), their ordered
+sequences than SMs: the segments' end states from a zero start
+(k_ssd_segment_states: one accumulated product B^T X'' per segment), their ordered
 combine into each segment's start state (the chunk decomposition of
 "分块推理…" §2.1-§2.2 with a segment as the chunk), and the full scan of every
 segment from its start state.  Compared with the fp64 oracle; the segment
@@ -98,7 +98,7 @@ def split(nseg, whole):
 def test_mixed_grid_matches_oracle(over, nseg, whole, input_dt):
     """The mixed layout: the first `whole` sequences scanned whole (from the
     caller's initial state to its final state) and the rest as segments
-    (lean end states, combine over the segmented sequences only, segment
+    (segment end states, combine over the segmented sequences only, segment
     scans), in one grid.  Every sequence of both kinds against the oracle."""
     wl = inputs.custom("mamba2_130m_layer", **over)
     host = inputs.generate(wl)

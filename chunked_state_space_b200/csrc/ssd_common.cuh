@@ -54,12 +54,23 @@ __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + 
 // only definition.
 __device__ int g_device_status = 0;
 
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute may start while the kernel before it on the
+// stream still runs; grid_dep_wait() returns once that kernel has completed
+// and its memory is visible (at once for an ordinary launch), and
+// grid_dep_launch() lets the next such kernel start early.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Launchers of the CUDA-core kernels (ssd_simt.cu).  They return
 // cudaSuccess or the launch error.
 cudaError_t launch_chunk_cumsum(const Problem& p, float* lam, cudaStream_t st);
 cudaError_t launch_chunk_state_simt(const Problem& p, const float* lam, float* states, cudaStream_t st);
+// programmatic: launched so that it may start while the kernel before it on
+// the stream finishes (it waits for that kernel's results itself)
 cudaError_t launch_state_passing(const Problem& p, const float* states, const float* lam,
-                                 const float* init, float* prev, float* final_state, cudaStream_t st);
+                                 const float* init, float* prev, float* final_state, cudaStream_t st,
+                                 bool programmatic = false);
 cudaError_t launch_chunk_scan_simt(const Problem& p, const float* lam, const float* prev, cudaStream_t st);
 cudaError_t launch_ssd_step(const Problem& p, float* state, cudaStream_t st);
 cudaError_t launch_rmsnorm(int64_t rows, int64_t features, int io, const void* in, float eps, void* out,

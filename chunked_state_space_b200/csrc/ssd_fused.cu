@@ -703,6 +703,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     };
     uint4 xcur[8];
     float s[P];
+    if (chunked) grid_dep_wait();  // start states from the kernel before (a programmatic launch)
     if (init_ptr) {
       const float4* src = reinterpret_cast<const float4*>(init_ptr + (int64_t)r * P);
 #pragma unroll
@@ -948,6 +949,7 @@ struct GridSplit {
   int64_t whole = 0, seq0 = 0;
   const float* init = nullptr;
   float* final_state = nullptr;
+  bool programmatic = false;  // may start while the kernel before it finishes
 };
 
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
@@ -988,7 +990,7 @@ cudaError_t launch_fused(const Problem& p, const float* init, float* final_state
       pc.H = p.B * p.H - w;
     }
     e = launch_state_passing(pc, states, decays, init ? init + w * NP : nullptr, states,
-                             final_state ? final_state + w * NP : nullptr, st);
+                             final_state ? final_state + w * NP : nullptr, st, /*programmatic=*/true);
     if (e != cudaSuccess) return e;
     return launch_segment_scan(ps, w, states, init, final_state, st);
   }
@@ -1015,6 +1017,7 @@ cudaError_t launch_segment_scan(const Problem& p, int64_t whole, const float* pr
   sp.seq0 = whole;
   sp.init = init;
   sp.final_state = final_state;
+  sp.programmatic = true;  // its prologue and the whole sequences overlap the combine
   return launch_mode(p, fused::MODE_CHUNK_SCAN, nullptr, prev, nullptr, p.y, nullptr, st, 0, nullptr, sp);
 }
 
@@ -1115,16 +1118,20 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   // the dt-scaled input whenever dt is read here (the whole scan, and the step
   // modes without a step-1 output)
   const bool xdt = p.input_dt && (mode == fused::MODE_SCAN || !lam), nrm = kp.ss_in != nullptr || kp.ss_out != nullptr;
-  const dim3 grid((unsigned)ctas);
-  if (xdt && nrm)
-    k_ssd_fused<true, true><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
-  else if (xdt)
-    k_ssd_fused<true, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
-  else if (nrm)
-    k_ssd_fused<false, true><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
-  else
-    k_ssd_fused<false, false><<<grid, THREADS, SMEM_BYTES, st>>>(kp, mx, mb, mc, my);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ctas);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = split.programmatic ? 1 : 0;
+  if (xdt && nrm) return cudaLaunchKernelEx(&cfg, k_ssd_fused<true, true>, kp, mx, mb, mc, my);
+  if (xdt) return cudaLaunchKernelEx(&cfg, k_ssd_fused<true, false>, kp, mx, mb, mc, my);
+  if (nrm) return cudaLaunchKernelEx(&cfg, k_ssd_fused<false, true>, kp, mx, mb, mc, my);
+  return cudaLaunchKernelEx(&cfg, k_ssd_fused<false, false>, kp, mx, mb, mc, my);
 }
 
 }  // namespace ssd

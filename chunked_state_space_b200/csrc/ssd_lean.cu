@@ -107,6 +107,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
 
+  grid_dep_launch();  // the combine may be scheduled now (it waits for this grid's results)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // sequence-fastest: CTAs that run together read the same tokens of
   // neighbouring heads (whole rows of x, shared tiles of B)

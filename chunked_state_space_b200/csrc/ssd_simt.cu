@@ -131,6 +131,8 @@ template <bool VEC>
 __global__ void __launch_bounds__(128) k_state_passing(const float* states, const float* __restrict__ lam,
                                                        const float* init, float* prev, float* final_state,
                                                        int H, int nc, int Q, int NP) {
+  grid_dep_wait();    // the chunk states and decays of the kernel before (a programmatic launch)
+  grid_dep_launch();  // and the scan after it may start its prologue
   const int h = blockIdx.y, b = blockIdx.z;
   const int e0 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
   const int lane = threadIdx.x & 31;
@@ -178,16 +180,23 @@ __global__ void __launch_bounds__(128) k_state_passing(const float* states, cons
 }
 
 cudaError_t launch_state_passing(const Problem& p, const float* states, const float* lam, const float* init,
-                                 float* prev, float* final_state, cudaStream_t st) {
+                                 float* prev, float* final_state, cudaStream_t st, bool programmatic) {
   const int NP = (int)(p.N * p.P);
   dim3 grid((unsigned)ceil_div(NP, 512), (unsigned)p.H, (unsigned)p.B);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = programmatic ? 1 : 0;
+  const int H = (int)p.H, nc = (int)p.nc, Q = (int)p.Q;
   if (NP % 4 == 0)
-    k_state_passing<true><<<grid, 128, 0, st>>>(states, lam, init, prev, final_state, (int)p.H, (int)p.nc,
-                                                (int)p.Q, NP);
-  else
-    k_state_passing<false><<<grid, 128, 0, st>>>(states, lam, init, prev, final_state, (int)p.H, (int)p.nc,
-                                                 (int)p.Q, NP);
-  return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, k_state_passing<true>, states, lam, init, prev, final_state, H, nc, Q, NP);
+  return cudaLaunchKernelEx(&cfg, k_state_passing<false>, states, lam, init, prev, final_state, H, nc, Q, NP);
 }
 
 // ---------------------------------------------------------------------------

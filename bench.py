@@ -359,8 +359,8 @@ def main():
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    # ssd_scan_fwd_host: the batch streams through the device one sequence at a
-    # time, copies in and out overlapped with the scan
+    # ssd_scan_fwd_host: the batch streams through the device in slices of one
+    # sequence and up to 4096 tokens, copies in and out overlapped with the scan
     host_ws = torch.empty(ssd.ssd_scan_fwd_host_workspace_size(dims), dtype=torch.uint8, device=dev)
 
     def e2e_step():

@@ -158,20 +158,25 @@ ssd_status ssd_scan_fwd_strided(const ssd_dims* d, const void* x, int64_t x_bstr
 
 /*
  * Bytes of DEVICE workspace ssd_scan_fwd_host needs for `d`: A and D, and two
- * one-sequence slice buffers (inputs, outputs and the scan's scratch).
+ * slice buffers (one sequence, up to 4096 tokens: inputs, outputs, the end
+ * state and the scan's scratch).
  */
 ssd_status ssd_scan_fwd_host_workspace_size(const ssd_dims* d, size_t* bytes);
 
 /*
  * ssd_scan_fwd with every tensor in HOST memory (same shapes, layouts and
  * meaning; init_state, final_state and D may be NULL as there), the copies
- * overlapped with the scan: the batch flows through the device workspace one
- * sequence at a time, slice b+1 copied in and slice b-1 copied out while slice
- * b is scanned on `stream`.  Host buffers should be page-locked
- * (cudaHostAlloc / cudaHostRegister): pageable memory works but its copies do
- * not overlap.  The host buffers must stay valid and unchanged until the work
- * on `stream` completes; y and final_state are written by then.  Results equal
- * ssd_scan_fwd's bitwise.  The two copy streams and their events belong to the
+ * overlapped with the scan: the batch flows through the device workspace in
+ * slices of one sequence and up to 4096 tokens (a whole number of chunks),
+ * slice s+1 copied in and slice s-1 copied out while slice s is scanned on
+ * `stream`, each slice from the end state of the slice before it in its
+ * sequence (the chunk recursion of "分块推理…" §2.2 with the slice as the chunk).
+ * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister):
+ * pageable memory works but its copies do not overlap.  The host buffers must
+ * stay valid and unchanged until the work on `stream` completes; y and
+ * final_state are written by then.  Results equal ssd_scan_fwd's up to
+ * rounding (bitwise when the sequence is one slice and both choose the same
+ * split of the sequences over SMs).  The two copy streams and their events belong to the
  * library (one set per device, created on first use, kept until the process
  * exits); each call forks them from `stream` and joins them back.  Calls from
  * several host threads on one device are serialised while they enqueue.

@@ -1,7 +1,9 @@
 """ssd_scan_fwd_host: the scan from and to host memory, copies overlapped with
-the scan one sequence at a time.  Its results must equal ssd_scan_fwd's on the
-same inputs bitwise (the same kernels run every (batch, head) sequence), and
-the oracle's within the io dtype's tolerance."""
+the scan in slices of one sequence and up to 4096 tokens, the state carried
+from slice to slice.  Its results must equal ssd_scan_fwd's on the same
+inputs bitwise where a sequence is one slice (the same kernels run every
+(batch, head) sequence), and the oracle's within the io dtype's tolerance
+(also where sequences are cut into several slices)."""
 import numpy as np
 import pytest
 import torch
@@ -57,3 +59,33 @@ def test_host_io_without_optional_tensors():
     y_d, _ = ssd.ssd_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], None, None, chunk=wl.chunk)
     torch.cuda.synchronize()
     assert torch.equal(y_h, y_d.cpu())
+
+
+@pytest.mark.parametrize("case", [
+    dict(base="mamba2_130m_layer", batch=2, seqlen=10000, nheads=4, ngroups=2, init_var=0.1),  # 3 slices, ragged
+    dict(base="tiny_f32", batch=2, seqlen=8200, nheads=2, ngroups=1, init_var=0.5),            # CUDA-core path
+])
+@pytest.mark.parametrize("want_final", [True, False])
+def test_host_io_long_sequences_in_slices(case, want_final):
+    """Sequences longer than a slice: several slices per sequence, each scanned
+    from the end state of the slice before; y and the final state against the
+    oracle and against ssd_scan_fwd (to rounding)."""
+    case = dict(case)
+    base = case.pop("base")
+    wl = inputs.custom(base, **case)
+    host = inputs.generate(wl)
+    h = host_inputs(host, True)
+    y_h, f_h = ssd.ssd_scan_fwd_host(h["x"], h["dt"], h["A"], h["B"], h["C"], h["D"], h["init"], chunk=wl.chunk,
+                                     want_final=want_final)
+    torch.cuda.synchronize()
+    y_ref, f_ref = oracle.scan_recurrence(*oracle_args(host))
+    assert rel_err(to_np64(y_h), y_ref) <= TOL[wl.io]
+    if want_final:
+        assert rel_err(to_np64(f_h), f_ref) <= TOL[wl.io]
+    else:
+        assert f_h is None
+    dev = device_inputs(host)
+    y_d, _ = ssd.ssd_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init"],
+                              chunk=wl.chunk)
+    torch.cuda.synchronize()
+    assert rel_err(to_np64(y_h), to_np64(y_d.cpu())) <= TOL[wl.io]

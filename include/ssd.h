@@ -126,7 +126,8 @@ ssd_status ssd_scan_workspace_size(const ssd_dims* d, size_t* bytes);
  *   workspace: device scratch of at least ssd_scan_workspace_size bytes,
  *   owned by the caller, contents need not be initialised.
  * Picks the tensor-core path for bf16 io when the sizes allow it, else the
- * CUDA-core path.  Errors: every status above.
+ * CUDA-core path (ssd_scan_path says which, and how many launches).
+ * Errors: every status above.
  */
 ssd_status ssd_scan_fwd(const ssd_dims* d, const void* x, const float* dt, const float* A,
                         const void* Bm, const void* Cm, const float* D, const float* init_state,
@@ -193,11 +194,18 @@ ssd_status ssd_scan_fwd_host(const ssd_dims* d, const void* x, const float* dt, 
  * steps 2 and 4 on tcgen05 tensor cores), SSD_PATH_FUSED (one tensor-core
  * kernel) or SSD_PATH_FUSED_PAIR (one tensor-core kernel, two heads of a
  * group per CTA sharing their B and C tiles; SSD_FLAG_TWO_HEADS_PER_CTA).
- * The one-head kernel runs one (batch, head) sequence per CTA.  The two-head
- * kernel, given the workspace of ssd_scan_workspace_size and more head pairs
- * than SMs, cuts the concatenated sequences into equal ranges, one persistent
- * CTA per SM, and hands the state across range boundaries through the
- * workspace; otherwise it runs whole sequences;
+ * The one-head kernel runs one (batch, head) sequence per CTA; where that
+ * leaves SMs idle (fewer sequences than SMs, or B*H a whole number of rounds
+ * of CTAs on the SMs plus a partial round) and a cost model of CTA rounds
+ * predicts a gain, it runs the segmented form instead (three launches: the
+ * end state of every segment of the affected sequences from a zero start,
+ * their ordered combine, then one grid scanning the other sequences whole and
+ * every segment from its start state), which needs the workspace of
+ * ssd_scan_workspace_size (without it, whole sequences).  The two-head
+ * kernel, given that workspace and more head pairs than SMs, cuts every
+ * sequence into segments scheduled in rounds on one persistent CTA per SM and
+ * hands the state across segment boundaries through the workspace; otherwise
+ * it runs whole sequences;
  * *kernels = kernel launches per call.  Either output pointer may be NULL.
  * Errors: as ssd_scan_workspace_size.
  */

@@ -3,6 +3,8 @@
 // fp32 or bf16 io, plus the layer-to-layer RMS normalisation.  This is the
 // exact path (fp32 io is checked at 1e-5) and the fallback for sizes the
 // tensor-core kernels do not cover.
+#include <type_traits>
+
 #include "ssd_common.cuh"
 
 namespace ssd {
@@ -51,7 +53,9 @@ cudaError_t launch_chunk_cumsum(const Problem& p, float* lam, cudaStream_t st) {
 // Step 2 (CUDA cores): chunk_states[b,h,c,n,p] = sum_s exp(lam_end - lam_s) B[s,n] x[s,p].
 // grid (nc, H, B), block 256.  Thread layout: p = tid % P fixed, rows n = tid / P
 // + k * (256 / P).  smem: B tile [32][N], x tile [32][P], weights [32].
-template <typename T>
+// MAXE: state rows per thread, at least ceil(N / (256 / P)) (the launcher picks
+// the smallest power of two), so no thread walks rows it does not own.
+template <typename T, int MAXE>
 __global__ void __launch_bounds__(256) k_chunk_state_simt(Problem p, const float* __restrict__ lam,
                                                           float* __restrict__ states) {
   extern __shared__ float sm[];
@@ -71,7 +75,6 @@ __global__ void __launch_bounds__(256) k_chunk_state_simt(Problem p, const float
   const int tid = threadIdx.x;
   const bool active = tid < rpp * P;
   const int pc = tid % P, n0 = tid / P;
-  constexpr int MAXE = 32;  // ceil(128 / (256/64))
   float acc[MAXE];
 #pragma unroll
   for (int k = 0; k < MAXE; ++k) acc[k] = 0.f;
@@ -113,10 +116,20 @@ __global__ void __launch_bounds__(256) k_chunk_state_simt(Problem p, const float
 cudaError_t launch_chunk_state_simt(const Problem& p, const float* lam, float* states, cudaStream_t st) {
   dim3 grid((unsigned)p.nc, (unsigned)p.H, (unsigned)p.B);
   size_t smem = sizeof(float) * (32 * p.N + 32 * p.P + 32);
-  if (p.io == SSD_BF16)
-    k_chunk_state_simt<__nv_bfloat16><<<grid, 256, smem, st>>>(p, lam, states);
-  else
-    k_chunk_state_simt<float><<<grid, 256, smem, st>>>(p, lam, states);
+  const int64_t rows = ceil_div(p.N, (int64_t)(256 / p.P));  // state rows per thread
+  auto go = [&](auto tag) {
+    constexpr int E = decltype(tag)::value;
+    if (p.io == SSD_BF16)
+      k_chunk_state_simt<__nv_bfloat16, E><<<grid, 256, smem, st>>>(p, lam, states);
+    else
+      k_chunk_state_simt<float, E><<<grid, 256, smem, st>>>(p, lam, states);
+  };
+  if (rows <= 1) go(std::integral_constant<int, 1>());
+  else if (rows <= 2) go(std::integral_constant<int, 2>());
+  else if (rows <= 4) go(std::integral_constant<int, 4>());
+  else if (rows <= 8) go(std::integral_constant<int, 8>());
+  else if (rows <= 16) go(std::integral_constant<int, 16>());
+  else go(std::integral_constant<int, 32>());
   return cudaGetLastError();
 }
 
@@ -205,7 +218,9 @@ cudaError_t launch_state_passing(const Problem& p, const float* states, const fl
 // grid (nc * ceil(Q/64), H, B), block 256 = 64 rows x 4 column groups; each
 // thread owns columns p = pg, pg+4, ... of one row.  smem: C rows [64][N+1],
 // B tile [64][N+1], x tile [64][P+1], lam of rows and keys.
-template <typename T>
+// MAXP: output columns per thread, at least ceil(P / 4) (the launcher picks the
+// smallest power of two).
+template <typename T, int MAXP>
 __global__ void __launch_bounds__(256) k_chunk_scan_simt(Problem p, const float* __restrict__ lam,
                                                          const float* __restrict__ prev) {
   extern __shared__ float sm[];
@@ -235,7 +250,6 @@ __global__ void __launch_bounds__(256) k_chunk_scan_simt(Problem p, const float*
     Cs[j * NS + n] = j < nrows ? to_f32(Cg[(int64_t)j * G * N + n]) : 0.f;
   }
   if (tid < 64) lt[tid] = tid < nrows ? lamc[r0 + tid] : 0.f;
-  constexpr int MAXP = 16;
   float acc[MAXP];
 #pragma unroll
   for (int k = 0; k < MAXP; ++k) acc[k] = 0.f;
@@ -302,17 +316,26 @@ cudaError_t launch_chunk_scan_simt(const Problem& p, const float* lam, const flo
   const int64_t ntt = ceil_div(p.Q, 64);
   dim3 grid((unsigned)(p.nc * ntt), (unsigned)p.H, (unsigned)p.B);
   size_t smem = sizeof(float) * (2 * 64 * (p.N + 1) + 64 * (p.P + 1) + 128);
-  cudaError_t e;
-  if (p.io == SSD_BF16) {
-    e = cudaFuncSetAttribute(k_chunk_scan_simt<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
-    k_chunk_scan_simt<__nv_bfloat16><<<grid, 256, smem, st>>>(p, lam, prev);
-  } else {
-    e = cudaFuncSetAttribute(k_chunk_scan_simt<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k_chunk_scan_simt<float><<<grid, 256, smem, st>>>(p, lam, prev);
-  }
+  const int64_t cols = ceil_div(p.P, (int64_t)4);  // output columns per thread
+  cudaError_t e = cudaSuccess;
+  auto go = [&](auto tag) {
+    constexpr int M = decltype(tag)::value;
+    if (p.io == SSD_BF16) {
+      e = cudaFuncSetAttribute(k_chunk_scan_simt<__nv_bfloat16, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+      if (e == cudaSuccess) k_chunk_scan_simt<__nv_bfloat16, M><<<grid, 256, smem, st>>>(p, lam, prev);
+    } else {
+      e = cudaFuncSetAttribute(k_chunk_scan_simt<float, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+      if (e == cudaSuccess) k_chunk_scan_simt<float, M><<<grid, 256, smem, st>>>(p, lam, prev);
+    }
+  };
+  if (cols <= 1) go(std::integral_constant<int, 1>());
+  else if (cols <= 2) go(std::integral_constant<int, 2>());
+  else if (cols <= 4) go(std::integral_constant<int, 4>());
+  else if (cols <= 8) go(std::integral_constant<int, 8>());
+  else go(std::integral_constant<int, 16>());
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -119,7 +119,7 @@ ssd_status run_unfused(const Problem& p, const float* init, float* final_state, 
   cudaError_t e = launch_chunk_cumsum(p, lam, st);
   if (e == cudaSuccess) {
     if (tc_supported(p))
-      e = launch_chunk_state_tc(p, lam, states, st);
+      e = launch_chunk_states_seq(p, lam, states, st);
     else
       e = launch_chunk_state_simt(p, lam, states, st);
   }
@@ -307,7 +307,7 @@ ssd_status ssd_chunk_state(const ssd_dims* d, const void* x, const void* Bm, con
   Problem p = make_problem(d);
   p.x = x; p.Bm = Bm;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (tc_supported(p)) return cuda_status(launch_chunk_state_tc(p, lam, chunk_states, st));
+  if (tc_supported(p)) return cuda_status(launch_chunk_states_seq(p, lam, chunk_states, st));
   return cuda_status(launch_chunk_state_simt(p, lam, chunk_states, st));
 }
 

@@ -1021,12 +1021,6 @@ cudaError_t launch_segment_scan(const Problem& p, int64_t whole, const float* pr
   return launch_mode(p, fused::MODE_CHUNK_SCAN, nullptr, prev, nullptr, p.y, nullptr, st, 0, nullptr, sp);
 }
 
-// Step 2 on tensor cores: one CTA per (batch, head, chunk), zero start, the
-// chunk's end state written to states[b,h,c].
-cudaError_t launch_chunk_state_tc(const Problem& p, const float* lam, float* states, cudaStream_t st) {
-  return launch_mode(p, fused::MODE_CHUNK_STATE, lam, nullptr, states, nullptr, nullptr, st);
-}
-
 // Step 4 on tensor cores: one CTA per (batch, head, chunk), starting from
 // prev[b,h,c], writing the chunk's outputs.
 cudaError_t launch_chunk_scan_tc(const Problem& p, const float* lam, const float* prev, cudaStream_t st) {

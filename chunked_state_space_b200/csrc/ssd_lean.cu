@@ -23,6 +23,7 @@
 #include <atomic>
 
 #include "ssd_common.cuh"
+#include "ssd_split.cuh"
 #include "ssd_tc.cuh"
 #include "tma.cuh"
 #include "umma.cuh"
@@ -285,6 +286,204 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+
+// Step 2 of the step-by-step scan on tensor cores: the end state of every
+// chunk from a zero start, states[b,h,c] = sum over the chunk's tokens s of
+// exp(lam_end(c) - lam(c, s)) B_s x_s^T, with lam the chunk-local cumulative
+// sums of dt * A from step 1.  The same product as above, accumulated over
+// the chunk's tiles; one CTA walks cpb consecutive chunks of one (batch, head)
+// so its TMA pipeline stays full across chunk boundaries, and the read-out of
+// chunk c (two TMEM accumulators, 128 columns) overlaps the MMAs of chunk c+1.
+struct ChunkParams {
+  int64_t L, Q, nc;   // sequence length, chunk length (a multiple of 128), chunks per sequence
+  int H, G, cpb;      // heads, groups, chunks per CTA
+  int64_t nseq;       // B * H
+  const float* lam;   // [B,H,nc,Q] chunk-local cumulative sums of dt * A
+  float* states;      // [B,H,nc,N,P]
+};
+
+enum { CFULL0 = 3 * STAGES, CFREE0 = 3 * STAGES + 2, NBAR_C = 3 * STAGES + 4 };
+constexpr uint32_t SMEM_BYTES_C = OFF_BAR + NBAR_C * 8 + 16 + 1024;  // + alignment slack
+
+__global__ void __launch_bounds__(THREADS, 1)
+    k_ssd_chunk_states(ChunkParams p, const __grid_constant__ CUtensorMap map_x,
+                       const __grid_constant__ CUtensorMap map_b) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(sm);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_BAR + NBAR_C * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_BAR + NBAR_C * 8 + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // sequence-fastest, as the other chunk grids
+  const int64_t bh = (int64_t)blockIdx.x % p.nseq;
+  const int64_t c0 = (int64_t)blockIdx.x / p.nseq * p.cpb;          // first chunk of this CTA
+  const int nch = (int)min((int64_t)p.cpb, p.nc - c0);              // chunks of this CTA
+  const int b = (int)(bh / p.H), h = (int)(bh % p.H);
+  const int g = h / (p.H / p.G);
+  const int tpc = (int)(p.Q / T);                                     // tiles per whole chunk
+  auto tiles_of = [&](int i) {  // tiles of the CTA's chunk i (the sequence's last chunk may be short)
+    const int64_t t0 = (c0 + i) * p.Q;
+    return (int)ceil_div(min(p.Q, p.L - t0), (int64_t)T);
+  };
+
+  if (warp == 1) tmem_alloc(tmem_slot, 2 * TMEM_COLS);
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&bar[FULL0 + i], 1);
+      mbar_init(&bar[READY0 + i], BUILD);
+      mbar_init(&bar[EMPTY0 + i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[CFULL0 + i], 1);
+      mbar_init(&bar[CFREE0 + i], BUILD);
+    }
+    fence_mbar_init();
+    prefetch_tmap(&map_x);
+    prefetch_tmap(&map_b);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int k = 0, issued = 0;  // tile counter over the CTA's chunks
+      bool ok = true;
+      for (int i = 0; i < nch && ok; ++i) {
+        const int nt = tiles_of(i);
+        for (int tt = 0; tt < nt; ++tt, ++k) {
+          const int st = k % STAGES;
+          if (k >= STAGES && !wait_bar(&bar[EMPTY0 + st], ((k / STAGES) + 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int t0 = (int)((c0 + i) * p.Q + (int64_t)tt * T);
+          uint8_t* sx = sm + st * STAGE;
+          mbar_arrive_expect_tx(&bar[FULL0 + st], STAGE);
+          tma_load_4d(sx + OFF_X, &map_x, &bar[FULL0 + st], 0, h, t0, b);
+          tma_load_4d(sx + OFF_B, &map_b, &bar[FULL0 + st], 0, g, t0, b);
+          tma_load_4d(sx + OFF_B + TILE, &map_b, &bar[FULL0 + st], 64, g, t0, b);
+          issued = k + 1;
+        }
+      }
+      for (int q = (issued > STAGES ? issued - STAGES : 0); q < issued; ++q) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&bar[FULL0 + q % STAGES], (q / STAGES) & 1) && globaltimer_ns() - t0 < 1000000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idB = idesc_bf16(128, 64, true, true);
+      const uint64_t dB = smem_desc(sbase + OFF_B, TILE, 1024);
+      const uint64_t dX = smem_desc(sbase + OFF_X, TILE, 1024);
+      int k = 0;
+      bool ok = true;
+      for (int i = 0; i < nch && ok; ++i) {
+        const int a = i & 1;
+        // the accumulator of chunk i-2 has been read out
+        if (i >= 2 && !wait_bar(&bar[CFREE0 + a], ((i - 2) >> 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        const int nt = tiles_of(i);
+        for (int tt = 0; tt < nt; ++tt, ++k) {
+          const int st = k % STAGES;
+          if (!wait_bar(&bar[READY0 + st], (k / STAGES) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t cB = desc_advance(dB, st * STAGE), cX = desc_advance(dX, st * STAGE);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ss(tmem + a * TMEM_COLS, desc_advance(cB, ks * 2048), desc_advance(cX, ks * 2048), idB,
+                   (tt > 0 || ks > 0) ? 1u : 0u);
+          mma_commit(&bar[EMPTY0 + st]);
+        }
+        mma_commit(&bar[CFULL0 + a]);  // chunk i's state is complete (also after an abort)
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ weights, X'', read-out
+    const int r = threadIdx.x - 64;   // token row of the tile
+    const int q = warp & 3;           // TMEM lane quarter of the read-out
+    const int n = q * 32 + lane;      // state row n of the read-out
+    const float* lamh = p.lam + bh * p.nc * p.Q;
+    auto read_out = [&](int i) {      // chunk i's accumulator to states[b,h,c0+i]
+      const int a = i & 1;
+      const bool done = wait_bar(&bar[CFULL0 + a], (i >> 1) & 1, abort_flag);
+      tc_fence_after();
+      float* dst = p.states + ((bh * p.nc + c0 + i) * 128 + n) * (int64_t)P;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + a * TMEM_COLS + 32 * c, v);
+        tmem_wait_ld();
+        if (done) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + 32 * c + e) =
+                make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
+                            __uint_as_float(v[e + 3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar[CFREE0 + a]);
+    };
+    int k = 0;
+    bool ok = true;
+    for (int i = 0; i < nch; ++i) {
+      const float* lc = lamh + (c0 + i) * p.Q;
+      const float lend = lc[p.Q - 1] * kLog2e;  // past L, lam stays at its last value
+      const int nt = tiles_of(i);
+      for (int tt = 0; tt < nt; ++tt, ++k) {
+        const int st = k % STAGES;
+        const float w = ex2f_approx(lend - lc[tt * T + r] * kLog2e);
+        if (ok) ok = wait_bar(&bar[FULL0 + st], (k / STAGES) & 1, abort_flag);
+        if (ok) {
+          const uint32_t row = sbase + st * STAGE + OFF_X;
+          const float2 w2 = make_float2(w, w);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t ad = row + swz128((uint32_t)r, (uint32_t)(8 * c));
+            uint4 v;
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(ad));
+            uint32_t* u = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f =
+                  mul2(make_float2(__uint_as_float(u[e] << 16), __uint_as_float(u[e] & 0xFFFF0000u)), w2);
+              u[e] = pack_bf16(f.x, f.y);
+            }
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(ad), "r"(v.x), "r"(v.y), "r"(v.z),
+                         "r"(v.w)
+                         : "memory");
+          }
+          fence_async_smem();
+        }
+        mbar_arrive(&bar[READY0 + st]);
+      }
+      if (i > 0) read_out(i - 1);  // overlaps the MMAs of chunk i
+    }
+    if (nch > 0) read_out(nch - 1);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * TMEM_COLS);
+    tmem_relinquish();
+  }
+}
+
 }  // namespace lean
 
 // The segments of sequences seq0, seq0 + 1, ... (p.Q = the segment length, a
@@ -334,4 +533,55 @@ cudaError_t launch_segment_states(const Problem& p, int64_t seq0, float* states,
   return cudaGetLastError();
 }
 
+}  // namespace ssd
+
+namespace ssd {
+// Step 2 of the step-by-step scan on tensor cores (bf16, P = 64, N = 128, Q a
+// multiple of 128): chunk_states[b,h,c] from a zero start, lam from step 1.
+cudaError_t launch_chunk_states_seq(const Problem& p, const float* lam, float* states, cudaStream_t st) {
+  using namespace lean;
+  if (!p.x || !p.Bm || !lam || !states || p.Q % T != 0 || p.P != P || p.N != 128) return cudaErrorInvalidValue;
+  const int64_t nseq = p.B * p.H;
+  // chunks per CTA: enough CTAs for several waves on the SMs, and at least
+  // 16 tiles per CTA where the sequence has them (the pipeline fill of a CTA
+  // is a few tiles' time)
+  const int64_t tiles_per_chunk = p.Q / T;
+  int64_t cpb = ceil_div((int64_t)16, tiles_per_chunk);
+  const int64_t want = 4 * (int64_t)split::sm_count();
+  while (cpb > 1 && nseq * ceil_div(p.nc, cpb) < want) cpb = ceil_div(cpb, (int64_t)2);
+  if (cpb > p.nc) cpb = p.nc;
+  const int64_t ctas = nseq * ceil_div(p.nc, cpb);
+  if (ctas <= 0 || ctas >= (1ll << 31)) return cudaErrorInvalidValue;
+  CUtensorMap mx, mb;
+  const uint32_t box[4] = {64, 1, (uint32_t)T, 1};
+  const uint64_t dx[4] = {(uint64_t)P, (uint64_t)p.H, (uint64_t)p.L, (uint64_t)p.B};
+  const uint64_t sx[3] = {(uint64_t)P * 2, (uint64_t)p.ldx * 2, (uint64_t)p.sx * 2};
+  const uint64_t dbc[4] = {(uint64_t)128, (uint64_t)p.G, (uint64_t)p.L, (uint64_t)p.B};
+  const uint64_t sbc[3] = {(uint64_t)128 * 2, (uint64_t)p.ldbc * 2, (uint64_t)p.sbc * 2};
+  if (!tma::encode_bf16_4d_cached(&mx, p.x, dx, sx, box) || !tma::encode_bf16_4d_cached(&mb, p.Bm, dbc, sbc, box))
+    return cudaErrorInvalidValue;
+  ChunkParams kp;
+  kp.L = p.L;
+  kp.Q = p.Q;
+  kp.nc = p.nc;
+  kp.H = (int)p.H;
+  kp.G = (int)p.G;
+  kp.cpb = (int)cpb;
+  kp.nseq = nseq;
+  kp.lam = lam;
+  kp.states = states;
+  static std::atomic<unsigned long long> attr_set{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_set.load() & bit)) {
+    e = cudaFuncSetAttribute((const void*)k_ssd_chunk_states, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SMEM_BYTES_C);
+    if (e != cudaSuccess) return e;
+    attr_set.fetch_or(bit);
+  }
+  k_ssd_chunk_states<<<(unsigned)ctas, THREADS, SMEM_BYTES_C, st>>>(kp, mx, mb);
+  return cudaGetLastError();
+}
 }  // namespace ssd

@@ -22,7 +22,6 @@ int fused_kernels_per_call(const Problem& p);
 size_t tc_workspace_bytes(const Problem& p);
 size_t pair_workspace_bytes(const Problem& p);
 
-cudaError_t launch_chunk_state_tc(const Problem& p, const float* lam, float* states, cudaStream_t st);
 cudaError_t launch_chunk_scan_tc(const Problem& p, const float* lam, const float* prev, cudaStream_t st);
 // Segments per sequence of the two-head kernel's schedule: 0 = chosen from
 // the shape (the default), n > 0 = n wherever n divides the sub-chunks
@@ -38,6 +37,9 @@ cudaError_t launch_segment_states(const Problem& p, int64_t whole, float* states
                                   cudaStream_t st);
 cudaError_t launch_segment_scan(const Problem& p, int64_t whole, const float* prev, const float* init,
                                 float* final_state, cudaStream_t st);
+// Step 2 on tensor cores: every chunk's end state from a zero start, several
+// consecutive chunks of one (batch, head) per CTA (csrc/ssd_lean.cu).
+cudaError_t launch_chunk_states_seq(const Problem& p, const float* lam, float* states, cudaStream_t st);
 // The whole scan in one launch.  With a workspace of pair_workspace_bytes
 // the two-head kernel runs segments of the sequences round-robin on one
 // persistent CTA per SM; without one (NULL / too small) every CTA runs whole

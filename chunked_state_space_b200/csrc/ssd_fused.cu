@@ -88,6 +88,7 @@ struct Params {
   // rows of x, shared tiles of B and C), chunk slot (sequence - seq0) * nc +
   // chunk.
   int64_t whole, seq0, nseq;
+  int cpc;  // MULTI: chunks per CTA (consecutive chunks of one sequence; state reloaded at each)
   const __nv_bfloat16* x;
   int64_t sx, ldx;    // batch and token strides of x
   __nv_bfloat16* y;
@@ -199,9 +200,10 @@ __device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
 
 // XDT: the dt-scaled input variant; NORM: a layer of a stack with the RMS norm
 // fused (input scaled from ss_in when given, sums of squares to ss_out when
-// given).  Separate instantiations, so that the plain scan carries none of
-// their per-column factors and sums.
-template <bool XDT, bool NORM>
+// given); MULTI: the chunk-scan step with cpc consecutive chunks per CTA, each
+// started from its given state.  Separate instantiations, so that the plain
+// scan carries none of their per-column factors, sums and reloads.
+template <bool XDT, bool NORM, bool MULTI = false>
 __global__ void __launch_bounds__(THREADS, 1)
     k_ssd_fused(Params p, const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
                 const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_y) {
@@ -225,11 +227,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   const bool chunked = p.mode != MODE_SCAN && (int64_t)blockIdx.x >= p.whole;
   const int64_t cb = (int64_t)blockIdx.x - p.whole;                // chunk CTA index (step modes)
   const int64_t bh = chunked ? p.seq0 + cb % p.nseq : (int64_t)blockIdx.x;
-  const int64_t cidx = chunked ? cb / p.nseq : 0;                  // chunk of this CTA (step modes)
+  // chunk of this CTA (step modes; MULTI: its first of cpc)
+  const int64_t cidx = chunked ? (MULTI ? cb / p.nseq * p.cpc : cb / p.nseq) : 0;
   const int b = (int)(bh / p.H), h = (int)(bh % p.H);
   const int g = h / (p.H / p.G);
   const int t_base = (int)(cidx * p.Q);                          // first token of this CTA
-  const int nsub = chunked ? (int)ceil_div(min((int64_t)p.Q, p.L - t_base), (int64_t)T) : p.nsub;
+  const int nsub = chunked ? (int)ceil_div(min((MULTI ? p.cpc : 1) * p.Q, p.L - t_base), (int64_t)T) : p.nsub;
   const int64_t cslot = (bh - p.seq0) * p.nc + cidx;            // chunk slot (step modes)
   const float* init_ptr = chunked ? (p.mode == MODE_CHUNK_SCAN ? p.chunk_init + cslot * NS * P : nullptr)
                                   : (p.init ? p.init + bh * NS * P : nullptr);
@@ -512,8 +515,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       float lam1 = v + pre;       // token 2a+1
       float lam0 = lam1 - l1;     // token 2a
       if (lamc) {                 // step modes: sub-chunk-local sums from step 1's output
-        const float* ls = lamc + jt * T;
-        const float base0 = (jt == 0) ? 0.f : ls[-1];
+        const float* ls = lamc + jt * T;  // chunks of one sequence are contiguous in step 1's output
+        bool chunk_start = jt == 0;
+        if constexpr (MULTI) chunk_start = (jt * T) % p.Q == 0;
+        const float base0 = chunk_start ? 0.f : ls[-1];
         lam0 = ls[2 * a] - base0;
         lam1 = ls[2 * a + 1] - base0;
       }
@@ -755,6 +760,19 @@ __global__ void __launch_bounds__(THREADS, 1)
           s[32 * c + i + 1] = o.y;
         }
       }
+      if constexpr (MULTI) {
+        // the next sub-chunk starts a chunk: its products take that chunk's given
+        // state, not this running one (y of this sub-chunk does not use it)
+        if (j + 1 < nsub && ((int64_t)(j + 1) * T) % p.Q == 0) {
+          const float4* src = reinterpret_cast<const float4*>(
+              p.chunk_init + (cslot + (int64_t)(j + 1) * T / p.Q) * NS * P + (int64_t)r * P);
+#pragma unroll
+          for (int i = 0; i < P / 4; ++i) {
+            const float4 v = src[i];
+            s[4 * i] = v.x; s[4 * i + 1] = v.y; s[4 * i + 2] = v.z; s[4 * i + 3] = v.w;
+          }
+        }
+      }
       if (ok) publish_state();
       if (r == 0) mark(j, EV_STATE_PUB);
       // y_t = y_intra + exp(lam_t) y_inter + D x_t, staged as a 128-B-swizzled tile
@@ -950,6 +968,7 @@ struct GridSplit {
   const float* init = nullptr;
   float* final_state = nullptr;
   bool programmatic = false;  // may start while the kernel before it finishes
+  int cpc = 0;                // chunk-scan step: consecutive chunks per CTA (0: one)
 };
 
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
@@ -1021,10 +1040,17 @@ cudaError_t launch_segment_scan(const Problem& p, int64_t whole, const float* pr
   return launch_mode(p, fused::MODE_CHUNK_SCAN, nullptr, prev, nullptr, p.y, nullptr, st, 0, nullptr, sp);
 }
 
-// Step 4 on tensor cores: one CTA per (batch, head, chunk), starting from
-// prev[b,h,c], writing the chunk's outputs.
+// Step 4 on tensor cores: consecutive chunks of one (batch, head) per CTA,
+// each started from prev[b,h,c], writing the chunks' outputs.
 cudaError_t launch_chunk_scan_tc(const Problem& p, const float* lam, const float* prev, cudaStream_t st) {
-  return launch_mode(p, fused::MODE_CHUNK_SCAN, lam, prev, nullptr, p.y, nullptr, st);
+  // consecutive chunks per CTA, as many as keep four CTAs per SM busy (up to
+  // 16 sub-chunks): the pipeline fill of a CTA is about two sub-chunks' time
+  GridSplit sp;
+  const int64_t spc = p.Q / fused::T, nseq = p.B * p.H, want = 4 * (int64_t)split::sm_count();
+  int64_t cpc = ceil_div((int64_t)16, spc);
+  while (cpc > 1 && nseq * ceil_div(p.nc, cpc) < want) cpc = ceil_div(cpc, (int64_t)2);
+  sp.cpc = (int)(cpc < p.nc ? cpc : p.nc);
+  return launch_mode(p, fused::MODE_CHUNK_SCAN, lam, prev, nullptr, p.y, nullptr, st, 0, nullptr, sp);
 }
 
 static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, const float* init, float* final_state,
@@ -1079,6 +1105,8 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   kp.whole = step_mode ? split.whole : 0;
   kp.seq0 = step_mode ? split.seq0 : 0;
   kp.nseq = p.B * p.H - kp.seq0;
+  kp.cpc = (mode == MODE_CHUNK_SCAN && split.cpc > 1) ? split.cpc : 1;
+  const bool multi = kp.cpc > 1;
   kp.x = static_cast<const __nv_bfloat16*>(p.x);
   kp.sx = p.sx;
   kp.ldx = p.ldx;
@@ -1099,14 +1127,16 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   if (e != cudaSuccess) return e;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set.load() & bit)) {
-    const void* fns[4] = {(const void*)k_ssd_fused<false, false>, (const void*)k_ssd_fused<true, false>,
-                          (const void*)k_ssd_fused<false, true>, (const void*)k_ssd_fused<true, true>};
-    for (int i = 0; i < 4 && e == cudaSuccess; ++i)
+    const void* fns[5] = {(const void*)k_ssd_fused<false, false>, (const void*)k_ssd_fused<true, false>,
+                          (const void*)k_ssd_fused<false, true>, (const void*)k_ssd_fused<true, true>,
+                          (const void*)k_ssd_fused<false, false, true>};
+    for (int i = 0; i < 5 && e == cudaSuccess; ++i)
       e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set.fetch_or(bit);
   }
-  const int64_t ctas = mode == fused::MODE_SCAN ? p.B * p.H : kp.whole + (p.B * p.H - kp.seq0) * p.nc;
+  const int64_t ctas = mode == fused::MODE_SCAN ? p.B * p.H
+                                                : kp.whole + (p.B * p.H - kp.seq0) * ceil_div(p.nc, (int64_t)kp.cpc);
   if (kp.whole < 0 || kp.whole > kp.seq0 || kp.seq0 > p.B * p.H || ctas <= 0 || ctas >= (1ll << 31))
     return cudaErrorInvalidValue;
   // the dt-scaled input whenever dt is read here (the whole scan, and the step
@@ -1122,6 +1152,10 @@ static cudaError_t launch_mode(const Problem& p, int mode, const float* lam, con
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = split.programmatic ? 1 : 0;
+  if (multi) {
+    if (xdt || nrm || kp.whole != 0) return cudaErrorInvalidValue;
+    return cudaLaunchKernelEx(&cfg, k_ssd_fused<false, false, true>, kp, mx, mb, mc, my);
+  }
   if (xdt && nrm) return cudaLaunchKernelEx(&cfg, k_ssd_fused<true, true>, kp, mx, mb, mc, my);
   if (xdt) return cudaLaunchKernelEx(&cfg, k_ssd_fused<true, false>, kp, mx, mb, mc, my);
   if (nrm) return cudaLaunchKernelEx(&cfg, k_ssd_fused<false, true>, kp, mx, mb, mc, my);

@@ -1046,10 +1046,7 @@ cudaError_t launch_chunk_scan_tc(const Problem& p, const float* lam, const float
   // consecutive chunks per CTA, as many as keep four CTAs per SM busy (up to
   // 16 sub-chunks): the pipeline fill of a CTA is about two sub-chunks' time
   GridSplit sp;
-  const int64_t spc = p.Q / fused::T, nseq = p.B * p.H, want = 4 * (int64_t)split::sm_count();
-  int64_t cpc = ceil_div((int64_t)16, spc);
-  while (cpc > 1 && nseq * ceil_div(p.nc, cpc) < want) cpc = ceil_div(cpc, (int64_t)2);
-  sp.cpc = (int)(cpc < p.nc ? cpc : p.nc);
+  sp.cpc = (int)step_chunks_per_cta(p);
   return launch_mode(p, fused::MODE_CHUNK_SCAN, lam, prev, nullptr, p.y, nullptr, st, 0, nullptr, sp);
 }
 

@@ -536,20 +536,27 @@ cudaError_t launch_segment_states(const Problem& p, int64_t seq0, float* states,
 }  // namespace ssd
 
 namespace ssd {
+static int g_step_cpc = 0;  // forced by a self-test (0: chosen from the shape)
+void set_step_chunks_per_cta(int n) { g_step_cpc = n > 0 ? n : 0; }
+// Consecutive chunks per CTA of the tensor-core step kernels (steps 2 and 4):
+// up to 16 tiles per CTA (a CTA's pipeline fill is a few tiles' time), fewer
+// where that would leave less than four CTAs per SM.
+int64_t step_chunks_per_cta(const Problem& p) {
+  int64_t cpc = g_step_cpc > 0 ? g_step_cpc : ceil_div((int64_t)16, p.Q / lean::T);
+  if (g_step_cpc <= 0) {
+    const int64_t nseq = p.B * p.H, want = 4 * (int64_t)split::sm_count();
+    while (cpc > 1 && nseq * ceil_div(p.nc, cpc) < want) cpc = ceil_div(cpc, (int64_t)2);
+  }
+  return cpc < p.nc ? cpc : (p.nc > 0 ? p.nc : 1);
+}
+
 // Step 2 of the step-by-step scan on tensor cores (bf16, P = 64, N = 128, Q a
 // multiple of 128): chunk_states[b,h,c] from a zero start, lam from step 1.
 cudaError_t launch_chunk_states_seq(const Problem& p, const float* lam, float* states, cudaStream_t st) {
   using namespace lean;
   if (!p.x || !p.Bm || !lam || !states || p.Q % T != 0 || p.P != P || p.N != 128) return cudaErrorInvalidValue;
   const int64_t nseq = p.B * p.H;
-  // chunks per CTA: enough CTAs for several waves on the SMs, and at least
-  // 16 tiles per CTA where the sequence has them (the pipeline fill of a CTA
-  // is a few tiles' time)
-  const int64_t tiles_per_chunk = p.Q / T;
-  int64_t cpb = ceil_div((int64_t)16, tiles_per_chunk);
-  const int64_t want = 4 * (int64_t)split::sm_count();
-  while (cpb > 1 && nseq * ceil_div(p.nc, cpb) < want) cpb = ceil_div(cpb, (int64_t)2);
-  if (cpb > p.nc) cpb = p.nc;
+  const int64_t cpb = step_chunks_per_cta(p);
   const int64_t ctas = nseq * ceil_div(p.nc, cpb);
   if (ctas <= 0 || ctas >= (1ll << 31)) return cudaErrorInvalidValue;
   CUtensorMap mx, mb;

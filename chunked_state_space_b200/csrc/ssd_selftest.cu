@@ -241,6 +241,13 @@ extern "C" ssd_status ssd_selftest_set_segments(int nseg) {
   return SSD_OK;
 }
 
+// Chunks per CTA of the tensor-core step kernels for the following launches.
+extern "C" ssd_status ssd_selftest_set_step_chunks(int n) {
+  if (n < 0) return SSD_ERR_INVALID_ARG;
+  ssd::set_step_chunks_per_cta(n);
+  return SSD_OK;
+}
+
 // The one-head kernel's segmented form for the following launches: the first
 // `whole` sequences whole, every later one in about nseg segments.
 extern "C" ssd_status ssd_selftest_set_split(int nseg, int64_t whole) {

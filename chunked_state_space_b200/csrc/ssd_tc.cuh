@@ -40,6 +40,10 @@ cudaError_t launch_segment_scan(const Problem& p, int64_t whole, const float* pr
 // Step 2 on tensor cores: every chunk's end state from a zero start, several
 // consecutive chunks of one (batch, head) per CTA (csrc/ssd_lean.cu).
 cudaError_t launch_chunk_states_seq(const Problem& p, const float* lam, float* states, cudaStream_t st);
+// Consecutive chunks per CTA of the tensor-core step kernels (steps 2 and 4),
+// and its self-test override (n > 0: n chunks per CTA; 0: from the shape).
+int64_t step_chunks_per_cta(const Problem& p);
+void set_step_chunks_per_cta(int n);
 // The whole scan in one launch.  With a workspace of pair_workspace_bytes
 // the two-head kernel runs segments of the sequences round-robin on one
 // persistent CTA per SM; without one (NULL / too small) every CTA runs whole

@@ -29,7 +29,8 @@ EXPORTED = ["ssd_status_string", "ssd_version", "ssd_scan_workspace_size", "ssd_
             "ssd_selftest_fused_trace", "ssd_scan_fwd_noalloc",
             "ssd_selftest_timeout", "ssd_scan_fwd_host", "ssd_scan_fwd_host_workspace_size",
             "ssd_scan_fwd_strided", "ssd_selftest_carry_timeout", "ssd_scan_fwd_vdecay",
-            "ssd_selftest_set_segments", "ssd_selftest_set_split", "ssd_scan_fwd_normed"]
+            "ssd_selftest_set_segments", "ssd_selftest_set_split", "ssd_selftest_set_step_chunks",
+            "ssd_scan_fwd_normed"]
 
 
 class SSDError(RuntimeError):
@@ -89,6 +90,7 @@ def lib() -> ctypes.CDLL:
         "ssd_selftest_carry_timeout": (ctypes.c_int, [D] + [_P] * 10 + [ctypes.c_size_t, _P]),
         "ssd_selftest_set_segments": (ctypes.c_int, [ctypes.c_int]),
         "ssd_selftest_set_split": (ctypes.c_int, [ctypes.c_int, ctypes.c_int64]),
+        "ssd_selftest_set_step_chunks": (ctypes.c_int, [ctypes.c_int]),
         "ssd_scan_fwd_normed": (ctypes.c_int, [D, _P, _P, ctypes.c_float] + [_P] * 10),
         "ssd_scan_fwd_vdecay": (ctypes.c_int, [D] + [_P] * 10),
     }
@@ -469,3 +471,9 @@ def ssd_selftest_set_split(nseg: int, whole: int) -> None:
     sequences whole, the rest in about `nseg` segments (nseg 0 = the cost
     model's choice)."""
     _check(lib().ssd_selftest_set_split(int(nseg), int(whole)), "ssd_selftest_set_split")
+
+
+def ssd_selftest_set_step_chunks(n: int) -> None:
+    """Chunks per CTA of the tensor-core step kernels for the following launches
+    (0 = chosen from the shape)."""
+    _check(lib().ssd_selftest_set_step_chunks(int(n)), "ssd_selftest_set_step_chunks")

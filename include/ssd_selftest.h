@@ -127,6 +127,16 @@ ssd_status ssd_selftest_set_segments(int nseg);
  */
 ssd_status ssd_selftest_set_split(int nseg, int64_t whole);
 
+/*
+ * ssd_selftest_set_step_chunks sets how many consecutive chunks of one
+ * (batch, head) sequence each CTA of the tensor-core step kernels handles
+ * (ssd_chunk_state and ssd_chunk_scan, and the step-by-step scan) for the
+ * following launches of this process (host state, not thread-safe): n > 0
+ * forces n (at most the chunks of a sequence), 0 restores the choice from the
+ * shape.  Same results either way.  Returns SSD_ERR_INVALID_ARG for n < 0.
+ */
+ssd_status ssd_selftest_set_step_chunks(int n);
+
 #ifdef __cplusplus
 }
 #endif

@@ -183,6 +183,41 @@ def test_steps_match_oracle_intermediates(case):
     assert rel_err(to_np64(y), ref["y"]) <= tol
 
 
+@pytest.mark.parametrize("chunk,cpc", [(256, 2), (256, 3), (128, 4), (128, 16)])
+def test_step_kernels_with_several_chunks_per_cta(chunk, cpc):
+    """Steps 2 and 4 on tcgen05 with cpc consecutive chunks of a sequence per
+    CTA (the chunk-scan kernel takes the next chunk's given state at each chunk
+    boundary): 1700 tokens give 7 or 14 chunks, so the last CTA of a sequence
+    holds fewer chunks and a ragged last chunk; the unfused scan runs the same
+    kernels end to end."""
+    wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=1700, nheads=3, ngroups=1, chunk=chunk,
+                       init_var=0.1)
+    tol = TOL[wl.io]
+    host = inputs.generate(wl, seed=5)
+    dev = device_inputs(host)
+    args = oracle_args(host)
+    ref = oracle.scan_chunked(*args[:5], wl.chunk, args[5], args[6])
+    x, Bm = dev["x"], dev["B"]
+    dims = ssd.make_dims(x, Bm, wl.chunk)
+    f32 = lambda a: torch.from_numpy(a.astype(np.float32)).cuda()
+    ssd.ssd_selftest_set_step_chunks(cpc)
+    try:
+        cs = ssd.ssd_chunk_state(x, Bm, f32(ref["lam"]), dims)
+        y = ssd.ssd_chunk_scan(x, Bm, dev["C"], f32(ref["lam"]), f32(ref["prev_states"]), dims, D=dev["D"])
+        y2, fin2 = run_scan(dev, wl, unfused=True)
+    finally:
+        ssd.ssd_selftest_set_step_chunks(0)
+    torch.cuda.synchronize()
+    assert rel_err(to_np64(cs), ref["chunk_states"]) <= tol
+    assert rel_err(to_np64(y), ref["y"]) <= tol
+    assert rel_err(to_np64(y2), ref["y"]) <= tol
+    assert rel_err(to_np64(fin2), ref["final"]) <= tol
+    # the chosen split gives the same chunk states to the fp32 rounding of the tiles
+    cs0 = ssd.ssd_chunk_state(x, Bm, f32(ref["lam"]), dims)
+    torch.cuda.synchronize()
+    assert rel_err(to_np64(cs0), to_np64(cs)) <= 1e-5
+
+
 @pytest.mark.parametrize("shape,dtype", [
     ((2, 37, 24, 64), torch.bfloat16),   # 74 rows (not a multiple of 8), 16-byte vectors
     ((1, 5, 3, 5), torch.bfloat16),      # 15 features: the scalar path

@@ -3,9 +3,11 @@ allocate device memory (graph capture in progress, engines that plan memory
 up front, fixed-budget runtimes).  Its scratch is a buffer compiled into
 libssd.so instead of a caller workspace.
 
-The test calls it through the C ABI twice in a row, on different inputs, and
-compares each result with ssd_scan_fwd_unfused (same kernels, caller
-workspace) and with the fp64 oracle, within the parity tolerances.  The file
+The tests call it through the C ABI twice in a row, on different inputs, and
+compare each result with ssd_scan_fwd_unfused (same kernels, caller
+workspace) and with the fp64 oracle, within the parity tolerances; and record
+it into a CUDA graph (where an allocation would fail the capture) and replay
+the graph on new inputs copied into the captured tensors.  The file
 is named so that pytest collects it last; it also passes alone in a fresh
 process.  The refusal of sizes beyond the built-in buffer needs no GPU and is
 checked in the CPU tier (tests/test_abi.py).
@@ -55,3 +57,34 @@ def test_noalloc_matches_unfused_twice(name, over):
         assert rel_err(to_np64(y), y64) <= TOL[wl.io]
         assert rel_err(to_np64(fin), f64) <= TOL[wl.io]
 
+
+def test_noalloc_recorded_in_cuda_graph():
+    """The call the entry point exists for: inside an open stream capture.  One
+    eager call first (the one-time set-up: kernel attributes, the scratch
+    address), then the call is captured and the graph replayed on two further
+    input sets copied into the same tensors."""
+    assert torch.cuda.is_available()
+    wl = inputs.custom("mamba2_130m_layer", batch=2, seqlen=1000, nheads=4, ngroups=2, init_var=0.1)
+    dev = device_inputs(inputs.generate(wl, seed=0))
+    s, _, _ = _noalloc(dev, wl)
+    torch.cuda.synchronize()
+    assert s == 0, ssd.status_string(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        s, y, fin = _noalloc(dev, wl)
+    assert s == 0, ssd.status_string(s)
+    for seed in (1, 2):
+        host = inputs.generate(wl, seed=seed)
+        new = device_inputs(host)
+        for k in dev:
+            dev[k].copy_(new[k])
+        g.replay()
+        y_ref, f_ref = ssd.ssd_scan_fwd_unfused(new["x"], new["dt"], new["A"], new["B"], new["C"], new["D"],
+                                                new["init"], chunk=wl.chunk)
+        torch.cuda.synchronize()
+        assert rel_err(to_np64(y), to_np64(y_ref)) <= TOL[wl.io]
+        assert rel_err(to_np64(fin), to_np64(f_ref)) <= TOL[wl.io]
+        y64, f64 = oracle.scan_recurrence(*oracle_args(host))
+        assert rel_err(to_np64(y), y64) <= TOL[wl.io]
+        assert rel_err(to_np64(fin), f64) <= TOL[wl.io]
+    del g

@@ -322,7 +322,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int nch = (int)min((int64_t)p.cpb, p.nc - c0);              // chunks of this CTA
   const int b = (int)(bh / p.H), h = (int)(bh % p.H);
   const int g = h / (p.H / p.G);
-  const int tpc = (int)(p.Q / T);                                     // tiles per whole chunk
   auto tiles_of = [&](int i) {  // tiles of the CTA's chunk i (the sequence's last chunk may be short)
     const int64_t t0 = (c0 + i) * p.Q;
     return (int)ceil_div(min(p.Q, p.L - t0), (int64_t)T);

@@ -659,6 +659,8 @@ def timed_steps(step, args, stream, dev, local, world, flush=None):
         step()
         ev[i][1].record(stream)
     t_end.record(stream)
+    while not t_end.query():  # wait without holding the GIL, so the clock sampler keeps polling
+        time.sleep(0.001)
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
     if world > 1:

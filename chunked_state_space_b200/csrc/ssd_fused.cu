@@ -13,7 +13,8 @@
 //   b_intra = B_j^T X'_j,  X'_j = diag(exp(lam_end - lam_s)) X_j
 //   (with the dt-scaled input every column s of P and row s of X' also
 //   carries dt_s)
-//   y_t     = y_intra + exp(lam_t) y_inter + D x_t    (fp32; x_t re-read from L2)
+//   y_t     = y_intra + exp(lam_t) y_inter + D x_t    (fp32; x_j copied from its stage
+//             tile into TMEM, over P's first 32 columns once the products are done)
 //   s_j     = exp(lam_end) s_{j-1} + b_intra              (fp32, registers)
 // Warp roles (384 threads): warp 2 issues TMA loads; warp 3 owns TMEM and
 // issues MMAs; warps 0-1 load dt one sub-chunk ahead, scan lam, form the
@@ -22,7 +23,7 @@
 // publish its bf16 copy.  The mask needs exp(lam_t - lam_s) only inside the
 // diagonal 32x32 blocks: below them it is exp(lam_t - lam_r) exp(lam_r - lam_s)
 // with r the last column of the block (both factors <= 1).
-// TMEM holds two 256-column buffers [S -> P | y_inter][y_intra][b_intra] so sub-chunk
+// TMEM holds two 256-column buffers [S -> P -> x | y_inter][y_intra][b_intra] so sub-chunk
 // j+1's S and mask overlap sub-chunk j's products and epilogue.  Every wait is bounded; a timeout
 // raises g_device_status and the roles drain without further waits.
 #include <atomic>
@@ -53,7 +54,7 @@ constexpr uint32_t OFF_DTS = OFF_ECOL + 4 * T * 4;   // float [4][128]: the inpu
 constexpr uint32_t OFF_RN = OFF_DTS + 4 * T * 4;     // float [4][128]: r_t of the normalised input
 constexpr uint32_t OFF_WTOT = OFF_RN + 4 * T * 4;
 constexpr uint32_t OFF_BAR = OFF_WTOT + 64;
-constexpr uint32_t NBAR = 20;
+constexpr uint32_t NBAR = 22;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
@@ -116,7 +117,8 @@ enum {
 // barrier indices
 enum {
   FULL0 = 0, EMPTY0 = 2, SFULL0 = 4, PFULL0 = 6, CFULL0 = 8, TEMPTY0 = 10, STATEFULL = 12, DRAIN = 13, LAMRDY0 = 14,
-  YFREE0 = 18  // [X' buffer]: the y tile staged there has been read by its TMA store
+  YFREE0 = 18,  // [X' buffer]: the y tile staged there has been read by its TMA store
+  XFULL0 = 20   // [TMEM buffer]: the sub-chunk's x tile copied into its columns 0-31
 };
 constexpr int AUX = 64;  // threads of warps 0-1
 // Warp w runs on SM sub-partition w % 4 and may only touch TMEM lane quarter
@@ -262,6 +264,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&bar[CFULL0 + i], 1);
       mbar_init(&bar[TEMPTY0 + i], T);
       mbar_init(&bar[YFREE0 + i], 1);
+      mbar_init(&bar[XFULL0 + i], 1);
     }
     mbar_init(&bar[STATEFULL], T);
     mbar_init(&bar[DRAIN], 1);
@@ -320,11 +323,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == W_MMA) {
     // ------------------------------------------------------------ MMA issuer
-    // Polls two queues and issues whichever is ready: the products c(jc) of
-    // sub-chunk jc (on the state's critical path, checked first) and S(js) of
-    // a later sub-chunk.  S(js) needs its stage loaded and its TMEM buffer
-    // released by the epilogue of js-2; c(jc) needs P and X' (PFULL) and the
-    // bf16 state b(jc-1) (STATEFULL).
+    // Polls three queues and issues whichever is ready: the products c(jc) of
+    // sub-chunk jc (on the state's critical path, checked first), the copy of
+    // the x tile of sub-chunk jx into TMEM for the epilogue's skip term, and
+    // S(js) of a later sub-chunk.  S(js) needs its stage loaded and its TMEM
+    // buffer released by the epilogue of js-2; c(jc) needs P and X' (PFULL) and
+    // the bf16 state b(jc-1) (STATEFULL); the copy goes over P's first 32
+    // columns, so it waits for the products of jx to complete (an MMA and a
+    // later tcgen05.cp of one thread are not ordered by the pipe), and the
+    // stage of jx is released only after it.
     if (lane == 0) {
       const uint32_t idS = idesc_bf16(128, 128, false, false);
       const uint32_t idY = idesc_bf16(128, 64, false, true);
@@ -337,10 +344,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint64_t dX = smem_desc(sbase + OFF_X, TILE, 1024);    // MN-major (B of y_intra)
       const uint64_t dXp = smem_desc(sbase + OFF_XP, TILE, 1024);  // MN-major (B of b_intra)
       const uint64_t dPrev = smem_desc(sbase + OFF_PREV, TILE, 1024);
-      int js = 0, jc = 0;
+      const uint64_t dXk = smem_desc(sbase + OFF_X, 16, 1024);     // K-major rows (the copy's source)
+      int js = 0, jc = 0, jx = 0;
       uint32_t idle = 0;
       uint64_t t_last = globaltimer_ns();
-      while (jc < nsub) {
+      while (jx < nsub) {
         bool progress = false;
         if (jc < js && mbar_test_wait(&bar[PFULL0 + (jc & 1)], (jc >> 1) & 1) &&
             mbar_test_wait(&bar[STATEFULL], jc & 1)) {
@@ -362,9 +370,20 @@ __global__ void __launch_bounds__(THREADS, 1)
             mma_ss(base + 64, desc_advance(cC, (ks >> 2) * TILE + (ks & 3) * 32), desc_advance(dPrev, ks * 2048), idY,
                    ks > 0);
           mma_commit(&bar[CFULL0 + buf]);
-          mma_commit(&bar[EMPTY0 + st]);
           mark(jc, EV_C_ISSUED);
           ++jc;
+          progress = true;
+        }
+        if (jx < jc && mbar_test_wait(&bar[CFULL0 + (jx & 1)], (jx >> 1) & 1)) {
+          const int st = jx & 1, buf = jx & 1;
+          tc_fence_after();
+          const uint64_t xs = desc_advance(dXk, st * STAGE);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)  // x row t -> lane t, bf16 pairs in columns 8k .. 8k+7
+            tmem_cp_128x256b(tmem + buf * 256 + 8 * k, desc_advance(xs, k * 32));
+          mma_commit(&bar[XFULL0 + buf]);
+          mma_commit(&bar[EMPTY0 + st]);
+          ++jx;
           progress = true;
         }
         if (js < nsub && mbar_test_wait(&bar[FULL0 + (js & 1)], (js >> 1) & 1) &&
@@ -692,21 +711,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int r = q * 32 + lane;  // state row n and output row t
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
     const float Dh = p.D ? p.D[h] : 0.f;
-    // x row of the sub-chunk, loaded before waiting for its products (it is in L2
-    // from the TMA load; the wait hides the latency)
-    const __nv_bfloat16* xg = p.x + (int64_t)b * p.sx + (int64_t)h * P;
-    auto load_x = [&](int j, uint4* xv) {
-      const int64_t tg = (int64_t)t_base + (int64_t)j * T + r;
-      if (j < nsub && tg < p.L) {
-        const uint4* src = reinterpret_cast<const uint4*>(xg + tg * p.ldx);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) xv[c] = src[c];
-      } else {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) xv[c] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    };
-    uint4 xcur[8];
+    // x of each sub-chunk comes from TMEM: the issuer copies the stage's x
+    // tile there once the products are done (the skip term D x_t)
     float s[P];
     if (chunked) grid_dep_wait();  // start states from the kernel before (a programmatic launch)
     if (init_ptr) {
@@ -737,7 +743,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     publish_state();
     for (int j = 0; j < nsub; ++j) {
       const int buf = j & 1;
-      load_x(j, xcur);
       bool ok = ctl.wait(CFULL0 + buf, (j >> 1) & 1);
       if (ok) ok = ctl.wait(LAMRDY0 + (j & 3), (j >> 2) & 1);      // acquire lam of this sub-chunk
       tc_fence_after();
@@ -775,6 +780,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (ok) publish_state();
       if (r == 0) mark(j, EV_STATE_PUB);
+      if (ok) ok = ctl.wait(XFULL0 + buf, (j >> 1) & 1);  // x of this sub-chunk in TMEM
+      tc_fence_after();
       // y_t = y_intra + exp(lam_t) y_inter + D x_t, staged as a 128-B-swizzled tile
       // in the X' buffer of this sub-chunk (free: its products have completed) and
       // written by one TMA store, coalesced, rows past L clipped by the copy.  Per-
@@ -788,14 +795,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       float ss = 0.f;  // sum of squares of the stored (bf16) y row
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t yi[16], ye[16];
+        uint32_t yi[16], ye[16], xr[8];
         tmem_ld16(base + 128 + 16 * c, yi);
         tmem_ld16(base + 64 + 16 * c, ye);
+        tmem_ld8(base + 8 * c, xr);
         tmem_wait_ld();
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           const int cc = 2 * c + h2;  // 8-column chunk
-          const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xcur[cc]);
+          const uint32_t* xu = xr + 4 * h2;
           uint4 ov;
           uint32_t* o = reinterpret_cast<uint32_t*>(&ov);
 #pragma unroll

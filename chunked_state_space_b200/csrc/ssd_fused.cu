@@ -684,19 +684,21 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int i = 0; i < 16; ++i) pk[i] = 0u;
         }
       };
+      // One 32-column block per TMEM round trip (load, wait, form, store): with
+      // two blocks per round trip, or the next block's load left in flight while
+      // this one is formed, the headline scan measured 6 % and 30 % slower.
 #pragma unroll 1
-      for (int kb = 0; kb < 4; kb += 2) {
-        uint32_t r0[32], r1[32], pk[16];
+      for (int kb = 0; kb < 4; ++kb) {
+        uint32_t r0[32], pk[16];
         // warp-uniform: only blocks on or below the diagonal block are read
-        if (kb <= q) tmem_ld32(tS + 32 * kb, r0);
-        if (kb + 1 <= q) tmem_ld32(tS + 32 * (kb + 1), r1);
-        tmem_wait_ld();
-        if (q == 3 && lane == 0) mark(j, kb == 0 ? EV_MASK_LD : EV_MASK_LD2);
+        if (kb <= q) {
+          tmem_ld32(tS + 32 * kb, r0);
+          tmem_wait_ld();
+        }
+        if (q == 3 && lane == 0 && (kb & 1) == 0) mark(j, kb == 0 ? EV_MASK_LD : EV_MASK_LD2);
         make_block(kb, r0, pk);
         tmem_st16(tS + 16 * kb, pk);
-        make_block(kb + 1, r1, pk);
-        tmem_st16(tS + 16 * (kb + 1), pk);
-        if (q == 3 && lane == 0) mark(j, kb == 0 ? EV_MASK_B01 : EV_MASK_B23);
+        if (q == 3 && lane == 0 && (kb & 1) == 1) mark(j, kb == 1 ? EV_MASK_B01 : EV_MASK_B23);
       }
       tmem_wait_st();
       if (q == 3 && lane == 0) mark(j, EV_MASK_WST);

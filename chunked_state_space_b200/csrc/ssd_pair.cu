@@ -702,17 +702,17 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int i = 0; i < 16; ++i) pk[i] = 0u;
           }
         };
+        // one 32-column block per TMEM round trip (as in the one-head kernel)
 #pragma unroll 1
-        for (int kb = 0; kb < 4; kb += 2) {
-          uint32_t r0[32], r1[32], pk[16];
+        for (int kb = 0; kb < 4; ++kb) {
+          uint32_t r0[32], pk[16];
           // warp-uniform: only blocks on or below the diagonal block are read
-          if (kb <= q) tmem_ld32(tS + 32 * kb, r0);
-          if (kb + 1 <= q) tmem_ld32(tS + 32 * (kb + 1), r1);
-          tmem_wait_ld();
+          if (kb <= q) {
+            tmem_ld32(tS + 32 * kb, r0);
+            tmem_wait_ld();
+          }
           make_block(kb, r0, pk);
           tmem_st16(tP + 16 * kb, pk);
-          make_block(kb + 1, r1, pk);
-          tmem_st16(tP + 16 * (kb + 1), pk);
         }
         tmem_wait_st();
         tc_fence_before();

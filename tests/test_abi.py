@@ -241,3 +241,17 @@ def test_vdecay_entry_rejects(lib):
     # y overlapping Av [H, N]
     assert lib.ssd_scan_fwd_vdecay(ctypes.byref(d), *ptrs[:7], ctypes.c_void_p(BASE + 3 * GB + 16), ptrs[8],
                                    None) == 1
+
+
+def test_selftest_setters_validate_and_reset(lib):
+    """The self-test overrides are host state only: negative values are refused,
+    zero restores the choice from the shape (no GPU needed)."""
+    invalid = ssd.STATUS_NAMES.index("SSD_ERR_INVALID_ARG")
+    assert lib.ssd_selftest_set_segments(-1) == invalid
+    assert lib.ssd_selftest_set_split(-1, 0) == invalid
+    assert lib.ssd_selftest_set_split(0, -1) == invalid
+    assert lib.ssd_selftest_set_step_chunks(-1) == invalid
+    for n in (3, 0):
+        ssd.ssd_selftest_set_segments(n)
+        ssd.ssd_selftest_set_split(n, n)
+        ssd.ssd_selftest_set_step_chunks(n)
